@@ -1,0 +1,200 @@
+"""Python binding of the B200 AQLM library (include/aqlm.h), via ctypes.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libaqlm_b200.so.  torch provides device memory and the current
+stream; outputs that the caller does not pass are allocated with torch.
+There is no CPU fallback: if the library is missing the calls raise.
+
+Layouts (see include/aqlm.h):
+  codes      [d_out, d_in/8, M]  uint8 (B = 8) or int16 (B = 16, read unsigned)
+  codebooks  [M, 2^B, 8]          float16
+  scales     [d_out]              float16 (a [d_out, 1, 1, 1] tensor is accepted)
+  x / y      [T, d_in] / [T, d_out] float16      (aqlm_gemv, T <= 16)
+  X / Y      [T, d_in] / [T, d_out] bfloat16     (aqlm_gemm)
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libaqlm_b200.so")
+
+AQLM_OK = 0
+AQLM_ERR_INVALID_ARG = 1
+AQLM_ERR_UNSUPPORTED = 2
+AQLM_ERR_MISALIGNED = 3
+AQLM_ERR_WORKSPACE = 4
+AQLM_ERR_CUDA = 5
+AQLM_ERR_TIMEOUT = 6
+GEMV_MAX_TOKENS = 16
+
+# Every entry point declared in include/aqlm.h.
+EXPORTS = ["aqlm_gemv", "aqlm_gemv_workspace_bytes", "aqlm_dequant", "aqlm_gemm",
+           "aqlm_gemm_workspace_bytes", "aqlm_gemm_check", "aqlm_bf16_gemm", "aqlm_decode_indices",
+           "aqlm_test_gemm_timeout", "aqlm_status_string", "aqlm_version"]
+
+
+class AqlmError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("d_out", ctypes.c_int32), ("d_in", ctypes.c_int32), ("group", ctypes.c_int32),
+                ("num_codebooks", ctypes.c_int32), ("codebook_bits", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load_library():
+    """Load libaqlm_b200.so and declare the C signatures (no CUDA call)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m additive_codebook_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz, u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_uint64
+    st = ctypes.c_int
+    sig = {
+        "aqlm_gemv": ([vp, vp, vp, vp, vp, i32, Shape, vp, sz, vp], st),
+        "aqlm_gemv_workspace_bytes": ([Shape, i32], sz),
+        "aqlm_dequant": ([vp, vp, vp, vp, Shape, vp], st),
+        "aqlm_gemm": ([vp, vp, vp, vp, vp, i32, Shape, vp, sz, vp], st),
+        "aqlm_gemm_workspace_bytes": ([Shape, i32], sz),
+        "aqlm_gemm_check": ([vp, sz, vp], st),
+        "aqlm_bf16_gemm": ([vp, vp, vp, i32, i32, i32, vp, vp], st),
+        "aqlm_decode_indices": ([vp, vp, Shape, vp], st),
+        "aqlm_test_gemm_timeout": ([vp, vp, vp, i32, i32, i32, vp, u64, vp], st),
+        "aqlm_status_string": ([st], ctypes.c_char_p),
+        "aqlm_version": ([], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def status_string(status):
+    return load_library().aqlm_status_string(int(status)).decode()
+
+
+def version():
+    return load_library().aqlm_version().decode()
+
+
+def _check(status, where):
+    if status != AQLM_OK:
+        raise AqlmError(status, where)
+
+
+def _p(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def shape_of(codes, d_in=None):
+    """aqlm_shape from a codes tensor [d_out, G, M] (B from its dtype)."""
+    d_out, G, M = codes.shape
+    B = 8 if codes.dtype == torch.uint8 else 16
+    return Shape(d_out, d_in if d_in is not None else G * 8, 8, M, B)
+
+
+def _flat_scales(scales):
+    return scales.reshape(-1)
+
+
+def gemv_workspace_bytes(shape, tokens):
+    return int(load_library().aqlm_gemv_workspace_bytes(shape, tokens))
+
+
+def gemm_workspace_bytes(shape, tokens):
+    return int(load_library().aqlm_gemm_workspace_bytes(shape, tokens))
+
+
+def aqlm_gemv(codes, codebooks, scales, x, y=None, workspace=None, stream=None):
+    """y[T, d_out] = fp16(W^ . x) for x [T, d_in] float16, 1 <= T <= 16."""
+    lib = load_library()
+    shape = shape_of(codes)
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    T = x.shape[0]
+    if y is None:
+        y = torch.empty((T, shape.d_out), dtype=torch.float16, device=x.device)
+    need = lib.aqlm_gemv_workspace_bytes(shape, T)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib.aqlm_gemv(_p(codes), _p(codebooks), _p(_flat_scales(scales)), _p(x), _p(y), T, shape,
+                         _p(workspace), wbytes, _stream(stream)), "aqlm_gemv")
+    return y
+
+
+def aqlm_dequant(codes, codebooks, scales, out=None, stream=None):
+    """W^[d_out, d_in] as bfloat16, bit-exact binary32 steps then RNE."""
+    lib = load_library()
+    shape = shape_of(codes)
+    if out is None:
+        out = torch.empty((shape.d_out, shape.d_in), dtype=torch.bfloat16, device=codes.device)
+    _check(lib.aqlm_dequant(_p(codes), _p(codebooks), _p(_flat_scales(scales)), _p(out), shape, _stream(stream)),
+           "aqlm_dequant")
+    return out
+
+
+def aqlm_gemm(codes, codebooks, scales, X, Y=None, workspace=None, stream=None):
+    """Y[T, d_out] = bf16(X . W^T): dequant into the workspace + tcgen05 GEMM."""
+    lib = load_library()
+    shape = shape_of(codes)
+    T = X.shape[0]
+    if Y is None:
+        Y = torch.empty((T, shape.d_out), dtype=torch.bfloat16, device=X.device)
+    if workspace is None:
+        workspace = torch.empty(lib.aqlm_gemm_workspace_bytes(shape, T), dtype=torch.uint8, device=X.device)
+    _check(lib.aqlm_gemm(_p(codes), _p(codebooks), _p(_flat_scales(scales)), _p(X), _p(Y), T, shape,
+                         _p(workspace), workspace.numel(), _stream(stream)), "aqlm_gemm")
+    return Y, workspace
+
+
+def aqlm_gemm_check(workspace, stream=None):
+    """Synchronise and return the status recorded in the GEMM workspace."""
+    lib = load_library()
+    return lib.aqlm_gemm_check(_p(workspace), workspace.numel(), _stream(stream))
+
+
+def aqlm_bf16_gemm(X, W, Y=None, status=None, stream=None):
+    """Y[T, n] = bf16(X[T, k] . W[n, k]^T) on the tensor cores."""
+    lib = load_library()
+    T, k = X.shape
+    n = W.shape[0]
+    if Y is None:
+        Y = torch.empty((T, n), dtype=torch.bfloat16, device=X.device)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=X.device)
+    _check(lib.aqlm_bf16_gemm(_p(X), _p(W), _p(Y), T, n, k, _p(status), _stream(stream)), "aqlm_bf16_gemm")
+    return Y, status
+
+
+def aqlm_decode_indices(codes, out=None, stream=None):
+    """Indices [d_out, G, M]: uint16 bit patterns held in an int16 tensor."""
+    lib = load_library()
+    shape = shape_of(codes)
+    if out is None:
+        out = torch.empty(codes.shape, dtype=torch.int16, device=codes.device)
+    _check(lib.aqlm_decode_indices(_p(codes), _p(out), shape, _stream(stream)), "aqlm_decode_indices")
+    return out
+
+
+def aqlm_test_gemm_timeout(X, W, Y, status, limit_ns, stream=None):
+    lib = load_library()
+    T, k = X.shape
+    n = W.shape[0]
+    return lib.aqlm_test_gemm_timeout(_p(X), _p(W), _p(Y), T, n, k, _p(status), limit_ns, _stream(stream))

@@ -1,0 +1,121 @@
+// common.cuh -- small device helpers shared by the library's kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+#include "aqlm.h"
+
+namespace aqlm {
+
+constexpr int kGroup = 8;  // g: inputs per group, every supported format
+
+// Layer geometry derived from an aqlm_shape.
+struct Dims {
+    int d_out;
+    int d_in;
+    int G;          // groups per row, d_in / 8
+    int M;          // codebooks
+    int B;          // bits per code
+    int row_bytes;  // bytes of codes per row, G * M * B / 8
+};
+
+inline Dims make_dims(const aqlm_shape &s) {
+    Dims d;
+    d.d_out = s.d_out;
+    d.d_in = s.d_in;
+    d.G = s.d_in / kGroup;
+    d.M = s.num_codebooks;
+    d.B = s.codebook_bits;
+    d.row_bytes = d.G * d.M * d.B / 8;
+    return d;
+}
+
+// ---- cache-hinted global loads (PTX ISA: ld with L1/L2 eviction priority) ----
+
+// L2 eviction policies (PTX createpolicy), passed to cache-hinted loads.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// Streaming read-only 16-byte load: not kept in L1, first out of L2.
+__device__ __forceinline__ uint4 ld_stream_u4(const void *p, uint64_t pol) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+
+// Read-only 16-byte load that should stay resident in L1 and L2 (codebooks).
+__device__ __forceinline__ uint4 ld_keep_u4(const void *p, uint64_t pol) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::evict_last.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+
+// Eight fp16 values packed in a uint4 -> eight floats (exact conversion).
+__device__ __forceinline__ void half8_to_float8(const uint4 &v, float *f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        __half2 h = *reinterpret_cast<const __half2 *>(&w[q]);
+        float2 p = __half22float2(h);
+        f[2 * q] = p.x;
+        f[2 * q + 1] = p.y;
+    }
+}
+
+// Launch through cudaLaunchKernelEx so that the returned error belongs to this
+// launch only.  `pdl` allows programmatic dependent launch: the kernel may
+// start while the previous kernel in the stream finishes, and must execute
+// griddepcontrol.wait before touching memory that kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                          bool pdl, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (pdl) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+inline int num_sms(int device) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device);
+    return n > 0 ? n : 148;
+}
+
+}  // namespace aqlm
+
+// Host-side launchers, one per kernel family (defined in the .cu files).
+namespace aqlm {
+cudaError_t launch_decode_indices(const void *codes, uint16_t *idx, const Dims &d, cudaStream_t st);
+cudaError_t launch_dequant(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                           uint16_t *W, const Dims &d, cudaStream_t st);
+size_t gemv_workspace_bytes(const Dims &d, int tokens);
+cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                        const uint16_t *x, uint16_t *y, int tokens, const Dims &d, float *workspace,
+                        cudaStream_t st);
+cudaError_t launch_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
+                             int32_t *status, cudaStream_t st);
+}  // namespace aqlm

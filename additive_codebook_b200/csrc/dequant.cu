@@ -1,0 +1,118 @@
+// dequant.cu -- code unpacking and bf16 dequantisation.
+//
+// "The AQLM Quantization Algorithm, Explained", section "What is
+// Multi-Codebook Quantization (MCQ)?": a group of g = 8 inputs of a row is
+// the sum of M codewords whose indices are the stored B-bit codes; the sum is
+// scaled by the row's scale.  Section "Why and what do we quantize?": the
+// weights are fetched compressed and dequantised at runtime before the
+// matmul.
+//
+// Both kernels are bound by HBM: decode_indices moves 2-4 bytes per group in
+// and 2M bytes out; dequant reads M*B/8 bytes of codes per group and writes
+// 16 bytes of bf16 (8 values).  One thread owns one group, so a warp's
+// stores cover 512 contiguous bytes and its code loads 64-128 contiguous
+// bytes; the grid is a multiple of the SM count and strides over groups.
+#include "common.cuh"
+
+namespace aqlm {
+namespace {
+
+// idx[n] = unsigned value of code n, n over [d_out][G][M].
+template <int B>
+__global__ void decode_indices_kernel(const void *__restrict__ codes, uint16_t *__restrict__ idx,
+                                      int64_t n_codes) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; n < n_codes; n += stride) {
+        if constexpr (B == 8) {
+            idx[n] = static_cast<const uint8_t *>(codes)[n];
+        } else {
+            idx[n] = static_cast<const uint16_t *>(codes)[n];
+        }
+    }
+}
+
+// W[i][8j+t] = bf16_rn(fp32(s_i) * (C_0[b0][t] + ... + C_{M-1}[b][t])), the
+// additions in codebook order, every operation rounded on its own.
+template <int M, int B>
+__global__ void __launch_bounds__(256) dequant_kernel(const uint8_t *__restrict__ codes,
+                                                      const uint4 *__restrict__ codebooks,
+                                                      const __half *__restrict__ scales,
+                                                      uint4 *__restrict__ W, int G,
+                                                      int64_t n_groups) {
+    constexpr int K = 1 << B;
+    constexpr int kCodeBytes = M * B / 8;
+    // 2x8: both codebooks (2 x 256 codewords x 16 B = 8 KiB) live in shared memory.
+    __shared__ uint4 cb_smem[B == 8 ? M * K : 1];
+    if constexpr (B == 8) {
+        for (int c = threadIdx.x; c < M * K; c += blockDim.x) cb_smem[c] = codebooks[c];
+        __syncthreads();
+    }
+    const uint64_t keep = policy_evict_last();
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t gi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; gi < n_groups; gi += stride) {
+        const uint8_t *cp = codes + gi * kCodeBytes;
+        uint32_t idx[M];
+        if constexpr (B == 8) {
+            const uint16_t pair = *reinterpret_cast<const uint16_t *>(cp);  // M == 2
+            idx[0] = pair & 0xffu;
+            idx[1] = pair >> 8;
+        } else if constexpr (M == 1) {
+            idx[0] = *reinterpret_cast<const uint16_t *>(cp);
+        } else {
+            const uint32_t both = *reinterpret_cast<const uint32_t *>(cp);
+            idx[0] = both & 0xffffu;
+            idx[1] = both >> 16;
+        }
+        float acc[kGroup];
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            const uint4 cw = (B == 8) ? cb_smem[m * K + idx[m]] : ld_keep_u4(codebooks + (size_t)m * K + idx[m], keep);
+            float f[kGroup];
+            half8_to_float8(cw, f);
+#pragma unroll
+            for (int t = 0; t < kGroup; ++t) acc[t] = (m == 0) ? f[t] : __fadd_rn(acc[t], f[t]);
+        }
+        const int64_t row = gi / G;
+        const float s = __half2float(scales[row]);
+        uint32_t out[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const __nv_bfloat16 lo = __float2bfloat16_rn(__fmul_rn(acc[2 * q], s));
+            const __nv_bfloat16 hi = __float2bfloat16_rn(__fmul_rn(acc[2 * q + 1], s));
+            out[q] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+        }
+        W[gi] = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+}
+
+int grid_for(int64_t work, int threads, int per_sm) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int64_t want = (work + threads - 1) / threads;
+    const int64_t cap = (int64_t)num_sms(dev) * per_sm;
+    return (int)(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_decode_indices(const void *codes, uint16_t *idx, const Dims &d, cudaStream_t st) {
+    const int64_t n = (int64_t)d.d_out * d.G * d.M;
+    const int grid = grid_for(n, 256, 8);
+    if (d.B == 8) return launch_kernel(decode_indices_kernel<8>, grid, 256, 0, st, false, codes, idx, n);
+    return launch_kernel(decode_indices_kernel<16>, grid, 256, 0, st, false, codes, idx, n);
+}
+
+cudaError_t launch_dequant(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                           uint16_t *W, const Dims &d, cudaStream_t st) {
+    const int64_t n = (int64_t)d.d_out * d.G;
+    const int grid = grid_for(n, 256, 8);
+    auto c = static_cast<const uint8_t *>(codes);
+    auto cb = reinterpret_cast<const uint4 *>(codebooks);
+    auto s = reinterpret_cast<const __half *>(scales);
+    auto w = reinterpret_cast<uint4 *>(W);
+    if (d.M == 1 && d.B == 16) return launch_kernel(dequant_kernel<1, 16>, grid, 256, 0, st, false, c, cb, s, w, d.G, n);
+    if (d.M == 2 && d.B == 8) return launch_kernel(dequant_kernel<2, 8>, grid, 256, 0, st, false, c, cb, s, w, d.G, n);
+    return launch_kernel(dequant_kernel<2, 16>, grid, 256, 0, st, false, c, cb, s, w, d.G, n);
+}
+
+}  // namespace aqlm

@@ -1,0 +1,386 @@
+// gemm_tcgen05.cu -- dense prefill GEMM on the 5th-generation tensor cores.
+//
+// Y[m][n] = sum_k X[m][k] * W[n][k]: X = the prefill activations [tokens][d_in]
+// and W = the dequantised layer [d_out][d_in], both bf16 and K-major; fp32
+// accumulation; bf16 output rounded to nearest even.  This is the matmul
+// "with dequantized, native-precision parameters" of section "What is
+// Multi-Codebook Quantization (MCQ)?" in "The AQLM Quantization Algorithm,
+// Explained".
+//
+// sm_100a design: a persistent kernel, one CTA per SM, 128x256 output tiles.
+//   warp 0      one thread issues TMA tile loads (128-byte swizzle) into a
+//               4-stage shared-memory ring, each stage guarded by a pair of
+//               mbarriers (full: bytes landed; empty: MMAs done reading);
+//   warp 1      allocates all 512 tensor-memory columns (two 128x256 fp32
+//               accumulators) and one thread issues tcgen05.mma
+//               (cta_group::1, kind::f16, M=128 N=256 K=16), releasing each
+//               ring stage with tcgen05.commit;
+//   warps 2-5   epilogue: tcgen05.ld from the accumulator of the previous
+//               tile while the MMAs of the next tile run into the other one,
+//               bf16 conversion, 16-byte global stores.
+// Every mbarrier wait is bounded in time.  A wait that gives up writes
+// AQLM_ERR_TIMEOUT to the status word, raises a CTA-wide abort flag that the
+// other roles poll, waits (bounded) for its TMA loads and MMAs in flight and
+// frees its tensor memory before returning; nothing traps.
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace aqlm {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int ACC_COLS = BN;           // fp32 columns per accumulator
+constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
+constexpr int kGemmThreads = 192;
+constexpr int kEpiWarps = 4;
+// bf16 x bf16 -> fp32, both operands K-major, M = 128, N = 256
+// (tcgen05 instruction descriptor: D format bits 4-5, A/B format bits 7-12,
+// N >> 3 at bits 17-22, M >> 4 at bits 24-28).
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+struct Bars {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+constexpr size_t kGemmSmem = 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + sizeof(Bars);
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t now_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase of `parity` to complete, for at most `limit_ns`.  On a
+// timeout record the status and raise the abort flag; give up early when
+// another role raised it.
+__device__ bool wait_bounded(uint32_t bar, uint32_t parity, Bars *bars, int32_t *status, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = now_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15) == 0) {
+            if (*reinterpret_cast<volatile int *>(&bars->abort_flag)) return false;
+            if (now_ns() - t0 > limit_ns) {
+                *reinterpret_cast<volatile int *>(&bars->abort_flag) = 1;
+                atomicExch(status, (int32_t)AQLM_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major tile written by TMA with the
+// 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address, 16-byte units
+    d |= (uint64_t)1 << 16;                    // leading byte offset (unused for this layout)
+    d |= (uint64_t)(1024 >> 4) << 32;          // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1 << 46;                    // descriptor version of sm_100
+    d |= (uint64_t)2 << 61;                    // 128-byte swizzle
+    return d;
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                  __nv_bfloat16 *__restrict__ Y, int m_total, int n_total, int k_total, int32_t *status,
+                  unsigned long long limit_ns, int stall_test) {
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte alignment for the swizzled tiles.
+    const uint32_t raw = smem_addr(smem_raw);
+    uint8_t *smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
+    Bars *bars = reinterpret_cast<Bars *>(smem + (size_t)STAGES * STAGE_BYTES);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m_tiles = (m_total + BM - 1) / BM;
+    const int n_tiles = (n_total + BN - 1) / BN;
+    const int num_tiles = m_tiles * n_tiles;
+    const int num_kb = (k_total + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_addr(&bars->full[s]), 1);
+            mbar_init(smem_addr(&bars->empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_addr(&bars->tfull[a]), 1);
+            mbar_init(smem_addr(&bars->tempty[a]), kEpiWarps);
+        }
+        mbar_init(smem_addr(&bars->mma_done), 1);
+        bars->abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(&bars->tmem_base)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0 && !stall_test) {
+            // ---- TMA producer ----
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued_parity[STAGES];
+            for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int mb = tile % m_tiles, nb = tile / m_tiles;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!wait_bounded(smem_addr(&bars->empty[stage]), phase ^ 1, bars, status, limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t full = smem_addr(&bars->full[stage]);
+                    const uint32_t dst = smem_addr(smem + (size_t)stage * STAGE_BYTES);
+                    mbar_expect_tx(full, STAGE_BYTES);
+                    tma_load_2d(dst, &tmap_x, kb * BK, mb * BM, full);
+                    tma_load_2d(dst + A_BYTES, &tmap_w, kb * BK, nb * BN, full);
+                    issued_parity[stage] = (int)phase;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            // No copy may still be landing in shared memory when the CTA exits.
+            for (int s = 0; s < STAGES; ++s) {
+                if (issued_parity[s] >= 0) {
+                    const uint32_t full = smem_addr(&bars->full[s]);
+                    const uint64_t t0 = now_ns();
+                    while (!mbar_try_wait(full, (uint32_t)issued_parity[s]) && now_ns() - t0 < limit_ns) {
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---- MMA issuer ----
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                if (!wait_bounded(smem_addr(&bars->tempty[acc]), acc_phase ^ 1, bars, status, limit_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(acc * ACC_COLS);
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!wait_bounded(smem_addr(&bars->full[stage]), phase, bars, status, limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_addr(smem + (size_t)stage * STAGE_BYTES);
+                    const uint32_t b0 = a0 + A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k) {
+                        // K step of 16 bf16 = 32 bytes inside the 128-byte swizzled row.
+                        mma_bf16(d_tmem, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), kIdesc,
+                                 (kb > 0 || k > 0) ? 1u : 0u);
+                    }
+                    mma_commit(smem_addr(&bars->empty[stage]));
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(smem_addr(&bars->tfull[acc]));
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_phase ^= 1;
+                }
+            }
+            // Tensor memory is freed below only after every issued MMA completed.
+            mma_commit(smem_addr(&bars->mma_done));
+            const uint64_t t0 = now_ns();
+            while (!mbar_try_wait(smem_addr(&bars->mma_done), 0) && now_ns() - t0 < limit_ns) {
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue: warps 2..5, TMEM lane quarter = warp % 4 ----
+        const int quarter = warp & 3;
+        const int row_in_tile = quarter * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            const int mb = tile % m_tiles, nb = tile / m_tiles;
+            bool ok = wait_bounded(smem_addr(&bars->tfull[acc]), acc_phase, bars, status, limit_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            const int m = mb * BM + row_in_tile;
+            const uint32_t t_base = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(t_base + (uint32_t)(c * 32), r);
+                const int n0 = nb * BN + c * 32;
+                if (m < m_total) {
+                    __nv_bfloat16 *dst = Y + (size_t)m * n_total + n0;
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        if (n0 + 8 * v < n_total) {
+                            uint32_t p[4];
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(
+                                    __uint_as_float(r[8 * v + 2 * h]), __uint_as_float(r[8 * v + 2 * h + 1]));
+                                p[h] = *reinterpret_cast<const uint32_t *>(&b2);
+                            }
+                            *reinterpret_cast<uint4 *>(dst + 8 * v) = make_uint4(p[0], p[1], p[2], p[3]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&bars->tempty[acc]));
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+    }
+}
+
+// ---- host side: tensor maps through the driver entry point ----
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return (EncodeTiledFn) nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// 2-D bf16 tensor [rows][cols] (cols contiguous), box = box_rows x 64 columns.
+bool make_map(CUtensorMap *map, const void *base, int rows, int cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+// Bound on any single wait of the GEMM (the whole GEMM takes well under this).
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+cudaError_t launch_bf16_gemm_ex(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
+                                int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test) {
+    CUtensorMap mx, mw;
+    if (!make_map(&mx, X, tokens, k, BM) || !make_map(&mw, W, n, k, BN)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kGemmSmem);
+    if (e != cudaSuccess) return e;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int tiles = ((tokens + BM - 1) / BM) * ((n + BN - 1) / BN);
+    const int sms = num_sms(dev);
+    const int grid = tiles < sms ? tiles : sms;
+    return launch_kernel(gemm_bf16_tcgen05, dim3(grid), dim3(kGemmThreads), kGemmSmem, st, false, mx, mw,
+                         reinterpret_cast<__nv_bfloat16 *>(Y), tokens, n, k, status, limit_ns, stall_test);
+}
+
+cudaError_t launch_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
+                             int32_t *status, cudaStream_t st) {
+    return launch_bf16_gemm_ex(X, W, Y, tokens, n, k, status, st, kWaitLimitNs, 0);
+}
+
+}  // namespace aqlm

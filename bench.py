@@ -1,0 +1,484 @@
+"""Benchmark of the AQLM inference path on B200: prints one JSON line.
+
+Headline workload: one AQLM 1x16 layer 4096x4096 (one 65536x8 fp16 codebook,
+fp16 scales, 2 bits/param in codes), batch 1, the decode-time matrix-vector
+product.  A step is one CUDA-graph replay of STEP_LAYERS back-to-back
+aqlm_gemv launches cycling over R distinct synthetic copies of the layer
+whose total footprint is more than 3x the L2 size, so no launch finds its
+codes in L2.  value = algorithmic bytes (codes + scales + x + y) of all
+launches of all ranks / max-over-ranks device time, in GB/s.
+
+The same JSON line carries, under "detail", every other workload of the
+scope: 2x8 4096^2, the Llama-2-7B decoder block (1x16 and 2x8), the
+Llama-2-70B layers (1x16 at 1/4/16 tokens, 2x16), and prefill (dequant +
+tcgen05 GEMM at 2048 tokens), each as us/layer and fraction of its roofline.
+
+--impl reference times the CPU oracle (the baseline of this build) on the
+same workload and prints the same line with "impl": "reference".
+Inputs are synthetic (seeded numpy draws; see synth/), not trained weights.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import LayerSpec, make_layer, LLAMA7B_SHAPES, LLAMA70B_SHAPES, PREFILL_SHAPES  # noqa: E402
+
+METRIC = "AQLM matvec µs/layer & achieved HBM GB/s vs roofline (1x16, 2x8); prefill TFLOP/s"
+HEADLINE = LayerSpec(4096, 4096, 1, 16)
+STEP_LAYERS = 1024
+L2_BYTES_FALLBACK = 126 * 1024 * 1024
+
+
+def algo_bytes(spec, T):
+    """Algorithmic bytes of one layer product: codes + scales + x + y."""
+    return spec.code_bytes() + 2 * spec.d_out + 2 * T * spec.d_in + 2 * T * spec.d_out
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "additive_codebook_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(f.encode())
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(kernel_key)
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples in the background (read-only query)."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.samples = []
+        self.loaded = threading.Event()
+        self._stop = threading.Event()
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((self.loaded.is_set(), parts))
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = [p for loaded, p in self.samples if loaded] or [p for _, p in self.samples]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(rows[0][2]),
+                "samples": len(rows), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+class Layers:
+    """R synthetic copies of one layer shape on the device (seeds seed..seed+R-1)."""
+
+    def __init__(self, spec, R, T, seed=0, x_dtype="fp16"):
+        import torch
+        self.spec, self.R, self.T = spec, R, T
+        self.copies = []
+        for r in range(R):
+            L = make_layer(spec, seed=seed + r, tokens=T if r == 0 else 0, x_dtype=x_dtype)
+            d = {"codes": torch.from_numpy(L["codes"]).cuda(), "codebooks": torch.from_numpy(L["codebooks"]).cuda(),
+                 "scales": torch.from_numpy(L["scales"]).cuda()}
+            self.copies.append(d)
+            if r == 0:
+                self.host0 = L
+        x = self.host0["x"]
+        self.x = (torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16) if x.dtype == np.uint16
+                  else torch.from_numpy(x).cuda())
+
+
+def copies_for(spec, T, l2_bytes, min_copies=2):
+    per = spec.code_bytes() + spec.codebook_bytes() + 2 * spec.d_out
+    return max(min_copies, int(np.ceil(3 * l2_bytes / per)))
+
+
+def gemv_graph(ac, layers, n_launch, ys, workspaces):
+    """Capture n_launch aqlm_gemv calls cycling over the copies in one graph."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for i in range(min(n_launch, layers.R)):   # warm-up outside capture (sets kernel attributes)
+            d = layers.copies[i]
+            ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], layers.x, y=ys[i % len(ys)],
+                         workspace=workspaces)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        for i in range(n_launch):
+            d = layers.copies[i % layers.R]
+            ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], layers.x, y=ys[i % len(ys)],
+                         workspace=workspaces)
+    return g
+
+
+def time_replays(g, steps, warmup, dist=None):
+    import torch
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        import torch.distributed as tdist
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    torch.cuda.synchronize()
+    return ms
+
+
+def bench_gemv(ac, spec, T, steps, warmup, l2_bytes, n_launch=STEP_LAYERS, dist=None):
+    import torch
+    R = copies_for(spec, T, l2_bytes)
+    layers = Layers(spec, R, T)
+    ys = [torch.empty((T, spec.d_out), dtype=torch.float16, device="cuda") for _ in range(4)]
+    need = ac.gemv_workspace_bytes(ac.shape_of(layers.copies[0]["codes"]), T)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda") if need else None
+    n_launch = max(n_launch, R)
+    g = gemv_graph(ac, layers, n_launch, ys, ws)
+    ms = time_replays(g, steps, warmup, dist)
+    us_layer = ms * 1e3 / (steps * n_launch)
+    launches_per_layer = 1 if need == 0 else 2
+    del g
+    return {"us_per_layer": us_layer, "bytes_per_layer": algo_bytes(spec, T), "copies": R,
+            "launches": steps * n_launch * launches_per_layer, "ms": ms, "layers": layers, "ws": ws}
+
+
+def bench_block(ac, fmt, steps, warmup, l2_bytes):
+    """Llama-2-7B decoder block: its 7 linears back to back, batch 1."""
+    import torch
+    M, B = fmt
+    specs = [LayerSpec(o, i, M, B) for _, o, i in LLAMA7B_SHAPES]
+    per_block = sum(s.code_bytes() + s.codebook_bytes() + 2 * s.d_out for s in specs)
+    R = max(2, int(np.ceil(3 * l2_bytes / per_block)))
+    blocks = [[Layers(s, 1, 1, seed=100 * r + k) for k, s in enumerate(specs)] for r in range(R)]
+    ys = {s.d_out: torch.empty((1, s.d_out), dtype=torch.float16, device="cuda") for s in specs}
+    x_in = {4096: blocks[0][0].x, 11008: blocks[0][6].x}
+    g = torch.cuda.CUDAGraph()
+    for blk in blocks:
+        for L in blk:
+            d = L.copies[0]
+            ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], x_in[L.spec.d_in], y=ys[L.spec.d_out])
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        for blk in blocks:
+            for L in blk:
+                d = L.copies[0]
+                ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], x_in[L.spec.d_in], y=ys[L.spec.d_out])
+    ms = time_replays(g, steps, warmup)
+    us_block = ms * 1e3 / (steps * R)
+    return {"us_per_block": us_block, "bytes_per_block": sum(algo_bytes(s, 1) for s in specs), "copies": R}
+
+
+def bench_prefill(ac, spec, tokens, reps, warmup):
+    import torch
+    L = Layers(spec, 1, tokens, x_dtype="bf16")
+    d = L.copies[0]
+    X = L.x
+    Y = torch.empty((tokens, spec.d_out), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(ac.gemm_workspace_bytes(ac.shape_of(d["codes"]), tokens), dtype=torch.uint8, device="cuda")
+    W = ws[256:].view(torch.bfloat16).view(spec.d_out, spec.d_in)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        out = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            out.append(e0.elapsed_time(e1) * 1e3)
+        return statistics.median(out)
+
+    t_total = timed(lambda: ac.aqlm_gemm(d["codes"], d["codebooks"], d["scales"], X, Y=Y, workspace=ws))
+    assert ac.aqlm_gemm_check(ws) == ac.AQLM_OK
+    t_deq = timed(lambda: ac.aqlm_dequant(d["codes"], d["codebooks"], d["scales"], out=W))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t_gemm = timed(lambda: ac.aqlm_bf16_gemm(X, W, Y=Y, status=status))
+    flops = 2.0 * tokens * spec.d_out * spec.d_in
+    deq_bytes = spec.code_bytes() + 2 * spec.d_out + 2 * spec.d_out * spec.d_in
+    return {"us_total": t_total, "us_dequant": t_deq, "us_gemm": t_gemm, "tflops": flops / t_total / 1e6,
+            "gemm_tflops": flops / t_gemm / 1e6, "dequant_gbs": deq_bytes / t_deq / 1e3}
+
+
+def e2e_gemv(ac, bench, steps, warmup):
+    """Through the public API with host buffers: per step H2D of x from pinned
+    memory, the layer calls, D2H of every layer's y."""
+    import torch
+    layers = bench["layers"]
+    spec, T = layers.spec, layers.T
+    R = layers.R
+    x_host = torch.from_numpy(layers.host0["x"]).pin_memory()
+    y_host = torch.empty((R, T, spec.d_out), dtype=torch.float16).pin_memory()
+    x_dev = torch.empty_like(layers.x)
+    y_dev = torch.empty((R, T, spec.d_out), dtype=torch.float16, device="cuda")
+    ws = bench["ws"]
+
+    def step():
+        x_dev.copy_(x_host, non_blocking=True)
+        for r in range(R):
+            d = layers.copies[r]
+            ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], x_dev, y=y_dev[r], workspace=ws)
+        y_host.copy_(y_dev, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    gbs = steps * R * algo_bytes(spec, T) / (ms * 1e-3) / 1e9
+    return {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": x_host.numel() * 2,
+            "d2h_bytes_per_step": y_host.numel() * 2, "layers_per_step": R,
+            "us_per_layer": ms * 1e3 / (steps * R)}
+
+
+def cpu_oracle_sample(spec, T, budget_s=10.0):
+    """The oracle as it stands on the host cores, repeated for about budget_s."""
+    import oracle
+    L = make_layer(spec, seed=0, tokens=T)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.gemv_f64(L["codes"], L["codebooks"], L["scales"], L["x"], spec.d_out, spec.d_in, 8, spec.M, spec.B)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": n * algo_bytes(spec, T) / el / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{n} full {spec.name} layer products, T={T}, {el:.1f} s"}
+
+
+def run_gpu(args):
+    import torch
+    import additive_codebook_b200 as ac
+    ac.load_library()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size or L2_BYTES_FALLBACK
+    peaks = load_peaks()
+    sampler = ClockSampler(local).__enter__()
+    time.sleep(0.3)
+    sampler.loaded.set()
+
+    head = bench_gemv(ac, HEADLINE, 1, args.steps, args.warmup, l2, dist=dist)
+    n_launch = max(STEP_LAYERS, head["copies"])
+    value = world * args.steps * n_launch * head["bytes_per_layer"] / (head["ms"] * 1e-3) / 1e9
+    achieved = head["bytes_per_layer"] / (head["us_per_layer"] * 1e-6) / 1e9
+    detail = {}
+    if not args.quick:
+        r = bench_gemv(ac, LayerSpec(4096, 4096, 2, 8), 1, max(3, args.steps // 2), args.warmup, l2)
+        detail["2x8 4096x4096 T1"] = _gemv_detail(r, peaks)
+        for fmt in ((1, 16), (2, 8)):
+            b = bench_block(ac, fmt, max(3, args.steps // 2), args.warmup, l2)
+            gbs = b["bytes_per_block"] / (b["us_per_block"] * 1e-6) / 1e9
+            detail[f"llama2-7b block {fmt[0]}x{fmt[1]} T1"] = {
+                "us_per_block": round(b["us_per_block"], 3), "gbs": round(gbs, 1),
+                "hbm_frac": round(gbs / peaks["hbm_gbs"], 4)}
+        for name, o, i in LLAMA70B_SHAPES:
+            for (M, B), Ts in (((1, 16), (1, 4, 16)), ((2, 16), (1,))):
+                for T in Ts:
+                    r = bench_gemv(ac, LayerSpec(o, i, M, B), T, 3, 2, l2, n_launch=64)
+                    detail[f"llama2-70b {name} {o}x{i} {M}x{B} T{T}"] = _gemv_detail(r, peaks, T=T)
+                    del r
+                    torch.cuda.empty_cache()
+        for o, i in PREFILL_SHAPES:
+            for M, B in ((1, 16), (2, 8)):
+                p = bench_prefill(ac, LayerSpec(o, i, M, B), 2048, reps=5, warmup=3)
+                detail[f"prefill {M}x{B} {o}x{i} T2048"] = {
+                    "us_per_layer": round(p["us_total"], 2), "tflops": round(p["tflops"], 1),
+                    "tensor_frac": round(p["tflops"] / peaks["bf16_tflops"], 4),
+                    "us_dequant": round(p["us_dequant"], 2), "dequant_gbs": round(p["dequant_gbs"], 1),
+                    "us_gemm": round(p["us_gemm"], 2), "gemm_tflops": round(p["gemm_tflops"], 1)}
+                torch.cuda.empty_cache()
+    e2e = e2e_gemv(ac, head, max(3, args.steps // 4), 2)
+    sampler.__exit__(None, None, None)
+    clocks = sampler.summary()
+
+    cpu = cpu_oracle_sample(HEADLINE, 1) if (rank == 0 and world == 1 and not args.quick) else None
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(head["ms"] / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp16 in, fp32 accumulate",
+        "data": "synthetic (seeded numpy draws: codebooks N(0,0.02), uniform codes, scales U[0.5,1.5], x N(0,1))",
+        "config": {"workload": "AQLM 1x16 layer 4096x4096 (group 8, one 65536x8 fp16 codebook), batch 1",
+                   "layers_per_step": n_launch, "distinct_layer_copies": head["copies"],
+                   "l2_policy": "inputs larger than L2: each step cycles over copies totalling > 3x L2",
+                   "parallelism": f"replicas x{world}"},
+        "us_per_layer": round(head["us_per_layer"], 4),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "traffic": recorded_traffic("gemv 1x16 4096x4096 T1"),
+                     "peak_source": f"{peaks['source']} copy bandwidth",
+                     "kernel": "gemv_kernel<1,16,1>",
+                     "algorithmic_bytes_per_launch": head["bytes_per_layer"]},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": head["launches"],
+        "clocks": clocks,
+        "detail": detail,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _gemv_detail(r, peaks, T=1):
+    gbs = r["bytes_per_layer"] / (r["us_per_layer"] * 1e-6) / 1e9
+    out = {"us_per_layer": round(r["us_per_layer"], 3), "gbs": round(gbs, 1),
+           "hbm_frac": round(gbs / peaks["hbm_gbs"], 4)}
+    if T > 1:
+        groups = r["layers"].spec.d_out * r["layers"].spec.groups
+        fma_t = groups * 8 * T / (r["us_per_layer"] * 1e-6) / 1e12
+        out["fma_tera_per_s"] = round(fma_t, 2)
+    return out
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    spec, T = HEADLINE, 1
+    L = make_layer(spec, seed=0, tokens=T)
+
+    def step():
+        oracle.gemv_f64(L["codes"], L["codebooks"], L["scales"], L["x"], spec.d_out, spec.d_in, 8, spec.M, spec.B)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = args.steps * algo_bytes(spec, T) / el / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(el * 1e3 / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "impl": "reference",
+        "data": "synthetic (seeded numpy draws)",
+        "config": {"workload": "AQLM 1x16 layer 4096x4096 (group 8, one 65536x8 fp16 codebook), batch 1",
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"{args.steps} full layer products after {args.warmup} warm-up"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--quick", action="store_true", help="headline workload only")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)   # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,191 @@
+/*
+ * aqlm.h -- C ABI of the B200 (sm_100a) AQLM inference library.
+ *
+ * AQLM ("Extreme Compression of Large Language Models via Additive
+ * Quantization", ICML 2024; explained in "The AQLM Quantization Algorithm,
+ * Explained", section "What is Multi-Codebook Quantization (MCQ)?") stores a
+ * weight matrix W of shape d_out x d_in as
+ *   - M codebooks of K = 2^B codewords, each codeword g = 8 values (16-bit);
+ *   - one 16-bit scale per output channel (row) i;
+ *   - for every group of g consecutive inputs of every row, M codes of B bits,
+ *     the indices of the codewords that are summed to approximate the group.
+ * The dequantised weight is
+ *   W^[i][8j + t] = s_i * sum_{m<M} C_m[ b(i, j, m) ][t],
+ * and a layer computes y = W^ . x for the activations of T tokens (W.X
+ * convention: rows of W are output channels).  The formats are named MxB
+ * after the naming scheme of section "Key AQLM quantization parameters":
+ * 1x16, 2x8 and 2x16 are supported.
+ *
+ * Memory layout (all row-major, every pointer is DEVICE memory unless stated):
+ *   codes      [d_out][d_in/8][M]   B = 8: uint8; B = 16: 16-bit words whose
+ *                                   index is the UNSIGNED value 0..65535
+ *                                   (pass int16 or uint16 storage alike)
+ *   codebooks  [M][2^B][8]          IEEE binary16 (fp16) bit patterns
+ *   scales     [d_out]              fp16
+ *   x, y       [T][d_in], [T][d_out] fp16           (aqlm_gemv)
+ *   X, Y       [T][d_in], [T][d_out] bfloat16       (aqlm_gemm)
+ *   W_out      [d_out][d_in]        bfloat16        (aqlm_dequant)
+ *
+ * Conventions for every entry point:
+ *   - The caller owns all memory.  The library allocates nothing, keeps no
+ *     pointer after a call returns and holds no mutable host state, so calls
+ *     from several host threads are safe.
+ *   - Work is enqueued on `stream` (NULL = the legacy default stream) and the
+ *     call returns without synchronising.  Outputs must not alias inputs.
+ *   - Validation happens on the host before any launch; a call that returns
+ *     anything but AQLM_OK has launched nothing, except AQLM_ERR_CUDA, which
+ *     reports the CUDA error of a launch (query it with cudaGetLastError
+ *     semantics: the library does not clear unrelated errors).
+ *   - No entry point prints, exits, throws or traps.
+ *   - Supported shapes: group == 8, (M, B) in {(1,16), (2,8), (2,16)},
+ *     d_out >= 1, d_in >= 8, d_in % 8 == 0 (else AQLM_ERR_UNSUPPORTED).
+ *   - Alignment: codes, codebooks, x/X, y/Y and W_out 16-byte aligned, and a
+ *     row of codes (d_in/8 * M * B/8 bytes) a multiple of 16 bytes, i.e.
+ *     d_in % 64 == 0 for 1x16 and 2x8, d_in % 32 == 0 for 2x16 (else
+ *     AQLM_ERR_MISALIGNED).  Scales need 2-byte alignment.
+ */
+#ifndef AQLM_B200_H
+#define AQLM_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define AQLM_API __attribute__((visibility("default")))
+#else
+#define AQLM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The CUDA runtime's cudaStream_t is `struct CUstream_st *`; declaring the
+ * same type here keeps this header free of CUDA includes. */
+struct CUstream_st;
+typedef struct CUstream_st *aqlm_stream_t;
+
+typedef enum {
+    AQLM_OK = 0,
+    AQLM_ERR_INVALID_ARG = 1,  /* null pointer, tokens out of range, bad sizes */
+    AQLM_ERR_UNSUPPORTED = 2,  /* format or shape outside the supported set   */
+    AQLM_ERR_MISALIGNED = 3,   /* pointer or row stride not 16-byte aligned   */
+    AQLM_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required  */
+    AQLM_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed         */
+    AQLM_ERR_TIMEOUT = 6       /* a bounded device-side wait gave up           */
+} aqlm_status;
+
+typedef struct {
+    int32_t d_out;          /* output channels (rows of W)                   */
+    int32_t d_in;           /* input features (columns of W)                 */
+    int32_t group;          /* g, inputs per group: must be 8                */
+    int32_t num_codebooks;  /* M                                             */
+    int32_t codebook_bits;  /* B: log2 of the codewords per codebook (8|16) */
+} aqlm_shape;
+
+/* Largest token count of the matrix-vector path. */
+#define AQLM_GEMV_MAX_TOKENS 16
+
+/*
+ * aqlm_gemv -- decode-time layer product, y = W^ . x, for 1 <= tokens <= 16.
+ *
+ * Defined by section "What is Multi-Codebook Quantization (MCQ)?": each
+ * group's codes select M codewords that are summed, the sum is scaled by the
+ * row's scale, and the product with the activations is taken.  Computed with
+ * fp32 accumulation; each y value is rounded once to fp16 (nearest even).
+ * The scale is applied to the row's accumulated sum (the same value in exact
+ * arithmetic as scaling every group).
+ *   codes, codebooks, scales: the layer, layout above.
+ *   x: [tokens][d_in] fp16.   y: [tokens][d_out] fp16 (written).
+ *   workspace/workspace_bytes: fp32 partial sums for shapes whose activations
+ *   do not fit on chip at once; aqlm_gemv_workspace_bytes() gives the size
+ *   (0 = none needed, NULL allowed).  Too small -> AQLM_ERR_WORKSPACE.
+ */
+AQLM_API aqlm_status aqlm_gemv(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                      const uint16_t *x, uint16_t *y, int32_t tokens, aqlm_shape shape,
+                      void *workspace, size_t workspace_bytes, aqlm_stream_t stream);
+
+/* Bytes of device workspace aqlm_gemv needs for this shape and token count
+ * (0 if none); returns 0 for invalid arguments too. */
+AQLM_API size_t aqlm_gemv_workspace_bytes(aqlm_shape shape, int32_t tokens);
+
+/*
+ * aqlm_dequant -- the runtime dequantisation of section "Why and what do we
+ * quantize?" (weights fetched compressed, turned back into native precision
+ * before the matmul) with the decode of section "What is Multi-Codebook
+ * Quantization (MCQ)?":
+ *   W_out[i][8j+t] = bf16_rn( fp32(s_i) * ( fp32(C_0[b0][t]) + ... + fp32(C_{M-1}[b][t]) ) )
+ * as separate IEEE binary32 operations in codebook order (no fused
+ * multiply-add), then one round-to-nearest-even to bfloat16.  The result is
+ * therefore bit-exact and deterministic.
+ *   W_out: [d_out][d_in] bf16 (written), 16-byte aligned.
+ */
+AQLM_API aqlm_status aqlm_dequant(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                         uint16_t *W_out, aqlm_shape shape, aqlm_stream_t stream);
+
+/*
+ * aqlm_gemm -- prefill product Y = X . W^T for many tokens: aqlm_dequant into
+ * the workspace, then a tcgen05 tensor-core GEMM (bf16 operands, fp32
+ * accumulation in tensor memory, bf16 output rounded to nearest even).
+ *   X: [tokens][d_in] bf16.  Y: [tokens][d_out] bf16 (written).  tokens >= 1.
+ *   workspace: at least aqlm_gemm_workspace_bytes(shape, tokens) bytes,
+ *   16-byte aligned; it holds the dequantised weight and a status word.
+ *   Every device-side wait of the GEMM is bounded; a wait that gives up
+ *   records AQLM_ERR_TIMEOUT in the workspace's status word (read it with
+ *   aqlm_gemm_check) and the kernel returns without trapping.
+ * Extra requirement: d_out % 8 == 0 (else AQLM_ERR_UNSUPPORTED).
+ */
+AQLM_API aqlm_status aqlm_gemm(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                      const uint16_t *X, uint16_t *Y, int32_t tokens, aqlm_shape shape,
+                      void *workspace, size_t workspace_bytes, aqlm_stream_t stream);
+
+AQLM_API size_t aqlm_gemm_workspace_bytes(aqlm_shape shape, int32_t tokens);
+
+/*
+ * aqlm_gemm_check -- synchronises `stream`, reads and clears the status word
+ * that aqlm_gemm calls with this workspace recorded.  Returns AQLM_OK,
+ * AQLM_ERR_TIMEOUT, or AQLM_ERR_CUDA if the stream itself reports an error.
+ */
+AQLM_API aqlm_status aqlm_gemm_check(void *workspace, size_t workspace_bytes, aqlm_stream_t stream);
+
+/*
+ * aqlm_bf16_gemm -- the tensor-core GEMM of aqlm_gemm on its own, for a dense
+ * bf16 weight: Y[tokens][n] = X[tokens][k] . W[n][k]^T.  n % 8 == 0, k % 8
+ * == 0, all matrices 16-byte aligned; `status` is a device int32 that
+ * receives AQLM_ERR_TIMEOUT if a bounded wait gives up (it is only ever
+ * written with a non-zero value; clear it yourself).
+ */
+AQLM_API aqlm_status aqlm_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int32_t tokens,
+                           int32_t n, int32_t k, int32_t *status, aqlm_stream_t stream);
+
+/*
+ * aqlm_decode_indices -- the code unpacking step on its own, for bit-exact
+ * checks: idx_out[(i*G + j)*M + m] = index of codebook m for group j of row
+ * i, as uint16 (G = d_in/8).  idx_out: d_out*G*M uint16, 2-byte aligned.
+ * Storing an index of B bits per codebook per group is the code
+ * representation of section "What is Multi-Codebook Quantization (MCQ)?".
+ */
+AQLM_API aqlm_status aqlm_decode_indices(const void *codes, uint16_t *idx_out, aqlm_shape shape,
+                                aqlm_stream_t stream);
+
+/*
+ * aqlm_test_gemm_timeout -- test hook for the GEMM's failure detection: runs
+ * the kernel of aqlm_bf16_gemm with its loads withheld, so that the first
+ * bounded wait runs out after `limit_ns` nanoseconds (1 ns .. 1 s).  The
+ * kernel must then write AQLM_ERR_TIMEOUT to *status, free its tensor
+ * memory and return; nothing faults or hangs.  Arguments as aqlm_bf16_gemm.
+ */
+AQLM_API aqlm_status aqlm_test_gemm_timeout(const uint16_t *X, const uint16_t *W, uint16_t *Y, int32_t tokens, int32_t n,
+                                   int32_t k, int32_t *status, uint64_t limit_ns, aqlm_stream_t stream);
+
+/* A static, human-readable name of a status code. */
+AQLM_API const char *aqlm_status_string(aqlm_status status);
+
+/* Library version, e.g. "0.1.0". */
+AQLM_API const char *aqlm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AQLM_B200_H */

@@ -1,0 +1,129 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/aqlm.h declares, and rejects bad arguments on the
+host before any CUDA call (validation never dereferences the pointers, so
+fake addresses are safe here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import additive_codebook_b200 as ac
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "aqlm.h")).read()
+    return re.findall(r"^AQLM_API\s+[\w\s\*]+?\b(aqlm_\w+)\s*\(", text, flags=re.M)
+
+
+def test_header_and_binding_agree():
+    names = header_functions()
+    assert len(names) == len(set(names)) and sorted(names) == sorted(ac.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ac.load_library()
+    for name in header_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings_and_version():
+    assert ac.status_string(ac.AQLM_OK) == "AQLM_OK"
+    assert ac.status_string(ac.AQLM_ERR_TIMEOUT) == "AQLM_ERR_TIMEOUT"
+    assert ac.status_string(99) == "AQLM_ERR_UNKNOWN"
+    assert re.match(r"^\d+\.\d+\.\d+$", ac.version())
+
+
+A16 = ctypes.c_void_p(0x10000)   # 16-byte aligned fake device addresses
+B16 = ctypes.c_void_p(0x20000)
+C16 = ctypes.c_void_p(0x30000)
+D16 = ctypes.c_void_p(0x40000)
+E16 = ctypes.c_void_p(0x50000)
+NULL = ctypes.c_void_p(0)
+ODD = ctypes.c_void_p(0x10008)
+
+
+def shape(d_out=256, d_in=512, M=2, B=8, g=8):
+    return ac.Shape(d_out, d_in, g, M, B)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(g=4), ac.AQLM_ERR_UNSUPPORTED),
+    (dict(M=3, B=8), ac.AQLM_ERR_UNSUPPORTED),
+    (dict(M=1, B=8), ac.AQLM_ERR_UNSUPPORTED),
+    (dict(M=2, B=12), ac.AQLM_ERR_UNSUPPORTED),
+    (dict(d_in=500), ac.AQLM_ERR_UNSUPPORTED),
+    (dict(d_in=520), ac.AQLM_ERR_MISALIGNED),          # 65 groups x 2 bytes: row not a 16-byte multiple
+    (dict(d_out=0), ac.AQLM_ERR_INVALID_ARG),
+    (dict(d_in=0), ac.AQLM_ERR_INVALID_ARG),
+    (dict(d_out=1 << 21), ac.AQLM_ERR_INVALID_ARG),
+])
+def test_shape_validation(kw, status):
+    lib = ac.load_library()
+    s = shape(**kw)
+    # every case fails validation, so nothing is launched with the fake pointers
+    assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 1, s, NULL, 0, NULL) == status
+
+
+def test_gemv_argument_errors():
+    lib = ac.load_library()
+    s = shape()
+    assert lib.aqlm_gemv(NULL, B16, C16, D16, E16, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemv(A16, NULL, C16, D16, E16, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemv(A16, B16, NULL, D16, E16, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemv(A16, B16, C16, NULL, E16, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemv(A16, B16, C16, D16, NULL, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 0, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 17, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemv(ODD, B16, C16, D16, E16, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_MISALIGNED
+    assert lib.aqlm_gemv(A16, ODD, C16, D16, E16, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_MISALIGNED
+    assert lib.aqlm_gemv(A16, B16, C16, ODD, E16, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_MISALIGNED
+
+
+def test_gemv_workspace_rules():
+    lib = ac.load_library()
+    big = ac.Shape(8192, 8192, 8, 1, 16)
+    assert lib.aqlm_gemv_workspace_bytes(shape(), 1) == 0
+    assert lib.aqlm_gemv_workspace_bytes(big, 1) == 0
+    need = lib.aqlm_gemv_workspace_bytes(big, 16)
+    assert need > 0 and need % (16 * 8192 * 4) == 0
+    assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 16, big, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 16, big, A16, need - 4, NULL) == ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 16, big, ODD, need, NULL) == ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_gemv_workspace_bytes(big, 0) == 0 and lib.aqlm_gemv_workspace_bytes(big, 17) == 0
+
+
+def test_gemm_argument_errors():
+    lib = ac.load_library()
+    s = ac.Shape(4096, 4096, 8, 1, 16)
+    need = lib.aqlm_gemm_workspace_bytes(s, 2048)
+    assert need == 256 + 4096 * 4096 * 2
+    assert lib.aqlm_gemm(A16, B16, C16, D16, E16, 2048, s, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_gemm(A16, B16, C16, D16, E16, 2048, s, A16, need - 1, NULL) == ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_gemm(A16, B16, C16, D16, E16, 0, s, A16, need, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemm(A16, B16, C16, ODD, E16, 16, s, A16, need, NULL) == ac.AQLM_ERR_MISALIGNED
+    s_odd = ac.Shape(4100, 4096, 8, 1, 16)
+    assert lib.aqlm_gemm(A16, B16, C16, D16, E16, 16, s_odd, A16, 1 << 40, NULL) == ac.AQLM_ERR_UNSUPPORTED
+    assert lib.aqlm_bf16_gemm(A16, B16, C16, 16, 100, 64, D16, NULL) == ac.AQLM_ERR_UNSUPPORTED
+    assert lib.aqlm_bf16_gemm(A16, B16, C16, 16, 128, 64, NULL, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemm_check(NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
+
+
+def test_dequant_and_decode_argument_errors():
+    lib = ac.load_library()
+    s = shape()
+    assert lib.aqlm_dequant(A16, B16, C16, NULL, s, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_dequant(A16, B16, C16, ODD, s, NULL) == ac.AQLM_ERR_MISALIGNED
+    assert lib.aqlm_decode_indices(NULL, A16, s, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_decode_indices(A16, ctypes.c_void_p(0x10001), s, NULL) == ac.AQLM_ERR_MISALIGNED
+    assert lib.aqlm_test_gemm_timeout(A16, B16, C16, 16, 128, 64, D16, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(ac, "_lib", None)
+    monkeypatch.setattr(ac, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        ac.load_library()

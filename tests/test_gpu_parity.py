@@ -1,0 +1,238 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Integer work (index unpacking) and the bf16 dequantisation are compared bit
+for bit; the fp16/bf16 layer outputs are held to the stated tolerance
+max|y - y_ref| <= 2e-3 ||x||_2 max_i ||(s . W^)_i||_2 and to a tighter bound
+derived from the arithmetic (one output rounding plus fp32 accumulation).
+Sizes span several CTA tiles with ragged tails; the full-size layers of the
+benchmark are checked on sampled rows/tokens the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import additive_codebook_b200 as ac
+import oracle
+from gpu_util import (DEV, bf16_to_np_bits, check_fp_output, layer, oracle_W, to_dev)
+from synth import LayerSpec, make_layer, make_x
+
+pytestmark = pytest.mark.gpu
+
+FORMATS = [(1, 16), (2, 8), (2, 16)]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu(cuda_device):
+    ac.load_library()
+    yield
+
+
+# ---------------------------------------------------------------- indices
+
+@pytest.mark.parametrize("M,B", FORMATS)
+def test_decode_indices_bit_exact(M, B):
+    spec = LayerSpec(200, 576, M, B)
+    L = make_layer(spec, seed=1, tokens=0)
+    d = to_dev(L)
+    got = ac.aqlm_decode_indices(d["codes"]).cpu().numpy().view(np.uint16)
+    want = oracle.decode_indices(L["codes"], spec.d_out, spec.d_in, 8, M, B)
+    assert np.array_equal(got, want)
+
+
+def test_decode_indices_edge_codes():
+    codes = np.array([0, 1, 32767, -32768, -1, 12345, -2, 255] * 8, dtype=np.int16).reshape(8, 8, 1)
+    got = ac.aqlm_decode_indices(torch.from_numpy(codes).to(DEV)).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, oracle.decode_indices(codes, 8, 64, 8, 1, 16))
+
+
+# ---------------------------------------------------------------- dequant
+
+@pytest.mark.parametrize("M,B", FORMATS)
+@pytest.mark.parametrize("d_out,d_in", [(200, 576), (1000, 1024)])
+def test_dequant_bit_exact(M, B, d_out, d_in):
+    spec = LayerSpec(d_out, d_in, M, B)
+    L = make_layer(spec, seed=2 + d_out, tokens=0)
+    L["scales"][:4] = np.array([1.0, -1.0, -0.75, 65504.0], dtype=np.float16)   # signs, overflow to inf
+    d = to_dev(L)
+    got = bf16_to_np_bits(ac.aqlm_dequant(d["codes"], d["codebooks"], d["scales"]))
+    want = oracle.dequant_bf16(L["codes"], L["codebooks"], L["scales"], d_out, d_in, 8, M, B)
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("M,B", FORMATS)
+def test_dequant_extreme_codes(M, B):
+    """All-zero and all-max codes (255 / 65535) and special codebook values."""
+    spec = LayerSpec(64, 512, M, B)
+    L = make_layer(spec, seed=3, tokens=0)
+    L["codes"][: 32] = 0
+    L["codes"][32:] = np.array(-1 if B == 16 else 255).astype(L["codes"].dtype)
+    L["codebooks"][:, 0, :3] = [0.0, -0.0, 6.0e-8]
+    L["codebooks"][:, -1, :3] = [65504.0, -65504.0, np.inf]
+    d = to_dev(L)
+    got = bf16_to_np_bits(ac.aqlm_dequant(d["codes"], d["codebooks"], d["scales"]))
+    want = oracle.dequant_bf16(L["codes"], L["codebooks"], L["scales"], 64, 512, 8, M, B)
+    assert np.array_equal(got, want)
+
+
+def test_dequant_deterministic():
+    spec = LayerSpec(512, 1024, 1, 16)
+    d = to_dev(make_layer(spec, seed=4, tokens=0))
+    a = ac.aqlm_dequant(d["codes"], d["codebooks"], d["scales"])
+    b = ac.aqlm_dequant(d["codes"], d["codebooks"], d["scales"])
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+# ---------------------------------------------------------------- gemv
+
+def _gemv_case(M, B, d_out, d_in, T, seed):
+    spec = LayerSpec(d_out, d_in, M, B)
+    L = make_layer(spec, seed=seed, tokens=T)
+    d = to_dev(L)
+    y = ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], d["x"]).cpu().numpy()
+    y_ref = oracle.gemv_f64(L["codes"], L["codebooks"], L["scales"], L["x"], d_out, d_in, 8, M, B)
+    W = oracle_W(L, spec)
+    return check_fp_output(y, y_ref, W, L["x"].astype(np.float64), out_rel=2.0 ** -10, acc_rel=2.0 ** -14)
+
+
+@pytest.mark.parametrize("M,B", FORMATS)
+@pytest.mark.parametrize("T", [1, 2, 3, 4, 7, 8, 16])
+def test_gemv_small(M, B, T):
+    # 200 rows: 7 row tiles, the last one ragged; 576 inputs: 72 groups, a
+    # chunk count that does not divide evenly over the 8 warps
+    _gemv_case(M, B, 200, 576, T, seed=10 + T)
+
+
+@pytest.mark.parametrize("M,B", FORMATS)
+@pytest.mark.parametrize("T", [1, 4, 16])
+def test_gemv_split_input_range(M, B, T):
+    # d_in = 4160 -> 520 groups; T = 16 needs the split over the input range
+    # (slabs of at most 256 groups), T = 4 and T = 1 do not
+    _gemv_case(M, B, 96, 4160, T, seed=20 + T)
+
+
+def test_gemv_one_hot_returns_columns():
+    """x = e_c returns column c of s . W^ (exact up to the fp16 rounding)."""
+    spec = LayerSpec(64, 512, 1, 16)
+    L = make_layer(spec, seed=5, tokens=0)
+    W = oracle_W(L, spec)
+    x = np.zeros((4, 512), dtype=np.float16)
+    cols = [0, 7, 300, 511]
+    for t, c in enumerate(cols):
+        x[t, c] = 1.0
+    d = to_dev(L)
+    y = ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], torch.from_numpy(x).to(DEV)).cpu().numpy()
+    for t, c in enumerate(cols):
+        assert np.array_equal(y[t], W[:, c].astype(np.float16))
+
+
+def test_gemv_two_calls_identical():
+    spec = LayerSpec(4096, 4096, 1, 16)
+    d = to_dev(make_layer(spec, seed=6, tokens=1))
+    a = ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], d["x"])
+    b = ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], d["x"])
+    assert torch.equal(a, b)
+
+
+FULL_GEMV = [
+    ("1x16 4096x4096", 4096, 4096, 1, 16, 1),
+    ("2x8 4096x4096", 4096, 4096, 2, 8, 1),
+    ("1x16 11008x4096", 11008, 4096, 1, 16, 1),
+    ("2x8 4096x11008", 4096, 11008, 2, 8, 1),
+    ("1x16 28672x8192 T4", 28672, 8192, 1, 16, 4),
+    ("1x16 8192x28672 T16", 8192, 28672, 1, 16, 16),
+    ("2x16 8192x8192", 8192, 8192, 2, 16, 1),
+    ("2x8 256x512", 256, 512, 2, 8, 1),
+]
+
+
+@pytest.mark.parametrize("name,d_out,d_in,M,B,T", FULL_GEMV, ids=[c[0] for c in FULL_GEMV])
+def test_gemv_full_size_sampled_rows(name, d_out, d_in, M, B, T):
+    spec = LayerSpec(d_out, d_in, M, B)
+    L = make_layer(spec, seed=0, tokens=T)
+    d = to_dev(L)
+    y = ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], d["x"]).cpu().numpy()
+    rng = np.random.Generator(np.random.PCG64(123))
+    rows = np.unique(np.concatenate([rng.choice(d_out, size=min(d_out, 256), replace=False), [0, d_out - 1]]))
+    sub = {"codes": np.ascontiguousarray(L["codes"][rows]), "codebooks": L["codebooks"],
+           "scales": np.ascontiguousarray(L["scales"][rows])}
+    y_ref = oracle.gemv_f64(sub["codes"], sub["codebooks"], sub["scales"], L["x"], len(rows), d_in, 8, M, B)
+    W = oracle.dequant_f64(sub["codes"], sub["codebooks"], sub["scales"], len(rows), d_in, 8, M, B)
+    check_fp_output(y[:, rows], y_ref, W, L["x"].astype(np.float64), out_rel=2.0 ** -10, acc_rel=2.0 ** -14)
+
+
+# ---------------------------------------------------------------- gemm
+
+def _gemm_check(Y, L, spec, X_bits, tokens_idx=None):
+    """Y [T, d_out] bf16 against (1) the exact layer and (2) the bf16-rounded W^."""
+    X64 = oracle.bf16_bits_to_f64(X_bits)
+    W_exact = oracle_W(L, spec)
+    Wb = oracle.bf16_bits_to_f64(oracle.dequant_bf16(L["codes"], L["codebooks"], L["scales"],
+                                                     spec.d_out, spec.d_in, 8, spec.M, spec.B))
+    if tokens_idx is not None:
+        X64 = X64[tokens_idx]
+        Y = Y[tokens_idx]
+    y_exact = oracle.matmul_f64(W_exact, X64)
+    y_bw = oracle.matmul_f64(Wb, X64)
+    Yf = oracle.bf16_bits_to_f64(Y)
+    # stated tolerance against the exact layer
+    check_fp_output(Yf, y_exact, W_exact, X64, out_rel=1.0, acc_rel=1.0)
+    # the tensor-core product of the bf16 operands: one bf16 rounding + fp32 accumulation
+    check_fp_output(Yf, y_bw, Wb, X64, out_rel=2.0 ** -8, acc_rel=2.0 ** -14)
+
+
+@pytest.mark.parametrize("M,B", FORMATS)
+@pytest.mark.parametrize("tokens,d_out,d_in", [(200, 520, 576), (256, 512, 1024), (130, 264, 64)])
+def test_gemm_small(M, B, tokens, d_out, d_in):
+    if (d_in // 8 * M * B // 8) % 16:
+        pytest.skip("row of codes not 16-byte aligned")
+    spec = LayerSpec(d_out, d_in, M, B)
+    L = make_layer(spec, seed=30 + tokens, tokens=tokens, x_dtype="bf16")
+    d = to_dev(L)
+    Y, ws = ac.aqlm_gemm(d["codes"], d["codebooks"], d["scales"], d["x"])
+    assert ac.aqlm_gemm_check(ws) == ac.AQLM_OK
+    _gemm_check(bf16_to_np_bits(Y), L, spec, L["x"])
+
+
+def test_bf16_gemm_matches_torch():
+    """The plain tensor-core GEMM against torch.matmul (fp32 accumulation) as a yardstick."""
+    g = torch.Generator(device="cpu").manual_seed(7)
+    X = torch.randn(384, 1536, generator=g).to(torch.bfloat16).to(DEV)
+    W = torch.randn(768, 1536, generator=g).to(torch.bfloat16).to(DEV)
+    Y, status = ac.aqlm_bf16_gemm(X, W)
+    ref = (X.float() @ W.float().T)
+    assert int(status.item()) == 0
+    err = (Y.float() - ref).abs()
+    assert float((err / (ref.abs() + 1e-2)).max()) < 2e-2
+    assert float(err.max()) < 0.25
+
+
+PREFILL = [(11008, 4096, 1, 16), (4096, 11008, 2, 8), (11008, 4096, 2, 8), (4096, 11008, 1, 16)]
+
+
+@pytest.mark.parametrize("d_out,d_in,M,B", PREFILL, ids=[f"{m}x{b} {o}x{i}" for o, i, m, b in PREFILL])
+def test_gemm_full_size_sampled_tokens(d_out, d_in, M, B):
+    spec = LayerSpec(d_out, d_in, M, B)
+    L = make_layer(spec, seed=0, tokens=2048, x_dtype="bf16")
+    d = to_dev(L)
+    Y, ws = ac.aqlm_gemm(d["codes"], d["codebooks"], d["scales"], d["x"])
+    assert ac.aqlm_gemm_check(ws) == ac.AQLM_OK
+    rng = np.random.Generator(np.random.PCG64(321))
+    toks = np.unique(np.concatenate([rng.choice(2048, size=12, replace=False), [0, 127, 128, 2047]]))
+    _gemm_check(bf16_to_np_bits(Y), L, spec, L["x"], tokens_idx=toks)
+
+
+def test_gemm_bounded_wait_reports_timeout():
+    """Loads withheld on purpose: the first wait runs out, the kernel records
+    AQLM_ERR_TIMEOUT, frees its tensor memory and returns; the context stays usable."""
+    X = torch.zeros(128, 64, dtype=torch.bfloat16, device=DEV)
+    W = torch.zeros(256, 64, dtype=torch.bfloat16, device=DEV)
+    Y = torch.empty(128, 256, dtype=torch.bfloat16, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    assert ac.aqlm_test_gemm_timeout(X, W, Y, status, 20_000_000) == ac.AQLM_OK
+    torch.cuda.synchronize()
+    assert int(status.item()) == ac.AQLM_ERR_TIMEOUT
+    # the device still works, and a normal GEMM afterwards is correct
+    Y2, st2 = ac.aqlm_bf16_gemm(torch.ones(128, 64, dtype=torch.bfloat16, device=DEV),
+                                torch.ones(256, 64, dtype=torch.bfloat16, device=DEV))
+    torch.cuda.synchronize()
+    assert int(st2.item()) == 0 and torch.all(Y2.float() == 64.0)
