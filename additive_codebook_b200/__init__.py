@@ -132,7 +132,7 @@ def aqlm_gemv(codes, codebooks, scales, x, y=None, workspace=None, stream=None):
         y = torch.empty((T, shape.d_out), dtype=torch.float16, device=x.device)
     need = lib.aqlm_gemv_workspace_bytes(shape, T)
     if need and workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+        workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
     wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(lib.aqlm_gemv(_p(codes), _p(codebooks), _p(_flat_scales(scales)), _p(x), _p(y), T, shape,
                          _p(workspace), wbytes, _stream(stream)), "aqlm_gemv")

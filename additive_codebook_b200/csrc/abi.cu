@@ -80,8 +80,8 @@ aqlm_status aqlm_gemv(const void *codes, const uint16_t *codebooks, const uint16
     const Dims d = aqlm::make_dims(shape);
     const size_t need = aqlm::gemv_workspace_bytes(d, tokens);
     if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16))) return AQLM_ERR_WORKSPACE;
-    return from_cuda(aqlm::launch_gemv(codes, codebooks, scales, x, y, tokens, d,
-                                       need > 0 ? static_cast<float *>(workspace) : nullptr, to_cuda(stream)));
+    return from_cuda(aqlm::launch_gemv(codes, codebooks, scales, x, y, tokens, d, need > 0 ? workspace : nullptr,
+                                       to_cuda(stream)));
 }
 
 size_t aqlm_gemm_workspace_bytes(aqlm_shape shape, int32_t tokens) {

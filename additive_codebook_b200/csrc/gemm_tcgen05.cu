@@ -2,10 +2,10 @@
 //
 // Y[m][n] = sum_k X[m][k] * W[n][k]: X = the prefill activations [tokens][d_in]
 // and W = the dequantised layer [d_out][d_in], both bf16 and K-major; fp32
-// accumulation; bf16 output rounded to nearest even.  This is the matmul
-// "with dequantized, native-precision parameters" of section "What is
-// Multi-Codebook Quantization (MCQ)?" in "The AQLM Quantization Algorithm,
-// Explained".
+// accumulation; bf16 output rounded to nearest even.  This is the product of
+// the activations with the dequantised weights in their native precision,
+// section "What is Multi-Codebook Quantization (MCQ)?" of "The AQLM
+// Quantization Algorithm, Explained".
 //
 // sm_100a design: a persistent kernel, one CTA per SM, 128x256 output tiles.
 //   warp 0      one thread issues TMA tile loads (128-byte swizzle) into a

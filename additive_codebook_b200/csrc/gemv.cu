@@ -1,51 +1,56 @@
-// gemv.cu -- host side of the decode-time product: work plan, launch, and
-// the fixed-order reduction of split partial sums.  The kernels are in
-// gemv_kernels.cuh, instantiated per format in gemv_1x16.cu, gemv_2x8.cu and
-// gemv_2x16.cu.
+// gemv.cu -- host side of the decode-time product: kernel choice, work plan,
+// workspace layout and the launch (with programmatic dependent launch).
+// The gather kernels are in gemv_kernels.cuh (instantiated per format in
+// gemv_1x16.cu, gemv_2x8.cu, gemv_2x16.cu); the batch-1 2x8 lookup-table
+// kernel is in gemv_lut.cu.
 #include "gemv_kernels.cuh"
 
 namespace aqlm {
+
+size_t gemv_lut_workspace_bytes(const Dims &d, int sms);
+cudaError_t launch_gemv_lut_2x8(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                                const uint16_t *x, uint16_t *y, const Dims &d, void *workspace, int sms,
+                                cudaStream_t st);
+
 namespace gemv_detail {
 namespace {
 
-// y[t][r] = fp16(s_r * sum over splits of partial[split][t][r]), splits in order.
-__global__ void gemv_finalize_kernel(const float *__restrict__ partial, const __half *__restrict__ scales,
-                                     __half *__restrict__ y, int d_out, int tokens, int splits) {
-    const int n = d_out * tokens;
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
-        const int r = i % d_out;
-        float sum = 0.f;
-        for (int s = 0; s < splits; ++s) sum += partial[(size_t)s * n + i];
-        y[i] = __float2half_rn(sum * __half2float(scales[r]));
-    }
-}
-
 struct Plan {
-    int slab_groups;  // groups of the input range one CTA covers
-    int splits;       // CTAs along the input dimension
-    size_t smem;      // dynamic shared memory per CTA
+    int tiles;             // row tiles of 32 rows (gridDim.x)
+    int splits;            // CTAs along the input range (gridDim.y)
+    int chunks_per_split;  // 16-byte code chunks per row per CTA
+    size_t smem;
 };
 
-// The whole row's activations (T x d_in fp32) stay on chip when they fit in
-// kXsBudget; otherwise the input range is cut into equal slabs (multiples of
-// 8 groups, so every slab holds whole 16-byte code chunks).
-Plan plan_gemv(const Dims &d, int T) {
-    int max_groups = kXsBudget / (kGroup * 4 * T);
-    max_groups -= max_groups % 8;
+inline size_t align16(size_t v) { return (v + 15) / 16 * 16; }
+
+// Split the input range when (a) T activations of the whole row exceed the
+// on-chip budget, or (b) there are too few row tiles to give every SM two
+// CTAs; never below one chunk per warp.
+Plan plan_gemv(const Dims &d, int T, int sms) {
+    const int gpc = 16 / (d.M * d.B / 8);
+    const int n_chunks = d.G / gpc;
     Plan p;
-    if (d.G <= max_groups) {
-        p.slab_groups = d.G;
-        p.splits = 1;
-    } else {
-        const int splits = (d.G + max_groups - 1) / max_groups;
-        int slab = (d.G + splits - 1) / splits;
-        slab = (slab + 7) / 8 * 8;
-        p.slab_groups = slab;
-        p.splits = (d.G + slab - 1) / slab;
-    }
-    const size_t cb = (d.B == 8) ? (size_t)d.M * 256 * 16 : 0;
-    p.smem = (size_t)T * p.slab_groups * kGroup * 4 + cb + (size_t)kWarps * T * 32 * 4;
+    p.tiles = (d.d_out + kRowsPerCta - 1) / kRowsPerCta;
+    int max_chunks = kXsBudget / (T * gpc * kGroup * 4);
+    if (max_chunks < 1) max_chunks = 1;
+    const int ks_min = (n_chunks + max_chunks - 1) / max_chunks;
+    int ks_par = (2 * sms) / p.tiles;
+    if (ks_par < 1) ks_par = 1;
+    int ks_cap = n_chunks / kWarps;
+    if (ks_cap < 1) ks_cap = 1;
+    int ks = ks_par < ks_cap ? ks_par : ks_cap;
+    if (ks < ks_min) ks = ks_min;
+    p.chunks_per_split = (n_chunks + ks - 1) / ks;
+    p.splits = (n_chunks + p.chunks_per_split - 1) / p.chunks_per_split;
+    p.smem = (size_t)T * p.chunks_per_split * gpc * kGroup * 4 + (size_t)kWarps * T * 32 * 4;
     return p;
+}
+
+size_t gather_workspace_bytes(const Dims &d, int T, int sms) {
+    const Plan p = plan_gemv(d, T, sms);
+    if (p.splits == 1) return 0;
+    return align16((size_t)p.splits * T * d.d_out * sizeof(float)) + (size_t)p.tiles * sizeof(uint32_t);
 }
 
 GemvFn pick(int M, int B, int T) {
@@ -54,39 +59,52 @@ GemvFn pick(int M, int B, int T) {
     return gemv_pick_2x16(T);
 }
 
+bool use_lut(const Dims &d, int T) { return d.M == 2 && d.B == 8 && T == 1; }
+
+int device_sms() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    return num_sms(dev);
+}
+
 }  // namespace
 }  // namespace gemv_detail
 
 size_t gemv_workspace_bytes(const Dims &d, int tokens) {
-    const gemv_detail::Plan p = gemv_detail::plan_gemv(d, tokens);
-    return p.splits > 1 ? (size_t)p.splits * tokens * d.d_out * sizeof(float) : 0;
+    using namespace gemv_detail;
+    const int sms = device_sms();
+    if (use_lut(d, tokens)) return gemv_lut_workspace_bytes(d, sms);
+    return gather_workspace_bytes(d, tokens, sms);
 }
 
 cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
-                        const uint16_t *x, uint16_t *y, int tokens, const Dims &d, float *workspace,
+                        const uint16_t *x, uint16_t *y, int tokens, const Dims &d, void *workspace,
                         cudaStream_t st) {
     using namespace gemv_detail;
-    const Plan p = plan_gemv(d, tokens);
+    const int sms = device_sms();
+    if (use_lut(d, tokens)) return launch_gemv_lut_2x8(codes, codebooks, scales, x, y, d, workspace, sms, st);
+    const Plan p = plan_gemv(d, tokens, sms);
     GemvFn fn = pick(d.M, d.B, tokens);
     if (p.smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
         if (e != cudaSuccess) return e;
     }
-    const dim3 grid((d.d_out + kRowsPerCta - 1) / kRowsPerCta, p.splits);
-    cudaError_t e = launch_kernel(fn, grid, dim3(kThreads), p.smem, st, false,
-                                  static_cast<const uint8_t *>(codes), reinterpret_cast<const uint4 *>(codebooks),
-                                  reinterpret_cast<const __half *>(scales), reinterpret_cast<const __half *>(x),
-                                  reinterpret_cast<__half *>(y), workspace, d.d_out, d.d_in, d.G, d.row_bytes,
-                                  p.slab_groups);
-    if (e != cudaSuccess || p.splits == 1) return e;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const int n = d.d_out * tokens;
-    int blocks = (n + 255) / 256;
-    if (blocks > num_sms(dev) * 8) blocks = num_sms(dev) * 8;
-    return launch_kernel(gemv_finalize_kernel, dim3(blocks), dim3(256), 0, st, false,
-                         static_cast<const float *>(workspace), reinterpret_cast<const __half *>(scales),
-                         reinterpret_cast<__half *>(y), d.d_out, tokens, p.splits);
+    GemvArgs a;
+    a.codes = static_cast<const uint8_t *>(codes);
+    a.codebooks = reinterpret_cast<const uint4 *>(codebooks);
+    a.scales = reinterpret_cast<const __half *>(scales);
+    a.x = reinterpret_cast<const __half *>(x);
+    a.y = reinterpret_cast<__half *>(y);
+    a.partial = static_cast<float *>(workspace);
+    a.counters = p.splits > 1 ? reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) +
+                                                             align16((size_t)p.splits * tokens * d.d_out * 4))
+                              : nullptr;
+    a.d_out = d.d_out;
+    a.d_in = d.d_in;
+    a.G = d.G;
+    a.row_bytes = d.row_bytes;
+    a.chunks_per_split = p.chunks_per_split;
+    return launch_kernel(fn, dim3(p.tiles, p.splits), dim3(kThreads), p.smem, st, true, a);
 }
 
 }  // namespace aqlm

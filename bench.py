@@ -213,7 +213,7 @@ def bench_gemv(ac, spec, T, steps, warmup, l2_bytes, n_launch=STEP_LAYERS, dist=
     layers = Layers(spec, R, T)
     ys = [torch.empty((T, spec.d_out), dtype=torch.float16, device="cuda") for _ in range(4)]
     need = ac.gemv_workspace_bytes(ac.shape_of(layers.copies[0]["codes"]), T)
-    ws = torch.empty(need, dtype=torch.uint8, device="cuda") if need else None
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda") if need else None
     n_launch = max(n_launch, R)
     g = gemv_graph(ac, layers, n_launch, ys, ws)
     ms = time_replays(g, steps, warmup, dist)

@@ -97,16 +97,24 @@ typedef struct {
  * arithmetic as scaling every group).
  *   codes, codebooks, scales: the layer, layout above.
  *   x: [tokens][d_in] fp16.   y: [tokens][d_out] fp16 (written).
- *   workspace/workspace_bytes: fp32 partial sums for shapes whose activations
- *   do not fit on chip at once; aqlm_gemv_workspace_bytes() gives the size
- *   (0 = none needed, NULL allowed).  Too small -> AQLM_ERR_WORKSPACE.
+ *   workspace/workspace_bytes: device scratch for fp32 partial sums and
+ *   arrival counters, used when a row's input range is split over several
+ *   CTAs; aqlm_gemv_workspace_bytes() gives the size for this device (0 =
+ *   none needed, NULL allowed).  Too small or not 16-byte aligned ->
+ *   AQLM_ERR_WORKSPACE.  The workspace must be zero-filled before its first
+ *   use; every completed call leaves it ready for the next one.  Calls that
+ *   share a workspace must not overlap on the GPU.
+ * Launch: with programmatic dependent launch.  codes, codebooks and scales
+ * are treated as constant weights and may be read before the preceding
+ * kernel in the stream has finished; x is read, and y and the workspace are
+ * written, only after it has finished.
  */
 AQLM_API aqlm_status aqlm_gemv(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                       const uint16_t *x, uint16_t *y, int32_t tokens, aqlm_shape shape,
                       void *workspace, size_t workspace_bytes, aqlm_stream_t stream);
 
 /* Bytes of device workspace aqlm_gemv needs for this shape and token count
- * (0 if none); returns 0 for invalid arguments too. */
+ * on the current device (0 if none); returns 0 for invalid arguments too. */
 AQLM_API size_t aqlm_gemv_workspace_bytes(aqlm_shape shape, int32_t tokens);
 
 /*

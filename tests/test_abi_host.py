@@ -89,7 +89,7 @@ def test_gemv_workspace_rules():
     assert lib.aqlm_gemv_workspace_bytes(shape(), 1) == 0
     assert lib.aqlm_gemv_workspace_bytes(big, 1) == 0
     need = lib.aqlm_gemv_workspace_bytes(big, 16)
-    assert need > 0 and need % (16 * 8192 * 4) == 0
+    assert need >= 2 * 16 * 8192 * 4            # at least two splits of fp32 partial sums
     assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 16, big, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
     assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 16, big, A16, need - 4, NULL) == ac.AQLM_ERR_WORKSPACE
     assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 16, big, ODD, need, NULL) == ac.AQLM_ERR_WORKSPACE

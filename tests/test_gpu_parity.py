@@ -133,6 +133,27 @@ def test_gemv_two_calls_identical():
     assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("M,B", FORMATS)
+def test_gemv_chain_reads_x_after_the_producer(M, B):
+    """Back-to-back layers where each x is the previous layer's y (programmatic
+    dependent launch must not read x early), with a torch kernel in between."""
+    specs = [LayerSpec(1024, 512, M, B), LayerSpec(512, 1024, M, B), LayerSpec(1024, 512, M, B)]
+    Ls = [make_layer(s, seed=40 + k, tokens=1 if k == 0 else 0) for k, s in enumerate(specs)]
+    ds = [to_dev(L) for L in Ls]
+    x = ds[0]["x"]
+    ys = []
+    for k, d in enumerate(ds):
+        y = ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], x)
+        ys.append(y)
+        x = y * 0.5 if k == 0 else y      # a torch kernel between the first two layers
+    torch.cuda.synchronize()
+    xin = [Ls[0]["x"], (ys[0] * 0.5).cpu().numpy(), ys[1].cpu().numpy()]
+    for k, (L, s) in enumerate(zip(Ls, specs)):
+        y_ref = oracle.gemv_f64(L["codes"], L["codebooks"], L["scales"], xin[k], s.d_out, s.d_in, 8, M, B)
+        check_fp_output(ys[k].cpu().numpy(), y_ref, oracle_W(L, s), xin[k].astype(np.float64),
+                        out_rel=2.0 ** -10, acc_rel=2.0 ** -14)
+
+
 FULL_GEMV = [
     ("1x16 4096x4096", 4096, 4096, 1, 16, 1),
     ("2x8 4096x4096", 4096, 4096, 2, 8, 1),
@@ -202,8 +223,10 @@ def test_bf16_gemm_matches_torch():
     ref = (X.float() @ W.float().T)
     assert int(status.item()) == 0
     err = (Y.float() - ref).abs()
-    assert float((err / (ref.abs() + 1e-2)).max()) < 2e-2
-    assert float(err.max()) < 0.25
+    # one bf16 rounding of the output (half an ulp, 2^-8 relative) plus fp32
+    # accumulation over k = 1536 terms
+    absdot = X.float().abs() @ W.float().abs().T
+    assert bool(torch.all(err <= 2.0 ** -8 * ref.abs() + 2.0 ** -14 * absdot + 1e-6))
 
 
 PREFILL = [(11008, 4096, 1, 16), (4096, 11008, 2, 8), (11008, 4096, 2, 8), (4096, 11008, 1, 16)]
