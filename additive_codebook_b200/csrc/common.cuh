@@ -65,6 +65,13 @@ __device__ __forceinline__ uint4 ld_keep_u4(const void *p, uint64_t pol) {
     return v;
 }
 
+// Asynchronous prefetch of [p, p + bytes) into L2 with an evict-last policy
+// (cp.async.bulk.prefetch; p and bytes multiples of 16).
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes, uint64_t pol) {
+    asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(p), "r"(bytes), "l"(pol)
+                 : "memory");
+}
+
 // Eight fp16 values packed in a uint4 -> eight floats (exact conversion).
 __device__ __forceinline__ void half8_to_float8(const uint4 &v, float *f) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};

@@ -7,11 +7,11 @@
 // weights are fetched compressed and dequantised at runtime before the
 // matmul.
 //
-// Both kernels are bound by HBM: decode_indices moves 2-4 bytes per group in
-// and 2M bytes out; dequant reads M*B/8 bytes of codes per group and writes
-// 16 bytes of bf16 (8 values).  One thread owns one group, so a warp's
-// stores cover 512 contiguous bytes and its code loads 64-128 contiguous
-// bytes; the grid is a multiple of the SM count and strides over groups.
+// decode_indices is bound by HBM (2-4 bytes per group in, 2M bytes out).
+// dequant reads M*B/8 bytes of codes per group and writes 16 bytes of bf16;
+// for 2x8 that write stream is the bound, for 1x16/2x16 the codeword gathers
+// from L2 (one 32-byte sector per 16-byte codeword) are.  The grids are a
+// multiple of the SM count and stride over the work.
 #include "common.cuh"
 
 namespace aqlm {
@@ -33,12 +33,17 @@ __global__ void decode_indices_kernel(const void *__restrict__ codes, uint16_t *
 
 // W[i][8j+t] = bf16_rn(fp32(s_i) * (C_0[b0][t] + ... + C_{M-1}[b][t])), the
 // additions in codebook order, every operation rounded on its own.
+// A warp owns a tile of 32 * kPerLane consecutive groups; lane l handles
+// groups l, l + 32, ...: each code load and each 16-byte store instruction of
+// the warp covers contiguous memory (64-128 and 512 bytes), and the lane's
+// kPerLane codeword gathers are in flight together.
+constexpr int kPerLane = 8;
+
 template <int M, int B>
 __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t *__restrict__ codes,
                                                       const uint4 *__restrict__ codebooks,
                                                       const __half *__restrict__ scales,
-                                                      uint4 *__restrict__ W, int G,
-                                                      int64_t n_groups) {
+                                                      uint4 *__restrict__ W, int G, int64_t n_groups) {
     constexpr int K = 1 << B;
     constexpr int kCodeBytes = M * B / 8;
     // 2x8: both codebooks (2 x 256 codewords x 16 B = 8 KiB) live in shared memory.
@@ -48,40 +53,76 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t *__restrict_
         __syncthreads();
     }
     const uint64_t keep = policy_evict_last();
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t gi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; gi < n_groups; gi += stride) {
-        const uint8_t *cp = codes + gi * kCodeBytes;
-        uint32_t idx[M];
-        if constexpr (B == 8) {
-            const uint16_t pair = *reinterpret_cast<const uint16_t *>(cp);  // M == 2
-            idx[0] = pair & 0xffu;
-            idx[1] = pair >> 8;
-        } else if constexpr (M == 1) {
-            idx[0] = *reinterpret_cast<const uint16_t *>(cp);
-        } else {
-            const uint32_t both = *reinterpret_cast<const uint32_t *>(cp);
-            idx[0] = both & 0xffffu;
-            idx[1] = both >> 16;
+    if constexpr (B == 16) {
+        // every layer has its own 1-2 MiB of codebooks, usually cold in L2:
+        // each CTA asks L2 for its share first
+        if (threadIdx.x == 0) {
+            const uint32_t cb_bytes = (uint32_t)M * K * 16;
+            const uint32_t share = ((cb_bytes + gridDim.x - 1) / gridDim.x + 255) & ~255u;
+            const uint32_t off = blockIdx.x * share;
+            if (off < cb_bytes)
+                prefetch_l2_bulk(reinterpret_cast<const uint8_t *>(codebooks) + off, min(share, cb_bytes - off), keep);
         }
-        float acc[kGroup];
+    }
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    constexpr int kTile = 32 * kPerLane;
+    for (int64_t tile = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); tile * kTile < n_groups;
+         tile += warps) {
+        const int64_t g0 = tile * kTile + lane;
+        uint32_t idx[kPerLane][M];
 #pragma unroll
-        for (int m = 0; m < M; ++m) {
-            const uint4 cw = (B == 8) ? cb_smem[m * K + idx[m]] : ld_keep_u4(codebooks + (size_t)m * K + idx[m], keep);
-            float f[kGroup];
-            half8_to_float8(cw, f);
-#pragma unroll
-            for (int t = 0; t < kGroup; ++t) acc[t] = (m == 0) ? f[t] : __fadd_rn(acc[t], f[t]);
+        for (int i = 0; i < kPerLane; ++i) {
+            const int64_t g = g0 + 32 * i;
+            uint32_t raw = 0;
+            if (g < n_groups) {
+                if constexpr (kCodeBytes == 2) {
+                    raw = __ldcs(reinterpret_cast<const uint16_t *>(codes) + g);
+                } else {
+                    raw = __ldcs(reinterpret_cast<const uint32_t *>(codes) + g);
+                }
+            }
+            if constexpr (M == 1) {
+                idx[i][0] = raw & 0xffffu;
+            } else if constexpr (B == 8) {
+                idx[i][0] = raw & 0xffu;
+                idx[i][1] = (raw >> 8) & 0xffu;
+            } else {
+                idx[i][0] = raw & 0xffffu;
+                idx[i][1] = raw >> 16;
+            }
         }
-        const int64_t row = gi / G;
-        const float s = __half2float(scales[row]);
-        uint32_t out[4];
+        uint4 cw[kPerLane][M];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const __nv_bfloat16 lo = __float2bfloat16_rn(__fmul_rn(acc[2 * q], s));
-            const __nv_bfloat16 hi = __float2bfloat16_rn(__fmul_rn(acc[2 * q + 1], s));
-            out[q] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+        for (int i = 0; i < kPerLane; ++i) {
+#pragma unroll
+            for (int m = 0; m < M; ++m) {
+                cw[i][m] = (B == 8) ? cb_smem[m * K + idx[i][m]] : ld_keep_u4(codebooks + (size_t)m * K + idx[i][m], keep);
+            }
         }
-        W[gi] = make_uint4(out[0], out[1], out[2], out[3]);
+#pragma unroll
+        for (int i = 0; i < kPerLane; ++i) {
+            const int64_t g = g0 + 32 * i;
+            if (g >= n_groups) break;
+            const float s = __half2float(scales[g / G]);
+            float acc[kGroup];
+            half8_to_float8(cw[i][0], acc);
+#pragma unroll
+            for (int m = 1; m < M; ++m) {
+                float f[kGroup];
+                half8_to_float8(cw[i][m], f);
+#pragma unroll
+                for (int t = 0; t < kGroup; ++t) acc[t] = __fadd_rn(acc[t], f[t]);
+            }
+            uint32_t out[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const __nv_bfloat16 lo = __float2bfloat16_rn(__fmul_rn(acc[2 * h], s));
+                const __nv_bfloat16 hi = __float2bfloat16_rn(__fmul_rn(acc[2 * h + 1], s));
+                out[h] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+            }
+            W[g] = make_uint4(out[0], out[1], out[2], out[3]);
+        }
     }
 }
 
@@ -105,7 +146,7 @@ cudaError_t launch_decode_indices(const void *codes, uint16_t *idx, const Dims &
 cudaError_t launch_dequant(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                            uint16_t *W, const Dims &d, cudaStream_t st) {
     const int64_t n = (int64_t)d.d_out * d.G;
-    const int grid = grid_for(n, 256, 8);
+    const int grid = grid_for((n + kPerLane - 1) / kPerLane, 256, 8);
     auto c = static_cast<const uint8_t *>(codes);
     auto cb = reinterpret_cast<const uint4 *>(codebooks);
     auto s = reinterpret_cast<const __half *>(scales);

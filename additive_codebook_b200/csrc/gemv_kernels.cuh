@@ -109,6 +109,18 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(const GemvArgs a) {
     const uint64_t stream_pol = policy_evict_first();
     const uint64_t keep_pol = policy_evict_last();
 
+    // The layer's codebooks are usually cold in L2 (every layer has its own):
+    // each CTA asks L2 for its share of them before anything else.
+    if (threadIdx.x == 0) {
+        const uint32_t cb_bytes = (uint32_t)M * F::K * 16;
+        const uint32_t n_cta = gridDim.x * gridDim.y;
+        const uint32_t share = ((cb_bytes + n_cta - 1) / n_cta + 255) & ~255u;
+        const uint32_t off = (blockIdx.y * gridDim.x + blockIdx.x) * share;
+        if (off < cb_bytes) {
+            prefetch_l2_bulk(reinterpret_cast<const uint8_t *>(a.codebooks) + off, min(share, cb_bytes - off),
+                             keep_pol);
+        }
+    }
     // Weights are constant: request the first two chunks before waiting on
     // the kernel that produces x.
     uint4 nxt0 = (valid && wc0 < wc1) ? ld_stream_u4(rowp + (size_t)wc0 * 16, stream_pol) : make_uint4(0, 0, 0, 0);

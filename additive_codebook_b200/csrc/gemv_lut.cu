@@ -14,10 +14,11 @@
 // j0 + l) and a range of rows.  Its tables L_m[j0 + l][k] live in shared
 // memory at word (m * 256 + k) * 32 + l, i.e. in bank l, so the 32 lanes of a
 // warp look up 32 different banks whatever their codes are: no bank
-// conflicts.  Each warp streams 8 rows at a time (lane l loads 16 bytes =
-// 8 groups of row r0 + l/4), stages them in shared memory, reads back its
-// own group's two code bytes per row, looks up and adds; a 5-step butterfly
-// then reduces the 8 row partials over the 32 lanes.  Slabs of one row
+// conflicts.  Each warp streams batches of 8 rows (lane l copies 16 bytes =
+// 8 groups of row r0 + l/4) through an 8-deep ring of asynchronous copies
+// (cp.async) in shared memory, so 64 KiB of codes per CTA are in flight;
+// it reads back its own group's two code bytes per row, looks up and adds; a
+// 5-step butterfly then reduces the 8 row partials over the 32 lanes.  Slabs of one row
 // range publish fp32 partial sums to the caller's workspace; the last CTA of
 // the row range to arrive (atomic counter, no waiting) adds them in slab
 // order (deterministic), scales by s_i, rounds to fp16 and resets the
@@ -29,12 +30,13 @@ namespace aqlm {
 namespace {
 
 constexpr int kSlab = 32;        // groups per slab, one per lane
-constexpr int kLutWarps = 8;
+constexpr int kLutWarps = 16;
 constexpr int kLutThreads = kLutWarps * 32;
 constexpr int kRowsPerBatch = 8;  // rows a warp stages at once (32 lanes x 16 bytes)
+constexpr int kStages = 8;        // batches in flight per warp (cp.async ring)
 constexpr size_t kLutSmem = (size_t)2 * 256 * kSlab * 4    // tables
                             + (size_t)2 * 256 * 8 * 4      // codebooks as fp32
-                            + (size_t)kLutWarps * kRowsPerBatch * kSlab * 2;  // code staging
+                            + (size_t)kLutWarps * kStages * 32 * 16;  // code ring
 
 struct LutArgs {
     const uint8_t *codes;
@@ -48,13 +50,23 @@ struct LutArgs {
 };
 
 __device__ __forceinline__ void gd_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// 16-byte asynchronous global -> shared copy; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void gd_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
 
 __global__ void __launch_bounds__(kLutThreads) gemv_lut_2x8_kernel(const LutArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     float *lut = reinterpret_cast<float *>(smem);               // [2][256][32]
     float *cbf = lut + 2 * 256 * kSlab;                          // [2][256][8]
-    uint4 *stage = reinterpret_cast<uint4 *>(cbf + 2 * 256 * 8);  // [warps][32] uint4
+    uint4 *ring = reinterpret_cast<uint4 *>(cbf + 2 * 256 * 8);  // [warps][stages][32] uint4
     __shared__ int s_last;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -62,21 +74,26 @@ __global__ void __launch_bounds__(kLutThreads) gemv_lut_2x8_kernel(const LutArgs
     const int j0 = slab * kSlab;
     const int row_begin = blockIdx.y * a.rows_per_chunk;
     const int row_end = min(a.d_out, row_begin + a.rows_per_chunk);
-    const uint64_t stream_pol = policy_evict_first();
 
     // This lane's 16-byte piece of a warp batch: row r0 + lane/4, groups
-    // j0 + 8*(lane%4) .. +7.  Groups past the row's end are not loaded.
+    // j0 + 8*(lane%4) .. +7.  Pieces past the row's end or past the last row
+    // are zero-filled instead of loaded.
     const int piece_row = lane >> 2;
     const int piece_group = j0 + 8 * (lane & 3);
     const bool piece_in_row = piece_group < a.G;
-    auto load_piece = [&](int r0) -> uint4 {
-        const int r = r0 + piece_row;
-        if (r < row_end && piece_in_row)
-            return ld_stream_u4(a.codes + (size_t)r * a.row_bytes + (size_t)piece_group * 2, stream_pol);
-        return make_uint4(0, 0, 0, 0);
+    uint4 *wring = ring + (size_t)warp * kStages * 32;
+    auto issue = [&](int batch, int slot) {
+        const int r = row_begin + (batch * kLutWarps + warp) * kRowsPerBatch + piece_row;
+        const bool ok = r < row_end && piece_in_row;
+        const uint8_t *src = ok ? a.codes + (size_t)r * a.row_bytes + (size_t)piece_group * 2 : a.codes;
+        cp_async16(wring + slot * 32 + lane, src, ok ? 16u : 0u);
+        cp_async_commit();
     };
-    int r0 = row_begin + warp * kRowsPerBatch;
-    uint4 nxt = (r0 < row_end) ? load_piece(r0) : make_uint4(0, 0, 0, 0);
+    const int rows = row_end - row_begin;
+    const int n_batches = (rows + kLutWarps * kRowsPerBatch - 1) / (kLutWarps * kRowsPerBatch);
+    // codes are constant weights: fill the ring before waiting on x's producer
+#pragma unroll
+    for (int b = 0; b < kStages; ++b) issue(b, b);
 
     // codebooks (constant weights) -> fp32 in shared memory
     for (int i = threadIdx.x; i < 2 * 256; i += kLutThreads) {
@@ -116,19 +133,19 @@ __global__ void __launch_bounds__(kLutThreads) gemv_lut_2x8_kernel(const LutArgs
 
     const float *lut0 = lut + lane;
     const float *lut1 = lut + 256 * kSlab + lane;
-    const uint16_t *wstage = reinterpret_cast<const uint16_t *>(stage + warp * 32);
-    for (; r0 < row_end; r0 += kLutWarps * kRowsPerBatch) {
-        stage[warp * 32 + lane] = nxt;
-        const int rn = r0 + kLutWarps * kRowsPerBatch;
-        nxt = (rn < row_end) ? load_piece(rn) : make_uint4(0, 0, 0, 0);
+    for (int b = 0; b < n_batches; ++b) {
+        const int slot = b % kStages;
+        cp_async_wait<kStages - 1>();   // the batch in `slot` has landed
         __syncwarp();
+        const uint16_t *codes16 = reinterpret_cast<const uint16_t *>(wring + slot * 32);
         float v[kRowsPerBatch];
 #pragma unroll
         for (int q = 0; q < kRowsPerBatch; ++q) {
-            const uint32_t code = wstage[q * kSlab + lane];  // byte 2l: codebook 0, byte 2l+1: codebook 1
+            const uint32_t code = codes16[q * kSlab + lane];  // byte 2l: codebook 0, byte 2l+1: codebook 1
             v[q] = lut0[(code & 0xffu) * kSlab] + lut1[(code >> 8) * kSlab];
         }
         __syncwarp();
+        issue(b + kStages, slot);   // refill the slot (zero-filled past the end)
         // butterfly: lane bits 4,3,2 select the row, the 4 lanes of a quad end
         // up with the full sum of row r0 + lane/4
         float u[4];
@@ -151,7 +168,7 @@ __global__ void __launch_bounds__(kLutThreads) gemv_lut_2x8_kernel(const LutArgs
         float z = (hi4 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, hi4 ? w2[0] : w2[1], 4);
         z += __shfl_xor_sync(0xffffffffu, z, 2);
         z += __shfl_xor_sync(0xffffffffu, z, 1);
-        const int r = r0 + (lane >> 2);
+        const int r = row_begin + (b * kLutWarps + warp) * kRowsPerBatch + (lane >> 2);
         if ((lane & 3) == 0 && r < row_end) {
             if (n_slabs == 1) {
                 a.y[r] = __float2half_rn(z * __half2float(a.scales[r]));
@@ -160,6 +177,7 @@ __global__ void __launch_bounds__(kLutThreads) gemv_lut_2x8_kernel(const LutArgs
             }
         }
     }
+    cp_async_wait<0>();   // nothing may still be landing in shared memory at exit
     if (n_slabs == 1) return;
 
     __threadfence();
