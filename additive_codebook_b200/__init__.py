@@ -32,7 +32,8 @@ GEMV_MAX_TOKENS = 16
 # Every entry point declared in include/aqlm.h.
 EXPORTS = ["aqlm_gemv", "aqlm_gemv_workspace_bytes", "aqlm_dequant", "aqlm_gemm",
            "aqlm_gemm_workspace_bytes", "aqlm_gemm_check", "aqlm_bf16_gemm", "aqlm_decode_indices",
-           "aqlm_test_gemm_timeout", "aqlm_status_string", "aqlm_version"]
+           "aqlm_test_gemm_timeout", "aqlm_gemv_noalloc", "aqlm_gemv_noalloc_max_scratch_bytes",
+           "aqlm_status_string", "aqlm_version"]
 
 
 class AqlmError(RuntimeError):
@@ -69,6 +70,8 @@ def load_library():
         "aqlm_bf16_gemm": ([vp, vp, vp, i32, i32, i32, vp, vp], st),
         "aqlm_decode_indices": ([vp, vp, Shape, vp], st),
         "aqlm_test_gemm_timeout": ([vp, vp, vp, i32, i32, i32, vp, u64, vp], st),
+        "aqlm_gemv_noalloc": ([vp, vp, vp, vp, vp, i32, Shape, vp], st),
+        "aqlm_gemv_noalloc_max_scratch_bytes": ([], sz),
         "aqlm_status_string": ([st], ctypes.c_char_p),
         "aqlm_version": ([], ctypes.c_char_p),
     }
@@ -136,6 +139,20 @@ def aqlm_gemv(codes, codebooks, scales, x, y=None, workspace=None, stream=None):
     wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(lib.aqlm_gemv(_p(codes), _p(codebooks), _p(_flat_scales(scales)), _p(x), _p(y), T, shape,
                          _p(workspace), wbytes, _stream(stream)), "aqlm_gemv")
+    return y
+
+
+def aqlm_gemv_noalloc(codes, codebooks, scales, x, y=None, stream=None):
+    """aqlm_gemv with the library's built-in scratch array (no workspace)."""
+    lib = load_library()
+    shape = shape_of(codes)
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    T = x.shape[0]
+    if y is None:
+        y = torch.empty((T, shape.d_out), dtype=torch.float16, device=x.device)
+    _check(lib.aqlm_gemv_noalloc(_p(codes), _p(codebooks), _p(_flat_scales(scales)), _p(x), _p(y), T, shape,
+                                 _stream(stream)), "aqlm_gemv_noalloc")
     return y
 
 

@@ -120,6 +120,7 @@ cudaError_t launch_decode_indices(const void *codes, uint16_t *idx, const Dims &
 cudaError_t launch_dequant(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                            uint16_t *W, const Dims &d, cudaStream_t st);
 size_t gemv_workspace_bytes(const Dims &d, int tokens);
+size_t gemv_workspace_counter_offset(const Dims &d, int tokens);
 cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                         const uint16_t *x, uint16_t *y, int tokens, const Dims &d, void *workspace,
                         cudaStream_t st);

@@ -8,6 +8,7 @@
 namespace aqlm {
 
 size_t gemv_lut_workspace_bytes(const Dims &d, int sms);
+size_t gemv_lut_workspace_counter_offset(const Dims &d, int sms);
 cudaError_t launch_gemv_lut_2x8(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                                 const uint16_t *x, uint16_t *y, const Dims &d, void *workspace, int sms,
                                 cudaStream_t st);
@@ -75,6 +76,17 @@ size_t gemv_workspace_bytes(const Dims &d, int tokens) {
     const int sms = device_sms();
     if (use_lut(d, tokens)) return gemv_lut_workspace_bytes(d, sms);
     return gather_workspace_bytes(d, tokens, sms);
+}
+
+// Offset of the arrival counters inside the workspace: the bytes from here to
+// the end of the workspace must be zero before a call.
+size_t gemv_workspace_counter_offset(const Dims &d, int tokens) {
+    using namespace gemv_detail;
+    const int sms = device_sms();
+    if (use_lut(d, tokens)) return gemv_lut_workspace_counter_offset(d, sms);
+    const Plan p = plan_gemv(d, tokens, sms);
+    if (p.splits == 1) return 0;
+    return align16((size_t)p.splits * tokens * d.d_out * sizeof(float));
 }
 
 cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint16_t *scales,

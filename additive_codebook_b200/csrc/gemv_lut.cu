@@ -226,6 +226,13 @@ size_t gemv_lut_workspace_bytes(const Dims &d, int sms) {
     return align16((size_t)p.n_slabs * d.d_out * sizeof(float)) + (size_t)p.row_chunks * sizeof(uint32_t);
 }
 
+// Offset of the arrival counters (the part that must be zero before a call).
+size_t gemv_lut_workspace_counter_offset(const Dims &d, int sms) {
+    const LutPlan p = plan_lut(d, sms);
+    if (p.n_slabs == 1) return 0;
+    return align16((size_t)p.n_slabs * d.d_out * sizeof(float));
+}
+
 cudaError_t launch_gemv_lut_2x8(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                                 const uint16_t *x, uint16_t *y, const Dims &d, void *workspace, int sms,
                                 cudaStream_t st) {

@@ -186,6 +186,33 @@ AQLM_API aqlm_status aqlm_decode_indices(const void *codes, uint16_t *idx_out, a
 AQLM_API aqlm_status aqlm_test_gemm_timeout(const uint16_t *X, const uint16_t *W, uint16_t *Y, int32_t tokens, int32_t n,
                                    int32_t k, int32_t *status, uint64_t limit_ns, aqlm_stream_t stream);
 
+/*
+ * aqlm_gemv_noalloc -- aqlm_gemv without a caller-provided workspace, for
+ * callers that cannot allocate device memory (for example a plugin that its
+ * host engine hands only input and output pointers, or an engine that fixes
+ * its device memory at start-up and allows no allocation afterwards).  The
+ * paper has no counterpart of this entry point; it is a library convenience.
+ *
+ * The scratch it needs lives in a fixed array inside the library, 8 MiB per
+ * GPU (aqlm_gemv_noalloc_max_scratch_bytes()), held by every GPU that loads
+ * the library until the process exits.  A shape and token count whose
+ * scratch (aqlm_gemv_workspace_bytes) exceeds that is rejected with
+ * AQLM_ERR_WORKSPACE.  The first call on a device looks up the array's
+ * device address there (cudaGetSymbolAddress); make that first call before
+ * any stream capture.  The part of the array that must start at zero is
+ * cleared on `stream` at every call.  All calls on a device share the one
+ * array and it keeps the last call's contents: calls that overlap on the GPU
+ * (other streams, other host threads) race and must be avoided.  No
+ * cudaMalloc, cudaFree or other allocating routine is called.  Arguments,
+ * results and errors otherwise as aqlm_gemv.
+ */
+AQLM_API aqlm_status aqlm_gemv_noalloc(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                                       const uint16_t *x, uint16_t *y, int32_t tokens, aqlm_shape shape,
+                                       aqlm_stream_t stream);
+
+/* Size of aqlm_gemv_noalloc's built-in scratch array, in bytes. */
+AQLM_API size_t aqlm_gemv_noalloc_max_scratch_bytes(void);
+
 /* A static, human-readable name of a status code. */
 AQLM_API const char *aqlm_status_string(aqlm_status status);
 

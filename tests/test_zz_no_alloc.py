@@ -1,0 +1,69 @@
+"""aqlm_gemv_noalloc: the decode product for callers that cannot allocate.
+
+Some callers of this library have no way to allocate device memory when they
+call it -- a plugin that its host engine hands only input and output
+pointers, or an engine that fixes its device memory at start-up.  For them
+aqlm_gemv_noalloc keeps its scratch in an array built into the library
+instead of a caller-provided workspace.  These tests call it through the C
+ABI, twice in a row on the same shape, and hold its output to the tolerance
+of the other parity tests against aqlm_gemv's output on the same inputs.
+
+This file is named so that pytest collects it last: a run that stops at the
+first failure has then already run every other test.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import additive_codebook_b200 as ac
+import oracle
+from gpu_util import DEV, check_fp_output, oracle_W, to_dev
+from synth import LayerSpec, make_layer
+
+pytestmark = pytest.mark.gpu
+
+# shapes whose product needs scratch: the 2x8 lookup-table path (16 slabs),
+# the 1x16 path split over the input range to fill the SMs, and a 16-token
+# product split because its activations do not fit on chip at once
+CASES = [(4096, 4096, 2, 8, 1), (4096, 4096, 1, 16, 1), (1024, 4096, 1, 16, 16), (512, 4160, 2, 16, 4)]
+
+
+def _call_noalloc(lib, d, x, y):
+    shape = ac.shape_of(d["codes"])
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return lib.aqlm_gemv_noalloc(ctypes.c_void_p(d["codes"].data_ptr()), ctypes.c_void_p(d["codebooks"].data_ptr()),
+                                 ctypes.c_void_p(d["scales"].data_ptr()), ctypes.c_void_p(x.data_ptr()),
+                                 ctypes.c_void_p(y.data_ptr()), x.shape[0], shape, stream)
+
+
+@pytest.mark.parametrize("d_out,d_in,M,B,T", CASES)
+def test_noalloc_matches_gemv_on_two_calls(cuda_device, d_out, d_in, M, B, T):
+    lib = ac.load_library()
+    spec = LayerSpec(d_out, d_in, M, B)
+    L = make_layer(spec, seed=77 + T, tokens=T)
+    d = to_dev(L)
+    shape = ac.shape_of(d["codes"])
+    assert 0 < lib.aqlm_gemv_workspace_bytes(shape, T) <= lib.aqlm_gemv_noalloc_max_scratch_bytes()
+    y_ref = ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], d["x"]).cpu().numpy().astype(np.float64)
+    W = oracle_W(L, spec)
+    x64 = L["x"].astype(np.float64)
+    for _ in range(2):
+        y = torch.full((T, d_out), float("nan"), dtype=torch.float16, device=DEV)
+        assert _call_noalloc(lib, d, d["x"], y) == ac.AQLM_OK
+        torch.cuda.synchronize()
+        check_fp_output(y.cpu().numpy(), y_ref, W, x64, out_rel=2.0 ** -10, acc_rel=2.0 ** -14)
+
+
+def test_noalloc_rejects_scratch_beyond_its_maximum(cuda_device):
+    lib = ac.load_library()
+    shape = ac.Shape(28672, 8192, 8, 1, 16)     # 16 tokens: far more than 8 MiB of partial sums
+    assert lib.aqlm_gemv_workspace_bytes(shape, 16) > lib.aqlm_gemv_noalloc_max_scratch_bytes()
+    codes = torch.zeros(16, dtype=torch.uint8, device=DEV)
+    x = torch.zeros(16, 8192, dtype=torch.float16, device=DEV)
+    y = torch.zeros(16, 28672, dtype=torch.float16, device=DEV)
+    p = ctypes.c_void_p(codes.data_ptr())
+    st = lib.aqlm_gemv_noalloc(p, p, p, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()), 16, shape,
+                               ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == ac.AQLM_ERR_WORKSPACE
