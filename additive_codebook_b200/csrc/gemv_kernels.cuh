@@ -8,11 +8,13 @@
 // decoding is bound by memory traffic, so the codes (2 or 4 bytes per group)
 // are the only large stream and everything else stays on chip.
 //
-// Work decomposition (one CTA = 16 warps = a tile of 32 output rows):
+// Work decomposition (one CTA = 8 warps = a tile of 32 output rows):
 //   - lane l of every warp owns row (tile * 32 + l); the CTA's input range is
-//     a run of 16-byte code chunks (8 groups, or 4 for 2x16) that the 16
+//     a run of 16-byte code chunks (8 groups, or 4 for 2x16) that the 8
 //     warps split into contiguous pieces, so each lane streams its own row's
 //     codes with 128-bit loads that bypass L1 and leave L2 first;
+//   - software pipeline per lane: the codeword gathers of chunk c+1 and the
+//     code load of chunk c+2 are in flight while chunk c is multiplied;
 //   - the activations of the CTA's input range are staged once in shared
 //     memory as fp32; all lanes of a warp work on the same group at the same
 //     time, so every activation load is a broadcast;
@@ -30,9 +32,9 @@
 //     so the result is deterministic, and resets the counter;
 //   - the row's sum is scaled by s_i and rounded once to fp16.
 // Programmatic dependent launch: the weights (codes, codebooks, scales) are
-// constant, so the first code chunks are requested before
-// griddepcontrol.wait; x is read and y, the partial sums and the counters are
-// written only after it.
+// constant, so the first code chunks are loaded and the first chunk's
+// codewords gathered before griddepcontrol.wait; x is read and y, the partial
+// sums and the counters are written only after it.
 #pragma once
 
 #include <array>
@@ -44,7 +46,7 @@ namespace aqlm {
 namespace gemv_detail {
 
 constexpr int kRowsPerCta = 32;
-constexpr int kWarps = 16;
+constexpr int kWarps = 8;
 constexpr int kThreads = kRowsPerCta * kWarps;
 constexpr int kXsBudget = 64 * 1024;  // bytes of fp32 activations per CTA
 
@@ -82,6 +84,51 @@ struct GemvArgs {
     int d_out, d_in, G, row_bytes;
     int chunks_per_split;
 };
+
+// The codeword gathers of one 16-byte code chunk: GPC groups x M codebooks.
+template <int M, int B>
+__device__ __forceinline__ void gather_chunk(const uint4 &ch, const uint4 *__restrict__ codebooks, uint64_t pol,
+                                             uint4 (&cw)[Fmt<M, B>::kGroupsPerChunk][M]) {
+    using F = Fmt<M, B>;
+#pragma unroll
+    for (int q = 0; q < F::kGroupsPerChunk; ++q) {
+#pragma unroll
+        for (int m = 0; m < M; ++m) cw[q][m] = ld_keep_u4(codebooks + (size_t)m * F::K + chunk_index<M, B>(ch, q, m), pol);
+    }
+}
+
+// acc[t] += sum over the chunk's groups of < sum_m C_m[b], x_t[group] >, with
+// x read from shared memory as warp-wide broadcasts; two partial sums per
+// group shorten the dependent FMA chains.
+template <int M, int B, int T>
+__device__ __forceinline__ void fma_chunk(const uint4 (&cw)[Fmt<M, B>::kGroupsPerChunk][M], const float *xp,
+                                          int xs_stride, float (&acc)[T]) {
+    using F = Fmt<M, B>;
+#pragma unroll
+    for (int q = 0; q < F::kGroupsPerChunk; ++q) {
+        float w[kGroup];
+        half8_to_float8(cw[q][0], w);
+        if constexpr (M == 2) {
+            float f[kGroup];
+            half8_to_float8(cw[q][1], f);
+#pragma unroll
+            for (int e = 0; e < kGroup; ++e) w[e] += f[e];
+        }
+#pragma unroll
+        for (int t = 0; t < T; ++t) {
+            const float4 p = *reinterpret_cast<const float4 *>(xp + (size_t)t * xs_stride + q * kGroup);
+            const float4 r = *reinterpret_cast<const float4 *>(xp + (size_t)t * xs_stride + q * kGroup + 4);
+            float s0 = w[0] * p.x, s1 = w[1] * p.y;
+            s0 = fmaf(w[2], p.z, s0);
+            s1 = fmaf(w[3], p.w, s1);
+            s0 = fmaf(w[4], r.x, s0);
+            s1 = fmaf(w[5], r.y, s1);
+            s0 = fmaf(w[6], r.z, s0);
+            s1 = fmaf(w[7], r.w, s1);
+            acc[t] += s0 + s1;
+        }
+    }
+}
 
 template <int M, int B, int T>
 __global__ void __launch_bounds__(kThreads) gemv_kernel(const GemvArgs a) {
@@ -121,13 +168,17 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(const GemvArgs a) {
                              keep_pol);
         }
     }
-    // Weights are constant: request the first two chunks before waiting on
-    // the kernel that produces x.
-    uint4 nxt0 = (valid && wc0 < wc1) ? ld_stream_u4(rowp + (size_t)wc0 * 16, stream_pol) : make_uint4(0, 0, 0, 0);
-    uint4 nxt1 = (valid && wc0 + 1 < wc1) ? ld_stream_u4(rowp + (size_t)(wc0 + 1) * 16, stream_pol)
-                                           : make_uint4(0, 0, 0, 0);
-    grid_dependency_wait();
+    // Weights are constant: before waiting on the kernel that produces x,
+    // load the first two code chunks and gather the first chunk's codewords.
+    auto load_chunk = [&](int c) -> uint4 {
+        return (valid && c < wc1) ? ld_stream_u4(rowp + (size_t)c * 16, stream_pol) : make_uint4(0, 0, 0, 0);
+    };
+    uint4 ch_cur = load_chunk(wc0);
+    uint4 ch_nxt = load_chunk(wc0 + 1);
+    uint4 cwA[GPC][M], cwB[GPC][M];
+    gather_chunk<M, B>(ch_cur, a.codebooks, keep_pol, cwA);
 
+    grid_dependency_wait();
     for (int i = threadIdx.x; i < T * ng; i += kThreads) {
         const int t = i / ng, q = i - t * ng;
         const uint4 v = *reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.d_in + (size_t)(g0 + q) * kGroup);
@@ -144,51 +195,22 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(const GemvArgs a) {
 #pragma unroll
     for (int t = 0; t < T; ++t) acc[t] = 0.f;
 
+    // software pipeline, two chunks per trip so both codeword buffers stay in
+    // registers: at the top cwA holds chunk c's codewords and ch_nxt chunk
+    // c+1's codes; chunk c+1's codewords and chunk c+2's codes are in flight
+    // while chunk c is multiplied, and so on
     for (int c = wc0; c < wc1; c += 2) {
-        const uint4 cur[2] = {nxt0, nxt1};
-        if (c + 2 < wc1) nxt0 = valid ? ld_stream_u4(rowp + (size_t)(c + 2) * 16, stream_pol) : make_uint4(0, 0, 0, 0);
-        if (c + 3 < wc1) nxt1 = valid ? ld_stream_u4(rowp + (size_t)(c + 3) * 16, stream_pol) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            if (c + u >= wc1) break;
-            // all codeword gathers of the chunk first, so they are in flight together
-            uint4 cw[GPC][M];
-#pragma unroll
-            for (int q = 0; q < GPC; ++q) {
-#pragma unroll
-                for (int m = 0; m < M; ++m) {
-                    const uint32_t k = chunk_index<M, B>(cur[u], q, m);
-                    cw[q][m] = ld_keep_u4(a.codebooks + (size_t)m * F::K + k, keep_pol);
-                }
-            }
-#pragma unroll
-            for (int q = 0; q < GPC; ++q) {
-                float w[kGroup];
-                half8_to_float8(cw[q][0], w);
-                if constexpr (M == 2) {
-                    float f[kGroup];
-                    half8_to_float8(cw[q][1], f);
-#pragma unroll
-                    for (int e = 0; e < kGroup; ++e) w[e] += f[e];
-                }
-                const float *xp = xs + ((c + u) * GPC + q - g0) * kGroup;
-#pragma unroll
-                for (int t = 0; t < T; ++t) {
-                    const float4 p = *reinterpret_cast<const float4 *>(xp + (size_t)t * xs_stride);
-                    const float4 r = *reinterpret_cast<const float4 *>(xp + (size_t)t * xs_stride + 4);
-                    float s = acc[t];
-                    s = fmaf(w[0], p.x, s);
-                    s = fmaf(w[1], p.y, s);
-                    s = fmaf(w[2], p.z, s);
-                    s = fmaf(w[3], p.w, s);
-                    s = fmaf(w[4], r.x, s);
-                    s = fmaf(w[5], r.y, s);
-                    s = fmaf(w[6], r.z, s);
-                    s = fmaf(w[7], r.w, s);
-                    acc[t] = s;
-                }
-            }
+        if (c + 1 < wc1) {
+            gather_chunk<M, B>(ch_nxt, a.codebooks, keep_pol, cwB);
+            ch_nxt = load_chunk(c + 2);
         }
+        fma_chunk<M, B, T>(cwA, xs + (size_t)(c * GPC - g0) * kGroup, xs_stride, acc);
+        if (c + 1 >= wc1) break;
+        if (c + 2 < wc1) {
+            gather_chunk<M, B>(ch_nxt, a.codebooks, keep_pol, cwA);
+            ch_nxt = load_chunk(c + 3);
+        }
+        fma_chunk<M, B, T>(cwB, xs + (size_t)((c + 1) * GPC - g0) * kGroup, xs_stride, acc);
     }
 
 #pragma unroll
