@@ -72,6 +72,12 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes, 
                  : "memory");
 }
 
+// Programmatic dependent launch: wait until the preceding kernel in the
+// stream has completed (and its writes are visible); let the next kernel in
+// the stream start launching.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 // Eight fp16 values packed in a uint4 -> eight floats (exact conversion).
 __device__ __forceinline__ void half8_to_float8(const uint4 &v, float *f) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};

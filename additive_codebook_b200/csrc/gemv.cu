@@ -1,14 +1,19 @@
 // gemv.cu -- host side of the decode-time product: kernel choice, work plan,
 // workspace layout and the launch (with programmatic dependent launch).
-// The gather kernels are in gemv_kernels.cuh (instantiated per format in
-// gemv_1x16.cu, gemv_2x8.cu, gemv_2x16.cu); the batch-1 2x8 lookup-table
-// kernel is in gemv_lut.cu.
+// One token: gemv_rows.cu (coalesced row streaming); the 2x8 lookup-table
+// kernel in gemv_lut.cu is its alternative for 2x8.  Several tokens (and
+// one token with activations too large for shared memory): the gather
+// kernels of gemv_kernels.cuh, instantiated per format in gemv_1x16.cu,
+// gemv_2x8.cu and gemv_2x16.cu.
 #include "gemv_kernels.cuh"
 
 namespace aqlm {
 
 size_t gemv_lut_workspace_bytes(const Dims &d, int sms);
 size_t gemv_lut_workspace_counter_offset(const Dims &d, int sms);
+bool gemv_rows_supported(const Dims &d);
+cudaError_t launch_gemv_rows(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
+                             uint16_t *y, const Dims &d, int sms, cudaStream_t st);
 cudaError_t launch_gemv_lut_2x8(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                                 const uint16_t *x, uint16_t *y, const Dims &d, void *workspace, int sms,
                                 cudaStream_t st);
@@ -33,7 +38,8 @@ Plan plan_gemv(const Dims &d, int T, int sms) {
     const int n_chunks = d.G / gpc;
     Plan p;
     p.tiles = (d.d_out + kRowsPerCta - 1) / kRowsPerCta;
-    int max_chunks = kXsBudget / (T * gpc * kGroup * 4);
+    const int tp = (T == 1) ? 1 : ((T + 3) & ~3);  // tokens padded in shared memory
+    int max_chunks = kXsBudget / (tp * gpc * kGroup * 4);
     if (max_chunks < 1) max_chunks = 1;
     const int ks_min = (n_chunks + max_chunks - 1) / max_chunks;
     int ks_par = (2 * sms) / p.tiles;
@@ -44,7 +50,7 @@ Plan plan_gemv(const Dims &d, int T, int sms) {
     if (ks < ks_min) ks = ks_min;
     p.chunks_per_split = (n_chunks + ks - 1) / ks;
     p.splits = (n_chunks + p.chunks_per_split - 1) / p.chunks_per_split;
-    p.smem = (size_t)T * p.chunks_per_split * gpc * kGroup * 4 + (size_t)kWarps * T * 32 * 4;
+    p.smem = (size_t)tp * p.chunks_per_split * gpc * kGroup * 4 + (size_t)kWarps * T * 32 * 4;
     return p;
 }
 
@@ -60,7 +66,14 @@ GemvFn pick(int M, int B, int T) {
     return gemv_pick_2x16(T);
 }
 
-bool use_lut(const Dims &d, int T) { return d.M == 2 && d.B == 8 && T == 1; }
+// One token: whole rows per warp with coalesced code streaming (no
+// workspace) when the activations fit on chip; the 2x8 lookup-table kernel
+// is the alternative for 2x8.
+constexpr bool kPreferLut2x8 = true;
+bool use_rows(const Dims &d, int T) {
+    return T == 1 && gemv_rows_supported(d) && !(kPreferLut2x8 && d.M == 2 && d.B == 8);
+}
+bool use_lut(const Dims &d, int T) { return d.M == 2 && d.B == 8 && T == 1 && !use_rows(d, T); }
 
 int device_sms() {
     int dev = 0;
@@ -74,6 +87,7 @@ int device_sms() {
 size_t gemv_workspace_bytes(const Dims &d, int tokens) {
     using namespace gemv_detail;
     const int sms = device_sms();
+    if (use_rows(d, tokens)) return 0;
     if (use_lut(d, tokens)) return gemv_lut_workspace_bytes(d, sms);
     return gather_workspace_bytes(d, tokens, sms);
 }
@@ -83,6 +97,7 @@ size_t gemv_workspace_bytes(const Dims &d, int tokens) {
 size_t gemv_workspace_counter_offset(const Dims &d, int tokens) {
     using namespace gemv_detail;
     const int sms = device_sms();
+    if (use_rows(d, tokens)) return 0;
     if (use_lut(d, tokens)) return gemv_lut_workspace_counter_offset(d, sms);
     const Plan p = plan_gemv(d, tokens, sms);
     if (p.splits == 1) return 0;
@@ -94,6 +109,7 @@ cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint
                         cudaStream_t st) {
     using namespace gemv_detail;
     const int sms = device_sms();
+    if (use_rows(d, tokens)) return launch_gemv_rows(codes, codebooks, scales, x, y, d, sms, st);
     if (use_lut(d, tokens)) return launch_gemv_lut_2x8(codes, codebooks, scales, x, y, d, workspace, sms, st);
     const Plan p = plan_gemv(d, tokens, sms);
     GemvFn fn = pick(d.M, d.B, tokens);

@@ -16,8 +16,10 @@
 //   - software pipeline per lane: the codeword gathers of chunk c+1 and the
 //     code load of chunk c+2 are in flight while chunk c is multiplied;
 //   - the activations of the CTA's input range are staged once in shared
-//     memory as fp32; all lanes of a warp work on the same group at the same
-//     time, so every activation load is a broadcast;
+//     memory as fp32, token-interleaved ([group][element][token], tokens
+//     padded to a multiple of 4); all lanes of a warp work on the same group
+//     at the same time, so every activation load is a broadcast, and for
+//     several tokens one 16-byte load feeds two packed fp32x2 FMAs;
 //   - codewords are gathered through L1/L2 with an evict-last policy (the
 //     1-2 MiB of 1x16/2x16 codebooks stay cache resident; measured on B200,
 //     random 16-byte gathers from L2 run at about one 32-byte sector per SM
@@ -97,13 +99,34 @@ __device__ __forceinline__ void gather_chunk(const uint4 &ch, const uint4 *__res
     }
 }
 
-// acc[t] += sum over the chunk's groups of < sum_m C_m[b], x_t[group] >, with
-// x read from shared memory as warp-wide broadcasts; two partial sums per
-// group shorten the dependent FMA chains.
+// Tokens padded to a multiple of 4 in shared memory (one token stays 1).
+template <int T>
+struct TokPad {
+    static constexpr int value = (T == 1) ? 1 : ((T + 3) & ~3);
+};
+
+__device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+// Two fp32 FMAs in one instruction (sm_100 packed fp32): d = a * b + c lane-wise.
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b, unsigned long long c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// acc += sum over the chunk's groups of < sum_m C_m[b], x_t[group] > for every
+// token t.  Activations in shared memory as xs[(group * 8 + e) * TP + t]
+// (fp32), read as warp-wide broadcasts.  One token: two partial sums per
+// group shorten the dependent chain.  Several tokens: an LDS.128 brings 4
+// tokens of one element and packed FMAs update 2 tokens per instruction.
 template <int M, int B, int T>
-__device__ __forceinline__ void fma_chunk(const uint4 (&cw)[Fmt<M, B>::kGroupsPerChunk][M], const float *xp,
-                                          int xs_stride, float (&acc)[T]) {
+__device__ __forceinline__ void fma_chunk(const uint4 (&cw)[Fmt<M, B>::kGroupsPerChunk][M], const float *xg,
+                                          float (&acc1)[1], unsigned long long (&acc2)[(TokPad<T>::value + 1) / 2]) {
     using F = Fmt<M, B>;
+    constexpr int TP = TokPad<T>::value;
 #pragma unroll
     for (int q = 0; q < F::kGroupsPerChunk; ++q) {
         float w[kGroup];
@@ -114,10 +137,10 @@ __device__ __forceinline__ void fma_chunk(const uint4 (&cw)[Fmt<M, B>::kGroupsPe
 #pragma unroll
             for (int e = 0; e < kGroup; ++e) w[e] += f[e];
         }
-#pragma unroll
-        for (int t = 0; t < T; ++t) {
-            const float4 p = *reinterpret_cast<const float4 *>(xp + (size_t)t * xs_stride + q * kGroup);
-            const float4 r = *reinterpret_cast<const float4 *>(xp + (size_t)t * xs_stride + q * kGroup + 4);
+        const float *xq = xg + q * kGroup * TP;
+        if constexpr (T == 1) {
+            const float4 p = *reinterpret_cast<const float4 *>(xq);
+            const float4 r = *reinterpret_cast<const float4 *>(xq + 4);
             float s0 = w[0] * p.x, s1 = w[1] * p.y;
             s0 = fmaf(w[2], p.z, s0);
             s1 = fmaf(w[3], p.w, s1);
@@ -125,7 +148,18 @@ __device__ __forceinline__ void fma_chunk(const uint4 (&cw)[Fmt<M, B>::kGroupsPe
             s1 = fmaf(w[5], r.y, s1);
             s0 = fmaf(w[6], r.z, s0);
             s1 = fmaf(w[7], r.w, s1);
-            acc[t] += s0 + s1;
+            acc1[0] += s0 + s1;
+        } else {
+#pragma unroll
+            for (int e = 0; e < kGroup; ++e) {
+                const unsigned long long ww = pack2(w[e], w[e]);
+#pragma unroll
+                for (int t4 = 0; t4 < TP / 4; ++t4) {
+                    const float4 v = *reinterpret_cast<const float4 *>(xq + e * TP + 4 * t4);
+                    acc2[2 * t4] = ffma2(ww, pack2(v.x, v.y), acc2[2 * t4]);
+                    acc2[2 * t4 + 1] = ffma2(ww, pack2(v.z, v.w), acc2[2 * t4 + 1]);
+                }
+            }
         }
     }
 }
@@ -141,9 +175,9 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(const GemvArgs a) {
     const int c0 = split * a.chunks_per_split;
     const int c1 = min(n_chunks_row, c0 + a.chunks_per_split);
     const int g0 = c0 * GPC, ng = (c1 - c0) * GPC;
-    const int xs_stride = a.chunks_per_split * GPC * kGroup;  // floats per token
-    float *xs = reinterpret_cast<float *>(smem);
-    float *red = xs + (size_t)T * xs_stride;                  // [kWarps][T][32]
+    constexpr int TP = TokPad<T>::value;
+    float *xs = reinterpret_cast<float *>(smem);                              // [group][8][TP]
+    float *red = xs + (size_t)a.chunks_per_split * GPC * kGroup * TP;         // [kWarps][T][32]
     __shared__ int s_last;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -179,21 +213,25 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(const GemvArgs a) {
     gather_chunk<M, B>(ch_cur, a.codebooks, keep_pol, cwA);
 
     grid_dependency_wait();
-    for (int i = threadIdx.x; i < T * ng; i += kThreads) {
+    for (int i = threadIdx.x; i < TP * ng; i += kThreads) {  // padded tokens are zeros
         const int t = i / ng, q = i - t * ng;
-        const uint4 v = *reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.d_in + (size_t)(g0 + q) * kGroup);
         float f[kGroup];
-        half8_to_float8(v, f);
-        float4 *dst = reinterpret_cast<float4 *>(xs + (size_t)t * xs_stride + q * kGroup);
-        dst[0] = make_float4(f[0], f[1], f[2], f[3]);
-        dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+        if (t < T) {
+            half8_to_float8(*reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.d_in + (size_t)(g0 + q) * kGroup), f);
+        } else {
+#pragma unroll
+            for (int e = 0; e < kGroup; ++e) f[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < kGroup; ++e) xs[((size_t)q * kGroup + e) * TP + t] = f[e];
     }
     __syncthreads();
     grid_dependents_launch();
 
-    float acc[T];
+    float acc1[1] = {0.f};
+    unsigned long long acc2[(TP + 1) / 2];
 #pragma unroll
-    for (int t = 0; t < T; ++t) acc[t] = 0.f;
+    for (int i = 0; i < (TP + 1) / 2; ++i) acc2[i] = 0ull;
 
     // software pipeline, two chunks per trip so both codeword buffers stay in
     // registers: at the top cwA holds chunk c's codewords and ch_nxt chunk
@@ -204,15 +242,27 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(const GemvArgs a) {
             gather_chunk<M, B>(ch_nxt, a.codebooks, keep_pol, cwB);
             ch_nxt = load_chunk(c + 2);
         }
-        fma_chunk<M, B, T>(cwA, xs + (size_t)(c * GPC - g0) * kGroup, xs_stride, acc);
+        fma_chunk<M, B, T>(cwA, xs + (size_t)(c * GPC - g0) * kGroup * TP, acc1, acc2);
         if (c + 1 >= wc1) break;
         if (c + 2 < wc1) {
             gather_chunk<M, B>(ch_nxt, a.codebooks, keep_pol, cwA);
             ch_nxt = load_chunk(c + 3);
         }
-        fma_chunk<M, B, T>(cwB, xs + (size_t)((c + 1) * GPC - g0) * kGroup, xs_stride, acc);
+        fma_chunk<M, B, T>(cwB, xs + (size_t)((c + 1) * GPC - g0) * kGroup * TP, acc1, acc2);
     }
 
+    float acc[T];
+    if constexpr (T == 1) {
+        acc[0] = acc1[0];
+    } else {
+#pragma unroll
+        for (int i = 0; i < (TP + 1) / 2; ++i) {
+            float lo, hi;
+            asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(acc2[i]));
+            if (2 * i < T) acc[2 * i] = lo;
+            if (2 * i + 1 < T) acc[2 * i + 1] = hi;
+        }
+    }
 #pragma unroll
     for (int t = 0; t < T; ++t) red[(warp * T + t) * 32 + lane] = acc[t];
     __syncthreads();
@@ -251,8 +301,16 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(const GemvArgs a) {
         const int t = i >> 5, l = i & 31;
         const int r = tile_row0 + l;
         if (r >= a.d_out) continue;
+        // 8 partials in flight per thread, added in split order
         float sum = 0.f;
-        for (int s = 0; s < splits; ++s) sum += __ldcg(&a.partial[((size_t)s * T + t) * a.d_out + r]);
+        for (int s0 = 0; s0 < splits; s0 += 8) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                v[u] = (s0 + u < splits) ? __ldcg(&a.partial[((size_t)(s0 + u) * T + t) * a.d_out + r]) : 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) sum += v[u];
+        }
         a.y[(size_t)t * a.d_out + r] = __float2half_rn(sum * __half2float(a.scales[r]));
     }
     if (threadIdx.x == 0) a.counters[blockIdx.x] = 0u;

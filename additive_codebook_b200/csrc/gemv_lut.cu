@@ -189,9 +189,17 @@ __global__ void __launch_bounds__(kLutThreads) gemv_lut_2x8_kernel(const LutArgs
     __syncthreads();
     if (!s_last) return;
     __threadfence();
+    // 16 partials in flight per thread, added in slab order
     for (int r = row_begin + threadIdx.x; r < row_end; r += kLutThreads) {
         float sum = 0.f;
-        for (int s = 0; s < n_slabs; ++s) sum += __ldcg(&a.partial[(size_t)s * a.d_out + r]);
+        for (int s0 = 0; s0 < n_slabs; s0 += 16) {
+            float v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+                v[u] = (s0 + u < n_slabs) ? __ldcg(&a.partial[(size_t)(s0 + u) * a.d_out + r]) : 0.f;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) sum += v[u];
+        }
         a.y[r] = __float2half_rn(sum * __half2float(a.scales[r]));
     }
     if (threadIdx.x == 0) a.counters[blockIdx.y] = 0u;

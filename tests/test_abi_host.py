@@ -87,9 +87,11 @@ def test_gemv_workspace_rules():
     lib = ac.load_library()
     big = ac.Shape(8192, 8192, 8, 1, 16)
     assert lib.aqlm_gemv_workspace_bytes(big, 1) == 0          # enough row tiles: no split
-    small = lib.aqlm_gemv_workspace_bytes(shape(), 1)          # 2x8 lookup tables: 2 slabs
-    assert small >= 2 * 256 * 4
-    assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 1, shape(), NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_gemv_workspace_bytes(shape(), 1) == 0      # one token: whole rows per warp
+    wide = shape(d_in=4096)                                    # 8 row tiles: split to fill the SMs
+    small = lib.aqlm_gemv_workspace_bytes(wide, 2)
+    assert small >= 2 * 2 * 256 * 4
+    assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 2, wide, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
     need = lib.aqlm_gemv_workspace_bytes(big, 16)
     assert need >= 2 * 16 * 8192 * 4            # at least two splits of fp32 partial sums
     assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 16, big, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE

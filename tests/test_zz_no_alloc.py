@@ -24,10 +24,10 @@ from synth import LayerSpec, make_layer
 
 pytestmark = pytest.mark.gpu
 
-# shapes whose product needs scratch: the 2x8 lookup-table path (16 slabs),
-# the 1x16 path split over the input range to fill the SMs, and a 16-token
-# product split because its activations do not fit on chip at once
-CASES = [(4096, 4096, 2, 8, 1), (4096, 4096, 1, 16, 1), (1024, 4096, 1, 16, 16), (512, 4160, 2, 16, 4)]
+# shapes whose product needs scratch: few-token products split over the
+# input range to fill the SMs, and a 16-token product split because its
+# activations do not fit on chip at once
+CASES = [(4096, 4096, 1, 16, 2), (2048, 4096, 2, 8, 3), (1024, 4096, 1, 16, 16), (512, 4160, 2, 16, 4)]
 
 
 def _call_noalloc(lib, d, x, y):
