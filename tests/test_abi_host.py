@@ -87,7 +87,8 @@ def test_gemv_workspace_rules():
     lib = ac.load_library()
     big = ac.Shape(8192, 8192, 8, 1, 16)
     assert lib.aqlm_gemv_workspace_bytes(big, 1) == 0          # enough row tiles: no split
-    assert lib.aqlm_gemv_workspace_bytes(shape(), 1) == 0      # one token: whole rows per warp
+    assert lib.aqlm_gemv_workspace_bytes(shape(M=1, B=16), 1) == 0   # one token: whole rows per warp
+    assert lib.aqlm_gemv_workspace_bytes(shape(), 1) > 0       # 2x8, one token: lookup tables, 2 slabs
     wide = shape(d_in=4096)                                    # 8 row tiles: split to fill the SMs
     small = lib.aqlm_gemv_workspace_bytes(wide, 2)
     assert small >= 2 * 2 * 256 * 4
