@@ -408,7 +408,7 @@ def run_gpu(args):
                      "frac": round(achieved / peaks["hbm_gbs"], 4),
                      "traffic": recorded_traffic("gemv 1x16 4096x4096 T1"),
                      "peak_source": f"{peaks['source']} copy bandwidth",
-                     "kernel": "gemv_kernel<1,16,1>",
+                     "kernel": "gemv_rows_kernel<1,16>",
                      "algorithmic_bytes_per_launch": head["bytes_per_layer"]},
         "cpu_baseline": cpu,
         "e2e": e2e,
