@@ -198,13 +198,25 @@ def time_replays(g, steps, warmup, dist=None):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     if dist is not None:
-        import torch.distributed as tdist
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dist)
         dist.barrier()
     torch.cuda.synchronize()
     return ms
+
+
+def max_over_ranks(value, dist):
+    """The largest of every rank's value (all ranks get it): the job's time is
+    its slowest replica's time."""
+    import torch
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(value)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world, steps, launches_per_step, bytes_per_launch, max_ms):
+    """Whole-job throughput: the bytes every replica processed / the slowest time."""
+    return world * steps * launches_per_step * bytes_per_launch / (max_ms * 1e-3) / 1e9
 
 
 def bench_gemv(ac, spec, T, steps, warmup, l2_bytes, n_launch=STEP_LAYERS, dist=None):
@@ -361,7 +373,7 @@ def run_gpu(args):
 
     head = bench_gemv(ac, HEADLINE, 1, args.steps, args.warmup, l2, dist=dist)
     n_launch = max(STEP_LAYERS, head["copies"])
-    value = world * args.steps * n_launch * head["bytes_per_layer"] / (head["ms"] * 1e-3) / 1e9
+    value = whole_job_gbs(world, args.steps, n_launch, head["bytes_per_layer"], head["ms"])
     achieved = head["bytes_per_layer"] / (head["us_per_layer"] * 1e-6) / 1e9
     detail = {}
     if not args.quick:
