@@ -5,7 +5,7 @@
 // one token with activations too large for shared memory): the gather
 // kernels of gemv_kernels.cuh, instantiated per format in gemv_1x16.cu,
 // gemv_2x8.cu and gemv_2x16.cu.
-#include "gemv_kernels.cuh"
+#include "gemv_multi.cuh"
 
 namespace aqlm {
 
@@ -54,10 +54,41 @@ Plan plan_gemv(const Dims &d, int T, int sms) {
     return p;
 }
 
+Plan plan_multi(const Dims &d, int T, int sms);
+
 size_t gather_workspace_bytes(const Dims &d, int T, int sms) {
-    const Plan p = plan_gemv(d, T, sms);
+    const Plan p = T > 1 ? plan_multi(d, T, sms) : plan_gemv(d, T, sms);
     if (p.splits == 1) return 0;
     return align16((size_t)p.splits * T * d.d_out * sizeof(float)) + (size_t)p.tiles * sizeof(uint32_t);
+}
+
+// Several tokens: tiles of 32*R rows, the same split rules with the fp16
+// token-interleaved activation budget and about three CTAs per SM.
+Plan plan_multi(const Dims &d, int T, int sms) {
+    const int gpc = 16 / (d.M * d.B / 8);
+    const int n_chunks = d.G / gpc;
+    const int R = 4, tp8 = (T + 7) & ~7;
+    Plan p;
+    p.tiles = (d.d_out + 32 * R - 1) / (32 * R);
+    int max_chunks = kXsBudget / (tp8 * gpc * kGroup * 2);
+    if (max_chunks < 1) max_chunks = 1;
+    const int ks_min = (n_chunks + max_chunks - 1) / max_chunks;
+    int ks_par = (3 * sms) / p.tiles;
+    if (ks_par < 1) ks_par = 1;
+    int ks_cap = n_chunks / kMultiWarps;
+    if (ks_cap < 1) ks_cap = 1;
+    int ks = ks_par < ks_cap ? ks_par : ks_cap;
+    if (ks < ks_min) ks = ks_min;
+    p.chunks_per_split = (n_chunks + ks - 1) / ks;
+    p.splits = (n_chunks + p.chunks_per_split - 1) / p.chunks_per_split;
+    p.smem = (size_t)tp8 * p.chunks_per_split * gpc * kGroup * 2 + (size_t)kMultiWarps * T * 32 * R * 4;
+    return p;
+}
+
+GemvFn pick_multi(int M, int B, int T) {
+    if (M == 1) return gemv_multi_pick_1x16(T);
+    if (B == 8) return gemv_multi_pick_2x8(T);
+    return gemv_multi_pick_2x16(T);
 }
 
 GemvFn pick(int M, int B, int T) {
@@ -99,7 +130,7 @@ size_t gemv_workspace_counter_offset(const Dims &d, int tokens) {
     const int sms = device_sms();
     if (use_rows(d, tokens)) return 0;
     if (use_lut(d, tokens)) return gemv_lut_workspace_counter_offset(d, sms);
-    const Plan p = plan_gemv(d, tokens, sms);
+    const Plan p = tokens > 1 ? plan_multi(d, tokens, sms) : plan_gemv(d, tokens, sms);
     if (p.splits == 1) return 0;
     return align16((size_t)p.splits * tokens * d.d_out * sizeof(float));
 }
@@ -111,8 +142,9 @@ cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint
     const int sms = device_sms();
     if (use_rows(d, tokens)) return launch_gemv_rows(codes, codebooks, scales, x, y, d, sms, st);
     if (use_lut(d, tokens)) return launch_gemv_lut_2x8(codes, codebooks, scales, x, y, d, workspace, sms, st);
-    const Plan p = plan_gemv(d, tokens, sms);
-    GemvFn fn = pick(d.M, d.B, tokens);
+    const bool multi = tokens > 1;
+    const Plan p = multi ? plan_multi(d, tokens, sms) : plan_gemv(d, tokens, sms);
+    GemvFn fn = multi ? pick_multi(d.M, d.B, tokens) : pick(d.M, d.B, tokens);
     if (p.smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
         if (e != cudaSuccess) return e;
@@ -132,7 +164,7 @@ cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint
     a.G = d.G;
     a.row_bytes = d.row_bytes;
     a.chunks_per_split = p.chunks_per_split;
-    return launch_kernel(fn, dim3(p.tiles, p.splits), dim3(kThreads), p.smem, st, true, a);
+    return launch_kernel(fn, dim3(p.tiles, p.splits), dim3(multi ? kMultiThreads : kThreads), p.smem, st, true, a);
 }
 
 }  // namespace aqlm
