@@ -11,9 +11,9 @@ namespace aqlm {
 
 size_t gemv_lut_workspace_bytes(const Dims &d, int sms);
 size_t gemv_lut_workspace_counter_offset(const Dims &d, int sms);
-bool gemv_rows_supported(const Dims &d);
+bool gemv_rows_supported(const Dims &d, int T);
 cudaError_t launch_gemv_rows(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
-                             uint16_t *y, const Dims &d, int sms, cudaStream_t st);
+                             uint16_t *y, int tokens, const Dims &d, int sms, cudaStream_t st);
 cudaError_t launch_gemv_lut_2x8(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                                 const uint16_t *x, uint16_t *y, const Dims &d, void *workspace, int sms,
                                 cudaStream_t st);
@@ -97,12 +97,12 @@ GemvFn pick(int M, int B, int T) {
     return gemv_pick_2x16(T);
 }
 
-// One token: whole rows per warp with coalesced code streaming (no
-// workspace) when the activations fit on chip; the 2x8 lookup-table kernel
-// is the alternative for 2x8.
+// Up to four tokens: whole rows per warp with coalesced code streaming (no
+// workspace) when the activations fit on chip; for one token of 2x8 the
+// lookup-table kernel is the alternative.
 constexpr bool kPreferLut2x8 = true;
 bool use_rows(const Dims &d, int T) {
-    return T == 1 && gemv_rows_supported(d) && !(kPreferLut2x8 && d.M == 2 && d.B == 8);
+    return gemv_rows_supported(d, T) && !(kPreferLut2x8 && T == 1 && d.M == 2 && d.B == 8);
 }
 bool use_lut(const Dims &d, int T) { return d.M == 2 && d.B == 8 && T == 1 && !use_rows(d, T); }
 
@@ -140,7 +140,7 @@ cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint
                         cudaStream_t st) {
     using namespace gemv_detail;
     const int sms = device_sms();
-    if (use_rows(d, tokens)) return launch_gemv_rows(codes, codebooks, scales, x, y, d, sms, st);
+    if (use_rows(d, tokens)) return launch_gemv_rows(codes, codebooks, scales, x, y, tokens, d, sms, st);
     if (use_lut(d, tokens)) return launch_gemv_lut_2x8(codes, codebooks, scales, x, y, d, workspace, sms, st);
     const bool multi = tokens > 1;
     const Plan p = multi ? plan_multi(d, tokens, sms) : plan_gemv(d, tokens, sms);

@@ -1,19 +1,20 @@
-// gemv_rows.cu -- batch-1 layer product with coalesced code streaming.
+// gemv_rows.cu -- layer product for 1..4 tokens with coalesced code streaming.
 //
 // "The AQLM Quantization Algorithm, Explained", section "What is
 // Multi-Codebook Quantization (MCQ)?": y_i = s_i * sum_j < sum_m C_m[b(i,j,m)],
 // x_j >.  Section "Why and what do we quantize?": decoding is bound by
 // memory traffic, and the codes are the only large stream.
 //
-// Design for one token: a warp owns whole rows; its 32 lanes take the row's
+// Design for few tokens: a warp owns whole rows; its 32 lanes take the row's
 // 16-byte code chunks l, l + 32, l + 64, ... so every code load of the warp
 // reads 512 contiguous bytes of one row (full DRAM bursts; measured on B200,
 // reading the codes in row-strided 16-byte pieces instead cost about 5 us
 // per 4096x4096 layer).  Each lane gathers the codewords of its chunk's
 // groups (1x16 / 2x16 through L1/L2 with an evict-last policy; 2x8 from
-// shared memory), multiplies them with the activations and keeps one fp32
-// partial sum; at the end of a row five shuffles add the 32 partials, lane 0
-// scales by s_i and rounds once to fp16.  No split, no workspace.
+// shared memory), multiplies them with every token's activations and keeps
+// one fp32 partial sum per token; at the end of a row five shuffles per token
+// add the 32 partials, lane 0 scales by s_i and rounds once to fp16.  No
+// split, no workspace.
 //   - Activations are staged once per CTA in shared memory as fp16,
 //     transposed by chunk ([group within chunk][chunk]) so that the lanes of
 //     a warp, which work on consecutive chunks, read consecutive 16 bytes.
@@ -59,14 +60,14 @@ __device__ __forceinline__ uint32_t code_index(const uint4 &ch, int q, int m) {
     }
 }
 
-template <int M, int B>
+template <int M, int B, int T>
 __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a) {
     using F = RowFmt<M, B>;
     constexpr int GPC = F::GPC;
     extern __shared__ __align__(16) unsigned char smem[];
     const int n_chunks = a.G / GPC;
-    uint4 *xs = reinterpret_cast<uint4 *>(smem);  // [GPC][n_chunks] groups of 8 fp16
-    uint4 *cbs = xs + a.G;                        // 2x8: [M][256] codewords
+    uint4 *xs = reinterpret_cast<uint4 *>(smem);  // [T][GPC][n_chunks] groups of 8 fp16
+    uint4 *cbs = xs + (size_t)T * a.G;            // 2x8: [M][256] codewords
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int total_warps = gridDim.x * kRowWarps;
@@ -118,25 +119,31 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
         const uint4 ch0 = load_code(0);
         if constexpr (!F::kSmemCodebook) gather(ch0, 0, cwA);
         grid_dep_wait();
-        for (int i = threadIdx.x; i < a.G; i += kRowThreads) {  // stage x, transposed by chunk
-            const int c = i / GPC, q = i - c * GPC;
-            xs[q * n_chunks + c] = *reinterpret_cast<const uint4 *>(a.x + (size_t)i * kGroup);
+        for (int i = threadIdx.x; i < T * a.G; i += kRowThreads) {  // stage x, transposed by chunk
+            const int t = i / a.G, g = i - t * a.G;
+            const int c = g / GPC, q = g - c * GPC;
+            xs[((size_t)t * GPC + q) * n_chunks + c] = *reinterpret_cast<const uint4 *>(a.x + (size_t)i * kGroup);
         }
         __syncthreads();
         if constexpr (F::kSmemCodebook) gather(ch0, 0, cwA);
     }
     grid_dep_launch();
 
-    float acc = 0.f;
+    float acc[T];
+#pragma unroll
+    for (int t = 0; t < T; ++t) acc[t] = 0.f;
     // y for the item's row once its last chunk slot has been added
     auto finish_item = [&](int k) {
         if (k % cpw != cpw - 1) return;
-        float v = acc;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         const int r = item_row(k);
-        if (lane == 0 && r < a.d_out) a.y[r] = __float2half_rn(v * __half2float(a.scales[r]));
-        acc = 0.f;
+#pragma unroll
+        for (int t = 0; t < T; ++t) {
+            float v = acc[t];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0 && r < a.d_out) a.y[(size_t)t * a.d_out + r] = __float2half_rn(v * __half2float(a.scales[r]));
+            acc[t] = 0.f;
+        }
     };
     auto multiply = [&](const uint4 (&cw)[GPC][M], int k) {
         const int c = lane + 32 * (k % cpw);
@@ -151,15 +158,18 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
 #pragma unroll
                 for (int e = 0; e < kGroup; ++e) w[e] += f[e];
             }
-            half8_to_float8(xs[q * n_chunks + c], xv);
-            float s0 = w[0] * xv[0], s1 = w[1] * xv[1];
-            s0 = fmaf(w[2], xv[2], s0);
-            s1 = fmaf(w[3], xv[3], s1);
-            s0 = fmaf(w[4], xv[4], s0);
-            s1 = fmaf(w[5], xv[5], s1);
-            s0 = fmaf(w[6], xv[6], s0);
-            s1 = fmaf(w[7], xv[7], s1);
-            acc += s0 + s1;
+#pragma unroll
+            for (int t = 0; t < T; ++t) {
+                half8_to_float8(xs[((size_t)t * GPC + q) * n_chunks + c], xv);
+                float s0 = w[0] * xv[0], s1 = w[1] * xv[1];
+                s0 = fmaf(w[2], xv[2], s0);
+                s1 = fmaf(w[3], xv[3], s1);
+                s0 = fmaf(w[4], xv[4], s0);
+                s1 = fmaf(w[5], xv[5], s1);
+                s0 = fmaf(w[6], xv[6], s0);
+                s1 = fmaf(w[7], xv[7], s1);
+                acc[t] += s0 + s1;
+            }
         }
     };
 
@@ -179,11 +189,26 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
 
 }  // namespace
 
-// Rows fit on chip when d_in fp16 activations (+ 8 KiB of 2x8 codebooks) do.
-bool gemv_rows_supported(const Dims &d) { return (size_t)d.d_in * 2 + 8192 <= 160 * 1024; }
+constexpr int kRowsMaxTokens = 4;
+
+// Whole rows per warp when the tokens are few and T * d_in fp16 activations
+// (+ 8 KiB of 2x8 codebooks) fit on chip.
+bool gemv_rows_supported(const Dims &d, int T) {
+    return T >= 1 && T <= kRowsMaxTokens && (size_t)T * d.d_in * 2 + 8192 <= 160 * 1024;
+}
+
+template <int M, int B>
+void (*rows_fn(int T))(const RowArgs) {
+    switch (T) {
+        case 1: return gemv_rows_kernel<M, B, 1>;
+        case 2: return gemv_rows_kernel<M, B, 2>;
+        case 3: return gemv_rows_kernel<M, B, 3>;
+        default: return gemv_rows_kernel<M, B, 4>;
+    }
+}
 
 cudaError_t launch_gemv_rows(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
-                             uint16_t *y, const Dims &d, int sms, cudaStream_t st) {
+                             uint16_t *y, int tokens, const Dims &d, int sms, cudaStream_t st) {
     RowArgs a;
     a.codes = static_cast<const uint8_t *>(codes);
     a.codebooks = reinterpret_cast<const uint4 *>(codebooks);
@@ -193,16 +218,16 @@ cudaError_t launch_gemv_rows(const void *codes, const uint16_t *codebooks, const
     a.d_out = d.d_out;
     a.G = d.G;
     a.row_bytes = d.row_bytes;
-    const size_t smem = (size_t)d.G * 16 + ((d.B == 8) ? (size_t)d.M * 256 * 16 : 0);
+    const size_t smem = (size_t)tokens * d.G * 16 + ((d.B == 8) ? (size_t)d.M * 256 * 16 : 0);
     int grid = (d.d_out + kRowWarps - 1) / kRowWarps;
     if (grid > 2 * sms) grid = 2 * sms;
     void (*fn)(const RowArgs);
     if (d.M == 1) {
-        fn = gemv_rows_kernel<1, 16>;
+        fn = rows_fn<1, 16>(tokens);
     } else if (d.B == 8) {
-        fn = gemv_rows_kernel<2, 8>;
+        fn = rows_fn<2, 8>(tokens);
     } else {
-        fn = gemv_rows_kernel<2, 16>;
+        fn = rows_fn<2, 16>(tokens);
     }
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -89,10 +89,11 @@ def test_gemv_workspace_rules():
     assert lib.aqlm_gemv_workspace_bytes(big, 1) == 0          # enough row tiles: no split
     assert lib.aqlm_gemv_workspace_bytes(shape(M=1, B=16), 1) == 0   # one token: whole rows per warp
     assert lib.aqlm_gemv_workspace_bytes(shape(), 1) > 0       # 2x8, one token: lookup tables, 2 slabs
-    wide = shape(d_in=4096)                                    # 8 row tiles: split to fill the SMs
-    small = lib.aqlm_gemv_workspace_bytes(wide, 2)
-    assert small >= 2 * 2 * 256 * 4
-    assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 2, wide, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
+    wide = shape(d_in=4096)                                    # 8 tokens, 2 row tiles: split to fill the SMs
+    assert lib.aqlm_gemv_workspace_bytes(wide, 4) == 0         # up to 4 tokens: whole rows per warp
+    small = lib.aqlm_gemv_workspace_bytes(wide, 8)
+    assert small >= 2 * 8 * 256 * 4
+    assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 8, wide, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
     need = lib.aqlm_gemv_workspace_bytes(big, 16)
     assert need >= 2 * 16 * 8192 * 4            # at least two splits of fp32 partial sums
     assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 16, big, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE

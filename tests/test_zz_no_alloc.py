@@ -24,10 +24,11 @@ from synth import LayerSpec, make_layer
 
 pytestmark = pytest.mark.gpu
 
-# shapes whose product needs scratch: few-token products split over the
-# input range to fill the SMs, and a 16-token product split because its
-# activations do not fit on chip at once
-CASES = [(4096, 4096, 1, 16, 2), (2048, 4096, 2, 8, 3), (1024, 4096, 1, 16, 16), (512, 4160, 2, 16, 4)]
+# shapes whose product needs scratch: the one-token 2x8 lookup-table path
+# (slab partial sums), products of several tokens split over the input range
+# to fill the SMs, and a 16-token product split because its activations do
+# not fit on chip at once
+CASES = [(4096, 4096, 2, 8, 1), (2048, 4096, 2, 8, 6), (1024, 4096, 1, 16, 16), (512, 4160, 2, 16, 8)]
 
 
 def _call_noalloc(lib, d, x, y):
@@ -58,11 +59,11 @@ def test_noalloc_matches_gemv_on_two_calls(cuda_device, d_out, d_in, M, B, T):
 
 def test_noalloc_rejects_scratch_beyond_its_maximum(cuda_device):
     lib = ac.load_library()
-    shape = ac.Shape(28672, 8192, 8, 1, 16)     # 16 tokens: far more than 8 MiB of partial sums
+    shape = ac.Shape(131072, 8192, 8, 1, 16)    # 16 tokens: far more than 8 MiB of partial sums
     assert lib.aqlm_gemv_workspace_bytes(shape, 16) > lib.aqlm_gemv_noalloc_max_scratch_bytes()
-    codes = torch.zeros(16, dtype=torch.uint8, device=DEV)
-    x = torch.zeros(16, 8192, dtype=torch.float16, device=DEV)
-    y = torch.zeros(16, 28672, dtype=torch.float16, device=DEV)
+    codes = torch.zeros(16, dtype=torch.uint8, device=DEV)   # never read: the call is rejected first
+    x = torch.zeros(16, 16, dtype=torch.float16, device=DEV)
+    y = torch.zeros(16, 16, dtype=torch.float16, device=DEV)
     p = ctypes.c_void_p(codes.data_ptr())
     st = lib.aqlm_gemv_noalloc(p, p, p, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()), 16, shape,
                                ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
