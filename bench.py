@@ -151,8 +151,11 @@ class Layers:
             if r == 0:
                 self.host0 = L
         x = self.host0["x"]
-        self.x = (torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16) if x.dtype == np.uint16
-                  else torch.from_numpy(x).cuda())
+        if x is None:
+            self.x = None
+        else:
+            self.x = (torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16) if x.dtype == np.uint16
+                      else torch.from_numpy(x).cuda())
 
 
 def copies_for(spec, T, l2_bytes, min_copies=2):
