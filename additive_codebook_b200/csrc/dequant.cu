@@ -33,11 +33,43 @@ __global__ void decode_indices_kernel(const void *__restrict__ codes, uint16_t *
 
 // W[i][8j+t] = bf16_rn(fp32(s_i) * (C_0[b0][t] + ... + C_{M-1}[b][t])), the
 // additions in codebook order, every operation rounded on its own.
-// A warp owns a tile of 32 * kPerLane consecutive groups; lane l handles
-// groups l, l + 32, ...: each code load and each 16-byte store instruction of
-// the warp covers contiguous memory (64-128 and 512 bytes), and the lane's
-// kPerLane codeword gathers are in flight together.
-constexpr int kPerLane = 8;
+// A warp walks tiles of 32 * kPerLane consecutive groups (lane l handles
+// groups l, l + 32, ...: every code load and every 16-byte store of the warp
+// covers contiguous memory) in a software pipeline: the codes of tile k+2
+// and the codeword gathers of tile k+1 are in flight while tile k is
+// converted and stored.
+constexpr int kPerLane = 4;
+constexpr int kTile = 32 * kPerLane;
+
+template <int M, int B>
+struct DequantStep {
+    static constexpr int K = 1 << B;
+    static constexpr int kCodeBytes = M * B / 8;
+};
+
+template <int M, int B>
+__device__ __forceinline__ void load_codes(const uint8_t *__restrict__ codes, int64_t g0, int64_t n_groups,
+                                           uint32_t (&raw)[kPerLane]) {
+#pragma unroll
+    for (int i = 0; i < kPerLane; ++i) {
+        const int64_t g = g0 + 32 * i;
+        raw[i] = 0;
+        if (g < n_groups) {
+            if constexpr (DequantStep<M, B>::kCodeBytes == 2) {
+                raw[i] = __ldcs(reinterpret_cast<const uint16_t *>(codes) + g);
+            } else {
+                raw[i] = __ldcs(reinterpret_cast<const uint32_t *>(codes) + g);
+            }
+        }
+    }
+}
+
+template <int M, int B>
+__device__ __forceinline__ uint32_t raw_index(uint32_t raw, int m) {
+    if constexpr (M == 1) return raw & 0xffffu;
+    else if constexpr (B == 8) return (raw >> (8 * m)) & 0xffu;
+    else return (raw >> (16 * m)) & 0xffffu;
+}
 
 template <int M, int B>
 __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t *__restrict__ codes,
@@ -45,7 +77,6 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t *__restrict_
                                                       const __half *__restrict__ scales,
                                                       uint4 *__restrict__ W, int G, int64_t n_groups) {
     constexpr int K = 1 << B;
-    constexpr int kCodeBytes = M * B / 8;
     // 2x8: both codebooks (2 x 256 codewords x 16 B = 8 KiB) live in shared memory.
     __shared__ uint4 cb_smem[B == 8 ? M * K : 1];
     if constexpr (B == 8) {
@@ -65,44 +96,23 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t *__restrict_
         }
     }
     const int lane = threadIdx.x & 31;
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    constexpr int kTile = 32 * kPerLane;
-    for (int64_t tile = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); tile * kTile < n_groups;
-         tile += warps) {
-        const int64_t g0 = tile * kTile + lane;
-        uint32_t idx[kPerLane][M];
-#pragma unroll
-        for (int i = 0; i < kPerLane; ++i) {
-            const int64_t g = g0 + 32 * i;
-            uint32_t raw = 0;
-            if (g < n_groups) {
-                if constexpr (kCodeBytes == 2) {
-                    raw = __ldcs(reinterpret_cast<const uint16_t *>(codes) + g);
-                } else {
-                    raw = __ldcs(reinterpret_cast<const uint32_t *>(codes) + g);
-                }
-            }
-            if constexpr (M == 1) {
-                idx[i][0] = raw & 0xffffu;
-            } else if constexpr (B == 8) {
-                idx[i][0] = raw & 0xffu;
-                idx[i][1] = (raw >> 8) & 0xffu;
-            } else {
-                idx[i][0] = raw & 0xffffu;
-                idx[i][1] = raw >> 16;
-            }
-        }
-        uint4 cw[kPerLane][M];
+    const int64_t stride = (int64_t)gridDim.x * (blockDim.x >> 5) * kTile;  // groups between a warp's tiles
+    int64_t g0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kTile + lane;
+
+    auto gather = [&](const uint32_t (&raw)[kPerLane], uint4 (&cw)[kPerLane][M]) {
 #pragma unroll
         for (int i = 0; i < kPerLane; ++i) {
 #pragma unroll
             for (int m = 0; m < M; ++m) {
-                cw[i][m] = (B == 8) ? cb_smem[m * K + idx[i][m]] : ld_keep_u4(codebooks + (size_t)m * K + idx[i][m], keep);
+                const uint32_t k = raw_index<M, B>(raw[i], m);
+                cw[i][m] = (B == 8) ? cb_smem[m * K + k] : ld_keep_u4(codebooks + (size_t)m * K + k, keep);
             }
         }
+    };
+    auto emit = [&](const uint4 (&cw)[kPerLane][M], int64_t gt) {
 #pragma unroll
         for (int i = 0; i < kPerLane; ++i) {
-            const int64_t g = g0 + 32 * i;
+            const int64_t g = gt + 32 * i;
             if (g >= n_groups) break;
             const float s = __half2float(scales[g / G]);
             float acc[kGroup];
@@ -123,6 +133,22 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t *__restrict_
             }
             W[g] = make_uint4(out[0], out[1], out[2], out[3]);
         }
+    };
+
+    uint32_t rawA[kPerLane], rawB[kPerLane];
+    uint4 cwA[kPerLane][M], cwB[kPerLane][M];
+    load_codes<M, B>(codes, g0, n_groups, rawA);
+    load_codes<M, B>(codes, g0 + stride, n_groups, rawB);
+    gather(rawA, cwA);
+    // two tiles per trip so both buffers stay in registers
+    for (; g0 - lane < n_groups; g0 += 2 * stride) {
+        load_codes<M, B>(codes, g0 + 2 * stride, n_groups, rawA);
+        gather(rawB, cwB);
+        emit(cwA, g0);
+        if (g0 + stride - lane >= n_groups) break;
+        load_codes<M, B>(codes, g0 + 3 * stride, n_groups, rawB);
+        gather(rawA, cwA);
+        emit(cwB, g0 + stride);
     }
 }
 
@@ -146,7 +172,7 @@ cudaError_t launch_decode_indices(const void *codes, uint16_t *idx, const Dims &
 cudaError_t launch_dequant(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                            uint16_t *W, const Dims &d, cudaStream_t st) {
     const int64_t n = (int64_t)d.d_out * d.G;
-    const int grid = grid_for((n + kPerLane - 1) / kPerLane, 256, 8);
+    const int grid = grid_for((n + kPerLane - 1) / kPerLane, 256, 4);
     auto c = static_cast<const uint8_t *>(codes);
     auto cb = reinterpret_cast<const uint4 *>(codebooks);
     auto s = reinterpret_cast<const __half *>(scales);
