@@ -43,7 +43,6 @@ constexpr int kTile = 32 * kPerLane;
 
 template <int M, int B>
 struct DequantStep {
-    static constexpr int K = 1 << B;
     static constexpr int kCodeBytes = M * B / 8;
 };
 
