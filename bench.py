@@ -272,7 +272,7 @@ def bench_prefill(ac, spec, tokens, reps, warmup):
     X = L.x
     Y = torch.empty((tokens, spec.d_out), dtype=torch.bfloat16, device="cuda")
     ws = torch.empty(ac.gemm_workspace_bytes(ac.shape_of(d["codes"]), tokens), dtype=torch.uint8, device="cuda")
-    W = ws[256:].view(torch.bfloat16).view(spec.d_out, spec.d_in)
+    W = ws[ws.numel() - 2 * spec.d_out * spec.d_in:].view(torch.bfloat16).view(spec.d_out, spec.d_in)  # W^ region
     # L2 flush by READING a 256 MiB buffer: a write-based flush would leave
     # ~126 MB of dirty lines whose write-back the timed kernel would pay for
     flush = torch.zeros(32 * 1024 * 1024, dtype=torch.int64, device="cuda")
