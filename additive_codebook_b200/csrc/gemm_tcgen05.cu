@@ -145,7 +145,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 
 // ---- fused dequantisation (aqlm_gemm) ----
-// Four extra warps per CTA decode W^ (the same binary32 steps as
+// Twelve extra warps per CTA decode W^ (the same binary32 steps as
 // aqlm_dequant) block of 256 rows by block, in the order the tile schedule
 // consumes them; every CTA takes one slice of every block.  A CTA publishes
 // its slice through the block's arrival counter (release); the TMA producer
@@ -153,7 +153,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 // then orders its tensor-memory-access loads after them with a proxy fence.
 // The blocks of the first wave of tiles are decoded by the epilogue warps as
 // well (they are idle until the first accumulator is ready).
-constexpr int kDequantWarps = 4;
+constexpr int kDequantWarps = 12;
 constexpr int kFusedThreads = kGemmThreads + 32 * kDequantWarps;
 
 struct FuseArgs {
@@ -230,17 +230,18 @@ __device__ void dequant_groups(const FuseArgs &fa, int64_t lo, int64_t hi, int t
     }
 }
 
-// Decode part `part` of `parts` of this CTA's slice of block b, then publish it.
+// Decode parts [p_lo, p_hi) of `parts` of this CTA's slice of block b, then
+// publish them.
 template <int M, int B>
-__device__ void dequant_block_part(const FuseArgs &fa, int n_total, int b, int part, int parts, int tid, int nthreads,
-                                   int bar_id, uint64_t keep, const uint4 *cb_smem) {
+__device__ void dequant_block_part(const FuseArgs &fa, int n_total, int b, int p_lo, int p_hi, int parts, int tid,
+                                   int nthreads, int bar_id, uint64_t keep, const uint4 *cb_smem) {
     const int64_t row0 = (int64_t)b * BN;
     const int64_t rows = min((int64_t)BN, (int64_t)n_total - row0);
     const int64_t base = row0 * fa.G, total = rows * fa.G;
     const int64_t s_lo = base + total * blockIdx.x / gridDim.x;
     const int64_t s_hi = base + total * (blockIdx.x + 1) / gridDim.x;
-    const int64_t lo = s_lo + (s_hi - s_lo) * part / parts;
-    const int64_t hi = s_lo + (s_hi - s_lo) * (part + 1) / parts;
+    const int64_t lo = s_lo + (s_hi - s_lo) * p_lo / parts;
+    const int64_t hi = s_lo + (s_hi - s_lo) * p_hi / parts;
     dequant_groups<M, B>(fa, lo, hi, tid, nthreads, keep, cb_smem);
     __threadfence();
     asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(nthreads) : "memory");
@@ -428,7 +429,9 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
             // idle until the first accumulator: help decode the first wave's blocks
             const int b0 = first_wave_blocks(num_tiles, m_tiles);
             for (int b = 0; b < b0; ++b)
-                dequant_block_part<FM, FB>(fa, n_total, b, 1, 2, threadIdx.x - 64, 32 * kEpiWarps, 2, keep_pol, cb_smem);
+                dequant_block_part<FM, FB>(fa, n_total, b, kDequantWarps, kDequantWarps + kEpiWarps,
+                                           kDequantWarps + kEpiWarps, threadIdx.x - 64, 32 * kEpiWarps, 2, keep_pol,
+                                           cb_smem);
         }
         // ---- epilogue: warps 2..5, TMEM lane quarter = warp % 4 ----
         const int quarter = warp & 3;
@@ -478,8 +481,9 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
         const int b0 = first_wave_blocks(num_tiles, m_tiles);
         const int tid = threadIdx.x - kGemmThreads;
         for (int b = 0; b < n_tiles; ++b) {
-            const bool shared_block = b < b0;
-            dequant_block_part<FM, FB>(fa, n_total, b, 0, shared_block ? 2 : 1, tid, 32 * kDequantWarps, 1, keep_pol,
+            // first-wave blocks: the epilogue warps take their share (by warp count)
+            const int parts = b < b0 ? kDequantWarps + kEpiWarps : kDequantWarps;
+            dequant_block_part<FM, FB>(fa, n_total, b, 0, kDequantWarps, parts, tid, 32 * kDequantWarps, 1, keep_pol,
                                        cb_smem);
         }
     }
