@@ -84,16 +84,9 @@ aqlm_status aqlm_gemv(const void *codes, const uint16_t *codebooks, const uint16
                                        to_cuda(stream)));
 }
 
-// aqlm_gemm workspace: [status word, padded to 256 B][one arrival counter per
-// block of 256 rows, padded to 256 B][W^: d_out x d_in bf16]
-size_t gemm_counter_bytes(const aqlm_shape &shape) {
-    const size_t blocks = ((size_t)shape.d_out + 255) / 256;
-    return (blocks * 4 + 255) / 256 * 256;
-}
-
 size_t aqlm_gemm_workspace_bytes(aqlm_shape shape, int32_t tokens) {
     if (check_shape(shape) != AQLM_OK || tokens < 1) return 0;
-    return kStatusBytes + gemm_counter_bytes(shape) + (size_t)shape.d_out * shape.d_in * 2;
+    return kStatusBytes + (size_t)shape.d_out * shape.d_in * 2;
 }
 
 aqlm_status aqlm_gemm(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *X,
@@ -107,14 +100,13 @@ aqlm_status aqlm_gemm(const void *codes, const uint16_t *codebooks, const uint16
     const size_t need = aqlm_gemm_workspace_bytes(shape, tokens);
     if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return AQLM_ERR_WORKSPACE;
     const cudaStream_t cs = to_cuda(stream);
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    int32_t *status = reinterpret_cast<int32_t *>(ws);
-    uint32_t *ready = reinterpret_cast<uint32_t *>(ws + kStatusBytes);
-    const size_t counters = gemm_counter_bytes(shape);
-    uint16_t *W = reinterpret_cast<uint16_t *>(ws + kStatusBytes + counters);
-    if (cudaMemsetAsync(ws, 0, kStatusBytes + counters, cs) != cudaSuccess) return AQLM_ERR_CUDA;
-    return from_cuda(aqlm::launch_fused_gemm(codes, codebooks, scales, X, W, Y, tokens, aqlm::make_dims(shape), status,
-                                             ready, cs));
+    int32_t *status = static_cast<int32_t *>(workspace);
+    uint16_t *W = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(workspace) + kStatusBytes);
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), cs);
+    if (e != cudaSuccess) return AQLM_ERR_CUDA;
+    e = aqlm::launch_dequant(codes, codebooks, scales, W, aqlm::make_dims(shape), cs);
+    if (e != cudaSuccess) return AQLM_ERR_CUDA;
+    return from_cuda(aqlm::launch_bf16_gemm(X, W, Y, tokens, shape.d_out, shape.d_in, status, cs));
 }
 
 aqlm_status aqlm_gemm_check(void *workspace, size_t workspace_bytes, aqlm_stream_t stream) {

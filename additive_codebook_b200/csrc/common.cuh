@@ -132,7 +132,4 @@ cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint
                         cudaStream_t st);
 cudaError_t launch_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                              int32_t *status, cudaStream_t st);
-cudaError_t launch_fused_gemm(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *X,
-                              uint16_t *W, uint16_t *Y, int tokens, const Dims &d, int32_t *status, uint32_t *ready,
-                              cudaStream_t st);
 }  // namespace aqlm

@@ -53,7 +53,6 @@ struct Bars {
     int abort_flag;
 };
 constexpr size_t kGemmSmem = 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + sizeof(Bars);
-// (the fused 2x8 kernel adds 16 bytes of alignment and its 8 KiB of codebooks)
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -144,124 +143,10 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// ---- fused dequantisation (aqlm_gemm) ----
-// Twelve extra warps per CTA decode W^ (the same binary32 steps as
-// aqlm_dequant) block of 256 rows by block, in the order the tile schedule
-// consumes them; every CTA takes one slice of every block.  A CTA publishes
-// its slice through the block's arrival counter (release); the TMA producer
-// waits (acquire, bounded) until all slices of its tile's block have arrived,
-// then orders its tensor-memory-access loads after them with a proxy fence.
-// The blocks of the first wave of tiles are decoded by the epilogue warps as
-// well (they are idle until the first accumulator is ready).
-constexpr int kDequantWarps = 12;
-constexpr int kFusedThreads = kGemmThreads + 32 * kDequantWarps;
-
-struct FuseArgs {
-    const uint8_t *codes;
-    const uint4 *codebooks;
-    const __half *scales;
-    uint4 *W;            // W^ as 8 bf16 per group, [d_out][G]
-    uint32_t *ready;     // per block of 256 rows: arrivals of decoded slices
-    int G;               // groups per row
-};
-
-__device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Groups [lo, hi) of W^ (flattened [d_out][G] order), nthreads threads, four
-// groups per thread in flight.
-template <int M, int B>
-__device__ void dequant_groups(const FuseArgs &fa, int64_t lo, int64_t hi, int tid, int nthreads, uint64_t keep,
-                               const uint4 *cb_smem) {
-    constexpr int K = 1 << B;
-    constexpr int kCodeBytes = M * B / 8;
-    for (int64_t g = lo + tid; g < hi; g += 4 * (int64_t)nthreads) {
-        uint32_t raw[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int64_t gi = g + (int64_t)i * nthreads;
-            raw[i] = 0;
-            if (gi < hi) {
-                if constexpr (kCodeBytes == 2) {
-                    raw[i] = __ldcs(reinterpret_cast<const uint16_t *>(fa.codes) + gi);
-                } else {
-                    raw[i] = __ldcs(reinterpret_cast<const uint32_t *>(fa.codes) + gi);
-                }
-            }
-        }
-        uint4 cw[4][M];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-#pragma unroll
-            for (int m = 0; m < M; ++m) {
-                uint32_t k;
-                if constexpr (M == 1) k = raw[i] & 0xffffu;
-                else if constexpr (B == 8) k = (raw[i] >> (8 * m)) & 0xffu;
-                else k = (raw[i] >> (16 * m)) & 0xffffu;
-                cw[i][m] = (B == 8) ? cb_smem[m * K + k] : ld_keep_u4(fa.codebooks + (size_t)m * K + k, keep);
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int64_t gi = g + (int64_t)i * nthreads;
-            if (gi >= hi) break;
-            const float s = __half2float(fa.scales[gi / fa.G]);
-            float acc[kGroup];
-            half8_to_float8(cw[i][0], acc);
-#pragma unroll
-            for (int m = 1; m < M; ++m) {
-                float f[kGroup];
-                half8_to_float8(cw[i][m], f);
-#pragma unroll
-                for (int t = 0; t < kGroup; ++t) acc[t] = __fadd_rn(acc[t], f[t]);
-            }
-            uint32_t out[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                const __nv_bfloat16 lo2 = __float2bfloat16_rn(__fmul_rn(acc[2 * h], s));
-                const __nv_bfloat16 hi2 = __float2bfloat16_rn(__fmul_rn(acc[2 * h + 1], s));
-                out[h] = (uint32_t)__bfloat16_as_ushort(lo2) | ((uint32_t)__bfloat16_as_ushort(hi2) << 16);
-            }
-            fa.W[gi] = make_uint4(out[0], out[1], out[2], out[3]);
-        }
-    }
-}
-
-// Decode parts [p_lo, p_hi) of `parts` of this CTA's slice of block b, then
-// publish them.
-template <int M, int B>
-__device__ void dequant_block_part(const FuseArgs &fa, int n_total, int b, int p_lo, int p_hi, int parts, int tid,
-                                   int nthreads, int bar_id, uint64_t keep, const uint4 *cb_smem) {
-    const int64_t row0 = (int64_t)b * BN;
-    const int64_t rows = min((int64_t)BN, (int64_t)n_total - row0);
-    const int64_t base = row0 * fa.G, total = rows * fa.G;
-    const int64_t s_lo = base + total * blockIdx.x / gridDim.x;
-    const int64_t s_hi = base + total * (blockIdx.x + 1) / gridDim.x;
-    const int64_t lo = s_lo + (s_hi - s_lo) * p_lo / parts;
-    const int64_t hi = s_lo + (s_hi - s_lo) * p_hi / parts;
-    dequant_groups<M, B>(fa, lo, hi, tid, nthreads, keep, cb_smem);
-    __threadfence();
-    asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(nthreads) : "memory");
-    if (tid == 0) {
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        atomicAdd(&fa.ready[b], 1u);
-    }
-}
-
-// Blocks of 256 rows touched by the first wave of tiles (one tile per CTA).
-__device__ __forceinline__ int first_wave_blocks(int num_tiles, int m_tiles) {
-    const int first = num_tiles < (int)gridDim.x ? num_tiles : (int)gridDim.x;
-    return (first + m_tiles - 1) / m_tiles;
-}
-
-template <int FM, int FB>
-__global__ void __launch_bounds__(FM ? kFusedThreads : kGemmThreads, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                   __nv_bfloat16 *__restrict__ Y, int m_total, int n_total, int k_total, int32_t *status,
-                  unsigned long long limit_ns, int stall_test, const FuseArgs fa) {
+                  unsigned long long limit_ns, int stall_test) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled tiles.
     const uint32_t raw = smem_addr(smem_raw);
@@ -273,22 +158,6 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
     const int n_tiles = (n_total + BN - 1) / BN;
     const int num_tiles = m_tiles * n_tiles;
     const int num_kb = (k_total + BK - 1) / BK;
-
-    uint4 *cb_smem = reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(bars) + ((sizeof(Bars) + 15) & ~size_t(15)));
-    const uint64_t keep_pol = policy_evict_last();
-    if constexpr (FM == 2 && FB == 8) {
-        for (int c = threadIdx.x; c < 512; c += blockDim.x) cb_smem[c] = fa.codebooks[c];
-    }
-    if constexpr (FM != 0 && FB == 16) {
-        if (threadIdx.x == 0) {  // this CTA's share of the (usually cold) codebooks into L2
-            const uint32_t cb_bytes = (uint32_t)FM * 65536u * 16u;
-            const uint32_t share = ((cb_bytes + gridDim.x - 1) / gridDim.x + 255) & ~255u;
-            const uint32_t off = blockIdx.x * share;
-            if (off < cb_bytes)
-                prefetch_l2_bulk(reinterpret_cast<const uint8_t *>(fa.codebooks) + off, min(share, cb_bytes - off),
-                                 keep_pol);
-        }
-    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -324,29 +193,8 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
             int issued_parity[STAGES];
             for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
             bool ok = true;
-            const int b0 = first_wave_blocks(num_tiles, m_tiles);
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 const int mb = tile % m_tiles, nb = tile / m_tiles;
-                if constexpr (FM != 0) {
-                    // every slice of this tile's block of W^ must be decoded first
-                    const uint32_t need = (uint32_t)gridDim.x * (nb < b0 ? 2u : 1u);
-                    const uint64_t t0 = now_ns();
-                    while (ld_acquire(&fa.ready[nb]) < need) {
-                        if (*reinterpret_cast<volatile int *>(&bars->abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        if (now_ns() - t0 > limit_ns) {
-                            *reinterpret_cast<volatile int *>(&bars->abort_flag) = 1;
-                            atomicExch(status, (int32_t)AQLM_ERR_TIMEOUT);
-                            ok = false;
-                            break;
-                        }
-                        __nanosleep(128);
-                    }
-                    if (!ok) break;
-                    asm volatile("fence.proxy.async.global;" ::: "memory");
-                }
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!wait_bounded(smem_addr(&bars->empty[stage]), phase ^ 1, bars, status, limit_ns)) {
                         ok = false;
@@ -424,15 +272,7 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
             }
         }
         __syncwarp();
-    } else if (warp < 2 + kEpiWarps) {
-        if constexpr (FM != 0) {
-            // idle until the first accumulator: help decode the first wave's blocks
-            const int b0 = first_wave_blocks(num_tiles, m_tiles);
-            for (int b = 0; b < b0; ++b)
-                dequant_block_part<FM, FB>(fa, n_total, b, kDequantWarps, kDequantWarps + kEpiWarps,
-                                           kDequantWarps + kEpiWarps, threadIdx.x - 64, 32 * kEpiWarps, 2, keep_pol,
-                                           cb_smem);
-        }
+    } else {
         // ---- epilogue: warps 2..5, TMEM lane quarter = warp % 4 ----
         const int quarter = warp & 3;
         const int row_in_tile = quarter * 32 + lane;
@@ -475,16 +315,6 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
                 acc = 0;
                 acc_phase ^= 1;
             }
-        }
-    } else if constexpr (FM != 0) {
-        // ---- dequantisation warps 6..9: every block of W^, in schedule order ----
-        const int b0 = first_wave_blocks(num_tiles, m_tiles);
-        const int tid = threadIdx.x - kGemmThreads;
-        for (int b = 0; b < n_tiles; ++b) {
-            // first-wave blocks: the epilogue warps take their share (by warp count)
-            const int parts = b < b0 ? kDequantWarps + kEpiWarps : kDequantWarps;
-            dequant_block_part<FM, FB>(fa, n_total, b, 0, kDequantWarps, parts, tid, 32 * kDequantWarps, 1, keep_pol,
-                                       cb_smem);
         }
     }
 
@@ -536,71 +366,21 @@ cudaError_t launch_bf16_gemm_ex(const uint16_t *X, const uint16_t *W, uint16_t *
                                 int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test) {
     CUtensorMap mx, mw;
     if (!make_map(&mx, X, tokens, k, BM) || !make_map(&mw, W, n, k, BN)) return cudaErrorInvalidValue;
-    auto kern = gemm_bf16_tcgen05<0, 0>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
+    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kGemmSmem);
     if (e != cudaSuccess) return e;
     int dev = 0;
     cudaGetDevice(&dev);
     const int tiles = ((tokens + BM - 1) / BM) * ((n + BN - 1) / BN);
     const int sms = num_sms(dev);
     const int grid = tiles < sms ? tiles : sms;
-    FuseArgs none = {};
-    return launch_kernel(kern, dim3(grid), dim3(kGemmThreads), kGemmSmem, st, false, mx, mw,
-                         reinterpret_cast<__nv_bfloat16 *>(Y), tokens, n, k, status, limit_ns, stall_test, none);
+    return launch_kernel(gemm_bf16_tcgen05, dim3(grid), dim3(kGemmThreads), kGemmSmem, st, false, mx, mw,
+                         reinterpret_cast<__nv_bfloat16 *>(Y), tokens, n, k, status, limit_ns, stall_test);
 }
 
 cudaError_t launch_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                              int32_t *status, cudaStream_t st) {
     return launch_bf16_gemm_ex(X, W, Y, tokens, n, k, status, st, kWaitLimitNs, 0);
-}
-
-// Prefill with the dequantisation fused into the GEMM: W (the workspace's
-// W^ region) is written by the kernel's own dequantisation warps and read by
-// its TMA loads.  `ready` holds one zeroed counter per block of 256 rows.
-// Cooperative launch: every CTA is resident at once, which the producer's
-// wait on other CTAs' slices relies on.
-cudaError_t launch_fused_gemm(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *X,
-                              uint16_t *W, uint16_t *Y, int tokens, const Dims &d, int32_t *status, uint32_t *ready,
-                              cudaStream_t st) {
-    CUtensorMap mx, mw;
-    if (!make_map(&mx, X, tokens, d.d_in, BM) || !make_map(&mw, W, d.d_out, d.d_in, BN)) return cudaErrorInvalidValue;
-    void (*kern)(const CUtensorMap, const CUtensorMap, __nv_bfloat16 *, int, int, int, int32_t *, unsigned long long,
-                 int, const FuseArgs);
-    size_t smem = kGemmSmem + 16;
-    if (d.M == 1) {
-        kern = gemm_bf16_tcgen05<1, 16>;
-    } else if (d.B == 8) {
-        kern = gemm_bf16_tcgen05<2, 8>;
-        smem += 8192;
-    } else {
-        kern = gemm_bf16_tcgen05<2, 16>;
-    }
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const int tiles = ((tokens + BM - 1) / BM) * ((d.d_out + BN - 1) / BN);
-    const int sms = num_sms(dev);
-    const int grid = tiles < sms ? tiles : sms;
-    FuseArgs fa;
-    fa.codes = static_cast<const uint8_t *>(codes);
-    fa.codebooks = reinterpret_cast<const uint4 *>(codebooks);
-    fa.scales = reinterpret_cast<const __half *>(scales);
-    fa.W = reinterpret_cast<uint4 *>(W);
-    fa.ready = ready;
-    fa.G = d.G;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kFusedThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, mx, mw, reinterpret_cast<__nv_bfloat16 *>(Y), tokens, d.d_out, d.d_in,
-                              status, kWaitLimitNs, 0, fa);
 }
 
 }  // namespace aqlm

@@ -132,16 +132,12 @@ AQLM_API aqlm_status aqlm_dequant(const void *codes, const uint16_t *codebooks, 
                          uint16_t *W_out, aqlm_shape shape, aqlm_stream_t stream);
 
 /*
- * aqlm_gemm -- prefill product Y = X . W^T for many tokens: one kernel that
- * dequantises W^ to bf16 (exactly as aqlm_dequant) into the workspace with
- * some of its warps while the others run a tcgen05 tensor-core GEMM over the
- * blocks already decoded (bf16 operands, fp32 accumulation in tensor memory,
- * bf16 output rounded to nearest even).
+ * aqlm_gemm -- prefill product Y = X . W^T for many tokens: aqlm_dequant into
+ * the workspace, then a tcgen05 tensor-core GEMM (bf16 operands, fp32
+ * accumulation in tensor memory, bf16 output rounded to nearest even).
  *   X: [tokens][d_in] bf16.  Y: [tokens][d_out] bf16 (written).  tokens >= 1.
  *   workspace: at least aqlm_gemm_workspace_bytes(shape, tokens) bytes,
- *   16-byte aligned; it holds a status word, one counter per block of 256
- *   rows and the dequantised weight.  Launched cooperatively (all CTAs
- *   resident at once).
+ *   16-byte aligned; it holds the dequantised weight and a status word.
  *   Every device-side wait of the GEMM is bounded; a wait that gives up
  *   records AQLM_ERR_TIMEOUT in the workspace's status word (read it with
  *   aqlm_gemm_check) and the kernel returns without trapping.
