@@ -168,17 +168,37 @@ cudaError_t launch_decode_indices(const void *codes, uint16_t *idx, const Dims &
     return launch_kernel(decode_indices_kernel<16>, grid, 256, 0, st, false, codes, idx, n);
 }
 
+// One wave: as many CTAs as the SMs hold at once (by the kernel's register
+// use), so every warp's tiles flow through its software pipeline without a
+// second wave of CTAs waiting behind the first.
+template <typename Kern>
+int one_wave_grid(Kern kern, int64_t n_groups) {
+    int dev = 0, occ = 0;
+    cudaGetDevice(&dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 256, 0) != cudaSuccess || occ < 1) occ = 1;
+    const int64_t tiles = (n_groups + kTile - 1) / kTile;
+    const int64_t want = (tiles + 7) / 8;  // 8 warps per CTA
+    const int64_t cap = (int64_t)num_sms(dev) * occ;
+    return (int)(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
 cudaError_t launch_dequant(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                            uint16_t *W, const Dims &d, cudaStream_t st) {
     const int64_t n = (int64_t)d.d_out * d.G;
-    const int grid = grid_for((n + kPerLane - 1) / kPerLane, 256, 4);
     auto c = static_cast<const uint8_t *>(codes);
     auto cb = reinterpret_cast<const uint4 *>(codebooks);
     auto s = reinterpret_cast<const __half *>(scales);
     auto w = reinterpret_cast<uint4 *>(W);
-    if (d.M == 1 && d.B == 16) return launch_kernel(dequant_kernel<1, 16>, grid, 256, 0, st, false, c, cb, s, w, d.G, n);
-    if (d.M == 2 && d.B == 8) return launch_kernel(dequant_kernel<2, 8>, grid, 256, 0, st, false, c, cb, s, w, d.G, n);
-    return launch_kernel(dequant_kernel<2, 16>, grid, 256, 0, st, false, c, cb, s, w, d.G, n);
+    if (d.M == 1 && d.B == 16) {
+        auto k = dequant_kernel<1, 16>;
+        return launch_kernel(k, one_wave_grid(k, n), 256, 0, st, false, c, cb, s, w, d.G, n);
+    }
+    if (d.M == 2 && d.B == 8) {
+        auto k = dequant_kernel<2, 8>;
+        return launch_kernel(k, one_wave_grid(k, n), 256, 0, st, false, c, cb, s, w, d.G, n);
+    }
+    auto k = dequant_kernel<2, 16>;
+    return launch_kernel(k, one_wave_grid(k, n), 256, 0, st, false, c, cb, s, w, d.G, n);
 }
 
 }  // namespace aqlm
