@@ -78,15 +78,6 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes, 
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
 
-// 16-byte asynchronous global -> shared copy (cp.async, L2 only).
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-                 "l"(src)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
 // Eight fp16 values packed in a uint4 -> eight floats (exact conversion).
 __device__ __forceinline__ void half8_to_float8(const uint4 &v, float *f) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};

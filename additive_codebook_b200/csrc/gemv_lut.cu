@@ -51,13 +51,13 @@ struct LutArgs {
 
 __device__ __forceinline__ void gd_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // 16-byte asynchronous global -> shared copy; src_bytes = 0 writes zeros.
-__device__ __forceinline__ void cp_async16_zfill(void *dst, const void *src, uint32_t src_bytes) {
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
                      static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
                  "l"(src), "r"(src_bytes)
                  : "memory");
 }
-__device__ __forceinline__ void lut_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void gd_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
@@ -65,7 +65,7 @@ __device__ __forceinline__ void gd_launch() { asm volatile("griddepcontrol.launc
 __global__ void __launch_bounds__(kLutThreads) gemv_lut_2x8_kernel(const LutArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     float *lut = reinterpret_cast<float *>(smem);               // [2][256][32]
-    float *cbf = lut + 2 * 256 * kSlab;                          // codebooks, fp16 [2][256][8]
+    float *cbf = lut + 2 * 256 * kSlab;                          // [2][256][8]
     uint4 *ring = reinterpret_cast<uint4 *>(cbf + 2 * 256 * 8);  // [warps][stages][32] uint4
     __shared__ int s_last;
 
@@ -86,20 +86,23 @@ __global__ void __launch_bounds__(kLutThreads) gemv_lut_2x8_kernel(const LutArgs
         const int r = row_begin + (batch * kLutWarps + warp) * kRowsPerBatch + piece_row;
         const bool ok = r < row_end && piece_in_row;
         const uint8_t *src = ok ? a.codes + (size_t)r * a.row_bytes + (size_t)piece_group * 2 : a.codes;
-        cp_async16_zfill(wring + slot * 32 + lane, src, ok ? 16u : 0u);
-        lut_cp_commit();
+        cp_async16(wring + slot * 32 + lane, src, ok ? 16u : 0u);
+        cp_async_commit();
     };
     const int rows = row_end - row_begin;
     const int n_batches = (rows + kLutWarps * kRowsPerBatch - 1) / (kLutWarps * kRowsPerBatch);
     // codes are constant weights: fill the ring before waiting on x's producer
-    // the two codebooks (constant weights, 8 KiB of fp16) as their own group
-    // of asynchronous copies, committed before the ring's groups
-    uint4 *cbh = reinterpret_cast<uint4 *>(cbf);
-    for (int i = threadIdx.x; i < 2 * 256; i += kLutThreads)
-        cp_async16_zfill(cbh + i, reinterpret_cast<const uint4 *>(a.codebooks) + i, 16u);
-    lut_cp_commit();
 #pragma unroll
     for (int b = 0; b < kStages; ++b) issue(b, b);
+
+    // codebooks (constant weights) -> fp32 in shared memory
+    for (int i = threadIdx.x; i < 2 * 256; i += kLutThreads) {
+        float f[8];
+        half8_to_float8(reinterpret_cast<const uint4 *>(a.codebooks)[i], f);
+        float4 *dst = reinterpret_cast<float4 *>(cbf + i * 8);
+        dst[0] = make_float4(f[0], f[1], f[2], f[3]);
+        dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
 
     gd_wait();
     // this lane's activation group (zeros past the end of the row)
@@ -110,20 +113,19 @@ __global__ void __launch_bounds__(kLutThreads) gemv_lut_2x8_kernel(const LutArgs
 #pragma unroll
         for (int e = 0; e < 8; ++e) xv[e] = 0.f;
     }
-    cp_async_wait<kStages>();  // the codebooks' group has landed (the ring's may not have)
     __syncthreads();
     // L_m[j0 + lane][k] for the (m, k) pairs of this warp
     for (int p = warp; p < 2 * 256; p += kLutWarps) {
-        float c[8];
-        half8_to_float8(cbh[p], c);
-        float d = c[0] * xv[0];
-        d = fmaf(c[1], xv[1], d);
-        d = fmaf(c[2], xv[2], d);
-        d = fmaf(c[3], xv[3], d);
-        d = fmaf(c[4], xv[4], d);
-        d = fmaf(c[5], xv[5], d);
-        d = fmaf(c[6], xv[6], d);
-        d = fmaf(c[7], xv[7], d);
+        const float4 c0 = reinterpret_cast<const float4 *>(cbf + p * 8)[0];
+        const float4 c1 = reinterpret_cast<const float4 *>(cbf + p * 8)[1];
+        float d = c0.x * xv[0];
+        d = fmaf(c0.y, xv[1], d);
+        d = fmaf(c0.z, xv[2], d);
+        d = fmaf(c0.w, xv[3], d);
+        d = fmaf(c1.x, xv[4], d);
+        d = fmaf(c1.y, xv[5], d);
+        d = fmaf(c1.z, xv[6], d);
+        d = fmaf(c1.w, xv[7], d);
         lut[p * kSlab + lane] = d;
     }
     __syncthreads();

@@ -22,9 +22,8 @@
 //     item k+2 and the codeword gathers of item k+1 are in flight while item
 //     k is multiplied; it runs across row boundaries.
 //   - Programmatic dependent launch: codebooks are prefetched into L2 and
-//     the first items' codes requested before griddepcontrol.wait (weights
-//     are constant); x is copied asynchronously right after it, before the
-//     first gathers wait for their codes; y is written only after the wait.
+//     the first items' codes and codewords fetched before griddepcontrol.wait
+//     (weights are constant); x is read and y written only after it.
 #include "common.cuh"
 
 namespace aqlm {
@@ -117,19 +116,14 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
     uint4 cwA[GPC][M], cwB[GPC][M];
     uint4 ch_next = load_code(1);
     {
-        // The code loads are issued before the wait; x is copied asynchronously
-        // (cp.async) right after it, and only then does the first gather wait
-        // for its codes, so the latencies of the codes and of x overlap.
         const uint4 ch0 = load_code(0);
+        if constexpr (!F::kSmemCodebook) gather(ch0, 0, cwA);
         grid_dep_wait();
         for (int i = threadIdx.x; i < T * a.G; i += kRowThreads) {  // stage x, transposed by chunk
             const int t = i / a.G, g = i - t * a.G;
             const int c = g / GPC, q = g - c * GPC;
-            cp_async16(xs + ((size_t)t * GPC + q) * n_chunks + c, a.x + (size_t)i * kGroup);
+            xs[((size_t)t * GPC + q) * n_chunks + c] = *reinterpret_cast<const uint4 *>(a.x + (size_t)i * kGroup);
         }
-        cp_async_commit();
-        if constexpr (!F::kSmemCodebook) gather(ch0, 0, cwA);
-        cp_async_wait_all();
         __syncthreads();
         if constexpr (F::kSmemCodebook) gather(ch0, 0, cwA);
     }
