@@ -18,14 +18,12 @@
 //   - Activations are staged once per CTA in shared memory as fp16,
 //     transposed by chunk ([group within chunk][chunk]) so that the lanes of
 //     a warp, which work on consecutive chunks, read consecutive 16 bytes.
-//   - Software pipeline over the warp's (row, chunk) items: the codeword
-//     gathers of item k+1 and the code loads of items k+2, k+3 are in flight
-//     while item k is multiplied; it runs across row boundaries.
+//   - Software pipeline over the warp's (row, chunk) items: the code load of
+//     item k+2 and the codeword gathers of item k+1 are in flight while item
+//     k is multiplied; it runs across row boundaries.
 //   - Programmatic dependent launch: codebooks are prefetched into L2 and
-//     the codes of the first four items and the codewords of the first two
-//     fetched before griddepcontrol.wait (weights are constant), so in a
-//     chain of layers they overlap the previous kernel; x is read and y
-//     written only after it.
+//     the first items' codes and codewords fetched before griddepcontrol.wait
+//     (weights are constant); x is read and y written only after it.
 #include "common.cuh"
 
 namespace aqlm {
@@ -116,15 +114,10 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
     };
 
     uint4 cwA[GPC][M], cwB[GPC][M];
-    // Weights are constant: the codes of items 0..3 and the codewords of items
-    // 0 and 1 are requested before waiting on the kernel that produces x.
-    uint4 ch_a = load_code(2), ch_b = load_code(3);
+    uint4 ch_next = load_code(1);
     {
-        const uint4 ch0 = load_code(0), ch1 = load_code(1);
-        if constexpr (!F::kSmemCodebook) {
-            gather(ch0, 0, cwA);
-            gather(ch1, 1, cwB);
-        }
+        const uint4 ch0 = load_code(0);
+        if constexpr (!F::kSmemCodebook) gather(ch0, 0, cwA);
         grid_dep_wait();
         for (int i = threadIdx.x; i < T * a.G; i += kRowThreads) {  // stage x, transposed by chunk
             const int t = i / a.G, g = i - t * a.G;
@@ -132,10 +125,7 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
             xs[((size_t)t * GPC + q) * n_chunks + c] = *reinterpret_cast<const uint4 *>(a.x + (size_t)i * kGroup);
         }
         __syncthreads();
-        if constexpr (F::kSmemCodebook) {
-            gather(ch0, 0, cwA);
-            gather(ch1, 1, cwB);
-        }
+        if constexpr (F::kSmemCodebook) gather(ch0, 0, cwA);
     }
     grid_dep_launch();
 
@@ -183,19 +173,17 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
         }
     };
 
-    // at the top of a trip: cwA / cwB hold (or are fetching) the codewords of
-    // items k / k+1, ch_a / ch_b the codes of items k+2 / k+3; while one item
-    // is multiplied the next one's codewords are in flight
+    // at the top of a trip: cwA holds item k's codewords, ch_next item k+1's codes
     for (int k = 0; item_row(k) < a.d_out; k += 2) {
+        gather(ch_next, k + 1, cwB);
+        ch_next = load_code(k + 2);
         multiply(cwA, k);
         finish_item(k);
-        gather(ch_a, k + 2, cwA);
-        ch_a = load_code(k + 4);
         if (item_row(k + 1) >= a.d_out) break;
+        gather(ch_next, k + 2, cwA);
+        ch_next = load_code(k + 3);
         multiply(cwB, k + 1);
         finish_item(k + 1);
-        gather(ch_b, k + 3, cwB);
-        ch_b = load_code(k + 5);
     }
 }
 
