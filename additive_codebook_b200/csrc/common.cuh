@@ -90,6 +90,15 @@ __device__ __forceinline__ void half8_to_float8(const uint4 &v, float *f) {
     }
 }
 
+// The kernels here hold at most a few bytes of static shared memory; opt in
+// to the dynamic size whenever static + dynamic could pass the 48 KiB that a
+// launch gets without the attribute.
+template <typename... KArgs>
+cudaError_t opt_in_dynamic_smem(void (*kern)(KArgs...), size_t bytes) {
+    if (bytes + 1024 <= 48 * 1024) return cudaSuccess;
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
 // Launch through cudaLaunchKernelEx so that the returned error belongs to this
 // launch only.  `pdl` allows programmatic dependent launch: the kernel may
 // start while the previous kernel in the stream finishes, and must execute

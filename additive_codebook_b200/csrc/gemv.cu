@@ -1,19 +1,21 @@
 // gemv.cu -- host side of the decode-time product: kernel choice, work plan,
 // workspace layout and the launch (with programmatic dependent launch).
-// One token: gemv_rows.cu (coalesced row streaming); the 2x8 lookup-table
-// kernel in gemv_lut.cu is its alternative for 2x8.  Several tokens (and
-// one token with activations too large for shared memory): the gather
-// kernels of gemv_kernels.cuh, instantiated per format in gemv_1x16.cu,
-// gemv_2x8.cu and gemv_2x16.cu.
+// 1..4 tokens: gemv_rows.cu (coalesced row streaming, the input range split
+// when the activations do not fit on chip); for one token of 2x8 the
+// lookup-table kernel of gemv_lut.cu.  5..16 tokens: the several-rows-per-lane
+// kernel of gemv_multi.cuh, instantiated per format in gemv_multi_1x16.cu,
+// gemv_multi_2x8.cu and gemv_multi_2x16.cu.
 #include "gemv_multi.cuh"
 
 namespace aqlm {
 
 size_t gemv_lut_workspace_bytes(const Dims &d, int sms);
 size_t gemv_lut_workspace_counter_offset(const Dims &d, int sms);
-bool gemv_rows_supported(const Dims &d, int T);
+bool gemv_rows_supported(int T);
+size_t gemv_rows_workspace_bytes(const Dims &d, int T, int sms);
+size_t gemv_rows_counter_offset(const Dims &d, int T, int sms);
 cudaError_t launch_gemv_rows(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
-                             uint16_t *y, int tokens, const Dims &d, int sms, cudaStream_t st);
+                             uint16_t *y, int tokens, const Dims &d, void *workspace, int sms, cudaStream_t st);
 cudaError_t launch_gemv_lut_2x8(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                                 const uint16_t *x, uint16_t *y, const Dims &d, void *workspace, int sms,
                                 cudaStream_t st);
@@ -30,40 +32,10 @@ struct Plan {
 
 inline size_t align16(size_t v) { return (v + 15) / 16 * 16; }
 
-// Split the input range when (a) T activations of the whole row exceed the
-// on-chip budget, or (b) there are too few row tiles to give every SM two
-// CTAs; never below one chunk per warp.
-Plan plan_gemv(const Dims &d, int T, int sms) {
-    const int gpc = 16 / (d.M * d.B / 8);
-    const int n_chunks = d.G / gpc;
-    Plan p;
-    p.tiles = (d.d_out + kRowsPerCta - 1) / kRowsPerCta;
-    const int tp = (T == 1) ? 1 : ((T + 3) & ~3);  // tokens padded in shared memory
-    int max_chunks = kXsBudget / (tp * gpc * kGroup * 4);
-    if (max_chunks < 1) max_chunks = 1;
-    const int ks_min = (n_chunks + max_chunks - 1) / max_chunks;
-    int ks_par = (2 * sms) / p.tiles;
-    if (ks_par < 1) ks_par = 1;
-    int ks_cap = n_chunks / kWarps;
-    if (ks_cap < 1) ks_cap = 1;
-    int ks = ks_par < ks_cap ? ks_par : ks_cap;
-    if (ks < ks_min) ks = ks_min;
-    p.chunks_per_split = (n_chunks + ks - 1) / ks;
-    p.splits = (n_chunks + p.chunks_per_split - 1) / p.chunks_per_split;
-    p.smem = (size_t)tp * p.chunks_per_split * gpc * kGroup * 4 + (size_t)kWarps * T * 32 * 4;
-    return p;
-}
-
-Plan plan_multi(const Dims &d, int T, int sms);
-
-size_t gather_workspace_bytes(const Dims &d, int T, int sms) {
-    const Plan p = T > 1 ? plan_multi(d, T, sms) : plan_gemv(d, T, sms);
-    if (p.splits == 1) return 0;
-    return align16((size_t)p.splits * T * d.d_out * sizeof(float)) + (size_t)p.tiles * sizeof(uint32_t);
-}
-
-// Several tokens: tiles of 32*R rows, the same split rules with the fp16
-// token-interleaved activation budget and about three CTAs per SM.
+// Several tokens: tiles of 32*R rows.  The input range is split over
+// gridDim.y CTAs when (a) T activations of the whole row exceed the on-chip
+// budget, or (b) there are too few row tiles to give every SM three CTAs;
+// never below one chunk per warp.
 Plan plan_multi(const Dims &d, int T, int sms) {
     const int gpc = 16 / (d.M * d.B / 8);
     const int n_chunks = d.G / gpc;
@@ -85,26 +57,22 @@ Plan plan_multi(const Dims &d, int T, int sms) {
     return p;
 }
 
+size_t multi_workspace_bytes(const Dims &d, int T, int sms) {
+    const Plan p = plan_multi(d, T, sms);
+    if (p.splits == 1) return 0;
+    return align16((size_t)p.splits * T * d.d_out * sizeof(float)) + (size_t)p.tiles * sizeof(uint32_t);
+}
+
 GemvFn pick_multi(int M, int B, int T) {
     if (M == 1) return gemv_multi_pick_1x16(T);
     if (B == 8) return gemv_multi_pick_2x8(T);
     return gemv_multi_pick_2x16(T);
 }
 
-GemvFn pick(int M, int B, int T) {
-    if (M == 1) return gemv_pick_1x16(T);
-    if (B == 8) return gemv_pick_2x8(T);
-    return gemv_pick_2x16(T);
-}
-
-// Up to four tokens: whole rows per warp with coalesced code streaming (no
-// workspace) when the activations fit on chip; for one token of 2x8 the
-// lookup-table kernel is the alternative.
-constexpr bool kPreferLut2x8 = true;
-bool use_rows(const Dims &d, int T) {
-    return gemv_rows_supported(d, T) && !(kPreferLut2x8 && T == 1 && d.M == 2 && d.B == 8);
-}
-bool use_lut(const Dims &d, int T) { return d.M == 2 && d.B == 8 && T == 1 && !use_rows(d, T); }
+// Up to four tokens: whole rows per warp with coalesced code streaming; for
+// one token of 2x8 the lookup-table kernel (measured faster on B200).
+bool use_lut(const Dims &d, int T) { return d.M == 2 && d.B == 8 && T == 1; }
+bool use_rows(const Dims &d, int T) { return gemv_rows_supported(T) && !use_lut(d, T); }
 
 int device_sms() {
     int dev = 0;
@@ -118,9 +86,9 @@ int device_sms() {
 size_t gemv_workspace_bytes(const Dims &d, int tokens) {
     using namespace gemv_detail;
     const int sms = device_sms();
-    if (use_rows(d, tokens)) return 0;
     if (use_lut(d, tokens)) return gemv_lut_workspace_bytes(d, sms);
-    return gather_workspace_bytes(d, tokens, sms);
+    if (use_rows(d, tokens)) return gemv_rows_workspace_bytes(d, tokens, sms);
+    return multi_workspace_bytes(d, tokens, sms);
 }
 
 // Offset of the arrival counters inside the workspace: the bytes from here to
@@ -128,9 +96,9 @@ size_t gemv_workspace_bytes(const Dims &d, int tokens) {
 size_t gemv_workspace_counter_offset(const Dims &d, int tokens) {
     using namespace gemv_detail;
     const int sms = device_sms();
-    if (use_rows(d, tokens)) return 0;
     if (use_lut(d, tokens)) return gemv_lut_workspace_counter_offset(d, sms);
-    const Plan p = tokens > 1 ? plan_multi(d, tokens, sms) : plan_gemv(d, tokens, sms);
+    if (use_rows(d, tokens)) return gemv_rows_counter_offset(d, tokens, sms);
+    const Plan p = plan_multi(d, tokens, sms);
     if (p.splits == 1) return 0;
     return align16((size_t)p.splits * tokens * d.d_out * sizeof(float));
 }
@@ -140,15 +108,12 @@ cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint
                         cudaStream_t st) {
     using namespace gemv_detail;
     const int sms = device_sms();
-    if (use_rows(d, tokens)) return launch_gemv_rows(codes, codebooks, scales, x, y, tokens, d, sms, st);
     if (use_lut(d, tokens)) return launch_gemv_lut_2x8(codes, codebooks, scales, x, y, d, workspace, sms, st);
-    const bool multi = tokens > 1;
-    const Plan p = multi ? plan_multi(d, tokens, sms) : plan_gemv(d, tokens, sms);
-    GemvFn fn = multi ? pick_multi(d.M, d.B, tokens) : pick(d.M, d.B, tokens);
-    if (p.smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
-        if (e != cudaSuccess) return e;
-    }
+    if (use_rows(d, tokens)) return launch_gemv_rows(codes, codebooks, scales, x, y, tokens, d, workspace, sms, st);
+    const Plan p = plan_multi(d, tokens, sms);
+    GemvFn fn = pick_multi(d.M, d.B, tokens);
+    const cudaError_t e = opt_in_dynamic_smem(fn, p.smem);
+    if (e != cudaSuccess) return e;
     GemvArgs a;
     a.codes = static_cast<const uint8_t *>(codes);
     a.codebooks = reinterpret_cast<const uint4 *>(codebooks);
@@ -164,7 +129,7 @@ cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint
     a.G = d.G;
     a.row_bytes = d.row_bytes;
     a.chunks_per_split = p.chunks_per_split;
-    return launch_kernel(fn, dim3(p.tiles, p.splits), dim3(multi ? kMultiThreads : kThreads), p.smem, st, true, a);
+    return launch_kernel(fn, dim3(p.tiles, p.splits), dim3(kMultiThreads), p.smem, st, true, a);
 }
 
 }  // namespace aqlm

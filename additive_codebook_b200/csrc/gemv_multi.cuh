@@ -1,4 +1,4 @@
-// gemv_multi.cuh -- layer product for 2..16 tokens, several rows per lane.
+// gemv_multi.cuh -- layer product for 5..16 tokens, several rows per lane.
 //
 // "The AQLM Quantization Algorithm, Explained", section "What is
 // Multi-Codebook Quantization (MCQ)?": y_i = s_i * sum_j < sum_m C_m[b(i,j,m)],
@@ -23,10 +23,65 @@
 //   - programmatic dependent launch: weights only before griddepcontrol.wait.
 #pragma once
 
-#include "gemv_kernels.cuh"
+#include <array>
+#include <utility>
+
+#include "common.cuh"
 
 namespace aqlm {
 namespace gemv_detail {
+
+// Bytes of staged activations per CTA: small, so that L1 keeps room for the
+// codeword gathers in flight (measured on B200, 24 KiB beat 64 KiB by 3-18%
+// from 8 to 16 tokens).
+constexpr int kXsBudget = 24 * 1024;
+
+template <int M, int B>
+struct Fmt {
+    static constexpr int K = 1 << B;
+    static constexpr int kCodeBytes = M * B / 8;             // per group
+    static constexpr int kGroupsPerChunk = 16 / kCodeBytes;  // per 16-byte load
+};
+
+// Index of codebook m for group q (0 <= q < groups per chunk) of a 16-byte chunk.
+template <int M, int B>
+__device__ __forceinline__ uint32_t chunk_index(const uint4 &ch, int q, int m) {
+    const uint32_t w[4] = {ch.x, ch.y, ch.z, ch.w};
+    if constexpr (M == 1 && B == 16) {
+        return (w[q >> 1] >> (16 * (q & 1))) & 0xffffu;
+    } else if constexpr (B == 8) {  // 2x8: byte 2q is codebook 0, byte 2q+1 codebook 1
+        return (w[q >> 1] >> (16 * (q & 1) + 8 * m)) & 0xffu;
+    } else {  // 2x16: word q holds codebook 0 in its low half, codebook 1 in its high half
+        return (w[q] >> (16 * m)) & 0xffffu;
+    }
+}
+
+struct GemvArgs {
+    const uint8_t *codes;
+    const uint4 *codebooks;
+    const __half *scales;
+    const __half *x;
+    __half *y;
+    float *partial;      // [splits][T][d_out] when splits > 1
+    uint32_t *counters;  // [row tiles] when splits > 1, zero between calls
+    int d_out, d_in, G, row_bytes;
+    int chunks_per_split;
+};
+
+using GemvFn = void (*)(const GemvArgs);
+
+__device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+// Two fp32 FMAs in one instruction (sm_100 packed fp32): d = a * b + c lane-wise.
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b, unsigned long long c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
 
 constexpr int kMultiWarps = 4;
 constexpr int kMultiThreads = kMultiWarps * 32;
@@ -222,12 +277,14 @@ __global__ void __launch_bounds__(kMultiThreads) gemv_multi_kernel(const GemvArg
     if (threadIdx.x == 0) a.counters[blockIdx.x] = 0u;
 }
 
+constexpr int kMultiMinTokens = 5;  // fewer tokens run on the row kernel
+
 template <int M, int B, int... Ts>
 constexpr std::array<GemvFn, sizeof...(Ts)> gemv_multi_table(std::integer_sequence<int, Ts...>) {
-    return std::array<GemvFn, sizeof...(Ts)>{{&gemv_multi_kernel<M, B, Ts + 2>...}};
+    return std::array<GemvFn, sizeof...(Ts)>{{&gemv_multi_kernel<M, B, Ts + kMultiMinTokens>...}};
 }
 
-// Kernel tables for 2..16 tokens, one per format, each in its own translation unit.
+// Kernel tables for 5..16 tokens, one per format, each in its own translation unit.
 GemvFn gemv_multi_pick_1x16(int tokens);
 GemvFn gemv_multi_pick_2x8(int tokens);
 GemvFn gemv_multi_pick_2x16(int tokens);

@@ -13,17 +13,22 @@
 // groups (1x16 / 2x16 through L1/L2 with an evict-last policy; 2x8 from
 // shared memory), multiplies them with every token's activations and keeps
 // one fp32 partial sum per token; at the end of a row five shuffles per token
-// add the 32 partials, lane 0 scales by s_i and rounds once to fp16.  No
-// split, no workspace.
+// add the 32 partials, lane 0 scales by s_i and rounds once to fp16.
 //   - Activations are staged once per CTA in shared memory as fp16,
 //     transposed by chunk ([group within chunk][chunk]) so that the lanes of
 //     a warp, which work on consecutive chunks, read consecutive 16 bytes.
 //   - Software pipeline over the warp's (row, chunk) items: the code load of
 //     item k+2 and the codeword gathers of item k+1 are in flight while item
 //     k is multiplied; it runs across row boundaries.
+//   - When T activations of the whole row do not fit the shared-memory
+//     budget, the row's chunks are split over gridDim.y CTAs (each stages only
+//     its slice of x); each writes fp32 row partials to the caller's workspace
+//     and the last CTA of a row set to arrive (an atomic counter, no waiting)
+//     adds them in split order, scales, rounds, and resets the counter.
 //   - Programmatic dependent launch: codebooks are prefetched into L2 and
 //     the first items' codes and codewords fetched before griddepcontrol.wait
-//     (weights are constant); x is read and y written only after it.
+//     (weights are constant); x is read and y, the partials and the counters
+//     are written only after it.
 #include "common.cuh"
 
 namespace aqlm {
@@ -38,7 +43,10 @@ struct RowArgs {
     const __half *scales;
     const __half *x;
     __half *y;
-    int d_out, G, row_bytes;
+    float *partial;        // [gridDim.y][T][d_out] when the input range is split
+    uint32_t *counters;    // [gridDim.x] when split; zero between calls
+    int d_out, d_in, G, row_bytes;
+    int chunks_per_split;  // 16-byte code chunks of a row per CTA
 };
 
 template <int M, int B>
@@ -65,9 +73,13 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
     using F = RowFmt<M, B>;
     constexpr int GPC = F::GPC;
     extern __shared__ __align__(16) unsigned char smem[];
-    const int n_chunks = a.G / GPC;
-    uint4 *xs = reinterpret_cast<uint4 *>(smem);  // [T][GPC][n_chunks] groups of 8 fp16
-    uint4 *cbs = xs + (size_t)T * a.G;            // 2x8: [M][256] codewords
+    __shared__ int s_last;
+    const int split = blockIdx.y, splits = gridDim.y;
+    const int xstride = a.chunks_per_split;
+    const int c0 = split * xstride;                       // first chunk of this CTA's slice
+    const int n_chunks = min(a.G / GPC - c0, xstride);    // chunks in the slice
+    uint4 *xs = reinterpret_cast<uint4 *>(smem);          // [T][GPC][xstride] groups of 8 fp16
+    uint4 *cbs = xs + (size_t)T * GPC * xstride;          // 2x8: [M][256] codewords
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int total_warps = gridDim.x * kRowWarps;
@@ -94,7 +106,8 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
     auto load_code = [&](int k) -> uint4 {
         const int r = item_row(k);
         const int c = lane + 32 * (k % cpw);
-        if (r < a.d_out && c < n_chunks) return ld_stream_u4(a.codes + (size_t)r * a.row_bytes + (size_t)c * 16, stream_pol);
+        if (r < a.d_out && c < n_chunks)
+            return ld_stream_u4(a.codes + (size_t)r * a.row_bytes + (size_t)(c0 + c) * 16, stream_pol);
         return make_uint4(0, 0, 0, 0);
     };
     auto gather = [&](const uint4 &ch, int k, uint4 (&cw)[GPC][M]) {
@@ -119,10 +132,12 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
         const uint4 ch0 = load_code(0);
         if constexpr (!F::kSmemCodebook) gather(ch0, 0, cwA);
         grid_dep_wait();
-        for (int i = threadIdx.x; i < T * a.G; i += kRowThreads) {  // stage x, transposed by chunk
-            const int t = i / a.G, g = i - t * a.G;
+        const int ng = n_chunks * GPC;  // groups of the slice
+        for (int i = threadIdx.x; i < T * ng; i += kRowThreads) {  // stage x, transposed by chunk
+            const int t = i / ng, g = i - t * ng;
             const int c = g / GPC, q = g - c * GPC;
-            xs[((size_t)t * GPC + q) * n_chunks + c] = *reinterpret_cast<const uint4 *>(a.x + (size_t)i * kGroup);
+            xs[((size_t)t * GPC + q) * xstride + c] =
+                *reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.d_in + (size_t)(c0 * GPC + g) * kGroup);
         }
         __syncthreads();
         if constexpr (F::kSmemCodebook) gather(ch0, 0, cwA);
@@ -141,7 +156,13 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
             float v = acc[t];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0 && r < a.d_out) a.y[(size_t)t * a.d_out + r] = __float2half_rn(v * __half2float(a.scales[r]));
+            if (lane == 0 && r < a.d_out) {
+                if (splits == 1) {
+                    a.y[(size_t)t * a.d_out + r] = __float2half_rn(v * __half2float(a.scales[r]));
+                } else {
+                    a.partial[((size_t)split * T + t) * a.d_out + r] = v;
+                }
+            }
             acc[t] = 0.f;
         }
     };
@@ -160,7 +181,7 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
             }
 #pragma unroll
             for (int t = 0; t < T; ++t) {
-                half8_to_float8(xs[((size_t)t * GPC + q) * n_chunks + c], xv);
+                half8_to_float8(xs[((size_t)t * GPC + q) * xstride + c], xv);
                 float s0 = w[0] * xv[0], s1 = w[1] * xv[1];
                 s0 = fmaf(w[2], xv[2], s0);
                 s1 = fmaf(w[3], xv[3], s1);
@@ -185,17 +206,90 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
         multiply(cwB, k + 1);
         finish_item(k + 1);
     }
+    if (splits == 1) return;
+
+    // split input range: the last CTA of this row set adds the partials in split order
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = (atomicAdd(&a.counters[blockIdx.x], 1u) == (uint32_t)(splits - 1));
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const int rows_per_warp = (a.d_out + total_warps - 1) / total_warps;
+    for (int i = threadIdx.x; i < rows_per_warp * kRowWarps * T; i += kRowThreads) {
+        const int w = i % kRowWarps, t = (i / kRowWarps) % T, j = i / (kRowWarps * T);
+        const int r = blockIdx.x * kRowWarps + w + total_warps * j;
+        if (r >= a.d_out) continue;
+        float sum = 0.f;
+        for (int s0 = 0; s0 < splits; s0 += 4) {  // 4 partials in flight, added in split order
+            float v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                v[u] = (s0 + u < splits) ? __ldcg(&a.partial[((size_t)(s0 + u) * T + t) * a.d_out + r]) : 0.f;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) sum += v[u];
+        }
+        a.y[(size_t)t * a.d_out + r] = __float2half_rn(sum * __half2float(a.scales[r]));
+    }
+    if (threadIdx.x == 0) a.counters[blockIdx.x] = 0u;
 }
 
 }  // namespace
 
 constexpr int kRowsMaxTokens = 4;
+// Staged activations (+ 2x8 codebooks) per CTA.  Kept small on purpose: the
+// shared-memory carveout comes out of L1, and L1 holds the codeword gathers
+// in flight (measured on B200: a 4-token 8192x28672 layer with 114 KiB per
+// CTA ran at 299 us, with 32 KiB slices at 176 us).
+constexpr size_t kRowsSmemBudget = 32 * 1024;
 
-// Whole rows per warp when the tokens are few and T * d_in fp16 activations
-// (+ 8 KiB of 2x8 codebooks) fit on chip.
-bool gemv_rows_supported(const Dims &d, int T) {
-    return T >= 1 && T <= kRowsMaxTokens && (size_t)T * d.d_in * 2 + 8192 <= 160 * 1024;
+namespace {
+
+struct RowPlan {
+    int grid_x;            // row sets of 8 warps
+    int splits;            // CTAs along the input range (gridDim.y)
+    int chunks_per_split;  // 16-byte code chunks per row per CTA
+    size_t smem;
+};
+
+// Work plan: the input range is split only as far as the staged activations
+// require, in slices of whole 32-chunk lane slots (a slice of 75 chunks
+// would leave 21 of 32 lanes idle in its last slot); the row sets
+// (gridDim.x) fill two CTAs per SM over all splits.
+RowPlan plan_rows(const Dims &d, int T, int sms) {
+    const int gpc = 16 / (d.M * d.B / 8);
+    const int n_chunks = d.G / gpc;
+    const size_t cb = (d.B == 8) ? (size_t)d.M * 256 * 16 : 0;
+    const size_t per_chunk = (size_t)T * gpc * 16;  // activation bytes per chunk of the slice
+    const int max_slots = (int)((kRowsSmemBudget - cb) / (per_chunk * 32));
+    const int slots = (n_chunks + 31) / 32;         // lane slots of a whole row
+    RowPlan p;
+    p.splits = max_slots < 1 ? (n_chunks + 31) / 32 : (slots + max_slots - 1) / max_slots;
+    p.chunks_per_split = ((slots + p.splits - 1) / p.splits) * 32;
+    if (p.chunks_per_split > n_chunks) p.chunks_per_split = n_chunks;
+    p.splits = (n_chunks + p.chunks_per_split - 1) / p.chunks_per_split;
+    p.smem = per_chunk * p.chunks_per_split + cb;
+    const int cap = (2 * sms) / p.splits > 0 ? (2 * sms) / p.splits : 1;
+    const int sets = (d.d_out + kRowWarps - 1) / kRowWarps;
+    p.grid_x = sets < cap ? sets : cap;
+    return p;
 }
+
+}  // namespace
+
+size_t gemv_rows_counter_offset(const Dims &d, int T, int sms) {
+    const RowPlan p = plan_rows(d, T, sms);
+    if (p.splits == 1) return 0;
+    return ((size_t)p.splits * T * d.d_out * sizeof(float) + 15) / 16 * 16;
+}
+
+size_t gemv_rows_workspace_bytes(const Dims &d, int T, int sms) {
+    const RowPlan p = plan_rows(d, T, sms);
+    if (p.splits == 1) return 0;
+    return gemv_rows_counter_offset(d, T, sms) + (size_t)p.grid_x * sizeof(uint32_t);
+}
+
+bool gemv_rows_supported(int T) { return T >= 1 && T <= kRowsMaxTokens; }
 
 template <int M, int B>
 void (*rows_fn(int T))(const RowArgs) {
@@ -208,19 +302,23 @@ void (*rows_fn(int T))(const RowArgs) {
 }
 
 cudaError_t launch_gemv_rows(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
-                             uint16_t *y, int tokens, const Dims &d, int sms, cudaStream_t st) {
+                             uint16_t *y, int tokens, const Dims &d, void *workspace, int sms, cudaStream_t st) {
+    const RowPlan p = plan_rows(d, tokens, sms);
     RowArgs a;
     a.codes = static_cast<const uint8_t *>(codes);
     a.codebooks = reinterpret_cast<const uint4 *>(codebooks);
     a.scales = reinterpret_cast<const __half *>(scales);
     a.x = reinterpret_cast<const __half *>(x);
     a.y = reinterpret_cast<__half *>(y);
+    a.partial = static_cast<float *>(workspace);
+    a.counters = p.splits > 1 ? reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) +
+                                                             gemv_rows_counter_offset(d, tokens, sms))
+                              : nullptr;
     a.d_out = d.d_out;
+    a.d_in = d.d_in;
     a.G = d.G;
     a.row_bytes = d.row_bytes;
-    const size_t smem = (size_t)tokens * d.G * 16 + ((d.B == 8) ? (size_t)d.M * 256 * 16 : 0);
-    int grid = (d.d_out + kRowWarps - 1) / kRowWarps;
-    if (grid > 2 * sms) grid = 2 * sms;
+    a.chunks_per_split = p.chunks_per_split;
     void (*fn)(const RowArgs);
     if (d.M == 1) {
         fn = rows_fn<1, 16>(tokens);
@@ -229,11 +327,9 @@ cudaError_t launch_gemv_rows(const void *codes, const uint16_t *codebooks, const
     } else {
         fn = rows_fn<2, 16>(tokens);
     }
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    return launch_kernel(fn, dim3(grid), dim3(kRowThreads), smem, st, true, a);
+    const cudaError_t e = opt_in_dynamic_smem(fn, p.smem);
+    if (e != cudaSuccess) return e;
+    return launch_kernel(fn, dim3(p.grid_x, p.splits), dim3(kRowThreads), p.smem, st, true, a);
 }
 
 }  // namespace aqlm

@@ -424,7 +424,10 @@ def run_gpu(args):
                      "traffic": recorded_traffic("gemv 1x16 4096x4096 T1"),
                      "peak_source": f"{peaks['source']} copy bandwidth",
                      "kernel": "gemv_rows_kernel<1,16>",
-                     "algorithmic_bytes_per_launch": head["bytes_per_layer"]},
+                     "algorithmic_bytes_per_launch": head["bytes_per_layer"],
+                     # the roofline that actually binds a batch-1 1x16 layer: one random 16-byte
+                     # codeword gather from L2 per group
+                     "gather_bound": gather_roofline(HEADLINE, head["us_per_layer"])},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": head["launches"],
@@ -438,14 +441,38 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
+# Random 16-byte gathers from an L2-resident 1-2 MiB table, measured on this
+# B200 with a microbenchmark (indices generated in registers, 8 gathers in
+# flight per thread): about one 32-byte sector per SM clock.
+L2_GATHER_PEAK_G_PER_S = 305.0
+# fp32 FMA peak: 148 SMs x 128 FMA/clock x the 1965 MHz maximum clock.
+FMA_PEAK_TERA_PER_S = 148 * 128 * 1.965e9 / 1e12
+
+
+def gather_roofline(spec, us):
+    """Codeword gathers per second against the measured L2 gather rate (1x16 and
+    2x16 gather M codewords per group; 2x8 uses shared-memory tables instead)."""
+    if spec.B != 16:
+        return None
+    gathers = spec.d_out * spec.groups * spec.M
+    achieved = gathers / (us * 1e-6) / 1e9
+    return {"achieved": round(achieved, 1), "peak": L2_GATHER_PEAK_G_PER_S, "unit": "G gathers/s",
+            "frac": round(achieved / L2_GATHER_PEAK_G_PER_S, 4),
+            "peak_source": "random 16-byte gather microbenchmark on this B200"}
+
+
 def _gemv_detail(r, peaks, T=1):
     gbs = r["bytes_per_layer"] / (r["us_per_layer"] * 1e-6) / 1e9
+    spec = r["layers"].spec
     out = {"us_per_layer": round(r["us_per_layer"], 3), "gbs": round(gbs, 1),
            "hbm_frac": round(gbs / peaks["hbm_gbs"], 4)}
+    gr = gather_roofline(spec, r["us_per_layer"])
+    if gr is not None:
+        out["gather_frac"] = gr["frac"]
     if T > 1:
-        groups = r["layers"].spec.d_out * r["layers"].spec.groups
-        fma_t = groups * 8 * T / (r["us_per_layer"] * 1e-6) / 1e12
+        fma_t = spec.d_out * spec.groups * 8 * T / (r["us_per_layer"] * 1e-6) / 1e12
         out["fma_tera_per_s"] = round(fma_t, 2)
+        out["fma_frac"] = round(fma_t / FMA_PEAK_TERA_PER_S, 4)
     return out
 
 
@@ -487,6 +514,8 @@ PROFILE_CASES = {
     "gemv-1x16-4096": ("gemv", 4096, 4096, 1, 16, 1),
     "gemv-2x8-4096": ("gemv", 4096, 4096, 2, 8, 1),
     "gemv-1x16-8192-t16": ("gemv", 8192, 8192, 1, 16, 16),
+    "gemv-1x16-28672x8192-t4": ("gemv", 28672, 8192, 1, 16, 4),
+    "gemv-1x16-8192x28672-t4": ("gemv", 8192, 28672, 1, 16, 4),
     "gemv-2x16-8192": ("gemv", 8192, 8192, 2, 16, 1),
     "dequant-1x16-11008x4096": ("dequant", 11008, 4096, 1, 16, 0),
     "dequant-2x8-11008x4096": ("dequant", 11008, 4096, 2, 8, 0),

@@ -110,6 +110,16 @@ def test_gemv_split_input_range(M, B, T):
     _gemv_case(M, B, 96, 4160, T, seed=20 + T)
 
 
+@pytest.mark.parametrize("M,B,T,d_in", [(1, 16, 1, 82112), (2, 16, 1, 82144), (1, 16, 2, 28736)]
+                         + [(m, b, 3, 28736) for m, b in FORMATS] + [(m, b, 4, 20544) for m, b in FORMATS])
+def test_gemv_rows_split_input_range(M, B, T, d_in):
+    # up to 4 tokens whose activations exceed the row kernel's 32 KiB budget:
+    # the input range is split in slices of whole 32-chunk lane slots (4 to 11
+    # of them here, the last one ragged), partial sums meet in the workspace;
+    # 100 rows leave some warps without a row
+    _gemv_case(M, B, 100, d_in, T, seed=30 + T)
+
+
 def test_gemv_one_hot_returns_columns():
     """x = e_c returns column c of s . W^ (exact up to the fp16 rounding)."""
     spec = LayerSpec(64, 512, 1, 16)
@@ -160,6 +170,7 @@ FULL_GEMV = [
     ("1x16 11008x4096", 11008, 4096, 1, 16, 1),
     ("2x8 4096x11008", 4096, 11008, 2, 8, 1),
     ("1x16 28672x8192 T4", 28672, 8192, 1, 16, 4),
+    ("1x16 8192x28672 T4", 8192, 28672, 1, 16, 4),
     ("1x16 8192x28672 T16", 8192, 28672, 1, 16, 16),
     ("2x16 8192x8192", 8192, 8192, 2, 16, 1),
     ("2x8 256x512", 256, 512, 2, 8, 1),
