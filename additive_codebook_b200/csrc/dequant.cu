@@ -37,8 +37,10 @@ __global__ void decode_indices_kernel(const void *__restrict__ codes, uint16_t *
 // groups l, l + 32, ...: every code load and every 16-byte store of the warp
 // covers contiguous memory) in a software pipeline: the codes of tile k+2
 // and the codeword gathers of tile k+1 are in flight while tile k is
-// converted and stored.
-constexpr int kPerLane = 4;
+// converted and stored.  Two groups per lane and at least three CTAs per SM
+// (measured on B200: 2x8 11008x4096 took 28.7 us, against 36.9 us with four
+// groups per lane at two CTAs per SM).
+constexpr int kPerLane = 2;
 constexpr int kTile = 32 * kPerLane;
 
 template <int M, int B>
@@ -70,11 +72,38 @@ __device__ __forceinline__ uint32_t raw_index(uint32_t raw, int m) {
     else return (raw >> (16 * m)) & 0xffffu;
 }
 
+// Row of group g without a division per group: division by the invariant
+// G as a multiply and a shift (Granlund and Montgomery, "Division by
+// invariant integers using multiplication", 1994): with s = ceil(log2 G)
+// and m = floor(2^(31+s) / G) + 1 (< 2^32), floor(g * m / 2^(31+s)) = g / G
+// for every 0 <= g < 2^31 (the error term g * (m - 2^(31+s)/G) / 2^(31+s)
+// stays below 1/G).  Larger g take the plain 64-bit division.
+struct RowDivider {
+    int64_t G;
+    uint32_t m;
+    int shift;  // 31 + s
+};
+
+RowDivider make_row_divider(int G) {
+    int s = 0;
+    while ((1ll << s) < G) ++s;
+    RowDivider r;
+    r.G = G;
+    r.m = (uint32_t)((1ull << (31 + s)) / (uint64_t)G + 1);
+    r.shift = 31 + s;
+    return r;
+}
+
+__device__ __forceinline__ int64_t row_of(int64_t g, const RowDivider &rd) {
+    if (g < (1ll << 31)) return (int64_t)(((uint64_t)g * rd.m) >> rd.shift);
+    return g / rd.G;
+}
+
 template <int M, int B>
-__global__ void __launch_bounds__(256) dequant_kernel(const uint8_t *__restrict__ codes,
+__global__ void __launch_bounds__(256, 3) dequant_kernel(const uint8_t *__restrict__ codes,
                                                       const uint4 *__restrict__ codebooks,
                                                       const __half *__restrict__ scales,
-                                                      uint4 *__restrict__ W, int G, int64_t n_groups) {
+                                                      uint4 *__restrict__ W, const RowDivider rd, int64_t n_groups) {
     constexpr int K = 1 << B;
     // 2x8: both codebooks (2 x 256 codewords x 16 B = 8 KiB) live in shared memory.
     __shared__ uint4 cb_smem[B == 8 ? M * K : 1];
@@ -113,7 +142,7 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t *__restrict_
         for (int i = 0; i < kPerLane; ++i) {
             const int64_t g = gt + 32 * i;
             if (g >= n_groups) break;
-            const float s = __half2float(scales[g / G]);
+            const float s = __half2float(scales[row_of(g, rd)]);
             float acc[kGroup];
             half8_to_float8(cw[i][0], acc);
 #pragma unroll
@@ -189,16 +218,17 @@ cudaError_t launch_dequant(const void *codes, const uint16_t *codebooks, const u
     auto cb = reinterpret_cast<const uint4 *>(codebooks);
     auto s = reinterpret_cast<const __half *>(scales);
     auto w = reinterpret_cast<uint4 *>(W);
+    const RowDivider rd = make_row_divider(d.G);
     if (d.M == 1 && d.B == 16) {
         auto k = dequant_kernel<1, 16>;
-        return launch_kernel(k, one_wave_grid(k, n), 256, 0, st, false, c, cb, s, w, d.G, n);
+        return launch_kernel(k, one_wave_grid(k, n), 256, 0, st, false, c, cb, s, w, rd, n);
     }
     if (d.M == 2 && d.B == 8) {
         auto k = dequant_kernel<2, 8>;
-        return launch_kernel(k, one_wave_grid(k, n), 256, 0, st, false, c, cb, s, w, d.G, n);
+        return launch_kernel(k, one_wave_grid(k, n), 256, 0, st, false, c, cb, s, w, rd, n);
     }
     auto k = dequant_kernel<2, 16>;
-    return launch_kernel(k, one_wave_grid(k, n), 256, 0, st, false, c, cb, s, w, d.G, n);
+    return launch_kernel(k, one_wave_grid(k, n), 256, 0, st, false, c, cb, s, w, rd, n);
 }
 
 }  // namespace aqlm
