@@ -5,7 +5,9 @@
 // x_j >.  Section "Why and what do we quantize?": decoding is bound by
 // memory traffic, and the codes are the only large stream.
 //
-// Design for few tokens: a warp owns whole rows; its 32 lanes take the row's
+// Design for few tokens: each CTA owns an equal contiguous range of rows (so
+// every SM gets the same share of rows), and its warps own whole rows of
+// that range, round robin; a warp's 32 lanes take the row's
 // 16-byte code chunks l, l + 32, l + 64, ... so every code load of the warp
 // reads 512 contiguous bytes of one row (full DRAM bursts; measured on B200,
 // reading the codes in row-strided 16-byte pieces instead cost about 5 us
@@ -23,7 +25,7 @@
 //   - When T activations of the whole row do not fit the shared-memory
 //     budget, the row's chunks are split over gridDim.y CTAs (each stages only
 //     its slice of x); each writes fp32 row partials to the caller's workspace
-//     and the last CTA of a row set to arrive (an atomic counter, no waiting)
+//     and the last CTA of a row range to arrive (an atomic counter, no waiting)
 //     adds them in split order, scales, rounds, and resets the counter.
 //   - Programmatic dependent launch: codebooks are prefetched into L2 and
 //     the first items' codes and codewords fetched before griddepcontrol.wait
@@ -82,8 +84,10 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
     uint4 *cbs = xs + (size_t)T * GPC * xstride;          // 2x8: [M][256] codewords
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int total_warps = gridDim.x * kRowWarps;
-    const int gwarp = blockIdx.x * kRowWarps + warp;
+    // this CTA's rows: an equal contiguous share [r0, r1) of d_out, so that
+    // every SM gets the same number of rows whichever CTAs it holds
+    const int r0 = (int)((int64_t)blockIdx.x * a.d_out / gridDim.x);
+    const int r1 = (int)((int64_t)(blockIdx.x + 1) * a.d_out / gridDim.x);
     const int cpw = (n_chunks + 31) / 32;  // chunk slots per lane per row
     const uint64_t stream_pol = policy_evict_first();
     const uint64_t keep_pol = policy_evict_last();
@@ -101,17 +105,17 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
         for (int c = threadIdx.x; c < M * F::K; c += kRowThreads) cbs[c] = a.codebooks[c];
     }
 
-    // item k of this warp: row gwarp + total_warps * (k / cpw), chunk slot k % cpw
-    auto item_row = [&](int k) { return gwarp + total_warps * (k / cpw); };
+    // item k of this warp: row r0 + warp + 8 * (k / cpw), chunk slot k % cpw
+    auto item_row = [&](int k) { return r0 + warp + kRowWarps * (k / cpw); };
     auto load_code = [&](int k) -> uint4 {
         const int r = item_row(k);
         const int c = lane + 32 * (k % cpw);
-        if (r < a.d_out && c < n_chunks)
+        if (r < r1 && c < n_chunks)
             return ld_stream_u4(a.codes + (size_t)r * a.row_bytes + (size_t)(c0 + c) * 16, stream_pol);
         return make_uint4(0, 0, 0, 0);
     };
     auto gather = [&](const uint4 &ch, int k, uint4 (&cw)[GPC][M]) {
-        const bool live = item_row(k) < a.d_out && lane + 32 * (k % cpw) < n_chunks;
+        const bool live = item_row(k) < r1 && lane + 32 * (k % cpw) < n_chunks;
 #pragma unroll
         for (int q = 0; q < GPC; ++q) {
 #pragma unroll
@@ -156,7 +160,7 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
             float v = acc[t];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0 && r < a.d_out) {
+            if (lane == 0 && r < r1) {
                 if (splits == 1) {
                     a.y[(size_t)t * a.d_out + r] = __float2half_rn(v * __half2float(a.scales[r]));
                 } else {
@@ -195,12 +199,12 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
     };
 
     // at the top of a trip: cwA holds item k's codewords, ch_next item k+1's codes
-    for (int k = 0; item_row(k) < a.d_out; k += 2) {
+    for (int k = 0; item_row(k) < r1; k += 2) {
         gather(ch_next, k + 1, cwB);
         ch_next = load_code(k + 2);
         multiply(cwA, k);
         finish_item(k);
-        if (item_row(k + 1) >= a.d_out) break;
+        if (item_row(k + 1) >= r1) break;
         gather(ch_next, k + 2, cwA);
         ch_next = load_code(k + 3);
         multiply(cwB, k + 1);
@@ -208,18 +212,15 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
     }
     if (splits == 1) return;
 
-    // split input range: the last CTA of this row set adds the partials in split order
+    // split input range: the last CTA of this row range adds the partials in split order
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) s_last = (atomicAdd(&a.counters[blockIdx.x], 1u) == (uint32_t)(splits - 1));
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    const int rows_per_warp = (a.d_out + total_warps - 1) / total_warps;
-    for (int i = threadIdx.x; i < rows_per_warp * kRowWarps * T; i += kRowThreads) {
-        const int w = i % kRowWarps, t = (i / kRowWarps) % T, j = i / (kRowWarps * T);
-        const int r = blockIdx.x * kRowWarps + w + total_warps * j;
-        if (r >= a.d_out) continue;
+    for (int i = threadIdx.x; i < (r1 - r0) * T; i += kRowThreads) {
+        const int t = i / (r1 - r0), r = r0 + (i - t * (r1 - r0));
         float sum = 0.f;
         for (int s0 = 0; s0 < splits; s0 += 4) {  // 4 partials in flight, added in split order
             float v[4];
@@ -246,7 +247,7 @@ constexpr size_t kRowsSmemBudget = 32 * 1024;
 namespace {
 
 struct RowPlan {
-    int grid_x;            // row sets of 8 warps
+    int grid_x;            // CTAs along the rows, each an equal contiguous row range
     int splits;            // CTAs along the input range (gridDim.y)
     int chunks_per_split;  // 16-byte code chunks per row per CTA
     size_t smem;
@@ -254,7 +255,7 @@ struct RowPlan {
 
 // Work plan: the input range is split only as far as the staged activations
 // require, in slices of whole 32-chunk lane slots (a slice of 75 chunks
-// would leave 21 of 32 lanes idle in its last slot); the row sets
+// would leave 21 of 32 lanes idle in its last slot); the row ranges
 // (gridDim.x) fill two CTAs per SM over all splits.
 RowPlan plan_rows(const Dims &d, int T, int sms) {
     const int gpc = 16 / (d.M * d.B / 8);

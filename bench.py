@@ -54,23 +54,27 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def kernel_source_hash():
+def kernel_source_hash(files):
+    """Hash of the sources a kernel is compiled from (names relative to the
+    package's csrc/ or to include/)."""
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "additive_codebook_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(files):
+        path = os.path.join(ROOT, "additive_codebook_b200", "csrc", f)
+        if not os.path.exists(path):
+            path = os.path.join(ROOT, "include", f)
         h.update(f.encode())
-        h.update(open(os.path.join(csrc, f), "rb").read())
+        h.update(open(path, "rb").read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel_key):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources; else None."""
+    on the kernel's current sources; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     rec = json.load(open(path)).get(kernel_key)
-    if not rec or rec.get("source_hash") != kernel_source_hash():
+    if not rec or rec.get("source_hash") != kernel_source_hash(rec.get("sources", [])):
         return None
     return rec.get("dram_bytes_per_launch")
 
