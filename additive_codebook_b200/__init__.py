@@ -105,15 +105,39 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+_shapes = {}
+
+
 def shape_of(codes, d_in=None):
     """aqlm_shape from a codes tensor [d_out, G, M] (B from its dtype)."""
-    d_out, G, M = codes.shape
-    B = 8 if codes.dtype == torch.uint8 else 16
-    return Shape(d_out, d_in if d_in is not None else G * 8, 8, M, B)
+    key = (tuple(codes.shape), codes.dtype, d_in)
+    sh = _shapes.get(key)
+    if sh is None:
+        d_out, G, M = codes.shape
+        B = 8 if codes.dtype == torch.uint8 else 16
+        sh = Shape(d_out, d_in if d_in is not None else G * 8, 8, M, B)
+        if len(_shapes) < 4096:
+            _shapes[key] = sh
+    return sh
 
 
 def _flat_scales(scales):
-    return scales.reshape(-1)
+    # [d_out] or [d_out, 1, ...]: only the pointer is passed, which a
+    # contiguous tensor shares with its flat view
+    return scales if scales.is_contiguous() else scales.reshape(-1).contiguous()
+
+
+_gemv_ws = {}
+
+
+def _gemv_need(lib, shape, T, device):
+    key = (shape.d_out, shape.d_in, shape.num_codebooks, shape.codebook_bits, T, device)
+    need = _gemv_ws.get(key)
+    if need is None:
+        need = int(lib.aqlm_gemv_workspace_bytes(shape, T))
+        if len(_gemv_ws) < 4096:
+            _gemv_ws[key] = need
+    return need
 
 
 def gemv_workspace_bytes(shape, tokens):
@@ -133,7 +157,7 @@ def aqlm_gemv(codes, codebooks, scales, x, y=None, workspace=None, stream=None):
     T = x.shape[0]
     if y is None:
         y = torch.empty((T, shape.d_out), dtype=torch.float16, device=x.device)
-    need = lib.aqlm_gemv_workspace_bytes(shape, T)
+    need = _gemv_need(lib, shape, T, x.device.index)
     if need and workspace is None:
         workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
     wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0

@@ -1,7 +1,11 @@
 // common.cuh -- small device helpers shared by the library's kernels.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
+#include <mutex>
+#include <tuple>
+#include <vector>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
@@ -124,10 +128,43 @@ cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t 
     return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
+// SM count of a device, queried once per device.
 inline int num_sms(int device) {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> cached[kMaxDevices];
+    if (device >= 0 && device < kMaxDevices) {
+        const int c = cached[device].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
     int n = 0;
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device);
-    return n > 0 ? n : 148;
+    if (n <= 0) return 148;
+    if (device >= 0 && device < kMaxDevices) cached[device].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+// CTAs of `kern` resident per SM at this block size and dynamic shared
+// memory (at least 1), cached per (device, kernel, threads, bytes): the
+// occupancy query costs microseconds of host time per call.
+inline int resident_ctas(const void *kern, int threads, size_t smem) {
+    static std::mutex mu;
+    static std::vector<std::tuple<int, const void *, int, size_t, int>> cache;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (const auto &e : cache)
+            if (std::get<0>(e) == dev && std::get<1>(e) == kern && std::get<2>(e) == threads && std::get<3>(e) == smem)
+                return std::get<4>(e);
+    }
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem) != cudaSuccess || occ < 1) {
+        cudaGetLastError();  // leave no sticky error behind; fall back to one CTA per SM
+        return 1;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache.size() < 4096) cache.emplace_back(dev, kern, threads, smem, occ);
+    return occ;
 }
 
 }  // namespace aqlm

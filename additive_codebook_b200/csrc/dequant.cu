@@ -202,9 +202,9 @@ cudaError_t launch_decode_indices(const void *codes, uint16_t *idx, const Dims &
 // second wave of CTAs waiting behind the first.
 template <typename Kern>
 int one_wave_grid(Kern kern, int64_t n_groups) {
-    int dev = 0, occ = 0;
+    int dev = 0;
     cudaGetDevice(&dev);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 256, 0) != cudaSuccess || occ < 1) occ = 1;
+    const int occ = resident_ctas(reinterpret_cast<const void *>(kern), 256, 0);
     const int64_t tiles = (n_groups + kTile - 1) / kTile;
     const int64_t want = (tiles + 7) / 8;  // 8 warps per CTA
     const int64_t cap = (int64_t)num_sms(dev) * occ;

@@ -1,24 +1,18 @@
 // gemv.cu -- host side of the decode-time product: kernel choice, work plan,
 // workspace layout and the launch (with programmatic dependent launch).
 // 1..4 tokens: gemv_rows.cu (coalesced row streaming, the input range split
-// when the activations do not fit on chip); for one token of 2x8 the
-// lookup-table kernel of gemv_lut.cu.  5..16 tokens: the several-rows-per-lane
+// when the activations do not fit on chip).  5..16 tokens: the several-rows-per-lane
 // kernel of gemv_multi.cuh, instantiated per format in gemv_multi_1x16.cu,
 // gemv_multi_2x8.cu and gemv_multi_2x16.cu.
 #include "gemv_multi.cuh"
 
 namespace aqlm {
 
-size_t gemv_lut_workspace_bytes(const Dims &d, int sms);
-size_t gemv_lut_workspace_counter_offset(const Dims &d, int sms);
 bool gemv_rows_supported(int T);
 size_t gemv_rows_workspace_bytes(const Dims &d, int T, int sms);
 size_t gemv_rows_counter_offset(const Dims &d, int T, int sms);
 cudaError_t launch_gemv_rows(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
                              uint16_t *y, int tokens, const Dims &d, void *workspace, int sms, cudaStream_t st);
-cudaError_t launch_gemv_lut_2x8(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
-                                const uint16_t *x, uint16_t *y, const Dims &d, void *workspace, int sms,
-                                cudaStream_t st);
 
 namespace gemv_detail {
 namespace {
@@ -69,10 +63,8 @@ GemvFn pick_multi(int M, int B, int T) {
     return gemv_multi_pick_2x16(T);
 }
 
-// Up to four tokens: whole rows per warp with coalesced code streaming; for
-// one token of 2x8 the lookup-table kernel (measured faster on B200).
-bool use_lut(const Dims &d, int T) { return d.M == 2 && d.B == 8 && T == 1; }
-bool use_rows(const Dims &d, int T) { return gemv_rows_supported(T) && !use_lut(d, T); }
+// Up to four tokens: whole rows per warp with coalesced code streaming.
+bool use_rows(int T) { return gemv_rows_supported(T); }
 
 int device_sms() {
     int dev = 0;
@@ -86,8 +78,7 @@ int device_sms() {
 size_t gemv_workspace_bytes(const Dims &d, int tokens) {
     using namespace gemv_detail;
     const int sms = device_sms();
-    if (use_lut(d, tokens)) return gemv_lut_workspace_bytes(d, sms);
-    if (use_rows(d, tokens)) return gemv_rows_workspace_bytes(d, tokens, sms);
+    if (use_rows(tokens)) return gemv_rows_workspace_bytes(d, tokens, sms);
     return multi_workspace_bytes(d, tokens, sms);
 }
 
@@ -96,8 +87,7 @@ size_t gemv_workspace_bytes(const Dims &d, int tokens) {
 size_t gemv_workspace_counter_offset(const Dims &d, int tokens) {
     using namespace gemv_detail;
     const int sms = device_sms();
-    if (use_lut(d, tokens)) return gemv_lut_workspace_counter_offset(d, sms);
-    if (use_rows(d, tokens)) return gemv_rows_counter_offset(d, tokens, sms);
+    if (use_rows(tokens)) return gemv_rows_counter_offset(d, tokens, sms);
     const Plan p = plan_multi(d, tokens, sms);
     if (p.splits == 1) return 0;
     return align16((size_t)p.splits * tokens * d.d_out * sizeof(float));
@@ -108,8 +98,7 @@ cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint
                         cudaStream_t st) {
     using namespace gemv_detail;
     const int sms = device_sms();
-    if (use_lut(d, tokens)) return launch_gemv_lut_2x8(codes, codebooks, scales, x, y, d, workspace, sms, st);
-    if (use_rows(d, tokens)) return launch_gemv_rows(codes, codebooks, scales, x, y, tokens, d, workspace, sms, st);
+    if (use_rows(tokens)) return launch_gemv_rows(codes, codebooks, scales, x, y, tokens, d, workspace, sms, st);
     const Plan p = plan_multi(d, tokens, sms);
     GemvFn fn = pick_multi(d.M, d.B, tokens);
     const cudaError_t e = opt_in_dynamic_smem(fn, p.smem);

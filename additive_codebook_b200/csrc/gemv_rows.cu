@@ -132,8 +132,8 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
 
     uint4 cwA[GPC][M], cwB[GPC][M];
     uint4 ch_next = load_code(1);
+    const uint4 ch0 = load_code(0);
     {
-        const uint4 ch0 = load_code(0);
         if constexpr (!F::kSmemCodebook) gather(ch0, 0, cwA);
         grid_dep_wait();
         const int ng = n_chunks * GPC;  // groups of the slice
@@ -144,7 +144,6 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
                 *reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.d_in + (size_t)(c0 * GPC + g) * kGroup);
         }
         __syncthreads();
-        if constexpr (F::kSmemCodebook) gather(ch0, 0, cwA);
     }
     grid_dep_launch();
 
@@ -170,45 +169,65 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
             acc[t] = 0.f;
         }
     };
+    // the decoded group q of item k's chunk times every token's activations
+    auto dot_group = [&](const uint4 &cw0, const uint4 &cw1, int q, int c) {
+        float w[kGroup], xv[kGroup];
+        half8_to_float8(cw0, w);
+        if constexpr (M == 2) {
+            float f[kGroup];
+            half8_to_float8(cw1, f);
+#pragma unroll
+            for (int e = 0; e < kGroup; ++e) w[e] += f[e];
+        }
+#pragma unroll
+        for (int t = 0; t < T; ++t) {
+            half8_to_float8(xs[((size_t)t * GPC + q) * xstride + c], xv);
+            float s0 = w[0] * xv[0], s1 = w[1] * xv[1];
+            s0 = fmaf(w[2], xv[2], s0);
+            s1 = fmaf(w[3], xv[3], s1);
+            s0 = fmaf(w[4], xv[4], s0);
+            s1 = fmaf(w[5], xv[5], s1);
+            s0 = fmaf(w[6], xv[6], s0);
+            s1 = fmaf(w[7], xv[7], s1);
+            acc[t] += s0 + s1;
+        }
+    };
     auto multiply = [&](const uint4 (&cw)[GPC][M], int k) {
         const int c = lane + 32 * (k % cpw);
         if (c >= n_chunks) return;
 #pragma unroll
-        for (int q = 0; q < GPC; ++q) {
-            float w[kGroup], xv[kGroup];
-            half8_to_float8(cw[q][0], w);
-            if constexpr (M == 2) {
-                float f[kGroup];
-                half8_to_float8(cw[q][1], f);
-#pragma unroll
-                for (int e = 0; e < kGroup; ++e) w[e] += f[e];
-            }
-#pragma unroll
-            for (int t = 0; t < T; ++t) {
-                half8_to_float8(xs[((size_t)t * GPC + q) * xstride + c], xv);
-                float s0 = w[0] * xv[0], s1 = w[1] * xv[1];
-                s0 = fmaf(w[2], xv[2], s0);
-                s1 = fmaf(w[3], xv[3], s1);
-                s0 = fmaf(w[4], xv[4], s0);
-                s1 = fmaf(w[5], xv[5], s1);
-                s0 = fmaf(w[6], xv[6], s0);
-                s1 = fmaf(w[7], xv[7], s1);
-                acc[t] += s0 + s1;
-            }
-        }
+        for (int q = 0; q < GPC; ++q) dot_group(cw[q][0], cw[q][M - 1], q, c);
     };
 
-    // at the top of a trip: cwA holds item k's codewords, ch_next item k+1's codes
-    for (int k = 0; item_row(k) < r1; k += 2) {
-        gather(ch_next, k + 1, cwB);
-        ch_next = load_code(k + 2);
-        multiply(cwA, k);
-        finish_item(k);
-        if (item_row(k + 1) >= r1) break;
-        gather(ch_next, k + 2, cwA);
-        ch_next = load_code(k + 3);
-        multiply(cwB, k + 1);
-        finish_item(k + 1);
+    if constexpr (F::kSmemCodebook) {
+        // 2x8: codewords come from shared memory at use (short latency, so no
+        // register copies of a whole item ahead); the codes run two items ahead
+        uint4 ch = ch0;
+        for (int k = 0; item_row(k) < r1; ++k) {
+            const uint4 ch_after = load_code(k + 2);
+            const int c = lane + 32 * (k % cpw);
+            if (c < n_chunks) {
+#pragma unroll
+                for (int q = 0; q < GPC; ++q)
+                    dot_group(cbs[code_index<M, B>(ch, q, 0)], cbs[F::K + code_index<M, B>(ch, q, M - 1)], q, c);
+            }
+            finish_item(k);
+            ch = ch_next;
+            ch_next = ch_after;
+        }
+    } else {
+        // at the top of a trip: cwA holds item k's codewords, ch_next item k+1's codes
+        for (int k = 0; item_row(k) < r1; k += 2) {
+            gather(ch_next, k + 1, cwB);
+            ch_next = load_code(k + 2);
+            multiply(cwA, k);
+            finish_item(k);
+            if (item_row(k + 1) >= r1) break;
+            gather(ch_next, k + 2, cwA);
+            ch_next = load_code(k + 3);
+            multiply(cwB, k + 1);
+            finish_item(k + 1);
+        }
     }
     if (splits == 1) return;
 
@@ -247,17 +266,15 @@ constexpr size_t kRowsSmemBudget = 32 * 1024;
 namespace {
 
 struct RowPlan {
-    int grid_x;            // CTAs along the rows, each an equal contiguous row range
     int splits;            // CTAs along the input range (gridDim.y)
     int chunks_per_split;  // 16-byte code chunks per row per CTA
     size_t smem;
 };
 
-// Work plan: the input range is split only as far as the staged activations
-// require, in slices of whole 32-chunk lane slots (a slice of 75 chunks
-// would leave 21 of 32 lanes idle in its last slot); the row ranges
-// (gridDim.x) fill two CTAs per SM over all splits.
-RowPlan plan_rows(const Dims &d, int T, int sms) {
+// Work plan along the input range: split only as far as the staged
+// activations require, in slices of whole 32-chunk lane slots (a slice of 75
+// chunks would leave 21 of 32 lanes idle in its last slot).
+RowPlan plan_rows(const Dims &d, int T) {
     const int gpc = 16 / (d.M * d.B / 8);
     const int n_chunks = d.G / gpc;
     const size_t cb = (d.B == 8) ? (size_t)d.M * 256 * 16 : 0;
@@ -270,24 +287,31 @@ RowPlan plan_rows(const Dims &d, int T, int sms) {
     if (p.chunks_per_split > n_chunks) p.chunks_per_split = n_chunks;
     p.splits = (n_chunks + p.chunks_per_split - 1) / p.chunks_per_split;
     p.smem = per_chunk * p.chunks_per_split + cb;
-    const int cap = (2 * sms) / p.splits > 0 ? (2 * sms) / p.splits : 1;
-    const int sets = (d.d_out + kRowWarps - 1) / kRowWarps;
-    p.grid_x = sets < cap ? sets : cap;
     return p;
+}
+
+// Row ranges (gridDim.x): as many CTAs as the SMs hold at once over all
+// splits (by the kernel's registers and shared memory), at most one per 8 rows.
+int rows_grid_x(const Dims &d, const RowPlan &p, int ctas_per_sm, int sms) {
+    const int cap = (ctas_per_sm * sms) / p.splits > 0 ? (ctas_per_sm * sms) / p.splits : 1;
+    const int sets = (d.d_out + kRowWarps - 1) / kRowWarps;
+    return sets < cap ? sets : cap;
 }
 
 }  // namespace
 
 size_t gemv_rows_counter_offset(const Dims &d, int T, int sms) {
-    const RowPlan p = plan_rows(d, T, sms);
+    (void)sms;
+    const RowPlan p = plan_rows(d, T);
     if (p.splits == 1) return 0;
     return ((size_t)p.splits * T * d.d_out * sizeof(float) + 15) / 16 * 16;
 }
 
+// Partials, then one arrival counter per possible row range (at most one per 8 rows).
 size_t gemv_rows_workspace_bytes(const Dims &d, int T, int sms) {
-    const RowPlan p = plan_rows(d, T, sms);
+    const RowPlan p = plan_rows(d, T);
     if (p.splits == 1) return 0;
-    return gemv_rows_counter_offset(d, T, sms) + (size_t)p.grid_x * sizeof(uint32_t);
+    return gemv_rows_counter_offset(d, T, sms) + (size_t)((d.d_out + kRowWarps - 1) / kRowWarps) * sizeof(uint32_t);
 }
 
 bool gemv_rows_supported(int T) { return T >= 1 && T <= kRowsMaxTokens; }
@@ -304,7 +328,7 @@ void (*rows_fn(int T))(const RowArgs) {
 
 cudaError_t launch_gemv_rows(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
                              uint16_t *y, int tokens, const Dims &d, void *workspace, int sms, cudaStream_t st) {
-    const RowPlan p = plan_rows(d, tokens, sms);
+    const RowPlan p = plan_rows(d, tokens);
     RowArgs a;
     a.codes = static_cast<const uint8_t *>(codes);
     a.codebooks = reinterpret_cast<const uint4 *>(codebooks);
@@ -328,9 +352,10 @@ cudaError_t launch_gemv_rows(const void *codes, const uint16_t *codebooks, const
     } else {
         fn = rows_fn<2, 16>(tokens);
     }
-    const cudaError_t e = opt_in_dynamic_smem(fn, p.smem);
+    cudaError_t e = opt_in_dynamic_smem(fn, p.smem);
     if (e != cudaSuccess) return e;
-    return launch_kernel(fn, dim3(p.grid_x, p.splits), dim3(kRowThreads), p.smem, st, true, a);
+    const int occ = resident_ctas(reinterpret_cast<const void *>(fn), kRowThreads, p.smem);
+    return launch_kernel(fn, dim3(rows_grid_x(d, p, occ, sms), p.splits), dim3(kRowThreads), p.smem, st, true, a);
 }
 
 }  // namespace aqlm

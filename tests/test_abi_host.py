@@ -88,7 +88,7 @@ def test_gemv_workspace_rules():
     big = ac.Shape(8192, 8192, 8, 1, 16)
     assert lib.aqlm_gemv_workspace_bytes(big, 1) == 0          # enough row tiles: no split
     assert lib.aqlm_gemv_workspace_bytes(shape(M=1, B=16), 1) == 0   # one token: whole rows per warp
-    assert lib.aqlm_gemv_workspace_bytes(shape(), 1) > 0       # 2x8, one token: lookup tables, 2 slabs
+    assert lib.aqlm_gemv_workspace_bytes(shape(), 1) == 0      # 2x8, one token: 2 KiB of activations
     wide = shape(d_in=4096)                                    # 8 tokens, 2 row tiles: split to fill the SMs
     assert lib.aqlm_gemv_workspace_bytes(shape(d_in=4096, M=1, B=16), 4) == 0   # 32 KiB of activations: one slice
     small = lib.aqlm_gemv_workspace_bytes(wide, 8)

@@ -24,11 +24,11 @@ from synth import LayerSpec, make_layer
 
 pytestmark = pytest.mark.gpu
 
-# shapes whose product needs scratch: the one-token 2x8 lookup-table path
-# (slab partial sums), products of several tokens split over the input range
-# to fill the SMs, and a 16-token product split because its activations do
-# not fit on chip at once
-CASES = [(4096, 4096, 2, 8, 1), (2048, 4096, 2, 8, 6), (1024, 4096, 1, 16, 16), (512, 4160, 2, 16, 8)]
+# shapes whose product needs scratch: a 4-token row-kernel product whose
+# activations are split into slices (7 x 64 chunks of 28672 inputs),
+# products of several tokens split over the input range to fill the SMs, and
+# a 16-token product split because its activations do not fit on chip at once
+CASES = [(1024, 28672, 2, 8, 4), (2048, 4096, 2, 8, 6), (1024, 4096, 1, 16, 16), (512, 4160, 2, 16, 8)]
 
 
 def _call_noalloc(lib, d, x, y):
