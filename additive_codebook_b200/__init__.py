@@ -30,7 +30,7 @@ AQLM_ERR_TIMEOUT = 6
 GEMV_MAX_TOKENS = 16
 
 # Every entry point declared in include/aqlm.h.
-EXPORTS = ["aqlm_gemv", "aqlm_gemv_workspace_bytes", "aqlm_dequant", "aqlm_gemm",
+EXPORTS = ["aqlm_gemv", "aqlm_gemv_workspace_bytes", "aqlm_gemv_check", "aqlm_dequant", "aqlm_gemm",
            "aqlm_gemm_workspace_bytes", "aqlm_gemm_check", "aqlm_bf16_gemm", "aqlm_decode_indices",
            "aqlm_test_gemm_timeout", "aqlm_gemv_noalloc", "aqlm_gemv_noalloc_max_scratch_bytes",
            "aqlm_status_string", "aqlm_version"]
@@ -63,6 +63,7 @@ def load_library():
     sig = {
         "aqlm_gemv": ([vp, vp, vp, vp, vp, i32, Shape, vp, sz, vp], st),
         "aqlm_gemv_workspace_bytes": ([Shape, i32], sz),
+        "aqlm_gemv_check": ([Shape, i32, vp, sz, vp], st),
         "aqlm_dequant": ([vp, vp, vp, vp, Shape, vp], st),
         "aqlm_gemm": ([vp, vp, vp, vp, vp, i32, Shape, vp, sz, vp], st),
         "aqlm_gemm_workspace_bytes": ([Shape, i32], sz),
@@ -164,6 +165,14 @@ def aqlm_gemv(codes, codebooks, scales, x, y=None, workspace=None, stream=None):
     _check(lib.aqlm_gemv(_p(codes), _p(codebooks), _p(_flat_scales(scales)), _p(x), _p(y), T, shape,
                          _p(workspace), wbytes, _stream(stream)), "aqlm_gemv")
     return y
+
+
+def aqlm_gemv_check(codes, tokens, workspace, stream=None):
+    """Synchronise and return the status the aqlm_gemv calls with this layer
+    shape, token count and workspace recorded (AQLM_OK or AQLM_ERR_TIMEOUT)."""
+    lib = load_library()
+    wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return lib.aqlm_gemv_check(shape_of(codes), tokens, _p(workspace), wbytes, _stream(stream))
 
 
 def aqlm_gemv_noalloc(codes, codebooks, scales, x, y=None, stream=None):

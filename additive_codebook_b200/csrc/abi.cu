@@ -84,6 +84,27 @@ aqlm_status aqlm_gemv(const void *codes, const uint16_t *codebooks, const uint16
                                        to_cuda(stream)));
 }
 
+aqlm_status aqlm_gemv_check(aqlm_shape shape, int32_t tokens, void *workspace, size_t workspace_bytes,
+                            aqlm_stream_t stream) {
+    if (check_shape(shape) != AQLM_OK) return AQLM_ERR_UNSUPPORTED;
+    if (tokens < 1 || tokens > AQLM_GEMV_MAX_TOKENS) return AQLM_ERR_INVALID_ARG;
+    const Dims d = aqlm::make_dims(shape);
+    const long long off = aqlm::gemv_status_offset(d, tokens);
+    const cudaStream_t cs = to_cuda(stream);
+    if (off < 0) return cudaStreamSynchronize(cs) == cudaSuccess ? AQLM_OK : AQLM_ERR_CUDA;
+    if (!workspace || workspace_bytes < (size_t)off + sizeof(int32_t) || !aligned(workspace, 16))
+        return AQLM_ERR_WORKSPACE;
+    int32_t *word = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + off);
+    int32_t h = 0;
+    if (cudaMemcpyAsync(&h, word, sizeof(h), cudaMemcpyDeviceToHost, cs) != cudaSuccess) return AQLM_ERR_CUDA;
+    if (cudaStreamSynchronize(cs) != cudaSuccess) return AQLM_ERR_CUDA;
+    if (h != 0) {
+        if (cudaMemsetAsync(word, 0, sizeof(int32_t), cs) != cudaSuccess) return AQLM_ERR_CUDA;
+        if (cudaStreamSynchronize(cs) != cudaSuccess) return AQLM_ERR_CUDA;
+    }
+    return h == 0 ? AQLM_OK : AQLM_ERR_TIMEOUT;
+}
+
 size_t aqlm_gemm_workspace_bytes(aqlm_shape shape, int32_t tokens) {
     if (check_shape(shape) != AQLM_OK || tokens < 1) return 0;
     return kStatusBytes + (size_t)shape.d_out * shape.d_in * 2;

@@ -176,6 +176,7 @@ cudaError_t launch_dequant(const void *codes, const uint16_t *codebooks, const u
                            uint16_t *W, const Dims &d, cudaStream_t st);
 size_t gemv_workspace_bytes(const Dims &d, int tokens);
 size_t gemv_workspace_counter_offset(const Dims &d, int tokens);
+long long gemv_status_offset(const Dims &d, int tokens);
 cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                         const uint16_t *x, uint16_t *y, int tokens, const Dims &d, void *workspace,
                         cudaStream_t st);

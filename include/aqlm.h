@@ -99,11 +99,16 @@ typedef struct {
  *   x: [tokens][d_in] fp16.   y: [tokens][d_out] fp16 (written).
  *   workspace/workspace_bytes: device scratch for fp32 partial sums and
  *   arrival counters, used when a row's input range is split over several
- *   CTAs; aqlm_gemv_workspace_bytes() gives the size for this device (0 =
- *   none needed, NULL allowed).  Too small or not 16-byte aligned ->
- *   AQLM_ERR_WORKSPACE.  The workspace must be zero-filled before its first
- *   use; every completed call leaves it ready for the next one.  Calls that
- *   share a workspace must not overlap on the GPU.
+ *   CTAs, and (5 to 16 tokens) a status word; aqlm_gemv_workspace_bytes()
+ *   gives the size for this device (0 = none needed, NULL allowed).  Too
+ *   small or not 16-byte aligned -> AQLM_ERR_WORKSPACE.  The workspace must be
+ *   zero-filled before its first use; every completed call leaves it ready for
+ *   the next one.  Calls that share a workspace must not overlap on the GPU.
+ * Up to 4 tokens the kernels have no device waits.  From 5 tokens the
+ * product runs on the tensor cores with producer/consumer waits inside each
+ * CTA, each bounded in time: a wait that gives up records AQLM_ERR_TIMEOUT in
+ * the workspace's status word (y is then not valid, and the workspace must be
+ * zero-filled again); aqlm_gemv_check() reads it.
  * Launch: with programmatic dependent launch.  codes, codebooks and scales
  * are treated as constant weights and may be read before the preceding
  * kernel in the stream has finished; x is read, and y and the workspace are
@@ -116,6 +121,17 @@ AQLM_API aqlm_status aqlm_gemv(const void *codes, const uint16_t *codebooks, con
 /* Bytes of device workspace aqlm_gemv needs for this shape and token count
  * on the current device (0 if none); returns 0 for invalid arguments too. */
 AQLM_API size_t aqlm_gemv_workspace_bytes(aqlm_shape shape, int32_t tokens);
+
+/*
+ * aqlm_gemv_check -- synchronise `stream` and return the status that the
+ * aqlm_gemv calls with this shape, token count and workspace recorded:
+ * AQLM_OK, or AQLM_ERR_TIMEOUT (the word is then cleared).  Paths without
+ * device waits (up to 4 tokens) have no status word: AQLM_OK after the
+ * synchronisation.  Not a counterpart of anything on the pages: library
+ * plumbing for the bounded waits.
+ */
+AQLM_API aqlm_status aqlm_gemv_check(aqlm_shape shape, int32_t tokens, void *workspace, size_t workspace_bytes,
+                                     aqlm_stream_t stream);
 
 /*
  * aqlm_dequant -- the runtime dequantisation of section "Why and what do we

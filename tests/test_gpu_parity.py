@@ -120,6 +120,25 @@ def test_gemv_rows_split_input_range(M, B, T, d_in):
     _gemv_case(M, B, 100, d_in, T, seed=30 + T)
 
 
+@pytest.mark.parametrize("T", [5, 16])
+def test_gemv_tensor_core_ragged_stage(T):
+    # 2x16 with 516 groups: the last 8-group stage of the tensor-core path holds
+    # 4 groups (the rest are zeros in the decoded tile); 300 rows: 3 row tiles,
+    # the last ragged
+    _gemv_case(2, 16, 300, 4128, T, seed=50 + T)
+
+
+@pytest.mark.parametrize("M,B", FORMATS)
+def test_gemv_check_reports_ok(M, B):
+    spec = LayerSpec(256, 1024, M, B)
+    for T in (1, 8):
+        d = to_dev(make_layer(spec, seed=60 + T, tokens=T))
+        need = ac.gemv_workspace_bytes(ac.shape_of(d["codes"]), T)
+        ws = torch.zeros(max(need, 16), dtype=torch.uint8, device="cuda")
+        ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], d["x"], workspace=ws)
+        assert ac.aqlm_gemv_check(d["codes"], T, ws) == ac.AQLM_OK
+
+
 def test_gemv_one_hot_returns_columns():
     """x = e_c returns column c of s . W^ (exact up to the fp16 rounding)."""
     spec = LayerSpec(64, 512, 1, 16)
@@ -144,11 +163,12 @@ def test_gemv_two_calls_identical():
 
 
 @pytest.mark.parametrize("M,B", FORMATS)
-def test_gemv_chain_reads_x_after_the_producer(M, B):
+@pytest.mark.parametrize("T", [1, 8])
+def test_gemv_chain_reads_x_after_the_producer(M, B, T):
     """Back-to-back layers where each x is the previous layer's y (programmatic
     dependent launch must not read x early), with a torch kernel in between."""
     specs = [LayerSpec(1024, 512, M, B), LayerSpec(512, 1024, M, B), LayerSpec(1024, 512, M, B)]
-    Ls = [make_layer(s, seed=40 + k, tokens=1 if k == 0 else 0) for k, s in enumerate(specs)]
+    Ls = [make_layer(s, seed=40 + k, tokens=T if k == 0 else 0) for k, s in enumerate(specs)]
     ds = [to_dev(L) for L in Ls]
     x = ds[0]["x"]
     ys = []

@@ -59,12 +59,14 @@ def test_noalloc_matches_gemv_on_two_calls(cuda_device, d_out, d_in, M, B, T):
 
 def test_noalloc_rejects_scratch_beyond_its_maximum(cuda_device):
     lib = ac.load_library()
-    shape = ac.Shape(131072, 8192, 8, 1, 16)    # 16 tokens: far more than 8 MiB of partial sums
-    assert lib.aqlm_gemv_workspace_bytes(shape, 16) > lib.aqlm_gemv_noalloc_max_scratch_bytes()
+    # 4 tokens of 28672 inputs: seven activation slices, 7 x 4 x 131072 fp32
+    # partial sums (14.7 MB), far more than the 8 MiB built in
+    shape = ac.Shape(131072, 28672, 8, 1, 16)
+    assert lib.aqlm_gemv_workspace_bytes(shape, 4) > lib.aqlm_gemv_noalloc_max_scratch_bytes()
     codes = torch.zeros(16, dtype=torch.uint8, device=DEV)   # never read: the call is rejected first
     x = torch.zeros(16, 16, dtype=torch.float16, device=DEV)
     y = torch.zeros(16, 16, dtype=torch.float16, device=DEV)
     p = ctypes.c_void_p(codes.data_ptr())
-    st = lib.aqlm_gemv_noalloc(p, p, p, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()), 16, shape,
+    st = lib.aqlm_gemv_noalloc(p, p, p, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()), 4, shape,
                                ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == ac.AQLM_ERR_WORKSPACE
