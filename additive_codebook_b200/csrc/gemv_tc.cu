@@ -12,8 +12,15 @@
 // codebooks each gets its own A tile and its own MMA into the same
 // accumulator, (C_0[b0] + C_1[b1]) . x = C_0[b0] . x + C_1[b1] . x.
 //
-// One CTA = 128 output rows x a range of input stages (64 inputs = 8 groups
-// each), 6 warps:
+// Work decomposition (stream-K): the (row tile of 128, stage of 64 inputs =
+// 8 groups) units of the layer, tile-major, are cut into equal contiguous
+// ranges, one per CTA, two CTAs per SM, so every SM gets the same work
+// whatever the shape.  A CTA's range crosses at most a few tiles: it handles
+// them as segments, one accumulator each; a segment that covers its whole
+// tile is scaled and stored, the others publish fp32 partial sums to the
+// workspace and the last segment of the tile to arrive (an atomic counter,
+// no waiting) adds them in input order (deterministic), scales and stores.
+// One CTA has 6 warps:
 //   warps 0-3  decoders, one thread per row: read the row's codes of the
 //              stage from the code tile, gather the codewords (1x16 / 2x16
 //              through L1/L2 with an evict-last policy, 2x8 from shared
@@ -27,9 +34,7 @@
 //   warp 5     allocates 32 TMEM columns; one thread issues
 //              tcgen05.mma.cta_group::1.kind::f16 (M = 128, N = 16, K = 16)
 //              and releases each stage with tcgen05.commit.
-// An input range split over gridDim.y CTAs publishes fp32 partials to the
-// workspace; the last CTA of the row tile to arrive (atomic counter, no
-// waiting) adds them in split order.  Every mbarrier wait is bounded in time:
+// Every mbarrier wait is bounded in time:
 // one that gives up records AQLM_ERR_TIMEOUT in the workspace's status word,
 // raises a CTA abort flag that the other roles poll, lets its copies and MMAs
 // in flight finish (bounded) and frees its tensor memory; nothing traps.
@@ -88,12 +93,37 @@ struct TcArgs {
     const uint4 *codebooks;
     const __half *scales;
     __half *y;
-    float *partial;      // [splits][T][d_out] when gridDim.y > 1
-    uint32_t *counters;  // [row tiles] when gridDim.y > 1, zero between calls
+    float *partial;      // [tiles][max_segs][T][128] partial sums of split tiles
+    uint32_t *counters;  // [tiles], zero between calls
     int32_t *status;     // AQLM_ERR_TIMEOUT after a wait gave up
     int d_out, G, T;
-    int stages_per_split, n_stages;
+    int n_stages;        // stages of 64 inputs per row
+    int max_segs;        // segments of one tile, at most
+    long long units;     // row tiles x n_stages
 };
+
+// CTA c works on units [unit_start(c), unit_start(c + 1)).
+__device__ __forceinline__ long long unit_start(int c, const TcArgs &a) {
+    return (long long)c * a.units / (long long)gridDim.x;
+}
+// The CTA whose range holds unit u.
+__device__ int cta_of_unit(long long u, const TcArgs &a) {
+    int c = (int)(u * (long long)gridDim.x / a.units);
+    while (c + 1 < (int)gridDim.x && unit_start(c + 1, a) <= u) ++c;
+    while (c > 0 && unit_start(c, a) > u) --c;
+    return c;
+}
+struct Seg {
+    int tile, k0, len;  // stages [k0, k0 + len) of row tile `tile`
+};
+__device__ __forceinline__ Seg seg_at(long long u, long long u_end, const TcArgs &a) {
+    Seg g;
+    g.tile = (int)(u / a.n_stages);
+    g.k0 = (int)(u - (long long)g.tile * a.n_stages);
+    const long long left = u_end - u;
+    g.len = (int)min((long long)(a.n_stages - g.k0), left);
+    return g;
+}
 
 __device__ __forceinline__ uint32_t saddr(const void *p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 __device__ __forceinline__ uint64_t now_ns() {
@@ -211,11 +241,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) gemv_tc_kernel(const __grid_con
     TcBars *bars = reinterpret_cast<TcBars *>(reinterpret_cast<uint8_t *>(cbs) + F::kCbBytes);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tile_row0 = blockIdx.x * kTcRows;
-    const int split = blockIdx.y, splits = gridDim.y;
-    const int st0 = split * a.stages_per_split;
-    const int n_st = min(a.n_stages - st0, a.stages_per_split);  // stages of this CTA (> 0)
-    const int n_boxes = (n_st + F::kStagesPerBox - 1) / F::kStagesPerBox;
+    const long long u_begin = unit_start(blockIdx.x, a), u_end = unit_start(blockIdx.x + 1, a);
+    constexpr int SPB = F::kStagesPerBox;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < F::kStages; ++s) {
@@ -237,9 +264,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) gemv_tc_kernel(const __grid_con
         for (int c = threadIdx.x; c < M * F::K; c += kTcThreads) cbs[c] = a.codebooks[c];
     } else if (threadIdx.x == 32) {  // this CTA's share of the (usually cold) codebooks into L2
         const uint32_t cb_bytes = (uint32_t)M * F::K * 16;
-        const uint32_t n_cta = gridDim.x * gridDim.y;
-        const uint32_t share = ((cb_bytes + n_cta - 1) / n_cta + 255) & ~255u;
-        const uint32_t off = (blockIdx.y * gridDim.x + blockIdx.x) * share;
+        const uint32_t share = ((cb_bytes + gridDim.x - 1) / gridDim.x + 255) & ~255u;
+        const uint32_t off = blockIdx.x * share;
         if (off < cb_bytes)
             prefetch_l2_bulk(reinterpret_cast<const uint8_t *>(a.codebooks) + off, min(share, cb_bytes - off),
                              policy_evict_last());
@@ -259,44 +285,58 @@ __global__ void __launch_bounds__(kTcThreads, 2) gemv_tc_kernel(const __grid_con
         if (lane == 0) {
             // ---- TMA producer: code boxes (weights) first, activations after the grid dependency ----
             int code_issued[kCodeSlots] = {-1, -1};
-            int stage_issued[4] = {-1, -1, -1, -1};
+            int stage_issued[F::kStages];
+            for (int s = 0; s < F::kStages; ++s) stage_issued[s] = -1;
+            int slot_last[kCodeSlots] = {0, 0};  // global index of the last stage of the box in each slot
             bool ok = true;
-            int next_box = 0;
-            auto issue_box = [&](int b) -> bool {
-                const int slot = b % kCodeSlots;
-                const uint32_t par = (uint32_t)((b / kCodeSlots) & 1);
+            // box cursor: box bj of the segment starting at unit bu (global stage index bgi)
+            long long bu = u_begin;
+            int bj = 0, bgi = 0, gb = 0;
+            auto issue_box = [&]() -> bool {
+                const Seg g = seg_at(bu, u_end, a);
+                const int slot = gb % kCodeSlots;
+                const uint32_t par = (uint32_t)((gb / kCodeSlots) & 1);
                 if (!tc_wait(saddr(&bars->code_empty[slot]), par ^ 1, bars, a.status)) return false;
                 const uint32_t full = saddr(&bars->code_full[slot]);
                 mbar_expect_tx(full, kTcRows * kCodeBoxBytes);
                 tma_load_2d(saddr(codes_s + (size_t)slot * kTcRows * kCodeBoxBytes), &tmap_codes,
-                            (st0 + b * F::kStagesPerBox) * F::kStageCodeBytes, tile_row0, full);
+                            (g.k0 + bj * SPB) * F::kStageCodeBytes, g.tile * kTcRows, full);
                 code_issued[slot] = (int)par;
+                slot_last[slot] = bgi + min(g.len, (bj + 1) * SPB) - 1;
+                ++gb;
+                if (++bj * SPB >= g.len) {  // next segment
+                    bu += g.len;
+                    bgi += g.len;
+                    bj = 0;
+                }
                 return true;
             };
-            for (; next_box < n_boxes && next_box < kCodeSlots && ok; ++next_box) ok = issue_box(next_box);
+            while (bu < u_end && gb < kCodeSlots && ok) ok = issue_box();
             grid_dep_wait();
-            for (int i = 0; i < n_st && ok; ++i) {
-                const int s = i % F::kStages;
-                const uint32_t par = (uint32_t)((i / F::kStages) & 1);
-                if (!tc_wait(saddr(&bars->empty[s]), par ^ 1, bars, a.status)) {
-                    ok = false;
-                    break;
+            int gi = 0;
+            for (long long u = u_begin; u < u_end && ok;) {
+                const Seg g = seg_at(u, u_end, a);
+                for (int l = 0; l < g.len && ok; ++l, ++gi) {
+                    const int s = gi % F::kStages;
+                    const uint32_t par = (uint32_t)((gi / F::kStages) & 1);
+                    if (!tc_wait(saddr(&bars->empty[s]), par ^ 1, bars, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t full = saddr(&bars->full[s]);
+                    mbar_expect_tx(full, kXBytes);
+                    tma_load_2d(saddr(ring + (size_t)s * F::kStageBytes + (size_t)M * kTileBytes), &tmap_x,
+                                (g.k0 + l) * kStageK, 0, full);
+                    stage_issued[s] = (int)par;
+                    // box gb takes the slot of box gb - 2, which the decoders release when
+                    // they store that box's last stage: issue it once the activations of
+                    // that stage are on their way (the decoders and the MMAs can always
+                    // get that far), well ahead of its use
+                    while (ok && bu < u_end && slot_last[gb % kCodeSlots] <= gi) ok = issue_box();
                 }
-                const uint32_t full = saddr(&bars->full[s]);
-                mbar_expect_tx(full, kXBytes);
-                tma_load_2d(saddr(ring + (size_t)s * F::kStageBytes + (size_t)M * kTileBytes), &tmap_x,
-                            (st0 + i) * kStageK, 0, full);
-                stage_issued[s] = (int)par;
-                // code box b reuses the slot of box b - 2, which the decoders release
-                // when they store stage (b - 1) * stages-per-box - 1: issue it once
-                // the activations up to that stage are on their way (the decoders
-                // and the MMAs can always get that far), a box and more ahead of use
-                if (next_box < n_boxes && i >= (next_box - 1) * F::kStagesPerBox - 1) {
-                    ok = issue_box(next_box);
-                    ++next_box;
-                }
+                u += g.len;
             }
-            for (; next_box < n_boxes && ok; ++next_box) ok = issue_box(next_box);
+            while (ok && bu < u_end) ok = issue_box();
             // no copy may still be landing in shared memory when the CTA exits
             for (int s = 0; s < kCodeSlots; ++s)
                 if (code_issued[s] >= 0) tc_drain(saddr(&bars->code_full[s]), (uint32_t)code_issued[s]);
@@ -306,159 +346,173 @@ __global__ void __launch_bounds__(kTcThreads, 2) gemv_tc_kernel(const __grid_con
         __syncwarp();
     } else if (warp == 5) {
         if (lane == 0) {
-            // ---- MMA issuer ----
+            // ---- MMA issuer: one accumulator per segment, released by the epilogue ----
             bool ok = true;
-            for (int i = 0; i < n_st; ++i) {
-                const int s = i % F::kStages;
-                const uint32_t par = (uint32_t)((i / F::kStages) & 1);
-                if (!tc_wait(saddr(&bars->full[s]), par, bars, a.status)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t a0 = saddr(ring + (size_t)s * F::kStageBytes);
-                const uint32_t b0 = a0 + (uint32_t)(M * kTileBytes);
+            int gi = 0;
+            for (long long u = u_begin; u < u_end && ok;) {
+                const Seg g = seg_at(u, u_end, a);
+                for (int l = 0; l < g.len; ++l, ++gi) {
+                    const int s = gi % F::kStages;
+                    const uint32_t par = (uint32_t)((gi / F::kStages) & 1);
+                    if (!tc_wait(saddr(&bars->full[s]), par, bars, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = saddr(ring + (size_t)s * F::kStageBytes);
+                    const uint32_t b0 = a0 + (uint32_t)(M * kTileBytes);
 #pragma unroll
-                for (int k = 0; k < kStageK / 16; ++k) {
+                    for (int k = 0; k < kStageK / 16; ++k) {
 #pragma unroll
-                    for (int m = 0; m < M; ++m)
-                        mma_f16(tmem, sw128_desc(a0 + (uint32_t)(m * kTileBytes) + 32 * k), sw128_desc(b0 + 32 * k),
-                                (i > 0 || k > 0 || m > 0) ? 1u : 0u);
+                        for (int m = 0; m < M; ++m)
+                            mma_f16(tmem, sw128_desc(a0 + (uint32_t)(m * kTileBytes) + 32 * k),
+                                    sw128_desc(b0 + 32 * k), (l > 0 || k > 0 || m > 0) ? 1u : 0u);
+                    }
+                    mma_commit(saddr(&bars->empty[s]));
                 }
-                mma_commit(saddr(&bars->empty[s]));
+                if (ok) mma_commit(saddr(&bars->acc_full));
+                u += g.len;
             }
-            if (ok) mma_commit(saddr(&bars->acc_full));
             // tensor memory is freed only after every issued MMA completed
             mma_commit(saddr(&bars->mma_done));
             tc_drain(saddr(&bars->mma_done), 0);
         }
         __syncwarp();
     } else {
-        // ---- decoders (thread = row of the tile), then the epilogue ----
+        // ---- decoders (thread = row of the tile), then each segment's epilogue ----
         const int r = warp * 32 + lane;
-        const int row = tile_row0 + r;
         const uint64_t keep = policy_evict_last();
         bool ok = true;
         uint4 code[kCodeVecs];
         uint4 cwA[kStageGroups][M], cwB[kStageGroups][M];
-        // codes of stage i from its box; returns false on an abandoned wait
-        auto read_codes = [&](int i) -> bool {
-            const int b = i / F::kStagesPerBox, slot = b % kCodeSlots;
-            if (i % F::kStagesPerBox == 0) {
-                if (!tc_wait(saddr(&bars->code_full[slot]), (uint32_t)((b / kCodeSlots) & 1), bars, a.status))
-                    return false;
-            }
-            const uint4 *src = reinterpret_cast<const uint4 *>(codes_s + (size_t)slot * kTcRows * kCodeBoxBytes +
-                                                               (size_t)r * kCodeBoxBytes +
-                                                               (size_t)(i % F::kStagesPerBox) * F::kStageCodeBytes);
+        int gi0 = 0, gb0 = 0, j = 0;  // global stage and box index of the segment's start, segment count
+        bool waited_grid = false;
+        for (long long u = u_begin; u < u_end && ok; ++j) {
+            const Seg g = seg_at(u, u_end, a);
+            const int row = g.tile * kTcRows + r;
+            // codes of local stage l from its box
+            auto read_codes = [&](int l) -> bool {
+                const int gbox = gb0 + l / SPB, slot = gbox % kCodeSlots;
+                if (l % SPB == 0) {
+                    if (!tc_wait(saddr(&bars->code_full[slot]), (uint32_t)((gbox / kCodeSlots) & 1), bars, a.status))
+                        return false;
+                }
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    codes_s + (size_t)slot * kTcRows * kCodeBoxBytes + (size_t)r * kCodeBoxBytes +
+                    (size_t)(l % SPB) * F::kStageCodeBytes);
 #pragma unroll
-            for (int v = 0; v < kCodeVecs; ++v) code[v] = src[v];
-            return true;
-        };
-        auto gather = [&](uint4 (&cw)[kStageGroups][M]) {
+                for (int v = 0; v < kCodeVecs; ++v) code[v] = src[v];
+                return true;
+            };
+            auto gather = [&](uint4 (&cw)[kStageGroups][M]) {
 #pragma unroll
-            for (int q = 0; q < kStageGroups; ++q) {
+                for (int q = 0; q < kStageGroups; ++q) {
 #pragma unroll
-                for (int m = 0; m < M; ++m) {
-                    const uint32_t idx = tc_index<M, B, kCodeVecs>(code, q, m);
-                    if constexpr (B == 8) {
-                        cw[q][m] = cbs[m * F::K + idx];
-                    } else {
-                        cw[q][m] = ld_keep_u4(a.codebooks + (size_t)m * F::K + idx, keep);
+                    for (int m = 0; m < M; ++m) {
+                        const uint32_t idx = tc_index<M, B, kCodeVecs>(code, q, m);
+                        if constexpr (B == 8) {
+                            cw[q][m] = cbs[m * F::K + idx];
+                        } else {
+                            cw[q][m] = ld_keep_u4(a.codebooks + (size_t)m * F::K + idx, keep);
+                        }
                     }
                 }
-            }
-        };
-        // stage i's codewords into its A tiles (groups past the row end as zeros)
-        auto store = [&](const uint4 (&cw)[kStageGroups][M], int i) -> bool {
-            const int s = i % F::kStages;
-            if (!tc_wait(saddr(&bars->empty[s]), (uint32_t)(((i / F::kStages) & 1) ^ 1), bars, a.status)) return false;
-            const int g0 = (st0 + i) * kStageGroups;
-            uint8_t *tile = ring + (size_t)s * F::kStageBytes + (size_t)r * 128;
+            };
+            // local stage l's codewords into its A tiles (groups past the row end as zeros)
+            auto store = [&](const uint4 (&cw)[kStageGroups][M], int l) -> bool {
+                const int gi = gi0 + l, s = gi % F::kStages;
+                if (!tc_wait(saddr(&bars->empty[s]), (uint32_t)(((gi / F::kStages) & 1) ^ 1), bars, a.status))
+                    return false;
+                const int grp0 = (g.k0 + l) * kStageGroups;
+                uint8_t *tile = ring + (size_t)s * F::kStageBytes + (size_t)r * 128;
 #pragma unroll
-            for (int q = 0; q < kStageGroups; ++q) {
-                const bool live = g0 + q < a.G;
+                for (int q = 0; q < kStageGroups; ++q) {
+                    const bool live = grp0 + q < a.G;
 #pragma unroll
-                for (int m = 0; m < M; ++m)
-                    *reinterpret_cast<uint4 *>(tile + (size_t)m * kTileBytes + ((q ^ (r & 7)) << 4)) =
-                        live ? cw[q][m] : make_uint4(0, 0, 0, 0);
-            }
-            fence_async_smem();
-            mbar_arrive(saddr(&bars->full[s]));
-            // the box's codes were consumed by this stage's gathers: its slot may
-            // be refilled (released here, after the shared-memory reads of the
-            // codes have certainly completed and after the proxy fence, not
-            // right after the reads themselves)
-            if (i % F::kStagesPerBox == F::kStagesPerBox - 1 || i == n_st - 1)
-                mbar_arrive(saddr(&bars->code_empty[(i / F::kStagesPerBox) % kCodeSlots]));
-            return true;
-        };
-        if (n_st > 0) {
+                    for (int m = 0; m < M; ++m)
+                        *reinterpret_cast<uint4 *>(tile + (size_t)m * kTileBytes + ((q ^ (r & 7)) << 4)) =
+                            live ? cw[q][m] : make_uint4(0, 0, 0, 0);
+                }
+                fence_async_smem();
+                mbar_arrive(saddr(&bars->full[s]));
+                // the box's codes were consumed by this stage's gathers: release its
+                // slot here (after the gathers that read the code registers and the
+                // proxy fence), not right after the shared-memory reads of the codes
+                if (l % SPB == SPB - 1 || l == g.len - 1)
+                    mbar_arrive(saddr(&bars->code_empty[(gb0 + l / SPB) % kCodeSlots]));
+                return true;
+            };
             ok = read_codes(0);
             if (ok) gather(cwA);
-        }
-        // two stages per trip so both codeword buffers stay in registers
-        for (int i = 0; i < n_st && ok; i += 2) {
-            if (i + 1 < n_st) {
-                ok = read_codes(i + 1);
-                if (ok) gather(cwB);
+            // two stages per trip so both codeword buffers stay in registers
+            for (int l = 0; l < g.len && ok; l += 2) {
+                if (l + 1 < g.len) {
+                    ok = read_codes(l + 1);
+                    if (ok) gather(cwB);
+                }
+                if (ok) ok = store(cwA, l);
+                if (!ok || l + 1 >= g.len) break;
+                if (l + 2 < g.len) {
+                    ok = read_codes(l + 2);
+                    if (ok) gather(cwA);
+                }
+                if (ok) ok = store(cwB, l + 1);
             }
-            if (ok) ok = store(cwA, i);
-            if (!ok || i + 1 >= n_st) break;
-            if (i + 2 < n_st) {
-                ok = read_codes(i + 2);
-                if (ok) gather(cwA);
-            }
-            if (ok) ok = store(cwB, i + 1);
-        }
 
-        // ---- epilogue ----
-        grid_dep_wait();
-        ok = ok && tc_wait(saddr(&bars->acc_full), 0, bars, a.status);
-        ok = __all_sync(0xffffffffu, ok);
-        if (ok) {
+            // ---- the segment's epilogue ----
+            if (!waited_grid) {
+                grid_dep_wait();
+                waited_grid = true;
+            }
+            ok = ok && tc_wait(saddr(&bars->acc_full), (uint32_t)(j & 1), bars, a.status);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
             tc_fence_after();
             uint32_t v[16];
             tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), v);
-            if (row < a.d_out) {
-                if (splits == 1) {
-                    const float sc = __half2float(a.scales[row]);
-                    for (int t = 0; t < a.T; ++t) a.y[(size_t)t * a.d_out + row] = __float2half_rn(__uint_as_float(v[t]) * sc);
-                } else {
-                    for (int t = 0; t < a.T; ++t)
-                        a.partial[((size_t)split * a.T + t) * a.d_out + row] = __uint_as_float(v[t]);
-                }
-            }
-        }
-        if (splits > 1) {
-            // the last CTA of the row tile adds the partials in split order
-            __threadfence();
-            asm volatile("bar.sync 1, %0;" ::"n"(kDecoders) : "memory");
-            if (threadIdx.x == 0) {
-                const int all_ok = !*reinterpret_cast<volatile int *>(&bars->abort_flag);
-                bars->last = all_ok && (atomicAdd(&a.counters[blockIdx.x], 1u) == (uint32_t)(splits - 1));
-            }
-            asm volatile("bar.sync 1, %0;" ::"n"(kDecoders) : "memory");
-            if (bars->last) {
-                __threadfence();
+            tc_fence_before();  // the next segment's MMAs overwrite the accumulator
+            if (g.len == a.n_stages) {
                 if (row < a.d_out) {
                     const float sc = __half2float(a.scales[row]);
-                    for (int t = 0; t < a.T; ++t) {
-                        float sum = 0.f;
-                        for (int s0 = 0; s0 < splits; s0 += 4) {  // 4 partials in flight, added in split order
-                            float p[4];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u)
-                                p[u] = (s0 + u < splits) ? __ldcg(&a.partial[((size_t)(s0 + u) * a.T + t) * a.d_out + row])
-                                                         : 0.f;
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) sum += p[u];
-                        }
-                        a.y[(size_t)t * a.d_out + row] = __float2half_rn(sum * sc);
-                    }
+                    for (int t = 0; t < a.T; ++t)
+                        a.y[(size_t)t * a.d_out + row] = __float2half_rn(__uint_as_float(v[t]) * sc);
                 }
-                if (threadIdx.x == 0) a.counters[blockIdx.x] = 0u;
+            } else {
+                const long long t_u0 = (long long)g.tile * a.n_stages;
+                const int c_lo = cta_of_unit(t_u0, a);
+                const int n_seg = cta_of_unit(t_u0 + a.n_stages - 1, a) - c_lo + 1;
+                float *part = a.partial + (size_t)g.tile * a.max_segs * a.T * kTcRows;
+                for (int t = 0; t < a.T; ++t)
+                    part[((size_t)(blockIdx.x - c_lo) * a.T + t) * kTcRows + r] = __uint_as_float(v[t]);
+                __threadfence();
+                asm volatile("bar.sync 1, %0;" ::"n"(kDecoders) : "memory");
+                if (threadIdx.x == 0)
+                    bars->last = (atomicAdd(&a.counters[g.tile], 1u) == (uint32_t)(n_seg - 1));
+                asm volatile("bar.sync 1, %0;" ::"n"(kDecoders) : "memory");
+                if (bars->last) {  // the last segment of the tile: add all of them in input order
+                    __threadfence();
+                    if (row < a.d_out) {
+                        const float sc = __half2float(a.scales[row]);
+                        for (int t = 0; t < a.T; ++t) {
+                            float sum = 0.f;
+                            for (int s0 = 0; s0 < n_seg; s0 += 4) {  // 4 partials in flight
+                                float pv[4];
+#pragma unroll
+                                for (int q = 0; q < 4; ++q)
+                                    pv[q] = (s0 + q < n_seg) ? __ldcg(&part[((size_t)(s0 + q) * a.T + t) * kTcRows + r]) : 0.f;
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) sum += pv[q];
+                            }
+                            a.y[(size_t)t * a.d_out + row] = __float2half_rn(sum * sc);
+                        }
+                    }
+                    if (threadIdx.x == 0) a.counters[g.tile] = 0u;
+                }
+                asm volatile("bar.sync 1, %0;" ::"n"(kDecoders) : "memory");  // bars->last is reused
             }
+            u += g.len;
+            gi0 += g.len;
+            gb0 += (g.len + SPB - 1) / SPB;
         }
     }
 
@@ -500,28 +554,30 @@ bool encode_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base, uin
 }
 
 struct TcPlan {
-    int tiles;             // row tiles of 128 (gridDim.x)
-    int splits;            // CTAs along the input range (gridDim.y)
-    int stages_per_split;  // stages of 64 inputs per CTA, whole code boxes
-    int n_stages;
+    int ctas;           // persistent CTAs, two per SM at most
+    int tiles;          // row tiles of 128
+    int n_stages;       // stages of 64 inputs per row
+    long long units;    // tiles x n_stages
+    int max_segs;       // segments of one tile, at most
 };
 
-int stages_per_box(const Dims &d) { return kCodeBoxBytes / (kStageGroups * d.M * d.B / 8); }
-
-// About two waves of CTAs (two resident per SM), each a whole number of code
-// boxes and at least two of them.
+// Stream-K plan: two CTAs per SM, each with an equal contiguous range of at
+// least 8 stage units (fewer CTAs for small layers).
 TcPlan plan_tc(const Dims &d, int sms) {
     TcPlan p;
     p.tiles = (d.d_out + kTcRows - 1) / kTcRows;
     p.n_stages = (d.G + kStageGroups - 1) / kStageGroups;
-    const int spb = stages_per_box(d);
-    int splits = (4 * sms + p.tiles - 1) / p.tiles;
-    if (splits < 1) splits = 1;
-    int sps = (p.n_stages + splits - 1) / splits;
-    sps = (sps + spb - 1) / spb * spb;
-    if (sps < 2 * spb) sps = 2 * spb;
-    p.stages_per_split = sps;
-    p.splits = (p.n_stages + sps - 1) / sps;
+    p.units = (long long)p.tiles * p.n_stages;
+    constexpr long long kMinUnits = 8;
+    long long ctas = 2ll * sms;
+    if (ctas > p.units / kMinUnits) ctas = p.units / kMinUnits;
+    if (ctas < 1) ctas = 1;
+    p.ctas = (int)ctas;
+    // a tile's units meet at most floor(n / units-per-CTA) + 2 CTA ranges
+    const long long upc = p.units / ctas;
+    long long segs = p.n_stages / upc + 2;
+    if (segs > ctas) segs = ctas;
+    p.max_segs = (int)segs;
     return p;
 }
 
@@ -532,7 +588,7 @@ cudaError_t launch_tc(const CUtensorMap &mc, const CUtensorMap &mx, const TcArgs
     auto fn = gemv_tc_kernel<M, B>;
     const cudaError_t e = opt_in_dynamic_smem(fn, TcFmt<M, B>::kSmem);
     if (e != cudaSuccess) return e;
-    return launch_kernel(fn, dim3(p.tiles, p.splits), dim3(kTcThreads), TcFmt<M, B>::kSmem, st, true, mc, mx, a);
+    return launch_kernel(fn, dim3(p.ctas), dim3(kTcThreads), TcFmt<M, B>::kSmem, st, true, mc, mx, a);
 }
 
 }  // namespace
@@ -541,17 +597,16 @@ constexpr int kTcMinTokens = 5;
 
 bool gemv_tc_supported(int T) { return T >= kTcMinTokens && T <= AQLM_GEMV_MAX_TOKENS; }
 
-// Workspace: [fp32 partials][arrival counters][status word], the last two
-// zero before a call (the counters only when the input range is split).
+// Workspace: [fp32 partials of split tiles][arrival counters][status word],
+// the last two zero before a call.
 size_t gemv_tc_counter_offset(const Dims &d, int T, int sms) {
     const TcPlan p = plan_tc(d, sms);
-    return p.splits > 1 ? al16((size_t)p.splits * T * d.d_out * sizeof(float)) : 0;
+    return al16((size_t)p.tiles * p.max_segs * T * kTcRows * sizeof(float));
 }
 
 size_t gemv_tc_workspace_bytes(const Dims &d, int T, int sms) {
     const TcPlan p = plan_tc(d, sms);
-    const size_t counters = p.splits > 1 ? al16((size_t)p.tiles * sizeof(uint32_t)) : 0;
-    return gemv_tc_counter_offset(d, T, sms) + counters + 16;
+    return gemv_tc_counter_offset(d, T, sms) + al16((size_t)p.tiles * sizeof(uint32_t)) + 16;
 }
 
 size_t gemv_tc_status_offset(const Dims &d, int T, int sms) { return gemv_tc_workspace_bytes(d, T, sms) - 16; }
@@ -571,13 +626,14 @@ cudaError_t launch_gemv_tc(const void *codes, const uint16_t *codebooks, const u
     a.scales = reinterpret_cast<const __half *>(scales);
     a.y = reinterpret_cast<__half *>(y);
     a.partial = reinterpret_cast<float *>(ws);
-    a.counters = p.splits > 1 ? reinterpret_cast<uint32_t *>(ws + gemv_tc_counter_offset(d, tokens, sms)) : nullptr;
+    a.counters = reinterpret_cast<uint32_t *>(ws + gemv_tc_counter_offset(d, tokens, sms));
     a.status = reinterpret_cast<int32_t *>(ws + gemv_tc_status_offset(d, tokens, sms));
     a.d_out = d.d_out;
     a.G = d.G;
     a.T = tokens;
-    a.stages_per_split = p.stages_per_split;
     a.n_stages = p.n_stages;
+    a.max_segs = p.max_segs;
+    a.units = p.units;
     if (d.M == 1) return launch_tc<1, 16>(mc, mx, a, p, st);
     if (d.B == 8) return launch_tc<2, 8>(mc, mx, a, p, st);
     return launch_tc<2, 16>(mc, mx, a, p, st);
