@@ -1,7 +1,7 @@
 // gemv.cu -- host side of the decode-time product: the kernel choice and the
-// workspace layout.  1..4 tokens: gemv_rows.cu (coalesced row streaming on the
+// workspace layout.  1..3 tokens: gemv_rows.cu (coalesced row streaming on the
 // CUDA cores, the input range split when the activations do not fit on chip).
-// 5..16 tokens: gemv_tc.cu (the weights decoded into shared memory for
+// 4..16 tokens: gemv_tc.cu (the weights decoded into shared memory for
 // tcgen05 tensor-core MMAs).  Both launch with programmatic dependent launch.
 #include "common.cuh"
 

@@ -1,4 +1,4 @@
-// gemv_tc.cu -- layer product for 5..16 tokens on the 5th-generation tensor
+// gemv_tc.cu -- layer product for 4..16 tokens on the 5th-generation tensor
 // cores, decoding the weights into shared memory on the fly.
 //
 // "The AQLM Quantization Algorithm, Explained", section "What is
@@ -593,7 +593,7 @@ cudaError_t launch_tc(const CUtensorMap &mc, const CUtensorMap &mx, const TcArgs
 
 }  // namespace
 
-constexpr int kTcMinTokens = 5;
+constexpr int kTcMinTokens = 4;
 
 bool gemv_tc_supported(int T) { return T >= kTcMinTokens && T <= AQLM_GEMV_MAX_TOKENS; }
 

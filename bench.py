@@ -482,12 +482,12 @@ def _gemv_detail(r, peaks, T=1):
     if gr is not None:
         out["gather_frac"] = gr["frac"]
     if T > 1:
-        # multiply-adds of the product per second; up to 4 tokens they run on the
-        # CUDA cores (fraction of the FMA peak), from 5 on the tensor cores, where
+        # multiply-adds of the product per second; up to 3 tokens they run on the
+        # CUDA cores (fraction of the FMA peak), from 4 on the tensor cores, where
         # the codeword gathers (gather_frac) are what binds
         mac_t = spec.d_out * spec.groups * 8 * T / (r["us_per_layer"] * 1e-6) / 1e12
         out["mac_tera_per_s"] = round(mac_t, 2)
-        if T <= 4:
+        if T <= 3:
             out["path"] = "row kernel, CUDA cores"
             out["fma_frac"] = round(mac_t / FMA_PEAK_TERA_PER_S, 4)
         else:

@@ -99,12 +99,12 @@ typedef struct {
  *   x: [tokens][d_in] fp16.   y: [tokens][d_out] fp16 (written).
  *   workspace/workspace_bytes: device scratch for fp32 partial sums and
  *   arrival counters, used when a row's input range is split over several
- *   CTAs, and (5 to 16 tokens) a status word; aqlm_gemv_workspace_bytes()
+ *   CTAs, and (4 to 16 tokens) a status word; aqlm_gemv_workspace_bytes()
  *   gives the size for this device (0 = none needed, NULL allowed).  Too
  *   small or not 16-byte aligned -> AQLM_ERR_WORKSPACE.  The workspace must be
  *   zero-filled before its first use; every completed call leaves it ready for
  *   the next one.  Calls that share a workspace must not overlap on the GPU.
- * Up to 4 tokens the kernels have no device waits.  From 5 tokens the
+ * Up to 3 tokens the kernels have no device waits.  From 4 tokens the
  * product runs on the tensor cores with producer/consumer waits inside each
  * CTA, each bounded in time: a wait that gives up records AQLM_ERR_TIMEOUT in
  * the workspace's status word (y is then not valid, and the workspace must be
@@ -126,7 +126,7 @@ AQLM_API size_t aqlm_gemv_workspace_bytes(aqlm_shape shape, int32_t tokens);
  * aqlm_gemv_check -- synchronise `stream` and return the status that the
  * aqlm_gemv calls with this shape, token count and workspace recorded:
  * AQLM_OK, or AQLM_ERR_TIMEOUT (the word is then cleared).  Paths without
- * device waits (up to 4 tokens) have no status word: AQLM_OK after the
+ * device waits (up to 3 tokens) have no status word: AQLM_OK after the
  * synchronisation.  Not a counterpart of anything on the pages: library
  * plumbing for the bounded waits.
  */

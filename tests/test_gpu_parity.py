@@ -110,17 +110,17 @@ def test_gemv_split_input_range(M, B, T):
     _gemv_case(M, B, 96, 4160, T, seed=20 + T)
 
 
-@pytest.mark.parametrize("M,B,T,d_in", [(1, 16, 1, 82112), (2, 16, 1, 82144), (1, 16, 2, 28736)]
-                         + [(m, b, 3, 28736) for m, b in FORMATS] + [(m, b, 4, 20544) for m, b in FORMATS])
+@pytest.mark.parametrize("M,B,T,d_in", [(1, 16, 1, 82112), (2, 16, 1, 82144)]
+                         + [(m, b, 3, 28736) for m, b in FORMATS] + [(m, b, 2, 20544) for m, b in FORMATS])
 def test_gemv_rows_split_input_range(M, B, T, d_in):
-    # up to 4 tokens whose activations exceed the row kernel's 32 KiB budget:
-    # the input range is split in slices of whole 32-chunk lane slots (4 to 11
+    # up to 3 tokens whose activations exceed the row kernel's 32 KiB budget:
+    # the input range is split in slices of whole 32-chunk lane slots (3 to 11
     # of them here, the last one ragged), partial sums meet in the workspace;
     # 100 rows leave some warps without a row
     _gemv_case(M, B, 100, d_in, T, seed=30 + T)
 
 
-@pytest.mark.parametrize("T", [5, 16])
+@pytest.mark.parametrize("T", [4, 5, 16])
 def test_gemv_tensor_core_ragged_stage(T):
     # 2x16 with 516 groups: the last 8-group stage of the tensor-core path holds
     # 4 groups (the rest are zeros in the decoded tile); 300 rows: 3 row tiles,
@@ -191,6 +191,7 @@ FULL_GEMV = [
     ("2x8 4096x11008", 4096, 11008, 2, 8, 1),
     ("1x16 28672x8192 T4", 28672, 8192, 1, 16, 4),
     ("1x16 8192x28672 T4", 8192, 28672, 1, 16, 4),
+    ("1x16 8192x28672 T3", 8192, 28672, 1, 16, 3),
     ("1x16 8192x28672 T16", 8192, 28672, 1, 16, 16),
     ("2x16 8192x8192", 8192, 8192, 2, 16, 1),
     ("2x8 256x512", 256, 512, 2, 8, 1),

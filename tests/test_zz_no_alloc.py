@@ -24,11 +24,11 @@ from synth import LayerSpec, make_layer
 
 pytestmark = pytest.mark.gpu
 
-# shapes whose product needs scratch: a 4-token row-kernel product whose
+# shapes whose product needs scratch: a 3-token row-kernel product whose
 # activations are split into slices (7 x 64 chunks of 28672 inputs),
 # products of several tokens split over the input range to fill the SMs, and
 # a 16-token product split because its activations do not fit on chip at once
-CASES = [(1024, 28672, 2, 8, 4), (2048, 4096, 2, 8, 6), (1024, 4096, 1, 16, 16), (512, 4160, 2, 16, 8)]
+CASES = [(1024, 28672, 2, 8, 3), (2048, 4096, 2, 8, 6), (1024, 4096, 1, 16, 16), (512, 4160, 2, 16, 8)]
 
 
 def _call_noalloc(lib, d, x, y):
@@ -59,14 +59,14 @@ def test_noalloc_matches_gemv_on_two_calls(cuda_device, d_out, d_in, M, B, T):
 
 def test_noalloc_rejects_scratch_beyond_its_maximum(cuda_device):
     lib = ac.load_library()
-    # 4 tokens of 28672 inputs: seven activation slices, 7 x 4 x 131072 fp32
-    # partial sums (14.7 MB), far more than the 8 MiB built in
+    # 3 tokens of 28672 inputs on the row kernel: seven activation slices,
+    # 7 x 3 x 131072 fp32 partial sums (11 MB), more than the 8 MiB built in
     shape = ac.Shape(131072, 28672, 8, 1, 16)
-    assert lib.aqlm_gemv_workspace_bytes(shape, 4) > lib.aqlm_gemv_noalloc_max_scratch_bytes()
+    assert lib.aqlm_gemv_workspace_bytes(shape, 3) > lib.aqlm_gemv_noalloc_max_scratch_bytes()
     codes = torch.zeros(16, dtype=torch.uint8, device=DEV)   # never read: the call is rejected first
     x = torch.zeros(16, 16, dtype=torch.float16, device=DEV)
     y = torch.zeros(16, 16, dtype=torch.float16, device=DEV)
     p = ctypes.c_void_p(codes.data_ptr())
-    st = lib.aqlm_gemv_noalloc(p, p, p, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()), 4, shape,
+    st = lib.aqlm_gemv_noalloc(p, p, p, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()), 3, shape,
                                ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == ac.AQLM_ERR_WORKSPACE
