@@ -22,10 +22,12 @@
 // no waiting) adds them in input order (deterministic), scales and stores.
 // One CTA has 6 warps:
 //   warps 0-3  decoders, one thread per row: read the row's codes of the
-//              stage from the code tile, gather the codewords (1x16 / 2x16
-//              through L1/L2 with an evict-last policy, 2x8 from shared
-//              memory) one stage ahead, and write them into the stage's A
-//              tile in the 128-byte-swizzled K-major layout that the MMA reads;
+//              stage from the code tile and copy each codeword straight from
+//              the codebook (through L1, L2 evict-last) into the stage's A tile
+//              in the 128-byte-swizzled K-major layout that the MMA reads, with
+//              16-byte cp.async copies; the stage's full barrier counts a
+//              thread's arrival when its copies have landed, so a decoder never
+//              waits for its gathers and runs up to the ring depth ahead;
 //              after the last stage they are the epilogue (tcgen05.ld of their
 //              TMEM lane quarter, scale, fp16 store or fp32 partials);
 //   warp 4     one thread issues the TMA loads: code tiles (64 bytes x 128
@@ -69,12 +71,14 @@ struct TcFmt {
     static constexpr int kCodeBytesPerGroup = M * B / 8;
     static constexpr int kStageCodeBytes = kStageGroups * kCodeBytesPerGroup;   // 16 or 32
     static constexpr int kStagesPerBox = kCodeBoxBytes / kStageCodeBytes;       // 4 or 2
-    static constexpr int kStages = (M == 1) ? 4 : 2;                            // A/B ring depth
+    // A/B ring depth (4 stages of 18 KiB for one codebook, 2 of 34 KiB for two)
+    // and CTAs per SM (measured on B200: a 3-stage ring with three CTAs per SM
+    // ran 1.6x slower than this)
+    static constexpr int kStages = (M == 1) ? 4 : 2;
+    static constexpr int kCtasPerSm = 2;
     static constexpr int kStageBytes = M * kTileBytes + kXBytes;
-    static constexpr int kCbBytes = (B == 8) ? M * K * 16 : 0;
-    // ring (1024-aligned), code slots, 2x8 codebooks, barriers, + alignment slack
-    static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + (size_t)kCodeSlots * kTcRows * kCodeBoxBytes +
-                                    kCbBytes + 256;
+    // ring (1024-aligned), code slots, barriers, + alignment slack
+    static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + (size_t)kCodeSlots * kTcRows * kCodeBoxBytes + 256;
 };
 
 struct TcBars {
@@ -201,6 +205,18 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// 16-byte asynchronous global -> shared copy through L1 with an L2 cache
+// policy; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async16_keep(uint32_t dst, const void *src, uint32_t src_bytes, uint64_t pol) {
+    asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes), "l"(pol)
+                 : "memory");
+}
+// Arrive on an mbarrier once all of this thread's earlier cp.async copies have
+// completed (the arrival is part of the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
@@ -227,7 +243,7 @@ __device__ __forceinline__ uint32_t tc_index(const uint4 (&c)[V], int q, int m) 
 }
 
 template <int M, int B>
-__global__ void __launch_bounds__(kTcThreads, 2) gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_codes,
+__global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm) gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_codes,
                                                                const __grid_constant__ CUtensorMap tmap_x,
                                                                const TcArgs a) {
     using F = TcFmt<M, B>;
@@ -237,8 +253,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) gemv_tc_kernel(const __grid_con
     uint8_t *smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
     uint8_t *ring = smem;                                                       // [stage][M A tiles | B tile]
     uint8_t *codes_s = ring + (size_t)F::kStages * F::kStageBytes;              // [slot][128 rows][64 B]
-    uint4 *cbs = reinterpret_cast<uint4 *>(codes_s + (size_t)kCodeSlots * kTcRows * kCodeBoxBytes);  // 2x8
-    TcBars *bars = reinterpret_cast<TcBars *>(reinterpret_cast<uint8_t *>(cbs) + F::kCbBytes);
+    TcBars *bars = reinterpret_cast<TcBars *>(codes_s + (size_t)kCodeSlots * kTcRows * kCodeBoxBytes);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long u_begin = unit_start(blockIdx.x, a), u_end = unit_start(blockIdx.x + 1, a);
@@ -260,9 +275,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) gemv_tc_kernel(const __grid_con
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_codes)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
     }
-    if constexpr (B == 8) {
-        for (int c = threadIdx.x; c < M * F::K; c += kTcThreads) cbs[c] = a.codebooks[c];
-    } else if (threadIdx.x == 32) {  // this CTA's share of the (usually cold) codebooks into L2
+    if (threadIdx.x == 32) {  // this CTA's share of the (usually cold) codebooks into L2
         const uint32_t cb_bytes = (uint32_t)M * F::K * 16;
         const uint32_t share = ((cb_bytes + gridDim.x - 1) / gridDim.x + 255) & ~255u;
         const uint32_t off = blockIdx.x * share;
@@ -358,6 +371,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) gemv_tc_kernel(const __grid_con
                         ok = false;
                         break;
                     }
+                    // the A tiles were written by cp.async (generic proxy): order them
+                    // before the tensor cores' (async proxy) reads
+                    fence_async_smem();
                     tc_fence_after();
                     const uint32_t a0 = saddr(ring + (size_t)s * F::kStageBytes);
                     const uint32_t b0 = a0 + (uint32_t)(M * kTileBytes);
@@ -383,80 +399,52 @@ __global__ void __launch_bounds__(kTcThreads, 2) gemv_tc_kernel(const __grid_con
         const int r = warp * 32 + lane;
         const uint64_t keep = policy_evict_last();
         bool ok = true;
-        uint4 code[kCodeVecs];
-        uint4 cwA[kStageGroups][M], cwB[kStageGroups][M];
         int gi0 = 0, gb0 = 0, j = 0;  // global stage and box index of the segment's start, segment count
         bool waited_grid = false;
         for (long long u = u_begin; u < u_end && ok; ++j) {
             const Seg g = seg_at(u, u_end, a);
             const int row = g.tile * kTcRows + r;
-            // codes of local stage l from its box
-            auto read_codes = [&](int l) -> bool {
+            for (int l = 0; l < g.len; ++l) {
+                // the row's codes of local stage l, from its box
                 const int gbox = gb0 + l / SPB, slot = gbox % kCodeSlots;
-                if (l % SPB == 0) {
-                    if (!tc_wait(saddr(&bars->code_full[slot]), (uint32_t)((gbox / kCodeSlots) & 1), bars, a.status))
-                        return false;
+                if (l % SPB == 0 &&
+                    !tc_wait(saddr(&bars->code_full[slot]), (uint32_t)((gbox / kCodeSlots) & 1), bars, a.status)) {
+                    ok = false;
+                    break;
                 }
-                const uint4 *src = reinterpret_cast<const uint4 *>(
-                    codes_s + (size_t)slot * kTcRows * kCodeBoxBytes + (size_t)r * kCodeBoxBytes +
-                    (size_t)(l % SPB) * F::kStageCodeBytes);
+                uint4 code[kCodeVecs];
+                const uint4 *src = reinterpret_cast<const uint4 *>(codes_s + (size_t)slot * kTcRows * kCodeBoxBytes +
+                                                                   (size_t)r * kCodeBoxBytes +
+                                                                   (size_t)(l % SPB) * F::kStageCodeBytes);
 #pragma unroll
                 for (int v = 0; v < kCodeVecs; ++v) code[v] = src[v];
-                return true;
-            };
-            auto gather = [&](uint4 (&cw)[kStageGroups][M]) {
-#pragma unroll
-                for (int q = 0; q < kStageGroups; ++q) {
-#pragma unroll
-                    for (int m = 0; m < M; ++m) {
-                        const uint32_t idx = tc_index<M, B, kCodeVecs>(code, q, m);
-                        if constexpr (B == 8) {
-                            cw[q][m] = cbs[m * F::K + idx];
-                        } else {
-                            cw[q][m] = ld_keep_u4(a.codebooks + (size_t)m * F::K + idx, keep);
-                        }
-                    }
-                }
-            };
-            // local stage l's codewords into its A tiles (groups past the row end as zeros)
-            auto store = [&](const uint4 (&cw)[kStageGroups][M], int l) -> bool {
+                // the stage's A tiles are free once the MMAs of its previous use are done
                 const int gi = gi0 + l, s = gi % F::kStages;
-                if (!tc_wait(saddr(&bars->empty[s]), (uint32_t)(((gi / F::kStages) & 1) ^ 1), bars, a.status))
-                    return false;
+                if (!tc_wait(saddr(&bars->empty[s]), (uint32_t)(((gi / F::kStages) & 1) ^ 1), bars, a.status)) {
+                    ok = false;
+                    break;
+                }
+                // codewords copied straight from the codebooks into the swizzled A
+                // tiles (zeros past the row end); the stage's full barrier counts
+                // this thread's arrival when all of its copies have landed
                 const int grp0 = (g.k0 + l) * kStageGroups;
-                uint8_t *tile = ring + (size_t)s * F::kStageBytes + (size_t)r * 128;
+                const uint32_t tile = saddr(ring + (size_t)s * F::kStageBytes + (size_t)r * 128);
 #pragma unroll
                 for (int q = 0; q < kStageGroups; ++q) {
-                    const bool live = grp0 + q < a.G;
+                    const uint32_t bytes = (grp0 + q < a.G) ? 16u : 0u;
 #pragma unroll
                     for (int m = 0; m < M; ++m)
-                        *reinterpret_cast<uint4 *>(tile + (size_t)m * kTileBytes + ((q ^ (r & 7)) << 4)) =
-                            live ? cw[q][m] : make_uint4(0, 0, 0, 0);
+                        cp_async16_keep(tile + (uint32_t)(m * kTileBytes) + (uint32_t)((q ^ (r & 7)) << 4),
+                                        a.codebooks + (size_t)m * F::K + tc_index<M, B, kCodeVecs>(code, q, m), bytes,
+                                        keep);
                 }
-                fence_async_smem();
-                mbar_arrive(saddr(&bars->full[s]));
-                // the box's codes were consumed by this stage's gathers: release its
-                // slot here (after the gathers that read the code registers and the
-                // proxy fence), not right after the shared-memory reads of the codes
-                if (l % SPB == SPB - 1 || l == g.len - 1)
-                    mbar_arrive(saddr(&bars->code_empty[(gb0 + l / SPB) % kCodeSlots]));
-                return true;
-            };
-            ok = read_codes(0);
-            if (ok) gather(cwA);
-            // two stages per trip so both codeword buffers stay in registers
-            for (int l = 0; l < g.len && ok; l += 2) {
-                if (l + 1 < g.len) {
-                    ok = read_codes(l + 1);
-                    if (ok) gather(cwB);
+                cp_async_arrive_noinc(saddr(&bars->full[s]));
+                // the box's codes were read into registers and used above: its slot
+                // may be refilled once the last stage of the box is issued
+                if (l % SPB == SPB - 1 || l == g.len - 1) {
+                    fence_async_smem();
+                    mbar_arrive(saddr(&bars->code_empty[slot]));
                 }
-                if (ok) ok = store(cwA, l);
-                if (!ok || l + 1 >= g.len) break;
-                if (l + 2 < g.len) {
-                    ok = read_codes(l + 2);
-                    if (ok) gather(cwA);
-                }
-                if (ok) ok = store(cwB, l + 1);
             }
 
             // ---- the segment's epilogue ----
@@ -561,15 +549,17 @@ struct TcPlan {
     int max_segs;       // segments of one tile, at most
 };
 
-// Stream-K plan: two CTAs per SM, each with an equal contiguous range of at
-// least 8 stage units (fewer CTAs for small layers).
+// Stream-K plan: as many CTAs as are resident at once (two per SM), each
+// with an equal contiguous range of at least 8 stage units (fewer CTAs for
+// small layers).
 TcPlan plan_tc(const Dims &d, int sms) {
     TcPlan p;
+    const int per_sm = (d.M == 1) ? TcFmt<1, 16>::kCtasPerSm : TcFmt<2, 16>::kCtasPerSm;
     p.tiles = (d.d_out + kTcRows - 1) / kTcRows;
     p.n_stages = (d.G + kStageGroups - 1) / kStageGroups;
     p.units = (long long)p.tiles * p.n_stages;
     constexpr long long kMinUnits = 8;
-    long long ctas = 2ll * sms;
+    long long ctas = (long long)per_sm * sms;
     if (ctas > p.units / kMinUnits) ctas = p.units / kMinUnits;
     if (ctas < 1) ctas = 1;
     p.ctas = (int)ctas;
