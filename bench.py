@@ -237,10 +237,31 @@ def bench_gemv(ac, spec, T, steps, warmup, l2_bytes, n_launch=STEP_LAYERS, dist=
     g = gemv_graph(ac, layers, n_launch, ys, ws)
     ms = time_replays(g, steps, warmup, dist)
     us_layer = ms * 1e3 / (steps * n_launch)
-    launches_per_layer = 1 if need == 0 else 2
     del g
+    # one kernel launch per layer product (split reductions happen inside the kernel)
     return {"us_per_layer": us_layer, "bytes_per_layer": algo_bytes(spec, T), "copies": R,
-            "launches": steps * n_launch * launches_per_layer, "ms": ms, "layers": layers, "ws": ws}
+            "launches": steps * n_launch, "ms": ms, "layers": layers, "ws": ws}
+
+
+def single_call_us(ac, bench, reps=50):
+    """Latency of one aqlm_gemv call on its own (not in a graph, no neighbour to
+    overlap with): CUDA events around each call, median over `reps` calls that
+    cycle over the layer copies."""
+    import torch
+    layers, ws = bench["layers"], bench["ws"]
+    y = torch.empty((layers.T, layers.spec.d_out), dtype=torch.float16, device="cuda")
+    out = []
+    for i in range(reps + 5):
+        d = layers.copies[i % layers.R]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], layers.x, y=y, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 5:
+            out.append(e0.elapsed_time(e1) * 1e3)
+    return statistics.median(out)
 
 
 def bench_block(ac, fmt, steps, warmup, l2_bytes):
@@ -417,6 +438,7 @@ def run_gpu(args):
                     "us_gemm": round(p["us_gemm"], 2), "gemm_tflops": round(p["gemm_tflops"], 1)}
                 torch.cuda.empty_cache()
     e2e = e2e_gemv(ac, head, max(3, args.steps // 4), 2)
+    single_us = single_call_us(ac, head)
     sampler.__exit__(None, None, None)
     clocks = sampler.summary()
 
@@ -431,6 +453,7 @@ def run_gpu(args):
                    "l2_policy": "inputs larger than L2: each step cycles over copies totalling > 3x L2",
                    "parallelism": f"replicas x{world}"},
         "us_per_layer": round(head["us_per_layer"], 4),
+        "single_call_us": round(single_us, 3),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4),
                      "traffic": recorded_traffic("gemv 1x16 4096x4096 T1"),
