@@ -97,6 +97,21 @@ __device__ __forceinline__ void half8_to_float8(const uint4 &v, float *f) {
     }
 }
 
+// e += lo(c) * lo(x), o += hi(c) * hi(x): the fp16 halves of c and x
+// multiplied and accumulated in fp32 by the mixed-precision fma of sm_100
+// (PTX `fma.rn.f32.f16`).  The product of two fp16 values is exact in fp32,
+// so this rounds exactly like converting both to fp32 first and fusing the
+// multiply-add, without the conversions.
+__device__ __forceinline__ void fma2_f16_f32(float &e, float &o, uint32_t c, uint32_t x) {
+    asm("{.reg .f16 cl, ch, xl, xh;\n\t"
+        "mov.b32 {cl, ch}, %2;\n\t"
+        "mov.b32 {xl, xh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, cl, xl, %0;\n\t"
+        "fma.rn.f32.f16 %1, ch, xh, %1;}"
+        : "+f"(e), "+f"(o)
+        : "r"(c), "r"(x));
+}
+
 // The kernels here hold at most a few bytes of static shared memory; opt in
 // to the dynamic size whenever static + dynamic could pass the 48 KiB that a
 // launch gets without the attribute.

@@ -36,8 +36,9 @@
 namespace aqlm {
 namespace {
 
+// Fewest warps per CTA (the 1x16 / 2x16 kernels; 2x8 runs 16): the
+// workspace keeps one arrival counter per kRowWarps rows.
 constexpr int kRowWarps = 8;
-constexpr int kRowThreads = kRowWarps * 32;
 
 struct RowArgs {
     const uint8_t *codes;
@@ -56,7 +57,20 @@ struct RowFmt {
     static constexpr int K = 1 << B;
     static constexpr int GPC = 16 / (M * B / 8);  // groups per 16-byte chunk
     static constexpr bool kSmemCodebook = (B == 8);
+    // 2x8 runs 16 warps (64 registers each) in one CTA per SM, 1x16 / 2x16
+    // 8 warps (their codewords of two items ahead take 64 more registers).
+    static constexpr int kWarps = kSmemCodebook ? 16 : 8;
+    static constexpr int kThreads = kWarps * 32;
 };
+
+// 2x8 codebooks are held in shared memory as 8 copies, copy p in bank quad p
+// (banks 4p..4p+3): codeword e of copy p is 16-byte word 8e + p.  Lane l
+// reads copy l & 7, so the 8 lanes of each quarter warp touch 8 different
+// bank quads whatever their codes are -- a warp's 16-byte gathers take 4
+// shared-memory wavefronts, the minimum for 512 bytes, where one shared copy
+// takes about twice that from bank conflicts.
+constexpr int kCbCopies = 8;  // one per bank quad; the indexing below uses << 3 and & 7
+static_assert(kCbCopies == 8, "copy index is lane & 7");
 
 template <int M, int B>
 __device__ __forceinline__ uint32_t code_index(const uint4 &ch, int q, int m) {
@@ -71,7 +85,7 @@ __device__ __forceinline__ uint32_t code_index(const uint4 &ch, int q, int m) {
 }
 
 template <int M, int B, int T>
-__global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a) {
+__global__ void __launch_bounds__(RowFmt<M, B>::kThreads) gemv_rows_kernel(const RowArgs a) {
     using F = RowFmt<M, B>;
     constexpr int GPC = F::GPC;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -81,14 +95,17 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
     const int c0 = split * xstride;                       // first chunk of this CTA's slice
     const int n_chunks = min(a.G / GPC - c0, xstride);    // chunks in the slice
     uint4 *xs = reinterpret_cast<uint4 *>(smem);          // [T][GPC][xstride] groups of 8 fp16
-    uint4 *cbs = xs + (size_t)T * GPC * xstride;          // 2x8: [M][256] codewords
+    uint4 *cbs = xs + (size_t)T * GPC * xstride;          // 2x8: [M][256][8 copies] codewords
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // this CTA's rows: an equal contiguous share [r0, r1) of d_out, so that
-    // every SM gets the same number of rows whichever CTAs it holds
+    // every SM gets the same number of rows whichever CTAs it holds; warp w
+    // owns rows r0 + w + 8 j, j < n_rows
     const int r0 = (int)((int64_t)blockIdx.x * a.d_out / gridDim.x);
     const int r1 = (int)((int64_t)(blockIdx.x + 1) * a.d_out / gridDim.x);
+    const int n_rows = r1 - r0 > warp ? (r1 - r0 - warp + F::kWarps - 1) / F::kWarps : 0;
     const int cpw = (n_chunks + 31) / 32;  // chunk slots per lane per row
+    const int n_items = n_rows * cpw;      // item k = (row j = k / cpw, slot k % cpw)
     const uint64_t stream_pol = policy_evict_first();
     const uint64_t keep_pol = policy_evict_last();
 
@@ -102,42 +119,58 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
                                  keep_pol);
         }
     } else {
-        for (int c = threadIdx.x; c < M * F::K; c += kRowThreads) cbs[c] = a.codebooks[c];
+        for (int c = threadIdx.x; c < M * F::K * kCbCopies; c += F::kThreads) cbs[c] = a.codebooks[c >> 3];
     }
+    // the scales of the warp's first 32 rows, lane j holding row j's (weights:
+    // read before the grid-dependency wait, off the critical path)
+    const float scale_j = (splits == 1 && lane < n_rows) ? __half2float(a.scales[r0 + warp + F::kWarps * lane]) : 0.f;
 
-    // item k of this warp: row r0 + warp + 8 * (k / cpw), chunk slot k % cpw
-    auto item_row = [&](int k) { return r0 + warp + kRowWarps * (k / cpw); };
-    auto load_code = [&](int k) -> uint4 {
-        const int r = item_row(k);
-        const int c = lane + 32 * (k % cpw);
-        if (r < r1 && c < n_chunks)
-            return ld_stream_u4(a.codes + (size_t)r * a.row_bytes + (size_t)(c0 + c) * 16, stream_pol);
+    // (row, slot) of an item, advanced without divisions
+    struct Item {
+        int j, s;
+    };
+    auto next = [&](Item it) -> Item {
+        if (++it.s == cpw) {
+            it.s = 0;
+            ++it.j;
+        }
+        return it;
+    };
+    auto lane_live = [&](Item it) { return it.j < n_rows && lane + 32 * it.s < n_chunks; };
+    auto load_code = [&](Item it) -> uint4 {
+        if (lane_live(it))
+            return ld_stream_u4(a.codes + (size_t)(r0 + warp + F::kWarps * it.j) * a.row_bytes +
+                                    (size_t)(c0 + lane + 32 * it.s) * 16,
+                                stream_pol);
         return make_uint4(0, 0, 0, 0);
     };
-    auto gather = [&](const uint4 &ch, int k, uint4 (&cw)[GPC][M]) {
-        const bool live = item_row(k) < r1 && lane + 32 * (k % cpw) < n_chunks;
+    auto gather = [&](const uint4 &ch, Item it, uint4 (&cw)[GPC][M]) {
+        const bool live = lane_live(it);
 #pragma unroll
         for (int q = 0; q < GPC; ++q) {
 #pragma unroll
-            for (int m = 0; m < M; ++m) {
-                const uint32_t idx = code_index<M, B>(ch, q, m);
-                if constexpr (F::kSmemCodebook) {
-                    cw[q][m] = cbs[m * F::K + idx];
-                } else {
-                    cw[q][m] = live ? ld_keep_u4(a.codebooks + (size_t)m * F::K + idx, keep_pol) : make_uint4(0, 0, 0, 0);
-                }
-            }
+            for (int m = 0; m < M; ++m)
+                cw[q][m] = live ? ld_keep_u4(a.codebooks + (size_t)m * F::K + code_index<M, B>(ch, q, m), keep_pol)
+                                : make_uint4(0, 0, 0, 0);
         }
     };
 
-    uint4 cwA[GPC][M], cwB[GPC][M];
-    uint4 ch_next = load_code(1);
-    const uint4 ch0 = load_code(0);
+    // Weights only before the grid-dependency wait: the codes of the first
+    // four items and (1x16 / 2x16) the codewords of the first two.
+    Item it0 = {0, 0};
+    Item it1 = next(it0);
+    Item it2 = next(it1);
+    Item it3 = next(it2);
+    uint4 cwA[F::kSmemCodebook ? 1 : GPC][M], cwB[F::kSmemCodebook ? 1 : GPC][M];
+    uint4 ch0 = load_code(it0), ch1 = load_code(it1), ch2 = load_code(it2), ch3 = load_code(it3);
+    if constexpr (!F::kSmemCodebook) {
+        gather(ch0, it0, cwA);
+        gather(ch1, it1, cwB);
+    }
+    grid_dep_wait();
     {
-        if constexpr (!F::kSmemCodebook) gather(ch0, 0, cwA);
-        grid_dep_wait();
         const int ng = n_chunks * GPC;  // groups of the slice
-        for (int i = threadIdx.x; i < T * ng; i += kRowThreads) {  // stage x, transposed by chunk
+        for (int i = threadIdx.x; i < T * ng; i += F::kThreads) {  // stage x, transposed by chunk
             const int t = i / ng, g = i - t * ng;
             const int c = g / GPC, q = g - c * GPC;
             xs[((size_t)t * GPC + q) * xstride + c] =
@@ -147,86 +180,99 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
     }
     grid_dep_launch();
 
-    float acc[T];
+    // two fp32 chains per token (even and odd lanes of the groups)
+    float acc[T], acc2[T];
 #pragma unroll
-    for (int t = 0; t < T; ++t) acc[t] = 0.f;
+    for (int t = 0; t < T; ++t) acc[t] = acc2[t] = 0.f;
     // y for the item's row once its last chunk slot has been added
-    auto finish_item = [&](int k) {
-        if (k % cpw != cpw - 1) return;
-        const int r = item_row(k);
+    auto finish_item = [&](Item it) {
+        if (it.s != cpw - 1) return;
+        const int r = r0 + warp + F::kWarps * it.j;
+        const float sc = __shfl_sync(0xffffffffu, scale_j, it.j & 31);
 #pragma unroll
         for (int t = 0; t < T; ++t) {
-            float v = acc[t];
+            float v = acc[t] + acc2[t];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0 && r < r1) {
+            if (lane == 0) {
                 if (splits == 1) {
-                    a.y[(size_t)t * a.d_out + r] = __float2half_rn(v * __half2float(a.scales[r]));
+                    const float s_r = it.j < 32 ? sc : __half2float(a.scales[r]);
+                    a.y[(size_t)t * a.d_out + r] = __float2half_rn(v * s_r);
                 } else {
                     a.partial[((size_t)split * T + t) * a.d_out + r] = v;
                 }
             }
-            acc[t] = 0.f;
+            acc[t] = acc2[t] = 0.f;
         }
     };
-    // the decoded group q of item k's chunk times every token's activations
+    // the codewords of group q of the lane's chunk times every token's
+    // activations: fp16 x fp16 products accumulated in fp32 (exact products)
     auto dot_group = [&](const uint4 &cw0, const uint4 &cw1, int q, int c) {
-        float w[kGroup], xv[kGroup];
-        half8_to_float8(cw0, w);
-        if constexpr (M == 2) {
-            float f[kGroup];
-            half8_to_float8(cw1, f);
-#pragma unroll
-            for (int e = 0; e < kGroup; ++e) w[e] += f[e];
-        }
 #pragma unroll
         for (int t = 0; t < T; ++t) {
-            half8_to_float8(xs[((size_t)t * GPC + q) * xstride + c], xv);
-            float s0 = w[0] * xv[0], s1 = w[1] * xv[1];
-            s0 = fmaf(w[2], xv[2], s0);
-            s1 = fmaf(w[3], xv[3], s1);
-            s0 = fmaf(w[4], xv[4], s0);
-            s1 = fmaf(w[5], xv[5], s1);
-            s0 = fmaf(w[6], xv[6], s0);
-            s1 = fmaf(w[7], xv[7], s1);
-            acc[t] += s0 + s1;
+            const uint4 xv = xs[((size_t)t * GPC + q) * xstride + c];
+            fma2_f16_f32(acc[t], acc2[t], cw0.x, xv.x);
+            fma2_f16_f32(acc[t], acc2[t], cw0.y, xv.y);
+            fma2_f16_f32(acc[t], acc2[t], cw0.z, xv.z);
+            fma2_f16_f32(acc[t], acc2[t], cw0.w, xv.w);
+            if constexpr (M == 2) {
+                fma2_f16_f32(acc[t], acc2[t], cw1.x, xv.x);
+                fma2_f16_f32(acc[t], acc2[t], cw1.y, xv.y);
+                fma2_f16_f32(acc[t], acc2[t], cw1.z, xv.z);
+                fma2_f16_f32(acc[t], acc2[t], cw1.w, xv.w);
+            }
         }
-    };
-    auto multiply = [&](const uint4 (&cw)[GPC][M], int k) {
-        const int c = lane + 32 * (k % cpw);
-        if (c >= n_chunks) return;
-#pragma unroll
-        for (int q = 0; q < GPC; ++q) dot_group(cw[q][0], cw[q][M - 1], q, c);
     };
 
     if constexpr (F::kSmemCodebook) {
-        // 2x8: codewords come from shared memory at use (short latency, so no
-        // register copies of a whole item ahead); the codes run two items ahead
-        uint4 ch = ch0;
-        for (int k = 0; item_row(k) < r1; ++k) {
-            const uint4 ch_after = load_code(k + 2);
-            const int c = lane + 32 * (k % cpw);
+        // 2x8: codewords from the shared-memory copies at use (short latency,
+        // nothing held ahead in registers); codes four items ahead
+        const int copy = lane & 7;
+        Item it = it0, ahead = next(it3);
+        for (int k = 0; k < n_items; ++k) {
+            const uint4 ch_after = load_code(ahead);
+            ahead = next(ahead);
+            const int c = lane + 32 * it.s;
             if (c < n_chunks) {
 #pragma unroll
                 for (int q = 0; q < GPC; ++q)
-                    dot_group(cbs[code_index<M, B>(ch, q, 0)], cbs[F::K + code_index<M, B>(ch, q, M - 1)], q, c);
+                    dot_group(cbs[(code_index<M, B>(ch0, q, 0) << 3) | copy],
+                              cbs[((F::K + code_index<M, B>(ch0, q, M - 1)) << 3) | copy], q, c);
             }
-            finish_item(k);
-            ch = ch_next;
-            ch_next = ch_after;
+            finish_item(it);
+            it = next(it);
+            ch0 = ch1;
+            ch1 = ch2;
+            ch2 = ch3;
+            ch3 = ch_after;
         }
     } else {
-        // at the top of a trip: cwA holds item k's codewords, ch_next item k+1's codes
-        for (int k = 0; item_row(k) < r1; k += 2) {
-            gather(ch_next, k + 1, cwB);
-            ch_next = load_code(k + 2);
-            multiply(cwA, k);
-            finish_item(k);
-            if (item_row(k + 1) >= r1) break;
-            gather(ch_next, k + 2, cwA);
-            ch_next = load_code(k + 3);
-            multiply(cwB, k + 1);
-            finish_item(k + 1);
+        // at the top of a trip: cwA / cwB hold items k / k+1's codewords,
+        // ch2 / ch3 items k+2 / k+3's codes
+        auto multiply = [&](const uint4 (&cw)[GPC][M], Item it) {
+            const int c = lane + 32 * it.s;
+            if (c >= n_chunks) return;
+#pragma unroll
+            for (int q = 0; q < GPC; ++q) dot_group(cw[q][0], cw[q][M - 1], q, c);
+        };
+        Item it = it0, g = it2, l = it3;
+        auto refill = [&](uint4 (&cw)[GPC][M]) {  // gather item g, load the codes of item g + 2
+            gather(ch2, g, cw);
+            g = next(g);
+            l = next(l);
+            ch2 = ch3;
+            ch3 = load_code(l);
+        };
+        for (int k = 0; k < n_items; k += 2) {
+            multiply(cwA, it);
+            finish_item(it);
+            it = next(it);
+            refill(cwA);
+            if (k + 1 >= n_items) break;
+            multiply(cwB, it);
+            finish_item(it);
+            it = next(it);
+            refill(cwB);
         }
     }
     if (splits == 1) return;
@@ -238,7 +284,7 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    for (int i = threadIdx.x; i < (r1 - r0) * T; i += kRowThreads) {
+    for (int i = threadIdx.x; i < (r1 - r0) * T; i += F::kThreads) {
         const int t = i / (r1 - r0), r = r0 + (i - t * (r1 - r0));
         float sum = 0.f;
         for (int s0 = 0; s0 < splits; s0 += 4) {  // 4 partials in flight, added in split order
@@ -259,7 +305,7 @@ __global__ void __launch_bounds__(kRowThreads) gemv_rows_kernel(const RowArgs a)
 // From 4 tokens on the tensor-core kernel is faster (measured on B200: 4 tokens
 // 28672x8192 174 -> 149 us; at 3 tokens the two are even).
 constexpr int kRowsMaxTokens = 3;
-// Staged activations (+ 2x8 codebooks) per CTA.  Kept small on purpose: the
+// Staged activations per CTA (2x8 adds its 64 KiB of codebook copies).  Kept small on purpose: the
 // shared-memory carveout comes out of L1, and L1 holds the codeword gathers
 // in flight (measured on B200: a 4-token 8192x28672 layer with 114 KiB per
 // CTA ran at 299 us, with 32 KiB slices at 176 us).
@@ -279,9 +325,9 @@ struct RowPlan {
 RowPlan plan_rows(const Dims &d, int T) {
     const int gpc = 16 / (d.M * d.B / 8);
     const int n_chunks = d.G / gpc;
-    const size_t cb = (d.B == 8) ? (size_t)d.M * 256 * 16 : 0;
+    const size_t cb = (d.B == 8) ? (size_t)d.M * 256 * 16 * kCbCopies : 0;
     const size_t per_chunk = (size_t)T * gpc * 16;  // activation bytes per chunk of the slice
-    const int max_slots = (int)((kRowsSmemBudget - cb) / (per_chunk * 32));
+    const int max_slots = (int)(kRowsSmemBudget / (per_chunk * 32));
     const int slots = (n_chunks + 31) / 32;         // lane slots of a whole row
     RowPlan p;
     p.splits = max_slots < 1 ? (n_chunks + 31) / 32 : (slots + max_slots - 1) / max_slots;
@@ -292,11 +338,28 @@ RowPlan plan_rows(const Dims &d, int T) {
     return p;
 }
 
-// Row ranges (gridDim.x): as many CTAs as the SMs hold at once over all
-// splits (by the kernel's registers and shared memory), at most one per 8 rows.
+int row_warps(const Dims &d) { return d.B == 8 ? RowFmt<2, 8>::kWarps : RowFmt<1, 16>::kWarps; }
+
+// CTAs of one launch per SM.  2x8: one 16-warp CTA, half of what the SM
+// holds, so that the next layer's CTA finds a free slot and fills its
+// codebook copies and loads its first codes (before the grid-dependency
+// wait) while this launch computes; measured on B200 (graph of back-to-back
+// launches, 4096x4096): with every slot taken by one launch the next
+// launch's CTAs started only as this launch's CTAs ended, and each CTA spent
+// 2-3 us on loads before its first multiply.  1x16 / 2x16: every slot, as
+// the random codeword gathers need all the warps the SM holds (one 8-warp CTA
+// per SM and launch measured slower: 4096x4096 10.6 against 9.8 us).
+int ctas_per_sm_per_launch(const Dims &d, int resident) {
+    if (d.B == 8) return resident > 1 ? resident / 2 : 1;
+    return resident;
+}
+
+// Row ranges (gridDim.x): as many CTAs as that over all splits, at most one
+// per warp's worth of rows.
 int rows_grid_x(const Dims &d, const RowPlan &p, int ctas_per_sm, int sms) {
     const int cap = (ctas_per_sm * sms) / p.splits > 0 ? (ctas_per_sm * sms) / p.splits : 1;
-    const int sets = (d.d_out + kRowWarps - 1) / kRowWarps;
+    const int warps = row_warps(d);
+    const int sets = (d.d_out + warps - 1) / warps;
     return sets < cap ? sets : cap;
 }
 
@@ -356,8 +419,10 @@ cudaError_t launch_gemv_rows(const void *codes, const uint16_t *codebooks, const
     }
     cudaError_t e = opt_in_dynamic_smem(fn, p.smem);
     if (e != cudaSuccess) return e;
-    const int occ = resident_ctas(reinterpret_cast<const void *>(fn), kRowThreads, p.smem);
-    return launch_kernel(fn, dim3(rows_grid_x(d, p, occ, sms), p.splits), dim3(kRowThreads), p.smem, st, true, a);
+    const int threads = row_warps(d) * 32;
+    const int occ = resident_ctas(reinterpret_cast<const void *>(fn), threads, p.smem);
+    return launch_kernel(fn, dim3(rows_grid_x(d, p, ctas_per_sm_per_launch(d, occ), sms), p.splits), dim3(threads),
+                         p.smem, st, true, a);
 }
 
 }  // namespace aqlm
