@@ -205,12 +205,24 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-// 16-byte asynchronous global -> shared copy through L1 with an L2 cache
-// policy; src_bytes = 0 writes zeros.
+// 16-byte asynchronous global -> shared copy with an L2 cache policy;
+// src_bytes = 0 writes zeros.  kL1: through L1 (.ca) for the 8 KiB of 2x8
+// codebooks, which L1 holds; otherwise L2 only (.cg) for the 1-2 MiB
+// 1x16 / 2x16 codebooks, whose random codewords L1 cannot hold.  Measured on
+// B200: .cg instead of .ca made 1x16 8192x8192 with 4 tokens 46.9 -> 41.6 us
+// and 28672x8192 with 16 tokens 149.6 -> 130.8 us, while 2x8 through L2 only
+// was 9x slower.
+template <bool kL1>
 __device__ __forceinline__ void cp_async16_keep(uint32_t dst, const void *src, uint32_t src_bytes, uint64_t pol) {
-    asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst), "l"(src),
-                 "r"(src_bytes), "l"(pol)
-                 : "memory");
+    if constexpr (kL1) {
+        asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst), "l"(src),
+                     "r"(src_bytes), "l"(pol)
+                     : "memory");
+    } else {
+        asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst), "l"(src),
+                     "r"(src_bytes), "l"(pol)
+                     : "memory");
+    }
 }
 // Arrive on an mbarrier once all of this thread's earlier cp.async copies have
 // completed (the arrival is part of the barrier's expected count).
@@ -434,9 +446,9 @@ __global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm) gemv_tc_k
                     const uint32_t bytes = (grp0 + q < a.G) ? 16u : 0u;
 #pragma unroll
                     for (int m = 0; m < M; ++m)
-                        cp_async16_keep(tile + (uint32_t)(m * kTileBytes) + (uint32_t)((q ^ (r & 7)) << 4),
-                                        a.codebooks + (size_t)m * F::K + tc_index<M, B, kCodeVecs>(code, q, m), bytes,
-                                        keep);
+                        cp_async16_keep<B == 8>(
+                            tile + (uint32_t)(m * kTileBytes) + (uint32_t)((q ^ (r & 7)) << 4),
+                            a.codebooks + (size_t)m * F::K + tc_index<M, B, kCodeVecs>(code, q, m), bytes, keep);
                 }
                 cp_async_arrive_noinc(saddr(&bars->full[s]));
                 // the box's codes were read into registers and used above: its slot
