@@ -1,18 +1,18 @@
 // gemv.cu -- host side of the decode-time product: the kernel choice and the
-// workspace layout.  1..3 tokens: gemv_rows.cu (coalesced row streaming on the
+// workspace layout.  Few tokens: gemv_rows.cu (coalesced row streaming on the
 // CUDA cores, the input range split when the activations do not fit on chip).
-// 4..16 tokens: gemv_tc.cu (the weights decoded into shared memory for
-// tcgen05 tensor-core MMAs).  Both launch with programmatic dependent launch.
+// More tokens: gemv_tc.cu (the weights decoded into shared memory for tcgen05
+// tensor-core MMAs).  Both launch with programmatic dependent launch.
 #include "common.cuh"
 
 namespace aqlm {
 
-bool gemv_rows_supported(int T);
+bool gemv_rows_supported(const Dims &d, int T);
 size_t gemv_rows_workspace_bytes(const Dims &d, int T, int sms);
 size_t gemv_rows_counter_offset(const Dims &d, int T, int sms);
 cudaError_t launch_gemv_rows(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
                              uint16_t *y, int tokens, const Dims &d, void *workspace, int sms, cudaStream_t st);
-bool gemv_tc_supported(int T);
+bool gemv_tc_supported(const Dims &d, int T);
 size_t gemv_tc_workspace_bytes(const Dims &d, int T, int sms);
 size_t gemv_tc_counter_offset(const Dims &d, int T, int sms);
 size_t gemv_tc_status_offset(const Dims &d, int T, int sms);
@@ -31,8 +31,8 @@ int device_sms() {
 
 size_t gemv_workspace_bytes(const Dims &d, int tokens) {
     const int sms = device_sms();
-    if (gemv_rows_supported(tokens)) return gemv_rows_workspace_bytes(d, tokens, sms);
-    if (gemv_tc_supported(tokens)) return gemv_tc_workspace_bytes(d, tokens, sms);
+    if (gemv_rows_supported(d, tokens)) return gemv_rows_workspace_bytes(d, tokens, sms);
+    if (gemv_tc_supported(d, tokens)) return gemv_tc_workspace_bytes(d, tokens, sms);
     return 0;
 }
 
@@ -40,15 +40,15 @@ size_t gemv_workspace_bytes(const Dims &d, int tokens) {
 // the end of the workspace must be zero before a call.
 size_t gemv_workspace_counter_offset(const Dims &d, int tokens) {
     const int sms = device_sms();
-    if (gemv_rows_supported(tokens)) return gemv_rows_counter_offset(d, tokens, sms);
-    if (gemv_tc_supported(tokens)) return gemv_tc_counter_offset(d, tokens, sms);
+    if (gemv_rows_supported(d, tokens)) return gemv_rows_counter_offset(d, tokens, sms);
+    if (gemv_tc_supported(d, tokens)) return gemv_tc_counter_offset(d, tokens, sms);
     return 0;
 }
 
 // Offset of the status word inside the workspace, or -1 when the path for
 // this shape and token count has no device waits (and no status word).
 long long gemv_status_offset(const Dims &d, int tokens) {
-    if (gemv_rows_supported(tokens) || !gemv_tc_supported(tokens)) return -1;
+    if (gemv_rows_supported(d, tokens) || !gemv_tc_supported(d, tokens)) return -1;
     return (long long)gemv_tc_status_offset(d, tokens, device_sms());
 }
 
@@ -56,9 +56,9 @@ cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint
                         const uint16_t *x, uint16_t *y, int tokens, const Dims &d, void *workspace,
                         cudaStream_t st) {
     const int sms = device_sms();
-    if (gemv_rows_supported(tokens))
+    if (gemv_rows_supported(d, tokens))
         return launch_gemv_rows(codes, codebooks, scales, x, y, tokens, d, workspace, sms, st);
-    if (gemv_tc_supported(tokens))
+    if (gemv_tc_supported(d, tokens))
         return launch_gemv_tc(codes, codebooks, scales, x, y, tokens, d, workspace, sms, st);
     return cudaErrorInvalidValue;
 }

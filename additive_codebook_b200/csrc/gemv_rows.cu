@@ -302,9 +302,15 @@ __global__ void __launch_bounds__(RowFmt<M, B>::kThreads) gemv_rows_kernel(const
 
 }  // namespace
 
-// From 4 tokens on the tensor-core kernel is faster (measured on B200: 4 tokens
-// 28672x8192 174 -> 149 us; at 3 tokens the two are even).
-constexpr int kRowsMaxTokens = 3;
+// Most tokens per format on this kernel; past them the tensor-core kernel is
+// faster.  Measured on B200 (8192x8192, graphs of back-to-back launches, row
+// kernel / tensor-core kernel): 1x16 2 tokens 36.7 / 40.5 us, 3 tokens 44.1 /
+// 41.0 us; 2x16 3 tokens 69.3 / 72.5 us, 4 tokens 73.2 / 73.0 us; 2x8 (whose
+// codebooks this kernel reads from shared memory) 4 tokens 38.1 / 41.3 us.
+int rows_max_tokens(const Dims &d) {
+    if (d.B == 8) return 4;
+    return d.M == 2 ? 3 : 2;
+}
 // Staged activations per CTA (2x8 adds its 64 KiB of codebook copies).  Kept small on purpose: the
 // shared-memory carveout comes out of L1, and L1 holds the codeword gathers
 // in flight (measured on B200: a 4-token 8192x28672 layer with 114 KiB per
@@ -339,6 +345,11 @@ RowPlan plan_rows(const Dims &d, int T) {
 }
 
 int row_warps(const Dims &d) { return d.B == 8 ? RowFmt<2, 8>::kWarps : RowFmt<1, 16>::kWarps; }
+// the workspace holds one arrival counter per kRowWarps rows, and a launch
+// has at most one CTA per row_warps() rows
+static_assert(RowFmt<2, 8>::kWarps >= kRowWarps && RowFmt<1, 16>::kWarps >= kRowWarps &&
+                  RowFmt<2, 16>::kWarps >= kRowWarps,
+              "fewer warps per CTA than the workspace's counters allow");
 
 // CTAs of one launch per SM.  2x8: one 16-warp CTA, half of what the SM
 // holds, so that the next layer's CTA finds a free slot and fills its
@@ -379,7 +390,7 @@ size_t gemv_rows_workspace_bytes(const Dims &d, int T, int sms) {
     return gemv_rows_counter_offset(d, T, sms) + (size_t)((d.d_out + kRowWarps - 1) / kRowWarps) * sizeof(uint32_t);
 }
 
-bool gemv_rows_supported(int T) { return T >= 1 && T <= kRowsMaxTokens; }
+bool gemv_rows_supported(const Dims &d, int T) { return T >= 1 && T <= rows_max_tokens(d); }
 
 template <int M, int B>
 void (*rows_fn(int T))(const RowArgs) {

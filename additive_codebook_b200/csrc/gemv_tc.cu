@@ -595,9 +595,12 @@ cudaError_t launch_tc(const CUtensorMap &mc, const CUtensorMap &mx, const TcArgs
 
 }  // namespace
 
-constexpr int kTcMinTokens = 4;
-
-bool gemv_tc_supported(int T) { return T >= kTcMinTokens && T <= AQLM_GEMV_MAX_TOKENS; }
+// Any token count works (the MMA's N is 16 whatever T is); gemv.cu sends this
+// kernel the counts past the row kernel's.
+bool gemv_tc_supported(const Dims &d, int T) {
+    (void)d;
+    return T >= 1 && T <= AQLM_GEMV_MAX_TOKENS;
+}
 
 // Workspace: [fp32 partials of split tiles][arrival counters][status word],
 // the last two zero before a call.

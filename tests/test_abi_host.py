@@ -90,7 +90,7 @@ def test_gemv_workspace_rules():
     assert lib.aqlm_gemv_workspace_bytes(shape(M=1, B=16), 1) == 0   # one token: whole rows per warp
     assert lib.aqlm_gemv_workspace_bytes(shape(), 1) == 0      # 2x8, one token: 2 KiB of activations
     wide = shape(d_in=4096)                                    # 8 tokens, 2 row tiles: split to fill the SMs
-    assert lib.aqlm_gemv_workspace_bytes(shape(d_in=4096, M=1, B=16), 3) == 0   # 24 KiB of activations: one slice
+    assert lib.aqlm_gemv_workspace_bytes(shape(d_in=4096, M=1, B=16), 2) == 0   # 16 KiB of activations: one slice
     small = lib.aqlm_gemv_workspace_bytes(wide, 8)
     assert small >= 2 * 8 * 256 * 4
     assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 8, wide, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
@@ -100,17 +100,22 @@ def test_gemv_workspace_rules():
     assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 16, big, A16, need - 4, NULL) == ac.AQLM_ERR_WORKSPACE
     assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 16, big, ODD, need, NULL) == ac.AQLM_ERR_WORKSPACE
     assert lib.aqlm_gemv_workspace_bytes(big, 0) == 0 and lib.aqlm_gemv_workspace_bytes(big, 17) == 0
-    # up to 3 tokens: the row kernel splits the input range only when T * d_in fp16
-    # activations exceed its shared-memory budget (32 KiB), in slices of whole
-    # 32-chunk lane slots (448 chunks of 16 bytes per 8192x28672 row)
+    # the row kernel (1x16 up to 2 tokens, 2x16 up to 3, 2x8 up to 4) splits the
+    # input range only when T * d_in fp16 activations exceed its shared-memory
+    # budget (32 KiB), in slices of whole 32-chunk lane slots (448 chunks of 16
+    # bytes per 8192x28672 row in 1x16 and 2x8)
     down = ac.Shape(8192, 28672, 8, 1, 16)
+    down8 = ac.Shape(8192, 28672, 8, 2, 8)
     assert lib.aqlm_gemv_workspace_bytes(down, 1) >= 2 * 1 * 8192 * 4   # 56 KiB: two slices of 224 chunks
     assert lib.aqlm_gemv_workspace_bytes(down, 2) >= 4 * 2 * 8192 * 4   # 112 KiB: four slices of 128
-    assert lib.aqlm_gemv_workspace_bytes(down, 3) >= 7 * 3 * 8192 * 4   # 168 KiB: seven slices of 64
-    assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 3, down, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
-    # from 4 tokens: the tensor-core kernel, whose workspace always holds a status word
-    assert lib.aqlm_gemv_workspace_bytes(down, 4) >= 16
-    assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 4, down, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_gemv_workspace_bytes(down8, 3) >= 7 * 3 * 8192 * 4  # 168 KiB: seven slices of 64
+    assert lib.aqlm_gemv_workspace_bytes(down8, 4) >= 7 * 4 * 8192 * 4  # 224 KiB: seven slices of 64
+    assert lib.aqlm_gemv(A16, B16, C16, D16, E16, 2, down, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
+    # past those token counts: the tensor-core kernel, whose workspace always
+    # holds a status word
+    for s_, T in ((down, 3), (down, 16), (down8, 5), (ac.Shape(8192, 28672, 8, 2, 16), 4)):
+        assert lib.aqlm_gemv_workspace_bytes(s_, T) >= 16
+        assert lib.aqlm_gemv(A16, B16, C16, D16, E16, T, s_, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
     assert lib.aqlm_gemv_workspace_bytes(ac.Shape(8192, 16384, 8, 1, 16), 1) == 0   # exactly 32 KiB
 
 

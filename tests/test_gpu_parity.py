@@ -110,13 +110,15 @@ def test_gemv_split_input_range(M, B, T):
     _gemv_case(M, B, 96, 4160, T, seed=20 + T)
 
 
-@pytest.mark.parametrize("M,B,T,d_in", [(1, 16, 1, 82112), (2, 16, 1, 82144)]
-                         + [(m, b, 3, 28736) for m, b in FORMATS] + [(m, b, 2, 20544) for m, b in FORMATS])
+@pytest.mark.parametrize("M,B,T,d_in", [(1, 16, 1, 82112), (2, 16, 1, 82144), (1, 16, 2, 28736), (2, 16, 3, 28736),
+                                         (2, 8, 3, 28736), (2, 8, 4, 28736)]
+                         + [(m, b, 2, 20544) for m, b in FORMATS])
 def test_gemv_rows_split_input_range(M, B, T, d_in):
-    # up to 3 tokens whose activations exceed the row kernel's 32 KiB budget:
-    # the input range is split in slices of whole 32-chunk lane slots (3 to 11
-    # of them here, the last one ragged), partial sums meet in the workspace;
-    # 100 rows leave some warps without a row
+    # row-kernel token counts (1x16 up to 2, 2x16 up to 3, 2x8 up to 4) whose
+    # activations exceed the row kernel's 32 KiB budget: the input range is
+    # split in slices of whole 32-chunk lane slots (3 to 11 of them here, the
+    # last one ragged), partial sums meet in the workspace; 100 rows leave some
+    # warps without a row
     _gemv_case(M, B, 100, d_in, T, seed=30 + T)
 
 
@@ -192,6 +194,7 @@ FULL_GEMV = [
     ("1x16 28672x8192 T4", 28672, 8192, 1, 16, 4),
     ("1x16 8192x28672 T4", 8192, 28672, 1, 16, 4),
     ("1x16 8192x28672 T3", 8192, 28672, 1, 16, 3),
+    ("2x8 8192x28672 T4", 8192, 28672, 2, 8, 4),
     ("1x16 8192x28672 T16", 8192, 28672, 1, 16, 16),
     ("2x16 8192x8192", 8192, 8192, 2, 16, 1),
     ("2x8 256x512", 256, 512, 2, 8, 1),

@@ -59,9 +59,10 @@ def test_noalloc_matches_gemv_on_two_calls(cuda_device, d_out, d_in, M, B, T):
 
 def test_noalloc_rejects_scratch_beyond_its_maximum(cuda_device):
     lib = ac.load_library()
-    # 3 tokens of 28672 inputs on the row kernel: seven activation slices,
-    # 7 x 3 x 131072 fp32 partial sums (11 MB), more than the 8 MiB built in
-    shape = ac.Shape(131072, 28672, 8, 1, 16)
+    # 3 tokens of 28672 inputs on the row kernel (2x8): seven activation
+    # slices, 7 x 3 x 131072 fp32 partial sums (11 MB), more than the 8 MiB
+    # built in
+    shape = ac.Shape(131072, 28672, 8, 2, 8)
     assert lib.aqlm_gemv_workspace_bytes(shape, 3) > lib.aqlm_gemv_noalloc_max_scratch_bytes()
     codes = torch.zeros(16, dtype=torch.uint8, device=DEV)   # never read: the call is rejected first
     x = torch.zeros(16, 16, dtype=torch.float16, device=DEV)
