@@ -30,7 +30,8 @@ AQLM_ERR_TIMEOUT = 6
 GEMV_MAX_TOKENS = 16
 
 # Every entry point declared in include/aqlm.h.
-EXPORTS = ["aqlm_gemv", "aqlm_gemv_workspace_bytes", "aqlm_gemv_check", "aqlm_dequant", "aqlm_gemm",
+EXPORTS = ["aqlm_gemv", "aqlm_gemv_workspace_bytes", "aqlm_gemv_row_tokens", "aqlm_gemv_multi",
+           "aqlm_gemv_multi_workspace_bytes", "aqlm_gemv_check", "aqlm_dequant", "aqlm_gemm",
            "aqlm_gemm_workspace_bytes", "aqlm_gemm_check", "aqlm_bf16_gemm", "aqlm_decode_indices",
            "aqlm_test_gemm_timeout", "aqlm_gemv_noalloc", "aqlm_gemv_noalloc_max_scratch_bytes",
            "aqlm_status_string", "aqlm_version"]
@@ -45,6 +46,15 @@ class AqlmError(RuntimeError):
 class Shape(ctypes.Structure):
     _fields_ = [("d_out", ctypes.c_int32), ("d_in", ctypes.c_int32), ("group", ctypes.c_int32),
                 ("num_codebooks", ctypes.c_int32), ("codebook_bits", ctypes.c_int32)]
+
+
+MULTI_MAX_LAYERS = 4
+
+
+class Layer(ctypes.Structure):
+    """aqlm_layer: one layer of an aqlm_gemv_multi call (device pointers)."""
+    _fields_ = [("codes", ctypes.c_void_p), ("codebooks", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("d_out", ctypes.c_int32)]
 
 
 _lib = None
@@ -63,6 +73,9 @@ def load_library():
     sig = {
         "aqlm_gemv": ([vp, vp, vp, vp, vp, i32, Shape, vp, sz, vp], st),
         "aqlm_gemv_workspace_bytes": ([Shape, i32], sz),
+        "aqlm_gemv_row_tokens": ([Shape], i32),
+        "aqlm_gemv_multi": ([ctypes.POINTER(Layer), i32, vp, i32, Shape, vp, sz, vp], st),
+        "aqlm_gemv_multi_workspace_bytes": ([ctypes.POINTER(Layer), i32, Shape, i32], sz),
         "aqlm_gemv_check": ([Shape, i32, vp, sz, vp], st),
         "aqlm_dequant": ([vp, vp, vp, vp, Shape, vp], st),
         "aqlm_gemm": ([vp, vp, vp, vp, vp, i32, Shape, vp, sz, vp], st),
@@ -165,6 +178,45 @@ def aqlm_gemv(codes, codebooks, scales, x, y=None, workspace=None, stream=None):
     _check(lib.aqlm_gemv(_p(codes), _p(codebooks), _p(_flat_scales(scales)), _p(x), _p(y), T, shape,
                          _p(workspace), wbytes, _stream(stream)), "aqlm_gemv")
     return y
+
+
+def gemv_row_tokens(shape):
+    """Most tokens aqlm_gemv runs on the CUDA cores (and aqlm_gemv_multi takes)."""
+    return int(load_library().aqlm_gemv_row_tokens(shape))
+
+
+def _layers(layers, ys):
+    arr = (Layer * len(layers))()
+    for k, (d, y) in enumerate(zip(layers, ys)):
+        arr[k] = Layer(d["codes"].data_ptr(), d["codebooks"].data_ptr(), _flat_scales(d["scales"]).data_ptr(),
+                       y.data_ptr() if y is not None else 0, d["codes"].shape[0])
+    return arr
+
+
+def gemv_multi_workspace_bytes(layers, tokens):
+    lib = load_library()
+    return int(lib.aqlm_gemv_multi_workspace_bytes(_layers(layers, [None] * len(layers)), len(layers),
+                                                   shape_of(layers[0]["codes"]), tokens))
+
+
+def aqlm_gemv_multi(layers, x, ys=None, workspace=None, stream=None):
+    """[y_l] = [fp16(W^_l . x)] for layers (dicts with codes, codebooks, scales)
+    that read the same x [T, d_in], in one launch."""
+    lib = load_library()
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    T = x.shape[0]
+    if ys is None:
+        ys = [torch.empty((T, d["codes"].shape[0]), dtype=torch.float16, device=x.device) for d in layers]
+    arr = _layers(layers, ys)
+    shape = shape_of(layers[0]["codes"])
+    need = int(lib.aqlm_gemv_multi_workspace_bytes(arr, len(layers), shape, T))
+    if need and workspace is None:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
+    wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib.aqlm_gemv_multi(arr, len(layers), _p(x), T, shape, _p(workspace), wbytes, _stream(stream)),
+           "aqlm_gemv_multi")
+    return ys
 
 
 def aqlm_gemv_check(codes, tokens, workspace, stream=None):

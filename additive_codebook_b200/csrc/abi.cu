@@ -84,6 +84,63 @@ aqlm_status aqlm_gemv(const void *codes, const uint16_t *codebooks, const uint16
                                        to_cuda(stream)));
 }
 
+int32_t aqlm_gemv_row_tokens(aqlm_shape shape) {
+    if (check_shape(shape) != AQLM_OK) return 0;
+    return aqlm::gemv_row_tokens(aqlm::make_dims(shape));
+}
+
+}  // extern "C"
+
+namespace {
+
+// Validated multi-layer arguments: the layers as the launchers take them.
+aqlm_status multi_layers(const aqlm_layer *layers, int32_t n_layers, aqlm_shape shape, aqlm::RowLayerIn *out) {
+    if (!layers || n_layers < 1 || n_layers > AQLM_MULTI_MAX_LAYERS) return AQLM_ERR_INVALID_ARG;
+    for (int l = 0; l < n_layers; ++l) {
+        aqlm_shape s = shape;
+        s.d_out = layers[l].d_out;
+        const aqlm_status st = check_shape(s);
+        if (st != AQLM_OK) return st;
+        out[l] = {layers[l].codes, layers[l].codebooks, layers[l].scales, layers[l].y, layers[l].d_out};
+    }
+    return AQLM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t aqlm_gemv_multi_workspace_bytes(const aqlm_layer *layers, int32_t n_layers, aqlm_shape shape, int32_t tokens) {
+    aqlm::RowLayerIn in[AQLM_MULTI_MAX_LAYERS];
+    if (multi_layers(layers, n_layers, shape, in) != AQLM_OK) return 0;
+    const Dims d = aqlm::make_dims(shape);
+    if (tokens < 1 || tokens > aqlm::gemv_row_tokens(d)) return 0;
+    return aqlm::gemv_multi_workspace_bytes(in, n_layers, d, tokens);
+}
+
+aqlm_status aqlm_gemv_multi(const aqlm_layer *layers, int32_t n_layers, const uint16_t *x, int32_t tokens,
+                            aqlm_shape shape, void *workspace, size_t workspace_bytes, aqlm_stream_t stream) {
+    aqlm::RowLayerIn in[AQLM_MULTI_MAX_LAYERS];
+    aqlm_status st = multi_layers(layers, n_layers, shape, in);
+    if (st != AQLM_OK) return st;
+    for (int l = 0; l < n_layers; ++l) {
+        aqlm_shape s = shape;
+        s.d_out = in[l].d_out;
+        st = check_layer(in[l].codes, in[l].codebooks, in[l].scales, s);
+        if (st != AQLM_OK) return st;
+        if (!in[l].y) return AQLM_ERR_INVALID_ARG;
+        if (!aligned(in[l].y, 2)) return AQLM_ERR_MISALIGNED;
+    }
+    if (!x || tokens < 1 || tokens > AQLM_GEMV_MAX_TOKENS) return AQLM_ERR_INVALID_ARG;
+    if (!aligned(x, 16)) return AQLM_ERR_MISALIGNED;
+    const Dims d = aqlm::make_dims(shape);
+    if (tokens > aqlm::gemv_row_tokens(d)) return AQLM_ERR_UNSUPPORTED;
+    const size_t need = aqlm::gemv_multi_workspace_bytes(in, n_layers, d, tokens);
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16))) return AQLM_ERR_WORKSPACE;
+    return from_cuda(aqlm::launch_gemv_multi(in, n_layers, x, tokens, d, need > 0 ? workspace : nullptr,
+                                             to_cuda(stream)));
+}
+
 aqlm_status aqlm_gemv_check(aqlm_shape shape, int32_t tokens, void *workspace, size_t workspace_bytes,
                             aqlm_stream_t stream) {
     if (check_shape(shape) != AQLM_OK) return AQLM_ERR_UNSUPPORTED;

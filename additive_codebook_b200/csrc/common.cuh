@@ -37,6 +37,16 @@ inline Dims make_dims(const aqlm_shape &s) {
     return d;
 }
 
+// One layer of a decode launch that runs several layers reading the same
+// activations (device pointers; layout as in aqlm.h).
+struct RowLayerIn {
+    const void *codes;
+    const uint16_t *codebooks;
+    const uint16_t *scales;
+    uint16_t *y;
+    int d_out;
+};
+
 // ---- cache-hinted global loads (PTX ISA: ld with L1/L2 eviction priority) ----
 
 // L2 eviction policies (PTX createpolicy), passed to cache-hinted loads.
@@ -195,6 +205,11 @@ long long gemv_status_offset(const Dims &d, int tokens);
 cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                         const uint16_t *x, uint16_t *y, int tokens, const Dims &d, void *workspace,
                         cudaStream_t st);
+int gemv_row_tokens(const Dims &d);
+size_t gemv_multi_workspace_bytes(const RowLayerIn *layers, int n, const Dims &d, int tokens);
+size_t gemv_multi_counter_offset(const RowLayerIn *layers, int n, const Dims &d, int tokens);
+cudaError_t launch_gemv_multi(const RowLayerIn *layers, int n, const uint16_t *x, int tokens, const Dims &d,
+                              void *workspace, cudaStream_t st);
 cudaError_t launch_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                              int32_t *status, cudaStream_t st);
 }  // namespace aqlm

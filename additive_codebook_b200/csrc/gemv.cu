@@ -8,6 +8,11 @@
 namespace aqlm {
 
 bool gemv_rows_supported(const Dims &d, int T);
+int rows_max_tokens(const Dims &d);
+size_t gemv_rows_multi_workspace_bytes(const RowLayerIn *layers, int n, const Dims &d, int T);
+size_t gemv_rows_multi_counter_offset(const RowLayerIn *layers, int n, const Dims &d, int T);
+cudaError_t launch_gemv_rows_multi(const RowLayerIn *layers, int n, const uint16_t *x, int tokens, const Dims &d,
+                                   void *workspace, int sms, cudaStream_t st);
 size_t gemv_rows_workspace_bytes(const Dims &d, int T, int sms);
 size_t gemv_rows_counter_offset(const Dims &d, int T, int sms);
 cudaError_t launch_gemv_rows(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
@@ -61,6 +66,23 @@ cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint
     if (gemv_tc_supported(d, tokens))
         return launch_gemv_tc(codes, codebooks, scales, x, y, tokens, d, workspace, sms, st);
     return cudaErrorInvalidValue;
+}
+
+// Several layers that read the same activations, in one row-kernel launch
+// (the token counts of the row kernel only).
+int gemv_row_tokens(const Dims &d) { return rows_max_tokens(d); }
+
+size_t gemv_multi_workspace_bytes(const RowLayerIn *layers, int n, const Dims &d, int tokens) {
+    return gemv_rows_multi_workspace_bytes(layers, n, d, tokens);
+}
+
+size_t gemv_multi_counter_offset(const RowLayerIn *layers, int n, const Dims &d, int tokens) {
+    return gemv_rows_multi_counter_offset(layers, n, d, tokens);
+}
+
+cudaError_t launch_gemv_multi(const RowLayerIn *layers, int n, const uint16_t *x, int tokens, const Dims &d,
+                              void *workspace, cudaStream_t st) {
+    return launch_gemv_rows_multi(layers, n, x, tokens, d, workspace, device_sms(), st);
 }
 
 }  // namespace aqlm

@@ -39,16 +39,32 @@ namespace {
 // Fewest warps per CTA (the 1x16 / 2x16 kernels; 2x8 runs 16): the
 // workspace keeps one arrival counter per kRowWarps rows.
 constexpr int kRowWarps = 8;
+constexpr int kRowMaxLayers = AQLM_MULTI_MAX_LAYERS;
 
-struct RowArgs {
+// One layer of a launch.  A launch runs the layers that read the same x
+// (one layer, or e.g. the q, k and v projections of an attention block):
+// CTAs [cta0, next layer's cta0) own this layer's rows.
+struct RowLayer {
     const uint8_t *codes;
     const uint4 *codebooks;
     const __half *scales;
-    const __half *x;
     __half *y;
-    float *partial;        // [gridDim.y][T][d_out] when the input range is split
+    int d_out;
+    int row0;  // first row of the layer in the launch's concatenated rows
+    int cta0;  // first CTA (blockIdx.x) of the layer
+};
+
+// NL: layers the kernel is built for (1, or kRowMaxLayers for launches of
+// several layers; a single layer then skips the layer lookup and passes a
+// quarter of the parameters).
+template <int NL>
+struct RowArgs {
+    RowLayer layer[NL];
+    int n_layers;
+    const __half *x;
+    float *partial;        // [gridDim.y][T][total_rows] when the input range is split
     uint32_t *counters;    // [gridDim.x] when split; zero between calls
-    int d_out, d_in, G, row_bytes;
+    int total_rows, d_in, G, row_bytes;
     int chunks_per_split;  // 16-byte code chunks of a row per CTA
 };
 
@@ -84,8 +100,8 @@ __device__ __forceinline__ uint32_t code_index(const uint4 &ch, int q, int m) {
     }
 }
 
-template <int M, int B, int T>
-__global__ void __launch_bounds__(RowFmt<M, B>::kThreads) gemv_rows_kernel(const RowArgs a) {
+template <int M, int B, int T, int NL>
+__global__ void __launch_bounds__(RowFmt<M, B>::kThreads, 2) gemv_rows_kernel(const RowArgs<NL> a) {
     using F = RowFmt<M, B>;
     constexpr int GPC = F::GPC;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -98,11 +114,28 @@ __global__ void __launch_bounds__(RowFmt<M, B>::kThreads) gemv_rows_kernel(const
     uint4 *cbs = xs + (size_t)T * GPC * xstride;          // 2x8: [M][256][8 copies] codewords
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // this CTA's rows: an equal contiguous share [r0, r1) of d_out, so that
-    // every SM gets the same number of rows whichever CTAs it holds; warp w
-    // owns rows r0 + w + 8 j, j < n_rows
-    const int r0 = (int)((int64_t)blockIdx.x * a.d_out / gridDim.x);
-    const int r1 = (int)((int64_t)(blockIdx.x + 1) * a.d_out / gridDim.x);
+    // this CTA's layer (static indices only: the descriptors stay in the
+    // kernel's parameter space) and its CTAs [L.cta0, cta_end)
+    RowLayer L = a.layer[0];
+    int cta_end = (int)gridDim.x;
+#pragma unroll
+    for (int i = 1; i < NL; ++i) {
+        if (i < a.n_layers) {
+            if ((int)blockIdx.x >= a.layer[i].cta0) {
+                L = a.layer[i];
+            } else if (a.layer[i].cta0 < cta_end) {
+                cta_end = a.layer[i].cta0;
+            }
+        }
+    }
+    const int bx = NL == 1 ? (int)blockIdx.x : (int)blockIdx.x - L.cta0;
+    const int nbx = NL == 1 ? (int)gridDim.x : cta_end - L.cta0;
+    const int row0 = NL == 1 ? 0 : L.row0;
+    // this CTA's rows: an equal contiguous share [r0, r1) of the layer's
+    // d_out, so that every SM gets the same number of rows whichever CTAs it
+    // holds; warp w owns rows r0 + w + kWarps j, j < n_rows
+    const int r0 = (int)((int64_t)bx * L.d_out / nbx);
+    const int r1 = (int)((int64_t)(bx + 1) * L.d_out / nbx);
     const int n_rows = r1 - r0 > warp ? (r1 - r0 - warp + F::kWarps - 1) / F::kWarps : 0;
     const int cpw = (n_chunks + 31) / 32;  // chunk slots per lane per row
     const int n_items = n_rows * cpw;      // item k = (row j = k / cpw, slot k % cpw)
@@ -112,18 +145,18 @@ __global__ void __launch_bounds__(RowFmt<M, B>::kThreads) gemv_rows_kernel(const
     if constexpr (!F::kSmemCodebook) {
         if (threadIdx.x == 0) {  // this CTA's share of the (usually cold) codebooks into L2
             const uint32_t cb_bytes = (uint32_t)M * F::K * 16;
-            const uint32_t share = ((cb_bytes + gridDim.x - 1) / gridDim.x + 255) & ~255u;
-            const uint32_t off = blockIdx.x * share;
+            const uint32_t share = ((cb_bytes + nbx - 1) / nbx + 255) & ~255u;
+            const uint32_t off = bx * share;
             if (off < cb_bytes)
-                prefetch_l2_bulk(reinterpret_cast<const uint8_t *>(a.codebooks) + off, min(share, cb_bytes - off),
+                prefetch_l2_bulk(reinterpret_cast<const uint8_t *>(L.codebooks) + off, min(share, cb_bytes - off),
                                  keep_pol);
         }
     } else {
-        for (int c = threadIdx.x; c < M * F::K * kCbCopies; c += F::kThreads) cbs[c] = a.codebooks[c >> 3];
+        for (int c = threadIdx.x; c < M * F::K * kCbCopies; c += F::kThreads) cbs[c] = L.codebooks[c >> 3];
     }
     // the scales of the warp's first 32 rows, lane j holding row j's (weights:
     // read before the grid-dependency wait, off the critical path)
-    const float scale_j = (splits == 1 && lane < n_rows) ? __half2float(a.scales[r0 + warp + F::kWarps * lane]) : 0.f;
+    const float scale_j = (splits == 1 && lane < n_rows) ? __half2float(L.scales[r0 + warp + F::kWarps * lane]) : 0.f;
 
     // (row, slot) of an item, advanced without divisions
     struct Item {
@@ -139,7 +172,7 @@ __global__ void __launch_bounds__(RowFmt<M, B>::kThreads) gemv_rows_kernel(const
     auto lane_live = [&](Item it) { return it.j < n_rows && lane + 32 * it.s < n_chunks; };
     auto load_code = [&](Item it) -> uint4 {
         if (lane_live(it))
-            return ld_stream_u4(a.codes + (size_t)(r0 + warp + F::kWarps * it.j) * a.row_bytes +
+            return ld_stream_u4(L.codes + (size_t)(r0 + warp + F::kWarps * it.j) * a.row_bytes +
                                     (size_t)(c0 + lane + 32 * it.s) * 16,
                                 stream_pol);
         return make_uint4(0, 0, 0, 0);
@@ -150,7 +183,7 @@ __global__ void __launch_bounds__(RowFmt<M, B>::kThreads) gemv_rows_kernel(const
         for (int q = 0; q < GPC; ++q) {
 #pragma unroll
             for (int m = 0; m < M; ++m)
-                cw[q][m] = live ? ld_keep_u4(a.codebooks + (size_t)m * F::K + code_index<M, B>(ch, q, m), keep_pol)
+                cw[q][m] = live ? ld_keep_u4(L.codebooks + (size_t)m * F::K + code_index<M, B>(ch, q, m), keep_pol)
                                 : make_uint4(0, 0, 0, 0);
         }
     };
@@ -196,10 +229,10 @@ __global__ void __launch_bounds__(RowFmt<M, B>::kThreads) gemv_rows_kernel(const
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
             if (lane == 0) {
                 if (splits == 1) {
-                    const float s_r = it.j < 32 ? sc : __half2float(a.scales[r]);
-                    a.y[(size_t)t * a.d_out + r] = __float2half_rn(v * s_r);
+                    const float s_r = it.j < 32 ? sc : __half2float(L.scales[r]);
+                    L.y[(size_t)t * L.d_out + r] = __float2half_rn(v * s_r);
                 } else {
-                    a.partial[((size_t)split * T + t) * a.d_out + r] = v;
+                    a.partial[((size_t)split * T + t) * a.total_rows + row0 + r] = v;
                 }
             }
             acc[t] = acc2[t] = 0.f;
@@ -291,11 +324,11 @@ __global__ void __launch_bounds__(RowFmt<M, B>::kThreads) gemv_rows_kernel(const
             float v[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-                v[u] = (s0 + u < splits) ? __ldcg(&a.partial[((size_t)(s0 + u) * T + t) * a.d_out + r]) : 0.f;
+                v[u] = (s0 + u < splits) ? __ldcg(&a.partial[((size_t)(s0 + u) * T + t) * a.total_rows + row0 + r]) : 0.f;
 #pragma unroll
             for (int u = 0; u < 4; ++u) sum += v[u];
         }
-        a.y[(size_t)t * a.d_out + r] = __float2half_rn(sum * __half2float(a.scales[r]));
+        L.y[(size_t)t * L.d_out + r] = __float2half_rn(sum * __half2float(L.scales[r]));
     }
     if (threadIdx.x == 0) a.counters[blockIdx.x] = 0u;
 }
@@ -365,75 +398,146 @@ int ctas_per_sm_per_launch(const Dims &d, int resident) {
     return resident;
 }
 
-// Row ranges (gridDim.x): as many CTAs as that over all splits, at most one
-// per warp's worth of rows.
-int rows_grid_x(const Dims &d, const RowPlan &p, int ctas_per_sm, int sms) {
+// CTAs of each layer (gridDim.x is their sum): as many CTAs in all as the
+// launch's share of the SMs over all splits, dealt to the layers in
+// proportion to their rows, at least one and at most one per warp's worth of
+// rows each.
+void rows_grid(const int *d_outs, int n, const Dims &d, const RowPlan &p, int ctas_per_sm, int sms, int *ctas) {
     const int cap = (ctas_per_sm * sms) / p.splits > 0 ? (ctas_per_sm * sms) / p.splits : 1;
     const int warps = row_warps(d);
-    const int sets = (d.d_out + warps - 1) / warps;
-    return sets < cap ? sets : cap;
+    long long want = 0, rows = 0;
+    for (int l = 0; l < n; ++l) {
+        want += (d_outs[l] + warps - 1) / warps;
+        rows += d_outs[l];
+    }
+    for (int l = 0; l < n; ++l) {
+        const int most = (d_outs[l] + warps - 1) / warps;
+        int c = want <= cap ? most : (int)((long long)cap * d_outs[l] / rows);
+        ctas[l] = c < 1 ? 1 : (c > most ? most : c);
+    }
+}
+
+// Workspace: fp32 partials [splits][T][rows of all layers], then one arrival
+// counter per CTA (a layer has at most one CTA per kRowWarps rows).
+size_t rows_counter_offset(long long rows, const Dims &d, int T) {
+    const RowPlan p = plan_rows(d, T);
+    if (p.splits == 1) return 0;
+    return ((size_t)p.splits * T * rows * sizeof(float) + 15) / 16 * 16;
+}
+size_t rows_workspace_bytes(const int *d_outs, int n, const Dims &d, int T) {
+    const RowPlan p = plan_rows(d, T);
+    if (p.splits == 1) return 0;
+    long long rows = 0, counters = 0;
+    for (int l = 0; l < n; ++l) {
+        rows += d_outs[l];
+        counters += (d_outs[l] + kRowWarps - 1) / kRowWarps;
+    }
+    return rows_counter_offset(rows, d, T) + (size_t)counters * sizeof(uint32_t);
 }
 
 }  // namespace
 
 size_t gemv_rows_counter_offset(const Dims &d, int T, int sms) {
     (void)sms;
-    const RowPlan p = plan_rows(d, T);
-    if (p.splits == 1) return 0;
-    return ((size_t)p.splits * T * d.d_out * sizeof(float) + 15) / 16 * 16;
+    return rows_counter_offset(d.d_out, d, T);
 }
 
-// Partials, then one arrival counter per possible row range (at most one per 8 rows).
 size_t gemv_rows_workspace_bytes(const Dims &d, int T, int sms) {
-    const RowPlan p = plan_rows(d, T);
-    if (p.splits == 1) return 0;
-    return gemv_rows_counter_offset(d, T, sms) + (size_t)((d.d_out + kRowWarps - 1) / kRowWarps) * sizeof(uint32_t);
+    (void)sms;
+    return rows_workspace_bytes(&d.d_out, 1, d, T);
+}
+
+size_t gemv_rows_multi_counter_offset(const RowLayerIn *layers, int n, const Dims &d, int T) {
+    long long rows = 0;
+    for (int l = 0; l < n; ++l) rows += layers[l].d_out;
+    return rows_counter_offset(rows, d, T);
+}
+
+size_t gemv_rows_multi_workspace_bytes(const RowLayerIn *layers, int n, const Dims &d, int T) {
+    int d_outs[kRowMaxLayers];
+    for (int l = 0; l < n; ++l) d_outs[l] = layers[l].d_out;
+    return rows_workspace_bytes(d_outs, n, d, T);
 }
 
 bool gemv_rows_supported(const Dims &d, int T) { return T >= 1 && T <= rows_max_tokens(d); }
 
-template <int M, int B>
-void (*rows_fn(int T))(const RowArgs) {
+// The kernel for T tokens; token counts past the format's rows_max_tokens()
+// are not built (nullptr).
+template <int M, int B, int NL>
+void (*rows_fn(int T))(const RowArgs<NL>) {
+    constexpr int kMax = B == 8 ? 4 : (M == 2 ? 3 : 2);
     switch (T) {
-        case 1: return gemv_rows_kernel<M, B, 1>;
-        case 2: return gemv_rows_kernel<M, B, 2>;
-        case 3: return gemv_rows_kernel<M, B, 3>;
-        default: return gemv_rows_kernel<M, B, 4>;
+        case 1: return gemv_rows_kernel<M, B, 1, NL>;
+        case 2: return gemv_rows_kernel<M, B, 2, NL>;
+        case 3: if constexpr (kMax >= 3) return gemv_rows_kernel<M, B, 3, NL>; else return nullptr;
+        case 4: if constexpr (kMax >= 4) return gemv_rows_kernel<M, B, 4, NL>; else return nullptr;
+        default: return nullptr;
     }
 }
 
-cudaError_t launch_gemv_rows(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
-                             uint16_t *y, int tokens, const Dims &d, void *workspace, int sms, cudaStream_t st) {
+namespace {
+
+template <int NL>
+cudaError_t launch_rows(const RowLayerIn *layers, int n, const uint16_t *x, int tokens, const Dims &d,
+                        void *workspace, int sms, cudaStream_t st) {
     const RowPlan p = plan_rows(d, tokens);
-    RowArgs a;
-    a.codes = static_cast<const uint8_t *>(codes);
-    a.codebooks = reinterpret_cast<const uint4 *>(codebooks);
-    a.scales = reinterpret_cast<const __half *>(scales);
+    void (*fn)(const RowArgs<NL>);
+    if (d.M == 1) {
+        fn = rows_fn<1, 16, NL>(tokens);
+    } else if (d.B == 8) {
+        fn = rows_fn<2, 8, NL>(tokens);
+    } else {
+        fn = rows_fn<2, 16, NL>(tokens);
+    }
+    if (!fn) return cudaErrorInvalidValue;
+    const int threads = row_warps(d) * 32;
+    const int occ = resident_ctas(reinterpret_cast<const void *>(fn), threads, p.smem);
+    int d_outs[kRowMaxLayers], ctas[kRowMaxLayers];
+    for (int l = 0; l < n; ++l) d_outs[l] = layers[l].d_out;
+    rows_grid(d_outs, n, d, p, ctas_per_sm_per_launch(d, occ), sms, ctas);
+    RowArgs<NL> a = {};
+    int cta0 = 0, row0 = 0;
+    for (int l = 0; l < n; ++l) {
+        RowLayer &L = a.layer[l];
+        L.codes = static_cast<const uint8_t *>(layers[l].codes);
+        L.codebooks = reinterpret_cast<const uint4 *>(layers[l].codebooks);
+        L.scales = reinterpret_cast<const __half *>(layers[l].scales);
+        L.y = reinterpret_cast<__half *>(layers[l].y);
+        L.d_out = layers[l].d_out;
+        L.row0 = row0;
+        L.cta0 = cta0;
+        row0 += layers[l].d_out;
+        cta0 += ctas[l];
+    }
+    a.n_layers = n;
     a.x = reinterpret_cast<const __half *>(x);
-    a.y = reinterpret_cast<__half *>(y);
     a.partial = static_cast<float *>(workspace);
     a.counters = p.splits > 1 ? reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) +
-                                                             gemv_rows_counter_offset(d, tokens, sms))
+                                                             rows_counter_offset(row0, d, tokens))
                               : nullptr;
-    a.d_out = d.d_out;
+    a.total_rows = row0;
     a.d_in = d.d_in;
     a.G = d.G;
     a.row_bytes = d.row_bytes;
     a.chunks_per_split = p.chunks_per_split;
-    void (*fn)(const RowArgs);
-    if (d.M == 1) {
-        fn = rows_fn<1, 16>(tokens);
-    } else if (d.B == 8) {
-        fn = rows_fn<2, 8>(tokens);
-    } else {
-        fn = rows_fn<2, 16>(tokens);
-    }
     cudaError_t e = opt_in_dynamic_smem(fn, p.smem);
     if (e != cudaSuccess) return e;
-    const int threads = row_warps(d) * 32;
-    const int occ = resident_ctas(reinterpret_cast<const void *>(fn), threads, p.smem);
-    return launch_kernel(fn, dim3(rows_grid_x(d, p, ctas_per_sm_per_launch(d, occ), sms), p.splits), dim3(threads),
-                         p.smem, st, true, a);
+    return launch_kernel(fn, dim3(cta0, p.splits), dim3(threads), p.smem, st, true, a);
+}
+
+}  // namespace
+
+cudaError_t launch_gemv_rows_multi(const RowLayerIn *layers, int n, const uint16_t *x, int tokens, const Dims &d,
+                                   void *workspace, int sms, cudaStream_t st) {
+    if (n < 1 || n > kRowMaxLayers) return cudaErrorInvalidValue;
+    if (n == 1) return launch_rows<1>(layers, n, x, tokens, d, workspace, sms, st);
+    return launch_rows<kRowMaxLayers>(layers, n, x, tokens, d, workspace, sms, st);
+}
+
+cudaError_t launch_gemv_rows(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
+                             uint16_t *y, int tokens, const Dims &d, void *workspace, int sms, cudaStream_t st) {
+    const RowLayerIn layer = {codes, codebooks, scales, y, d.d_out};
+    return launch_gemv_rows_multi(&layer, 1, x, tokens, d, workspace, sms, st);
 }
 
 }  // namespace aqlm

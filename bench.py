@@ -264,30 +264,40 @@ def single_call_us(ac, bench, reps=50):
     return statistics.median(out)
 
 
-def bench_block(ac, fmt, steps, warmup, l2_bytes):
-    """Llama-2-7B decoder block: its 7 linears back to back, batch 1."""
+def bench_block(ac, fmt, steps, warmup, l2_bytes, fused=False):
+    """Llama-2-7B decoder block: its 7 linears back to back, batch 1.  fused:
+    q/k/v in one aqlm_gemv_multi launch and gate/up in another (they read the
+    same x), o and down alone -- 4 launches per block instead of 7."""
     import torch
     M, B = fmt
     specs = [LayerSpec(o, i, M, B) for _, o, i in LLAMA7B_SHAPES]
     per_block = sum(s.code_bytes() + s.codebook_bytes() + 2 * s.d_out for s in specs)
     R = max(2, int(np.ceil(3 * l2_bytes / per_block)))
     blocks = [[Layers(s, 1, 1, seed=100 * r + k) for k, s in enumerate(specs)] for r in range(R)]
-    ys = {s.d_out: torch.empty((1, s.d_out), dtype=torch.float16, device="cuda") for s in specs}
+    ys = [torch.empty((1, s.d_out), dtype=torch.float16, device="cuda") for s in specs]
     x_in = {4096: blocks[0][0].x, 11008: blocks[0][6].x}
+    groups = [[0, 1, 2], [3], [4, 5], [6]] if fused else [[k] for k in range(len(specs))]
+
+    def block(blk):
+        for grp in groups:
+            x = x_in[specs[grp[0]].d_in]
+            if len(grp) == 1:
+                d = blk[grp[0]].copies[0]
+                ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], x, y=ys[grp[0]])
+            else:
+                ac.aqlm_gemv_multi([blk[k].copies[0] for k in grp], x, ys=[ys[k] for k in grp])
+
     g = torch.cuda.CUDAGraph()
     for blk in blocks:
-        for L in blk:
-            d = L.copies[0]
-            ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], x_in[L.spec.d_in], y=ys[L.spec.d_out])
+        block(blk)
     torch.cuda.synchronize()
     with torch.cuda.graph(g, capture_error_mode="relaxed"):
         for blk in blocks:
-            for L in blk:
-                d = L.copies[0]
-                ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], x_in[L.spec.d_in], y=ys[L.spec.d_out])
+            block(blk)
     ms = time_replays(g, steps, warmup)
     us_block = ms * 1e3 / (steps * R)
-    return {"us_per_block": us_block, "bytes_per_block": sum(algo_bytes(s, 1) for s in specs), "copies": R}
+    return {"us_per_block": us_block, "bytes_per_block": sum(algo_bytes(s, 1) for s in specs), "copies": R,
+            "launches_per_block": len(groups)}
 
 
 def bench_prefill(ac, spec, tokens, reps, warmup):
@@ -416,11 +426,12 @@ def run_gpu(args):
         r = bench_gemv(ac, LayerSpec(4096, 4096, 2, 8), 1, max(3, args.steps // 2), args.warmup, l2)
         detail["2x8 4096x4096 T1"] = _gemv_detail(r, peaks)
         for fmt in ((1, 16), (2, 8)):
-            b = bench_block(ac, fmt, max(3, args.steps // 2), args.warmup, l2)
-            gbs = b["bytes_per_block"] / (b["us_per_block"] * 1e-6) / 1e9
-            detail[f"llama2-7b block {fmt[0]}x{fmt[1]} T1"] = {
-                "us_per_block": round(b["us_per_block"], 3), "gbs": round(gbs, 1),
-                "hbm_frac": round(gbs / peaks["hbm_gbs"], 4)}
+            for fused in (False, True):
+                b = bench_block(ac, fmt, max(3, args.steps // 2), args.warmup, l2, fused=fused)
+                gbs = b["bytes_per_block"] / (b["us_per_block"] * 1e-6) / 1e9
+                detail[f"llama2-7b block {fmt[0]}x{fmt[1]} T1" + (" fused qkv, gate+up" if fused else "")] = {
+                    "us_per_block": round(b["us_per_block"], 3), "gbs": round(gbs, 1),
+                    "hbm_frac": round(gbs / peaks["hbm_gbs"], 4), "launches": b["launches_per_block"]}
         for name, o, i in LLAMA70B_SHAPES:
             for (M, B), Ts in (((1, 16), (1, 4, 16)), ((2, 16), (1,))):
                 for T in Ts:

@@ -86,6 +86,19 @@ typedef struct {
 /* Largest token count of the matrix-vector path. */
 #define AQLM_GEMV_MAX_TOKENS 16
 
+/* Most layers of one aqlm_gemv_multi call. */
+#define AQLM_MULTI_MAX_LAYERS 4
+
+/* One layer of an aqlm_gemv_multi call: a host struct whose pointers are
+ * device memory, laid out as above. */
+typedef struct {
+    const void *codes;          /* [d_out][d_in/8][M]                       */
+    const uint16_t *codebooks;  /* [M][2^B][8] fp16                         */
+    const uint16_t *scales;     /* [d_out] fp16                             */
+    uint16_t *y;                /* [tokens][d_out] fp16, written            */
+    int32_t d_out;              /* rows of this layer                       */
+} aqlm_layer;
+
 /*
  * aqlm_gemv -- decode-time layer product, y = W^ . x, for 1 <= tokens <= 16.
  *
@@ -104,11 +117,12 @@ typedef struct {
  *   small or not 16-byte aligned -> AQLM_ERR_WORKSPACE.  The workspace must be
  *   zero-filled before its first use; every completed call leaves it ready for
  *   the next one.  Calls that share a workspace must not overlap on the GPU.
- * Up to 3 tokens the kernels have no device waits.  From 4 tokens the
- * product runs on the tensor cores with producer/consumer waits inside each
- * CTA, each bounded in time: a wait that gives up records AQLM_ERR_TIMEOUT in
- * the workspace's status word (y is then not valid, and the workspace must be
- * zero-filled again); aqlm_gemv_check() reads it.
+ * Up to AQLM_GEMV_ROW_TOKENS(shape) tokens (1x16: 2, 2x16: 3, 2x8: 4) the
+ * product runs on the CUDA cores with no device waits.  Past that it runs on
+ * the tensor cores with producer/consumer waits inside each CTA, each bounded
+ * in time: a wait that gives up records AQLM_ERR_TIMEOUT in the workspace's
+ * status word (y is then not valid, and the workspace must be zero-filled
+ * again); aqlm_gemv_check() reads it.
  * Launch: with programmatic dependent launch.  codes, codebooks and scales
  * are treated as constant weights and may be read before the preceding
  * kernel in the stream has finished; x is read, and y and the workspace are
@@ -122,12 +136,52 @@ AQLM_API aqlm_status aqlm_gemv(const void *codes, const uint16_t *codebooks, con
  * on the current device (0 if none); returns 0 for invalid arguments too. */
 AQLM_API size_t aqlm_gemv_workspace_bytes(aqlm_shape shape, int32_t tokens);
 
+/* Most tokens for which aqlm_gemv runs on the CUDA cores with no device waits
+ * (1x16: 2, 2x16: 3, 2x8: 4), which is also the most aqlm_gemv_multi takes;
+ * 0 for an unsupported shape.  The value belongs to this build of the library
+ * (it follows measurements of both kernels), so ask rather than hard-code it. */
+AQLM_API int32_t aqlm_gemv_row_tokens(aqlm_shape shape);
+
+/*
+ * aqlm_gemv_multi -- the products y_l = W^_l . x of 1 to AQLM_MULTI_MAX_LAYERS
+ * layers that read the SAME activations x, in one launch: e.g. the query, key
+ * and value projections of an attention block, or the gate and up
+ * projections of a feed-forward block.  Each layer is computed exactly as
+ * aqlm_gemv computes it (same section of the pages, same arithmetic and the
+ * same order of every addition, so each y_l is bit-for-bit aqlm_gemv's);
+ * one launch instead of n_layers saves the launch-to-launch gaps, and the
+ * layers' CTAs share the SMs in proportion to their rows.  Not a counterpart
+ * of anything on the pages: a batching of their product.
+ *   layers[n_layers]: HOST array; every layer has the format of `shape`
+ *   (shape.d_in, group, num_codebooks, codebook_bits; shape.d_out is ignored)
+ *   and its own codes, codebooks, scales, output and d_out >= 1.
+ *   x: [tokens][d_in] fp16, read by every layer.
+ *   tokens: 1 .. aqlm_gemv_row_tokens(shape); more -> AQLM_ERR_UNSUPPORTED
+ *   (call aqlm_gemv per layer for those).
+ *   workspace: as aqlm_gemv's, sized by aqlm_gemv_multi_workspace_bytes()
+ *   (0 = none needed, NULL allowed); zero-filled before its first use, left
+ *   ready for the next call; calls sharing it must not overlap on the GPU.
+ * Errors: n_layers outside 1..AQLM_MULTI_MAX_LAYERS or a NULL pointer ->
+ * AQLM_ERR_INVALID_ARG; alignment as aqlm_gemv (per layer) ->
+ * AQLM_ERR_MISALIGNED; no launch happens on any error but AQLM_ERR_CUDA.
+ * No device waits.  Launch: programmatic dependent launch, as aqlm_gemv.
+ */
+AQLM_API aqlm_status aqlm_gemv_multi(const aqlm_layer *layers, int32_t n_layers, const uint16_t *x, int32_t tokens,
+                                     aqlm_shape shape, void *workspace, size_t workspace_bytes,
+                                     aqlm_stream_t stream);
+
+/* Bytes of device workspace aqlm_gemv_multi needs for these layers (only
+ * their d_out is read), format and token count on the current device (0 if
+ * none); returns 0 for invalid arguments too. */
+AQLM_API size_t aqlm_gemv_multi_workspace_bytes(const aqlm_layer *layers, int32_t n_layers, aqlm_shape shape,
+                                                int32_t tokens);
+
 /*
  * aqlm_gemv_check -- synchronise `stream` and return the status that the
  * aqlm_gemv calls with this shape, token count and workspace recorded:
  * AQLM_OK, or AQLM_ERR_TIMEOUT (the word is then cleared).  Paths without
- * device waits (up to 3 tokens) have no status word: AQLM_OK after the
- * synchronisation.  Not a counterpart of anything on the pages: library
+ * device waits (up to AQLM_GEMV_ROW_TOKENS(shape) tokens) have no status word:
+ * AQLM_OK after the synchronisation.  Not a counterpart of anything on the pages: library
  * plumbing for the bounded waits.
  */
 AQLM_API aqlm_status aqlm_gemv_check(aqlm_shape shape, int32_t tokens, void *workspace, size_t workspace_bytes,

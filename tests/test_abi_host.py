@@ -150,3 +150,64 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(ac, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         ac.load_library()
+
+
+def test_row_tokens_per_format():
+    lib = ac.load_library()
+    assert lib.aqlm_gemv_row_tokens(shape(M=1, B=16)) == 2
+    assert lib.aqlm_gemv_row_tokens(shape(M=2, B=16)) == 3
+    assert lib.aqlm_gemv_row_tokens(shape(M=2, B=8)) == 4
+    assert lib.aqlm_gemv_row_tokens(shape(M=3, B=8)) == 0
+    assert lib.aqlm_gemv_row_tokens(shape(d_in=500)) == 0
+
+
+def _multi(*d_outs, codes=A16, y=E16):
+    arr = (ac.Layer * max(len(d_outs), 1))()
+    for k, n in enumerate(d_outs):
+        arr[k] = ac.Layer(codes.value, B16.value, C16.value, y.value if y.value else None, n)
+    return arr
+
+
+def test_gemv_multi_argument_errors():
+    # every call fails validation on the host, so the fake pointers are never used
+    lib = ac.load_library()
+    s = shape(d_out=0)   # d_out of the common shape is ignored
+    q = _multi(4096, 1024, 1024)
+    assert lib.aqlm_gemv_multi(q, 0, D16, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemv_multi(_multi(8, 8, 8, 8, 8), 5, D16, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemv_multi(None, 1, D16, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemv_multi(q, 3, NULL, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemv_multi(_multi(64, 0), 2, D16, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemv_multi(_multi(64, 64, y=NULL), 2, D16, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemv_multi(_multi(64, 64, codes=ODD), 2, D16, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_MISALIGNED
+    assert lib.aqlm_gemv_multi(_multi(64, 64, y=ctypes.c_void_p(0x50001)), 2, D16, 1, s, NULL, 0, NULL) == \
+        ac.AQLM_ERR_MISALIGNED
+    assert lib.aqlm_gemv_multi(q, 3, ODD, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_MISALIGNED
+    assert lib.aqlm_gemv_multi(q, 3, D16, 0, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemv_multi(q, 3, D16, 17, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    # past the row kernel's token count the call is refused (aqlm_gemv per layer instead)
+    assert lib.aqlm_gemv_multi(q, 3, D16, 5, s, NULL, 0, NULL) == ac.AQLM_ERR_UNSUPPORTED
+    s16 = shape(d_out=0, d_in=4096, M=1, B=16)
+    assert lib.aqlm_gemv_multi(q, 3, D16, 3, s16, NULL, 0, NULL) == ac.AQLM_ERR_UNSUPPORTED
+    assert lib.aqlm_gemv_multi(q, 3, D16, 1, shape(d_out=0, M=3), NULL, 0, NULL) == ac.AQLM_ERR_UNSUPPORTED
+
+
+def test_gemv_multi_workspace_rules():
+    lib = ac.load_library()
+    s = shape(d_out=0, d_in=4096, M=1, B=16)
+    q = _multi(4096, 1024, 1024)
+    assert lib.aqlm_gemv_multi_workspace_bytes(q, 3, s, 1) == 0       # 8 KiB of activations: no split
+    assert lib.aqlm_gemv_multi_workspace_bytes(q, 3, s, 3) == 0       # past the row kernel: invalid
+    assert lib.aqlm_gemv_multi_workspace_bytes(q, 0, s, 1) == 0
+    # 28672 inputs, 1 token: two activation slices; partials for all 6144
+    # rows, then one counter per 8 rows of each layer
+    wide = shape(d_out=0, d_in=28672, M=1, B=16)
+    need = lib.aqlm_gemv_multi_workspace_bytes(q, 3, wide, 1)
+    assert need == 2 * 1 * 6144 * 4 + (512 + 128 + 128) * 4
+    assert lib.aqlm_gemv_multi(q, 3, D16, 1, wide, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_gemv_multi(q, 3, D16, 1, wide, A16, need - 4, NULL) == ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_gemv_multi(q, 3, D16, 1, wide, ODD, need, NULL) == ac.AQLM_ERR_WORKSPACE
+    # one layer: the same workspace as aqlm_gemv
+    one = _multi(8192)
+    assert lib.aqlm_gemv_multi_workspace_bytes(one, 1, wide, 2) == \
+        lib.aqlm_gemv_workspace_bytes(ac.Shape(8192, 28672, 8, 1, 16), 2)
