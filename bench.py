@@ -469,7 +469,7 @@ def run_gpu(args):
                      "frac": round(achieved / peaks["hbm_gbs"], 4),
                      "traffic": recorded_traffic("gemv 1x16 4096x4096 T1"),
                      "peak_source": f"{peaks['source']} copy bandwidth",
-                     "kernel": "gemv_rows_kernel<1,16>",
+                     "kernel": "gemv_rows_kernel<1,16,1,1>",
                      "algorithmic_bytes_per_launch": head["bytes_per_layer"],
                      # the roofline that actually binds a batch-1 1x16 layer: one random 16-byte
                      # codeword gather from L2 per group
