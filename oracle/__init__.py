@@ -6,8 +6,11 @@ Python binding never do.  It shares no code with the CUDA path.
 
 Definitions follow "The AQLM Quantization Algorithm, Explained", section
 "What is Multi-Codebook Quantization (MCQ)?" (decode a group as the sum of M
-codewords, scale per output channel, multiply with the activations) and
-section "Memory footprint of AQLM-quantized models" (bits per parameter).
+codewords, scale per output channel, multiply with the activations), section
+"Memory footprint of AQLM-quantized models" (bits per parameter) and, for the
+encoding (aqlm_encode_oracle.c), section "AQLM quantization process"
+(codebooks initialised by residual k-means, codes learned with the codebooks
+fixed; readings E1-E6 in that file).
 
 Parity pins: tests/test_oracle.py checks every function here against closed
 forms, brute force and independent library routines.  No function is
@@ -41,6 +44,14 @@ def _configure(lib):
     lib.aqlm_oracle_float_to_bf16.argtypes = [ctypes.c_float]
     lib.aqlm_oracle_float_to_bf16.restype = ctypes.c_uint16
     lib.aqlm_oracle_num_threads.restype = ctypes.c_int
+    # encoding (aqlm_encode_oracle.c)
+    lib.aqlm_oracle_double_to_half.argtypes = [ctypes.c_double]
+    lib.aqlm_oracle_double_to_half.restype = ctypes.c_uint16
+    lib.aqlm_oracle_encode_scales.argtypes = [vp, i64, i64, vp, vp]
+    lib.aqlm_oracle_nearest.argtypes = [vp, i64, vp, i64, vp, vp]
+    lib.aqlm_oracle_kmeans_update.argtypes = [vp, vp, i64, i64, vp, vp, vp]
+    lib.aqlm_oracle_residual_kmeans.argtypes = [vp, i64, i32, i64, vp, i32, vp]
+    lib.aqlm_oracle_encode_greedy.argtypes = [vp, i64, vp, i32, i64, vp]
     return lib
 
 
@@ -157,3 +168,73 @@ def bf16_bits_to_f64(bits):
     """bfloat16 bit patterns -> float64 (the upper half of a binary32)."""
     b = np.ascontiguousarray(bits, dtype=np.uint16)
     return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+# --------------------------------------------------------------------------- encoding
+# "The AQLM Quantization Algorithm, Explained", section "AQLM quantization
+# process": codes are learned with fixed codebooks and scales, the codebooks
+# initialised by residual k-means.  Readings E1-E6 are stated in
+# aqlm_encode_oracle.c.
+
+def _f32(a, cols=None):
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    if cols is not None:
+        assert a.size % cols == 0
+    return a
+
+
+def double_to_half(x):
+    """binary16 bits of a real number, round to nearest even."""
+    return _load().aqlm_oracle_double_to_half(float(x))
+
+
+def encode_scales(W):
+    """E1, E2: (scales float16 [d_out], groups float32 [d_out * d_in / 8, 8])."""
+    W = _f32(W)
+    d_out, d_in = W.shape
+    sc = np.empty(d_out, dtype=np.uint16)
+    V = np.empty((d_out * d_in // 8, 8), dtype=np.float32)
+    assert _load().aqlm_oracle_encode_scales(_ptr(W), d_out, d_in, _ptr(sc), _ptr(V)) == 0
+    return sc.view(np.float16), V
+
+
+def nearest(V, C):
+    """E3: (index int32 [N], distance float32 [N]) of each group's nearest codeword."""
+    V, C = _f32(V, 8), _f32(C, 8)
+    N, K = V.size // 8, C.size // 8
+    idx = np.empty(N, dtype=np.int32)
+    dist = np.empty(N, dtype=np.float32)
+    assert _load().aqlm_oracle_nearest(_ptr(V), N, _ptr(C), K, _ptr(idx), _ptr(dist)) == 0
+    return idx, dist
+
+
+def kmeans_update(V, idx, C_prev):
+    """E4: (centroids float32 [K, 8], counts int64 [K])."""
+    V, C_prev = _f32(V, 8), _f32(C_prev, 8)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    N, K = V.size // 8, C_prev.size // 8
+    C = np.empty((K, 8), dtype=np.float32)
+    counts = np.empty(K, dtype=np.int64)
+    assert _load().aqlm_oracle_kmeans_update(_ptr(V), _ptr(idx), N, K, _ptr(C_prev), _ptr(C), _ptr(counts)) == 0
+    return C, counts
+
+
+def residual_kmeans(V, M, K, init_idx, iters):
+    """E5: codebooks float32 [M, K, 8]."""
+    V = _f32(V, 8)
+    init_idx = np.ascontiguousarray(init_idx, dtype=np.int32)
+    assert init_idx.size == M * K
+    C = np.empty((M, K, 8), dtype=np.float32)
+    assert _load().aqlm_oracle_residual_kmeans(_ptr(V), V.size // 8, M, K, _ptr(init_idx), iters, _ptr(C)) == 0
+    return C
+
+
+def encode_greedy(V, codebooks):
+    """E6: codes uint16 [N, M] against float16 codebooks [M, K, 8]."""
+    V = _f32(V, 8)
+    cb = _c16(codebooks)
+    M, K = cb.shape[0], cb.shape[1]
+    codes = np.empty((V.size // 8, M), dtype=np.uint16)
+    assert _load().aqlm_oracle_encode_greedy(_ptr(V), V.size // 8, _ptr(cb), M, K, _ptr(codes)) == 0
+    return codes
+

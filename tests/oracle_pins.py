@@ -312,7 +312,158 @@ def pin_worked_example():
     assert np.array_equal(y, np.array(ex["expected_y"], dtype=np.float64))
 
 
+# --------------------------------------------------------------------------- encoding
+# Section "AQLM quantization process": codebooks initialised by residual
+# k-means, codes learned with the codebooks fixed.  Readings E1-E6 are in
+# oracle/aqlm_encode_oracle.c.
+
+def pin_double_to_half():
+    """Rounding to binary16 agrees with numpy's float64 -> float16 conversion:
+    every binary16 value, the midpoints between neighbours (ties to even),
+    values just off the midpoints, the subnormal range and overflow."""
+    every = np.arange(65536, dtype=np.uint16).view(np.float16)
+    finite = every[np.isfinite(every)].astype(np.float64)
+    pos = np.unique(finite[finite >= 0])
+    mids = (pos[:-1] + pos[1:]) / 2
+    probes = np.concatenate([finite, mids, -mids, np.nextafter(mids, 0), np.nextafter(mids, 1e9),
+                             [65504.0, 65519.99, 65520.0, 1e6, 2.0 ** -25, 2.0 ** -25 * 1.0000001, 2.0 ** -26, 0.0, -0.0],
+                             _rng(5).standard_normal(4000) * np.exp(_rng(6).uniform(-18, 11, 4000))])
+    with np.errstate(over="ignore"):
+        want = probes.astype(np.float16).view(np.uint16)
+    got = np.array([oracle.double_to_half(v) for v in probes], dtype=np.uint16)
+    assert np.array_equal(got, want), np.flatnonzero(got != want)[:5]
+
+
+def pin_encode_scales():
+    """E1/E2: the scale is the row's root mean square rounded to binary16
+    (numpy float64 statistics, numpy rounding), 1.0 for an all-zero row, and
+    the groups are the row's values divided by it (numpy float32 division)."""
+    rng = _rng(21)
+    W = (rng.standard_normal((40, 256)) * rng.uniform(0.01, 3.0, (40, 1))).astype(np.float32)
+    W[7] = 0.0
+    sc, V = oracle.encode_scales(W)
+    rms = np.sqrt((W.astype(np.float64) ** 2).mean(axis=1)).astype(np.float16)
+    rms[7] = 1.0
+    assert np.array_equal(sc.view(np.uint16), rms.view(np.uint16))
+    want = (W / sc.astype(np.float32)[:, None]).reshape(-1, 8)
+    assert np.array_equal(V, want)
+
+
+def _brute_nearest(V, C):
+    d = ((V.astype(np.float64)[:, None, :] - C.astype(np.float64)[None, :, :]) ** 2).sum(-1)
+    return d
+
+
+def pin_nearest_codeword():
+    """E3: the chosen codeword is the nearest by the float64 distance (brute
+    force), exactly so wherever the two nearest are not within rounding of
+    each other; a group equal to a codeword gets that codeword at distance 0;
+    duplicated codewords resolve to the lowest index."""
+    rng = _rng(22)
+    C = rng.standard_normal((300, 8)).astype(np.float32)
+    V = rng.standard_normal((500, 8)).astype(np.float32)
+    V[:50] = C[rng.integers(0, 300, 50)]
+    idx, dist = oracle.nearest(V, C)
+    d = _brute_nearest(V, C)
+    best = d.min(axis=1)
+    chosen = d[np.arange(len(V)), idx]
+    assert np.all(chosen <= best * (1 + 1e-5) + 1e-12)
+    srt = np.sort(d, axis=1)
+    clear = srt[:, 1] > srt[:, 0] * (1 + 1e-4) + 1e-9
+    assert np.array_equal(idx[clear], d.argmin(axis=1)[clear])
+    assert np.allclose(dist, chosen, rtol=1e-5, atol=1e-12)
+    assert np.all(dist[:50] == 0)
+    # duplicates: codewords 10 and 20 equal, a group equal to them -> 10
+    C2 = C.copy()
+    C2[20] = C2[10]
+    i2, _ = oracle.nearest(C2[10:11] + np.float32(0), C2)
+    assert i2[0] == 10
+    i3, _ = oracle.nearest(C2[20:21], C2[::-1].copy())
+    assert i3[0] == 300 - 1 - 20
+
+
+def pin_kmeans_update():
+    """E4: centroids are the float64 means of their groups rounded to float32
+    (numpy, summing in the same order), counts exact, empty clusters keep
+    their previous value."""
+    rng = _rng(23)
+    V = rng.standard_normal((1000, 8)).astype(np.float32)
+    K = 40
+    idx = rng.integers(0, K - 5, 1000).astype(np.int32)   # the last 5 clusters stay empty
+    C_prev = rng.standard_normal((K, 8)).astype(np.float32)
+    C, counts = oracle.kmeans_update(V, idx, C_prev)
+    assert np.array_equal(counts, np.bincount(idx, minlength=K))
+    sums = np.zeros((K, 8), dtype=np.float64)
+    np.add.at(sums, idx, V.astype(np.float64))
+    want = C_prev.copy()
+    nz = counts > 0
+    want[nz] = (sums[nz] / counts[nz, None]).astype(np.float32)
+    assert np.array_equal(C, want)
+
+
+def pin_residual_kmeans_recovers_clusters():
+    """E5 closed forms: data drawn around K well-separated centres, started
+    from one member of each cluster, converge to the cluster means; the second
+    codebook (of residuals) is the k-means of the small offsets, and adding
+    it never raises the squared error of the codebook-0 approximation."""
+    rng = _rng(24)
+    K, per = 12, 40
+    centres = (rng.standard_normal((K, 8)) * 10).astype(np.float32)
+    lab = np.repeat(np.arange(K), per)
+    V = (centres[lab] + rng.standard_normal((K * per, 8)).astype(np.float32) * 0.05).astype(np.float32)
+    perm = rng.permutation(K * per)
+    V, lab = V[perm], lab[perm]
+    first = np.array([np.flatnonzero(lab == k)[0] for k in range(K)], dtype=np.int32)
+    init = np.stack([first, rng.choice(K * per, K, replace=False).astype(np.int32)])
+    C = oracle.residual_kmeans(V, 2, K, init, iters=4)
+    means = np.stack([V[lab == k].astype(np.float64).mean(0) for k in range(K)])
+    assert np.allclose(C[0], means, atol=1e-5)
+    d0 = _brute_nearest(V, C[0])
+    i0 = d0.argmin(1)
+    R = V - C[0][i0]
+    e1 = (R.astype(np.float64) ** 2).sum()
+    i1 = _brute_nearest(R, C[1]).argmin(1)
+    e2 = ((R - C[1][i1]).astype(np.float64) ** 2).sum()
+    assert e2 <= e1 and np.abs(C[1]).max() < 0.5
+
+
+def pin_greedy_codes_recover_sums():
+    """E6 closed form: with codebook 0 on a coarse grid and codebook 1 of
+    small offsets (all binary16-exact), a group that is exactly C0[b0] + C1[b1]
+    is encoded as (b0, b1); with one codebook a group equal to a codeword gets
+    its index (brute force agrees on random groups where the choice is clear)."""
+    rng = _rng(25)
+    K0, K1 = 64, 16
+    C0 = (rng.integers(-8, 8, (K0, 8)) * 4).astype(np.float16)
+    C0[1:] += (np.arange(1, K0)[:, None] % 4 == 0) * np.float16(1)    # distinct rows
+    C0 = np.unique(C0, axis=0)[:32]
+    C1 = (rng.integers(-3, 4, (K1, 8)) / 16).astype(np.float16)
+    C1 = np.unique(C1, axis=0)
+    k0, k1 = len(C0), len(C1)
+    b0 = rng.integers(0, k0, 400)
+    b1 = rng.integers(0, k1, 400)
+    V = (C0[b0].astype(np.float32) + C1[b1].astype(np.float32))
+    cb = np.zeros((2, max(k0, k1), 8), dtype=np.float16)
+    cb[0, :k0], cb[1, :k1] = C0, C1
+    cb[1, k1:] = np.float16(1000)                     # padding never chosen
+    cb[0, k0:] = np.float16(1000)
+    codes = oracle.encode_greedy(V, cb)
+    assert np.array_equal(codes[:, 0], b0) and np.array_equal(codes[:, 1], b1)
+    # one codebook, random groups: brute force where the nearest is clear
+    C = rng.standard_normal((1, 200, 8)).astype(np.float16)
+    Vr = rng.standard_normal((300, 8)).astype(np.float32)
+    c1 = oracle.encode_greedy(Vr, C)[:, 0]
+    d = _brute_nearest(Vr, C[0].astype(np.float32))
+    srt = np.sort(d, axis=1)
+    clear = srt[:, 1] > srt[:, 0] * (1 + 1e-4)
+    assert np.array_equal(c1[clear], d.argmin(1)[clear])
+
+
+ENCODE_PINS = [pin_double_to_half, pin_encode_scales, pin_nearest_codeword, pin_kmeans_update,
+               pin_residual_kmeans_recovers_clusters, pin_greedy_codes_recover_sums]
+
 ALL_PINS = [pin_half_conversion, pin_bf16_rounding, pin_decode_indices,
             pin_index_encoding_recovers_codes, pin_one_hot_activation, pin_linearity,
             pin_dense_special_case, pin_brute_force_tiny, pin_bf16_activations, pin_matmul,
-            pin_dequant_bf16_binary32_steps, pin_bits_per_parameter, pin_worked_example]
+            pin_dequant_bf16_binary32_steps, pin_bits_per_parameter, pin_worked_example,
+            *ENCODE_PINS]

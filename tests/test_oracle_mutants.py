@@ -1,10 +1,12 @@
 """Planted mistakes in the oracle must fail at least one pin (CPU only).
 
-Each case copies oracle/aqlm_oracle.c, changes one expression into a
+Each case copies one of the oracle's C files (aqlm_oracle.c, or
+aqlm_encode_oracle.c for the encoding), changes one expression into a
 plausible bug (a dropped term, a wrong sign, a swapped index, a transposed
-operand, an off-by-one, a wrong rounding rule), compiles the copy into a
-temporary directory and runs the pins of tests/oracle_pins.py against it.
-Every planted change keeps all memory accesses in bounds.
+operand, an off-by-one, a wrong rounding or tie rule), compiles the copy with
+the other file into a temporary directory and runs the pins of
+tests/oracle_pins.py against it.  Every planted change keeps all memory
+accesses in bounds.
 """
 import ctypes
 import os
@@ -15,7 +17,8 @@ import pytest
 import oracle
 from oracle_pins import ALL_PINS
 
-SRC = os.path.join(os.path.dirname(oracle.__file__), "aqlm_oracle.c")
+ORACLE_DIR = os.path.dirname(oracle.__file__)
+INFER, ENCODE = "aqlm_oracle.c", "aqlm_encode_oracle.c"
 
 MUTANTS = {
     "dequant_drops_scale": ("W[i * d_in + j * g + t] = s * sum;", "W[i * d_in + j * g + t] = sum;"),
@@ -37,19 +40,37 @@ MUTANTS = {
     "bpp_scale_term": ("double scale_bits = (double)d_out * 16.0;", "double scale_bits = (double)d_out * 32.0;"),
     "bpp_codebook_term": ("double codebook_bits = (double)M * ldexp(1.0, B) * g * 16.0;",
                           "double codebook_bits = ldexp(1.0, B) * g * 16.0;"),
+    # encoding
+    "half_ties_away": (ENCODE, "double q = rint(ldexp(a, 11 - e));", "double q = round(ldexp(a, 11 - e));"),
+    "scale_mean_abs": (ENCODE, "acc += (double)row[k] * (double)row[k];", "acc += fabs((double)row[k]);"),
+    "nearest_ties_high": (ENCODE, "const float dk = distance(V + n * 8, C + k * 8);\n            if (dk < bd) {",
+                          "const float dk = distance(V + n * 8, C + k * 8);\n            if (dk <= bd) {"),
+    "distance_drops_lane": (ENCODE, "o = fmaf(d[7], d[7], o);", "o = o;"),
+    "update_off_by_one": (ENCODE, "(float)(sums[k * 8 + t] / (double)counts[k])",
+                          "(float)(sums[k * 8 + t] / (double)(counts[k] + 1))"),
+    "residual_not_subtracted": (ENCODE, "R[n * 8 + t] = R[n * 8 + t] - C[(int64_t)idx[n] * 8 + t];",
+                                "R[n * 8 + t] = R[n * 8 + t] + 0.0f * C[(int64_t)idx[n] * 8 + t];"),
+    "greedy_residual_kept": (ENCODE, "for (int t = 0; t < 8; ++t) r[t] = r[t] - Cm[best * 8 + t];",
+                             "for (int t = 0; t < 8; ++t) r[t] = r[t] - 0.0f * Cm[best * 8 + t];"),
 }
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_planted_mistake_is_caught(name, tmp_path):
-    old, new = MUTANTS[name]
-    src = open(SRC).read()
-    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
-    mutated = tmp_path / "mutant.c"
-    mutated.write_text(src.replace(old, new))
+    case = MUTANTS[name]
+    fname, old, new = case if len(case) == 3 else (INFER, *case)
+    srcs = []
+    for f in (INFER, ENCODE):
+        text = open(os.path.join(ORACLE_DIR, f)).read()
+        if f == fname:
+            assert text.count(old) == 1, f"mutation site for {name} not found exactly once"
+            text = text.replace(old, new)
+        path = tmp_path / f
+        path.write_text(text)
+        srcs.append(str(path))
     lib_path = tmp_path / "libmutant.so"
     subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
-                    "-o", str(lib_path), str(mutated), "-lm"], check=True)
+                    "-o", str(lib_path), *srcs, "-lm"], check=True)
     mutant = oracle._configure(ctypes.CDLL(str(lib_path)))
     saved = oracle._load()
     oracle._lib = mutant
