@@ -34,7 +34,11 @@ EXPORTS = ["aqlm_gemv", "aqlm_gemv_workspace_bytes", "aqlm_gemv_row_tokens", "aq
            "aqlm_gemv_multi_workspace_bytes", "aqlm_gemv_check", "aqlm_dequant", "aqlm_gemm",
            "aqlm_gemm_workspace_bytes", "aqlm_gemm_check", "aqlm_bf16_gemm", "aqlm_decode_indices",
            "aqlm_test_gemm_timeout", "aqlm_gemv_noalloc", "aqlm_gemv_noalloc_max_scratch_bytes",
-           "aqlm_status_string", "aqlm_version"]
+           "aqlm_status_string", "aqlm_version",
+           "aqlm_encode_scales", "aqlm_nearest_workspace_bytes", "aqlm_nearest_codeword",
+           "aqlm_kmeans_workspace_bytes", "aqlm_kmeans_update", "aqlm_residual_kmeans_workspace_bytes",
+           "aqlm_residual_kmeans", "aqlm_encode_codes_workspace_bytes", "aqlm_encode_codes",
+           "aqlm_encode_layer_workspace_bytes", "aqlm_encode_layer"]
 
 
 class AqlmError(RuntimeError):
@@ -68,7 +72,7 @@ def load_library():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with `python -m additive_codebook_b200.build`")
     lib = ctypes.CDLL(LIB_PATH)
-    vp, i32, sz, u64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_uint64
+    vp, i32, sz, u64, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_uint64, ctypes.c_int64
     st = ctypes.c_int
     sig = {
         "aqlm_gemv": ([vp, vp, vp, vp, vp, i32, Shape, vp, sz, vp], st),
@@ -86,6 +90,17 @@ def load_library():
         "aqlm_test_gemm_timeout": ([vp, vp, vp, i32, i32, i32, vp, u64, vp], st),
         "aqlm_gemv_noalloc": ([vp, vp, vp, vp, vp, i32, Shape, vp], st),
         "aqlm_gemv_noalloc_max_scratch_bytes": ([], sz),
+        "aqlm_encode_scales": ([vp, i32, i32, vp, vp, vp], st),
+        "aqlm_nearest_workspace_bytes": ([i64], sz),
+        "aqlm_nearest_codeword": ([vp, i64, vp, i32, vp, vp, vp, sz, vp], st),
+        "aqlm_kmeans_workspace_bytes": ([i32], sz),
+        "aqlm_kmeans_update": ([vp, vp, i64, vp, i32, vp, vp, vp, sz, vp], st),
+        "aqlm_residual_kmeans_workspace_bytes": ([i64, i32, i32], sz),
+        "aqlm_residual_kmeans": ([vp, i64, i32, i32, vp, i32, vp, vp, sz, vp], st),
+        "aqlm_encode_codes_workspace_bytes": ([Shape], sz),
+        "aqlm_encode_codes": ([vp, vp, vp, Shape, vp, sz, vp], st),
+        "aqlm_encode_layer_workspace_bytes": ([Shape], sz),
+        "aqlm_encode_layer": ([vp, Shape, vp, i32, vp, vp, vp, vp, sz, vp], st),
         "aqlm_status_string": ([st], ctypes.c_char_p),
         "aqlm_version": ([], ctypes.c_char_p),
     }
@@ -300,3 +315,91 @@ def aqlm_test_gemm_timeout(X, W, Y, status, limit_ns, stream=None):
     T, k = X.shape
     n = W.shape[0]
     return lib.aqlm_test_gemm_timeout(_p(X), _p(W), _p(Y), T, n, k, _p(status), limit_ns, _stream(stream))
+
+
+# --------------------------------------------------------------------------- encoding
+
+def _ws(nbytes, device):
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def encode_scales(W, stream=None):
+    """(scales float16 [d_out], groups float32 [d_out*d_in/8, 8]) of W [d_out, d_in] float32."""
+    lib = load_library()
+    d_out, d_in = W.shape
+    scales = torch.empty(d_out, dtype=torch.float16, device=W.device)
+    groups = torch.empty((d_out * d_in // 8, 8), dtype=torch.float32, device=W.device)
+    _check(lib.aqlm_encode_scales(_p(W), d_out, d_in, _p(scales), _p(groups), _stream(stream)), "aqlm_encode_scales")
+    return scales, groups
+
+
+def nearest_codeword(groups, codebook, with_dist=False, stream=None):
+    """int32 index (and float32 distance) of each group's nearest codeword."""
+    lib = load_library()
+    n, K = groups.shape[0], codebook.shape[0]
+    idx = torch.empty(n, dtype=torch.int32, device=groups.device)
+    dist = torch.empty(n, dtype=torch.float32, device=groups.device) if with_dist else None
+    ws = _ws(lib.aqlm_nearest_workspace_bytes(n), groups.device)
+    _check(lib.aqlm_nearest_codeword(_p(groups), n, _p(codebook), K, _p(idx), _p(dist), _p(ws), ws.numel(),
+                                     _stream(stream)), "aqlm_nearest_codeword")
+    return (idx, dist) if with_dist else idx
+
+
+def kmeans_update(groups, idx, centroids, stream=None):
+    """(centroids float32 [K, 8], counts int32 [K]) after one k-means update."""
+    lib = load_library()
+    n, K = groups.shape[0], centroids.shape[0]
+    out = torch.empty_like(centroids)
+    counts = torch.empty(K, dtype=torch.int32, device=groups.device)
+    ws = _ws(lib.aqlm_kmeans_workspace_bytes(K), groups.device)
+    _check(lib.aqlm_kmeans_update(_p(groups), _p(idx), n, _p(centroids), K, _p(out), _p(counts), _p(ws), ws.numel(),
+                                  _stream(stream)), "aqlm_kmeans_update")
+    return out, counts
+
+
+def residual_kmeans(groups, M, K, init_idx, iters, stream=None):
+    """float32 codebooks [M, K, 8]; init_idx: host int32 array [M, K] of group indices."""
+    import numpy as np
+    lib = load_library()
+    n = groups.shape[0]
+    init = np.ascontiguousarray(init_idx, dtype=np.int32)
+    assert init.size == M * K
+    out = torch.empty((M, K, 8), dtype=torch.float32, device=groups.device)
+    ws = _ws(lib.aqlm_residual_kmeans_workspace_bytes(n, M, K), groups.device)
+    _check(lib.aqlm_residual_kmeans(_p(groups), n, M, K, init.ctypes.data_as(ctypes.c_void_p), iters, _p(out), _p(ws),
+                                    ws.numel(), _stream(stream)), "aqlm_residual_kmeans")
+    return out
+
+
+def _codes_out(d_out, d_in, M, B, device):
+    return torch.empty((d_out, d_in // 8, M), dtype=torch.uint8 if B == 8 else torch.int16, device=device)
+
+
+def encode_codes(groups, codebooks, d_out, d_in, stream=None):
+    """Greedy codes [d_out, d_in/8, M] of the groups against float16 codebooks [M, 2^B, 8]."""
+    lib = load_library()
+    M, K = codebooks.shape[0], codebooks.shape[1]
+    B = 8 if K == 256 else 16
+    shape = Shape(d_out, d_in, 8, M, B)
+    codes = _codes_out(d_out, d_in, M, B, groups.device)
+    ws = _ws(lib.aqlm_encode_codes_workspace_bytes(shape), groups.device)
+    _check(lib.aqlm_encode_codes(_p(groups), _p(codebooks), _p(codes), shape, _p(ws), ws.numel(), _stream(stream)),
+           "aqlm_encode_codes")
+    return codes
+
+
+def encode_layer(W, M, B, init_idx, iters, stream=None):
+    """{codes, codebooks (float16 [M, 2^B, 8]), scales (float16 [d_out])} of W [d_out, d_in] float32."""
+    import numpy as np
+    lib = load_library()
+    d_out, d_in = W.shape
+    shape = Shape(d_out, d_in, 8, M, B)
+    init = np.ascontiguousarray(init_idx, dtype=np.int32)
+    codes = _codes_out(d_out, d_in, M, B, W.device)
+    codebooks = torch.empty((M, 1 << B, 8), dtype=torch.float16, device=W.device)
+    scales = torch.empty(d_out, dtype=torch.float16, device=W.device)
+    ws = _ws(lib.aqlm_encode_layer_workspace_bytes(shape), W.device)
+    _check(lib.aqlm_encode_layer(_p(W), shape, init.ctypes.data_as(ctypes.c_void_p), iters, _p(codes), _p(codebooks),
+                                 _p(scales), _p(ws), ws.numel(), _stream(stream)), "aqlm_encode_layer")
+    return {"codes": codes, "codebooks": codebooks, "scales": scales}
+

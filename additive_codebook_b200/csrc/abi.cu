@@ -217,6 +217,156 @@ aqlm_status aqlm_test_gemm_timeout(const uint16_t *X, const uint16_t *W, uint16_
     return from_cuda(aqlm::launch_bf16_gemm_ex(X, W, Y, tokens, n, k, status, to_cuda(stream), limit_ns, 1));
 }
 
+// ---- encoding ----
+
+aqlm_status aqlm_encode_scales(const float *W, int32_t d_out, int32_t d_in, uint16_t *scales, float *groups,
+                               aqlm_stream_t stream) {
+    if (!W || !scales || !groups || d_out < 1 || d_in < 8 || d_out > kMaxDim || d_in > kMaxDim) {
+        return AQLM_ERR_INVALID_ARG;
+    }
+    if (d_in % 8) return AQLM_ERR_UNSUPPORTED;
+    if (!aligned(W, 16) || !aligned(groups, 16) || !aligned(scales, 2)) return AQLM_ERR_MISALIGNED;
+    return from_cuda(aqlm::launch_encode_scales(W, d_out, d_in, scales, groups, to_cuda(stream)));
+}
+
+size_t aqlm_nearest_workspace_bytes(int64_t n) { return n < 0 ? 0 : aqlm::nearest_workspace_bytes(n); }
+
+aqlm_status aqlm_nearest_codeword(const float *groups, int64_t n, const float *codebook, int32_t K, int32_t *idx,
+                                  float *dist, void *workspace, size_t workspace_bytes, aqlm_stream_t stream) {
+    if (n < 0 || K < 1 || (n > 0 && (!groups || !idx)) || !codebook) return AQLM_ERR_INVALID_ARG;
+    if (n > ((int64_t)1 << 40)) return AQLM_ERR_INVALID_ARG;
+    if (!aligned(groups, 16) || !aligned(codebook, 16) || !aligned(idx, 4) || !aligned(dist, 4))
+        return AQLM_ERR_MISALIGNED;
+    const size_t need = aqlm::nearest_workspace_bytes(n);
+    if (n > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16))) return AQLM_ERR_WORKSPACE;
+    return from_cuda(aqlm::launch_nearest(groups, n, codebook, K, idx, dist, workspace, to_cuda(stream)));
+}
+
+size_t aqlm_kmeans_workspace_bytes(int32_t K) { return K < 1 ? 0 : aqlm::kmeans_workspace_bytes(K); }
+
+aqlm_status aqlm_kmeans_update(const float *groups, const int32_t *idx, int64_t n, const float *centroids, int32_t K,
+                               float *centroids_out, int32_t *counts, void *workspace, size_t workspace_bytes,
+                               aqlm_stream_t stream) {
+    if (n < 0 || K < 1 || (n > 0 && (!groups || !idx)) || !centroids || !centroids_out) return AQLM_ERR_INVALID_ARG;
+    if (n > ((int64_t)1 << 40)) return AQLM_ERR_INVALID_ARG;
+    if (!aligned(groups, 16) || !aligned(idx, 4) || !aligned(centroids, 16) || !aligned(centroids_out, 16) ||
+        !aligned(counts, 4))
+        return AQLM_ERR_MISALIGNED;
+    const size_t need = aqlm::kmeans_workspace_bytes(K);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return AQLM_ERR_WORKSPACE;
+    return from_cuda(aqlm::launch_kmeans_update(groups, idx, n, centroids, K, centroids_out, counts, workspace,
+                                                to_cuda(stream)));
+}
+
+}  // extern "C"
+
+namespace {
+
+// Workspace head of the residual k-means: the copy of init_idx, then the
+// launcher's own workspace.
+size_t init_copy_bytes(int32_t M, int32_t K) { return ((size_t)M * K * sizeof(int32_t) + 255) / 256 * 256; }
+
+aqlm_status check_init(const int32_t *init_idx, int64_t n, int32_t M, int32_t K) {
+    if (!init_idx) return AQLM_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < (int64_t)M * K; ++i)
+        if (init_idx[i] < 0 || init_idx[i] >= n) return AQLM_ERR_INVALID_ARG;
+    return AQLM_OK;
+}
+
+// Residual k-means with init_idx already validated; ws has
+// aqlm_residual_kmeans_workspace_bytes(n, M, K) bytes.
+aqlm_status run_residual_kmeans(const float *groups, int64_t n, int32_t M, int32_t K, const int32_t *init_idx,
+                                int32_t iters, float *codebooks, void *ws, cudaStream_t cs) {
+    int32_t *init_dev = static_cast<int32_t *>(ws);
+    cudaError_t e = cudaMemcpyAsync(init_dev, init_idx, (size_t)M * K * sizeof(int32_t), cudaMemcpyHostToDevice, cs);
+    if (e != cudaSuccess) return AQLM_ERR_CUDA;
+    return from_cuda(aqlm::launch_residual_kmeans(groups, n, M, K, init_dev, iters, codebooks,
+                                                  static_cast<uint8_t *>(ws) + init_copy_bytes(M, K), cs));
+}
+
+size_t layer_groups(const aqlm_shape &s) { return (size_t)s.d_out * (s.d_in / 8); }
+inline size_t al256(size_t v) { return (v + 255) / 256 * 256; }
+
+}  // namespace
+
+extern "C" {
+
+size_t aqlm_residual_kmeans_workspace_bytes(int64_t n, int32_t M, int32_t K) {
+    if (n < 1 || M < 1 || K < 1) return 0;
+    return init_copy_bytes(M, K) + aqlm::residual_kmeans_workspace_bytes(n, K);
+}
+
+aqlm_status aqlm_residual_kmeans(const float *groups, int64_t n, int32_t M, int32_t K, const int32_t *init_idx,
+                                 int32_t iters, float *codebooks, void *workspace, size_t workspace_bytes,
+                                 aqlm_stream_t stream) {
+    if (!groups || !codebooks || n < 1 || M < 1 || M > 8 || K < 1 || iters < 0) return AQLM_ERR_INVALID_ARG;
+    if (n > ((int64_t)1 << 40)) return AQLM_ERR_INVALID_ARG;
+    aqlm_status st = check_init(init_idx, n, M, K);
+    if (st != AQLM_OK) return st;
+    if (!aligned(groups, 16) || !aligned(codebooks, 16)) return AQLM_ERR_MISALIGNED;
+    const size_t need = aqlm_residual_kmeans_workspace_bytes(n, M, K);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return AQLM_ERR_WORKSPACE;
+    return run_residual_kmeans(groups, n, M, K, init_idx, iters, codebooks, workspace, to_cuda(stream));
+}
+
+size_t aqlm_encode_codes_workspace_bytes(aqlm_shape shape) {
+    if (check_shape(shape) != AQLM_OK) return 0;
+    return aqlm::encode_codes_workspace_bytes((long long)layer_groups(shape), shape.num_codebooks,
+                                              1 << shape.codebook_bits);
+}
+
+aqlm_status aqlm_encode_codes(const float *groups, const uint16_t *codebooks, void *codes, aqlm_shape shape,
+                              void *workspace, size_t workspace_bytes, aqlm_stream_t stream) {
+    aqlm_status st = check_shape(shape);
+    if (st != AQLM_OK) return st;
+    if (!groups || !codebooks || !codes) return AQLM_ERR_INVALID_ARG;
+    if (!aligned(groups, 16) || !aligned(codebooks, 16) || !aligned(codes, 16)) return AQLM_ERR_MISALIGNED;
+    const size_t need = aqlm_encode_codes_workspace_bytes(shape);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return AQLM_ERR_WORKSPACE;
+    return from_cuda(aqlm::launch_encode_codes(groups, (long long)layer_groups(shape), codebooks, shape.num_codebooks,
+                                               1 << shape.codebook_bits, codes, shape.codebook_bits / 8, workspace,
+                                               to_cuda(stream)));
+}
+
+// Workspace of the whole encoding: groups, fp32 codebooks, then the larger of
+// the residual k-means' and the greedy codes' workspaces.
+size_t aqlm_encode_layer_workspace_bytes(aqlm_shape shape) {
+    if (check_shape(shape) != AQLM_OK) return 0;
+    const int64_t n = (int64_t)layer_groups(shape);
+    const int32_t M = shape.num_codebooks, K = 1 << shape.codebook_bits;
+    const size_t a = aqlm_residual_kmeans_workspace_bytes(n, M, K), b = aqlm_encode_codes_workspace_bytes(shape);
+    return al256((size_t)n * 8 * sizeof(float)) + al256((size_t)M * K * 8 * sizeof(float)) + (a > b ? a : b);
+}
+
+aqlm_status aqlm_encode_layer(const float *W, aqlm_shape shape, const int32_t *init_idx, int32_t iters, void *codes,
+                              uint16_t *codebooks, uint16_t *scales, void *workspace, size_t workspace_bytes,
+                              aqlm_stream_t stream) {
+    aqlm_status st = check_shape(shape);
+    if (st != AQLM_OK) return st;
+    if (!W || !codes || !codebooks || !scales || iters < 0) return AQLM_ERR_INVALID_ARG;
+    const int64_t n = (int64_t)layer_groups(shape);
+    const int32_t M = shape.num_codebooks, K = 1 << shape.codebook_bits;
+    st = check_init(init_idx, n, M, K);
+    if (st != AQLM_OK) return st;
+    if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(codebooks, 16) || !aligned(scales, 2))
+        return AQLM_ERR_MISALIGNED;
+    const size_t need = aqlm_encode_layer_workspace_bytes(shape);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return AQLM_ERR_WORKSPACE;
+    const cudaStream_t cs = to_cuda(stream);
+    uint8_t *w = static_cast<uint8_t *>(workspace);
+    float *groups = reinterpret_cast<float *>(w);
+    w += al256((size_t)n * 8 * sizeof(float));
+    float *cb32 = reinterpret_cast<float *>(w);
+    w += al256((size_t)M * K * 8 * sizeof(float));
+    cudaError_t e = aqlm::launch_encode_scales(W, shape.d_out, shape.d_in, scales, groups, cs);
+    if (e != cudaSuccess) return AQLM_ERR_CUDA;
+    st = run_residual_kmeans(groups, n, M, K, init_idx, iters, cb32, w, cs);
+    if (st != AQLM_OK) return st;
+    e = aqlm::launch_round_codebooks(cb32, (long long)M * K * 8, codebooks, cs);
+    if (e != cudaSuccess) return AQLM_ERR_CUDA;
+    return from_cuda(aqlm::launch_encode_codes(groups, n, codebooks, M, K, codes, shape.codebook_bits / 8, w, cs));
+}
+
 const char *aqlm_status_string(aqlm_status status) {
     switch (status) {
         case AQLM_OK: return "AQLM_OK";

@@ -212,4 +212,19 @@ cudaError_t launch_gemv_multi(const RowLayerIn *layers, int n, const uint16_t *x
                               void *workspace, cudaStream_t st);
 cudaError_t launch_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                              int32_t *status, cudaStream_t st);
+// encoding (encode.cu)
+cudaError_t launch_encode_scales(const float *W, int d_out, int d_in, uint16_t *scales, float *V, cudaStream_t st);
+size_t nearest_workspace_bytes(long long N);
+cudaError_t launch_nearest(const float *V, long long N, const float *C, int K, int32_t *idx, float *dist,
+                           void *workspace, cudaStream_t st);
+size_t kmeans_workspace_bytes(int K);
+cudaError_t launch_kmeans_update(const float *V, const int32_t *idx, long long N, const float *C_prev, int K,
+                                 float *C_out, int32_t *counts_out, void *workspace, cudaStream_t st);
+size_t residual_kmeans_workspace_bytes(long long N, int K);
+cudaError_t launch_residual_kmeans(const float *V, long long N, int M, int K, const int32_t *init_idx, int iters,
+                                   float *C_out, void *workspace, cudaStream_t st);
+size_t encode_codes_workspace_bytes(long long N, int M, int K);
+cudaError_t launch_encode_codes(const float *V, long long N, const uint16_t *codebooks, int M, int K, void *codes,
+                                int code_bytes, void *workspace, cudaStream_t st);
+cudaError_t launch_round_codebooks(const float *C, long long n, uint16_t *C16, cudaStream_t st);
 }  // namespace aqlm

@@ -283,6 +283,81 @@ AQLM_API aqlm_status aqlm_gemv_noalloc(const void *codes, const uint16_t *codebo
 /* Size of aqlm_gemv_noalloc's built-in scratch array, in bytes. */
 AQLM_API size_t aqlm_gemv_noalloc_max_scratch_bytes(void);
 
+/* ===========================================================================
+ * Encoding: scales, codebooks and codes of a layer from its weights.
+ *
+ * Section "AQLM quantization process" of "The AQLM Quantization Algorithm,
+ * Explained": codes are learned with the codebooks and scales fixed, the
+ * codebooks initialised "with a residual k-means approach".  The pages give
+ * no loss, search or update rule beyond that; the readings taken here are:
+ *   scale s_i   root mean square of row i rounded to fp16 (1.0 if it rounds to
+ *               0): the sum of squares in double, lane l of 32 summing inputs
+ *               l, l+32, ... in order, partial sums combined pairwise
+ *               (l + (l ^ 16), then ^ 8, ^ 4, ^ 2, ^ 1); sqrt(sum / d_in);
+ *   groups      v = W[i][8j .. 8j+7] / s_i (binary32 division), [d_out*d_in/8][8];
+ *   distance    squared Euclidean in binary32: e = chain of fused multiply-adds
+ *               of the squared differences of lanes 0, 2, 4, 6 (the first a plain
+ *               product), o the same for lanes 1, 3, 5, 7, distance = e + o;
+ *   nearest     least distance, ties to the lowest index;
+ *   k-means     a centroid becomes the mean of its groups (sums in double, one
+ *               rounding), one without groups keeps its value; codebook m is
+ *               k-means of the residuals left by codebooks 0..m-1;
+ *   codes       greedy, codebook by codebook: the nearest codeword of the
+ *               residual, which then loses that codeword (binary32).
+ * Every integer result (index, code, count) is deterministic; centroids sum
+ * in double with atomics, so their last binary32 bit may depend on order.
+ * The workspace of each call is device scratch of the size its
+ * *_workspace_bytes query gives; nothing needs to be zero beforehand.
+ * All float arrays are fp32, 16-byte aligned.
+ * ======================================================================== */
+
+/* E1/E2: scales[d_out] (fp16) and groups [d_out*d_in/8][8] (fp32) of W
+ * [d_out][d_in] (fp32).  d_in % 8 == 0. */
+AQLM_API aqlm_status aqlm_encode_scales(const float *W, int32_t d_out, int32_t d_in, uint16_t *scales, float *groups,
+                                        aqlm_stream_t stream);
+
+/* Nearest codeword of each of n groups [n][8] in a codebook [K][8]:
+ * idx[n] (int32) and, if dist is not NULL, its distance. */
+AQLM_API size_t aqlm_nearest_workspace_bytes(int64_t n);
+AQLM_API aqlm_status aqlm_nearest_codeword(const float *groups, int64_t n, const float *codebook, int32_t K,
+                                           int32_t *idx, float *dist, void *workspace, size_t workspace_bytes,
+                                           aqlm_stream_t stream);
+
+/* One k-means update: centroids_out[K][8] from the groups and their
+ * assignments idx[n] (indices outside 0..K-1 are ignored); counts (int32
+ * [K], may be NULL) receives the group count of every centroid. */
+AQLM_API size_t aqlm_kmeans_workspace_bytes(int32_t K);
+AQLM_API aqlm_status aqlm_kmeans_update(const float *groups, const int32_t *idx, int64_t n, const float *centroids,
+                                        int32_t K, float *centroids_out, int32_t *counts, void *workspace,
+                                        size_t workspace_bytes, aqlm_stream_t stream);
+
+/* Residual k-means: M codebooks [M][K][8] (fp32) of the n groups, `iters`
+ * updates each.  init_idx is a HOST array [M][K] of group indices (0..n-1,
+ * else AQLM_ERR_INVALID_ARG): codebook m starts from the residuals they name
+ * (the random draw of the initialisation, made by the caller).  Copies
+ * init_idx from pageable host memory, so it is not for stream capture. */
+AQLM_API size_t aqlm_residual_kmeans_workspace_bytes(int64_t n, int32_t M, int32_t K);
+AQLM_API aqlm_status aqlm_residual_kmeans(const float *groups, int64_t n, int32_t M, int32_t K,
+                                          const int32_t *init_idx, int32_t iters, float *codebooks, void *workspace,
+                                          size_t workspace_bytes, aqlm_stream_t stream);
+
+/* Greedy codes of the d_out*d_in/8 groups against fp16 codebooks
+ * [M][2^B][8], written as the codes of `shape` ([d_out][d_in/8][M], uint8 or
+ * 16-bit) -- the layout aqlm_gemv, aqlm_dequant and aqlm_gemm read. */
+AQLM_API size_t aqlm_encode_codes_workspace_bytes(aqlm_shape shape);
+AQLM_API aqlm_status aqlm_encode_codes(const float *groups, const uint16_t *codebooks, void *codes, aqlm_shape shape,
+                                       void *workspace, size_t workspace_bytes, aqlm_stream_t stream);
+
+/* The whole encoding of a layer W [d_out][d_in] (fp32): scales, residual
+ * k-means codebooks (iters updates each, started from init_idx, a HOST array
+ * [M][2^B] of group indices below d_out*d_in/8) rounded to fp16, greedy codes.
+ * Outputs in the inference layout: codes, codebooks [M][2^B][8] fp16, scales
+ * [d_out] fp16.  Not for stream capture (see aqlm_residual_kmeans). */
+AQLM_API size_t aqlm_encode_layer_workspace_bytes(aqlm_shape shape);
+AQLM_API aqlm_status aqlm_encode_layer(const float *W, aqlm_shape shape, const int32_t *init_idx, int32_t iters,
+                                       void *codes, uint16_t *codebooks, uint16_t *scales, void *workspace,
+                                       size_t workspace_bytes, aqlm_stream_t stream);
+
 /* A static, human-readable name of a status code. */
 AQLM_API const char *aqlm_status_string(aqlm_status status);
 

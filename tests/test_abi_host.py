@@ -211,3 +211,40 @@ def test_gemv_multi_workspace_rules():
     one = _multi(8192)
     assert lib.aqlm_gemv_multi_workspace_bytes(one, 1, wide, 2) == \
         lib.aqlm_gemv_workspace_bytes(ac.Shape(8192, 28672, 8, 1, 16), 2)
+
+
+def test_encode_argument_errors():
+    """The encoding entry points reject bad arguments on the host (nothing is
+    launched, so the fake device addresses are never touched)."""
+    lib = ac.load_library()
+    s = shape(d_out=64, d_in=512, M=2, B=8)
+    init_ok = (ctypes.c_int32 * (2 * 256))(*([3] * 512))
+    init_bad = (ctypes.c_int32 * (2 * 256))(*([3] * 511 + [64 * 64]))   # one index past the 4096 groups
+    ws = lib.aqlm_encode_layer_workspace_bytes(s)
+    assert ws > 0 and lib.aqlm_encode_layer_workspace_bytes(shape(M=3)) == 0
+    assert lib.aqlm_encode_layer(A16, s, init_bad, 2, B16, C16, D16, E16, ws, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_encode_layer(A16, s, None, 2, B16, C16, D16, E16, ws, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_encode_layer(A16, s, init_ok, -1, B16, C16, D16, E16, ws, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_encode_layer(ODD, s, init_ok, 2, B16, C16, D16, E16, ws, NULL) == ac.AQLM_ERR_MISALIGNED
+    assert lib.aqlm_encode_layer(A16, s, init_ok, 2, B16, C16, D16, E16, ws - 1, NULL) == ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_encode_layer(A16, shape(M=3), init_ok, 2, B16, C16, D16, E16, ws, NULL) == \
+        ac.AQLM_ERR_UNSUPPORTED
+    assert lib.aqlm_encode_scales(A16, 64, 500, B16, C16, NULL) == ac.AQLM_ERR_UNSUPPORTED
+    assert lib.aqlm_encode_scales(A16, 0, 512, B16, C16, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_encode_scales(ODD, 64, 512, B16, C16, NULL) == ac.AQLM_ERR_MISALIGNED
+    nws = lib.aqlm_nearest_workspace_bytes(1000)
+    assert nws >= 1000 * 8
+    assert lib.aqlm_nearest_codeword(A16, 1000, B16, 0, C16, NULL, D16, nws, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_nearest_codeword(A16, 1000, B16, 256, C16, NULL, D16, nws - 8, NULL) == ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_nearest_codeword(ODD, 1000, B16, 256, C16, NULL, D16, nws, NULL) == ac.AQLM_ERR_MISALIGNED
+    kws = lib.aqlm_kmeans_workspace_bytes(256)
+    assert kws >= 256 * 8 * 8 + 256 * 4
+    assert lib.aqlm_kmeans_update(A16, B16, 1000, C16, 256, D16, NULL, E16, kws - 1, NULL) == ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_kmeans_update(A16, B16, -1, C16, 256, D16, NULL, E16, kws, NULL) == ac.AQLM_ERR_INVALID_ARG
+    rws = lib.aqlm_residual_kmeans_workspace_bytes(4096, 2, 256)
+    assert lib.aqlm_residual_kmeans(A16, 4096, 2, 256, init_bad, 3, B16, C16, rws, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_residual_kmeans(A16, 4096, 2, 256, init_ok, 3, B16, C16, rws - 1, NULL) == ac.AQLM_ERR_WORKSPACE
+    cws = lib.aqlm_encode_codes_workspace_bytes(s)
+    assert cws >= 4096 * 8 * 4 + 4096 * 8 + 2 * 256 * 8 * 4
+    assert lib.aqlm_encode_codes(A16, B16, C16, s, D16, cws - 1, NULL) == ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_encode_codes(A16, B16, ODD, s, D16, cws, NULL) == ac.AQLM_ERR_MISALIGNED
