@@ -346,6 +346,41 @@ def bench_prefill(ac, spec, tokens, reps, warmup):
             "gemm_tflops": flops / t_gemm / 1e6, "dequant_gbs": deq_bytes / t_deq / 1e3}
 
 
+# Lane operations of one distance evaluation: 8 differences, 8 squares
+# accumulated by multiply / fused multiply-add, 1 addition of the two chains.
+DIST_LANE_OPS = 17
+
+
+def bench_encode(ac, spec, reps=3):
+    """Greedy codes of a whole layer (aqlm_encode_codes: one nearest-codeword
+    pass per codebook over every group of the layer), timed with CUDA events
+    on the current stream.  Reports distance evaluations per second against
+    the fp32 lane-operation peak of the CUDA cores."""
+    import torch
+    rng = np.random.Generator(np.random.PCG64(11))
+    n = spec.d_out * spec.groups
+    K = 1 << spec.B
+    groups = torch.from_numpy(rng.standard_normal((n, 8), dtype=np.float32)).cuda()
+    cb = torch.from_numpy((rng.standard_normal((spec.M, K, 8)) * 0.5).astype(np.float16)).cuda()
+    ac.encode_codes(groups, cb, spec.d_out, spec.d_in)     # warm-up
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        ac.encode_codes(groups, cb, spec.d_out, spec.d_in)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    dists = n * K * spec.M
+    rate = dists / (ms * 1e-3)
+    peak = FMA_PEAK_TERA_PER_S * 1e12 / DIST_LANE_OPS
+    return {"ms_per_layer": round(ms, 3), "distances_per_s": round(rate / 1e12, 4), "unit": "T distances/s",
+            "alu_frac": round(rate / peak, 4),
+            "alu_peak": f"{FMA_PEAK_TERA_PER_S:.1f} T fp32 lane-ops/s / {DIST_LANE_OPS} per distance"}
+
+
 def e2e_gemv(ac, bench, steps, warmup):
     """Through the public API with host buffers: per step H2D of x from pinned
     memory, the layer calls, D2H of every layer's y."""
@@ -439,6 +474,9 @@ def run_gpu(args):
                     detail[f"llama2-70b {name} {o}x{i} {M}x{B} T{T}"] = _gemv_detail(r, peaks, T=T)
                     del r
                     torch.cuda.empty_cache()
+        for M, B in ((1, 16), (2, 8)):
+            detail[f"encode codes {M}x{B} 4096x4096"] = bench_encode(ac, LayerSpec(4096, 4096, M, B))
+            torch.cuda.empty_cache()
         for o, i in PREFILL_SHAPES:
             for M, B in ((1, 16), (2, 8)):
                 p = bench_prefill(ac, LayerSpec(o, i, M, B), 2048, reps=5, warmup=3)
@@ -574,6 +612,7 @@ PROFILE_CASES = {
     "dequant-1x16-11008x4096": ("dequant", 11008, 4096, 1, 16, 0),
     "dequant-2x8-11008x4096": ("dequant", 11008, 4096, 2, 8, 0),
     "gemm-2048x11008x4096": ("gemm", 11008, 4096, 2, 8, 2048),
+    "encode-1x16-256x4096": ("encode", 256, 4096, 1, 16, 0),
 }
 
 
@@ -600,6 +639,12 @@ def run_profile_case(name, launches=12):
         out = torch.empty((o, i), dtype=torch.bfloat16, device="cuda")
         for _ in range(launches):
             ac.aqlm_dequant(d["codes"], d["codebooks"], d["scales"], out=out)
+    elif kind == "encode":
+        rng = np.random.Generator(np.random.PCG64(11))
+        groups = torch.from_numpy(rng.standard_normal((o * i // 8, 8), dtype=np.float32)).cuda()
+        cb = torch.from_numpy((rng.standard_normal((M, 1 << B, 8)) * 0.5).astype(np.float16)).cuda()
+        for _ in range(max(2, launches // 4)):
+            ac.encode_codes(groups, cb, o, i)
     else:
         layers = Layers(spec, 1, T, x_dtype="bf16")
         d = layers.copies[0]
