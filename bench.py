@@ -606,6 +606,7 @@ PROFILE_CASES = {
     "gemv-1x16-4096": ("gemv", 4096, 4096, 1, 16, 1),
     "gemv-2x8-4096": ("gemv", 4096, 4096, 2, 8, 1),
     "gemv-1x16-8192-t16": ("gemv", 8192, 8192, 1, 16, 16),
+    "gemv-1x16-8192-t4": ("gemv", 8192, 8192, 1, 16, 4),
     "gemv-1x16-28672x8192-t4": ("gemv", 28672, 8192, 1, 16, 4),
     "gemv-1x16-8192x28672-t4": ("gemv", 8192, 28672, 1, 16, 4),
     "gemv-2x16-8192": ("gemv", 8192, 8192, 2, 16, 1),
