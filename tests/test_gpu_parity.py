@@ -249,6 +249,25 @@ def test_gemm_small(M, B, tokens, d_out, d_in):
     _gemm_check(bf16_to_np_bits(Y), L, spec, L["x"])
 
 
+@pytest.mark.parametrize("tokens,n,k", [(200, 520, 576), (128, 256, 65536), (130, 264, 64)])
+def test_bf16_gemm_ragged_and_deep(tokens, n, k):
+    """Ragged tiles in every dimension (200 x 520 x 576), one tile with a long
+    k loop (1024 k blocks), and a single k block: against torch (fp32
+    accumulation), and bit-identical from call to call."""
+    g = torch.Generator(device="cpu").manual_seed(tokens + n)
+    X = (torch.randn(tokens, k, generator=g) / 4).to(torch.bfloat16).to(DEV)
+    W = (torch.randn(n, k, generator=g) / 4).to(torch.bfloat16).to(DEV)
+    Y1, s1 = ac.aqlm_bf16_gemm(X, W)
+    Y2, s2 = ac.aqlm_bf16_gemm(X, W)
+    torch.cuda.synchronize()
+    assert int(s1.item()) == 0 and int(s2.item()) == 0
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+    ref = X.float() @ W.float().T
+    absdot = X.float().abs() @ W.float().abs().T
+    err = (Y1.float() - ref).abs()
+    assert bool(torch.all(err <= 2.0 ** -8 * ref.abs() + 2.0 ** -14 * absdot + 1e-6))
+
+
 def test_bf16_gemm_matches_torch():
     """The plain tensor-core GEMM against torch.matmul (fp32 accumulation) as a yardstick."""
     g = torch.Generator(device="cpu").manual_seed(7)
