@@ -471,7 +471,8 @@ def run_gpu(args):
             for (M, B), Ts in (((1, 16), (1, 4, 16)), ((2, 16), (1,))):
                 for T in Ts:
                     r = bench_gemv(ac, LayerSpec(o, i, M, B), T, 3, 2, l2, n_launch=64)
-                    detail[f"llama2-70b {name} {o}x{i} {M}x{B} T{T}"] = _gemv_detail(r, peaks, T=T)
+                    detail[f"llama2-70b {name} {o}x{i} {M}x{B} T{T}"] = _gemv_detail(
+                        r, peaks, T=T, row_tokens=ac.gemv_row_tokens(ac.Shape(o, i, 8, M, B)))
                     del r
                     torch.cuda.empty_cache()
         for M, B in ((1, 16), (2, 8)):
@@ -546,7 +547,7 @@ def gather_roofline(spec, us):
             "peak_source": "random 16-byte gather microbenchmark on this B200"}
 
 
-def _gemv_detail(r, peaks, T=1):
+def _gemv_detail(r, peaks, T=1, row_tokens=None):
     gbs = r["bytes_per_layer"] / (r["us_per_layer"] * 1e-6) / 1e9
     spec = r["layers"].spec
     out = {"us_per_layer": round(r["us_per_layer"], 3), "gbs": round(gbs, 1),
@@ -555,12 +556,13 @@ def _gemv_detail(r, peaks, T=1):
     if gr is not None:
         out["gather_frac"] = gr["frac"]
     if T > 1:
-        # multiply-adds of the product per second; up to 3 tokens they run on the
-        # CUDA cores (fraction of the FMA peak), from 4 on the tensor cores, where
-        # the codeword gathers (gather_frac) are what binds
+        # multiply-adds of the product per second; up to the format's row-kernel
+        # token count (aqlm_gemv_row_tokens) they run on the CUDA cores (fraction
+        # of the FMA peak), past it on the tensor cores, where the codeword
+        # gathers (gather_frac) are what binds
         mac_t = spec.d_out * spec.groups * 8 * T / (r["us_per_layer"] * 1e-6) / 1e12
         out["mac_tera_per_s"] = round(mac_t, 2)
-        if T <= 3:
+        if row_tokens is not None and T <= row_tokens:
             out["path"] = "row kernel, CUDA cores"
             out["fma_frac"] = round(mac_t / FMA_PEAK_TERA_PER_S, 4)
         else:
