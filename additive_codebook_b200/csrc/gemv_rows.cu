@@ -392,7 +392,7 @@ static_assert(RowFmt<2, 8>::kWarps >= kRowWarps && RowFmt<1, 16>::kWarps >= kRow
 // launch's CTAs started only as this launch's CTAs ended, and each CTA spent
 // 2-3 us on loads before its first multiply.  1x16 / 2x16: every slot, as
 // the random codeword gathers need all the warps the SM holds (one 8-warp CTA
-// per SM and launch measured slower: 4096x4096 10.6 against 9.7 us).
+// per SM and launch measured slower: 4096x4096 10.6 against 9.8 us).
 int ctas_per_sm_per_launch(const Dims &d, int resident) {
     if (d.B == 8) return resident > 1 ? resident / 2 : 1;
     return resident;
