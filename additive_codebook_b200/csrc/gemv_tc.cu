@@ -493,18 +493,22 @@ __global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm) gemv_tc_k
                     __threadfence();
                     if (row < a.d_out) {
                         const float sc = __half2float(a.scales[row]);
-                        for (int t = 0; t < a.T; ++t) {
-                            float sum = 0.f;
-                            for (int s0 = 0; s0 < n_seg; s0 += 4) {  // 4 partials in flight
-                                float pv[4];
+                        // segment by segment, every token's partial at once (up to 16
+                        // loads in flight); each token's sum still runs in segment order
+                        float sum[kTcN];
 #pragma unroll
-                                for (int q = 0; q < 4; ++q)
-                                    pv[q] = (s0 + q < n_seg) ? __ldcg(&part[((size_t)(s0 + q) * a.T + t) * kTcRows + r]) : 0.f;
+                        for (int t = 0; t < kTcN; ++t) sum[t] = 0.f;
+                        for (int sg = 0; sg < n_seg; ++sg) {
+                            float pv[kTcN];
 #pragma unroll
-                                for (int q = 0; q < 4; ++q) sum += pv[q];
-                            }
-                            a.y[(size_t)t * a.d_out + row] = __float2half_rn(sum * sc);
+                            for (int t = 0; t < kTcN; ++t)
+                                pv[t] = t < a.T ? __ldcg(&part[((size_t)sg * a.T + t) * kTcRows + r]) : 0.f;
+#pragma unroll
+                            for (int t = 0; t < kTcN; ++t) sum[t] += pv[t];
                         }
+#pragma unroll
+                        for (int t = 0; t < kTcN; ++t)
+                            if (t < a.T) a.y[(size_t)t * a.d_out + row] = __float2half_rn(sum[t] * sc);
                     }
                     if (threadIdx.x == 0) a.counters[g.tile] = 0u;
                 }
