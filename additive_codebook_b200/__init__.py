@@ -31,7 +31,7 @@ GEMV_MAX_TOKENS = 16
 
 # Every entry point declared in include/aqlm.h.
 EXPORTS = ["aqlm_gemv", "aqlm_gemv_workspace_bytes", "aqlm_gemv_row_tokens", "aqlm_gemv_multi",
-           "aqlm_gemv_multi_workspace_bytes", "aqlm_gemv_check", "aqlm_dequant", "aqlm_gemm",
+           "aqlm_gemv_multi_workspace_bytes", "aqlm_gemv_multi_check", "aqlm_gemv_check", "aqlm_dequant", "aqlm_gemm",
            "aqlm_gemm_workspace_bytes", "aqlm_gemm_check", "aqlm_bf16_gemm", "aqlm_decode_indices",
            "aqlm_test_gemm_timeout", "aqlm_gemv_noalloc", "aqlm_gemv_noalloc_max_scratch_bytes",
            "aqlm_status_string", "aqlm_version",
@@ -80,6 +80,7 @@ def load_library():
         "aqlm_gemv_row_tokens": ([Shape], i32),
         "aqlm_gemv_multi": ([ctypes.POINTER(Layer), i32, vp, i32, Shape, vp, sz, vp], st),
         "aqlm_gemv_multi_workspace_bytes": ([ctypes.POINTER(Layer), i32, Shape, i32], sz),
+        "aqlm_gemv_multi_check": ([ctypes.POINTER(Layer), i32, Shape, i32, vp, sz, vp], st),
         "aqlm_gemv_check": ([Shape, i32, vp, sz, vp], st),
         "aqlm_dequant": ([vp, vp, vp, vp, Shape, vp], st),
         "aqlm_gemm": ([vp, vp, vp, vp, vp, i32, Shape, vp, sz, vp], st),
@@ -232,6 +233,15 @@ def aqlm_gemv_multi(layers, x, ys=None, workspace=None, stream=None):
     _check(lib.aqlm_gemv_multi(arr, len(layers), _p(x), T, shape, _p(workspace), wbytes, _stream(stream)),
            "aqlm_gemv_multi")
     return ys
+
+
+def aqlm_gemv_multi_check(layers, tokens, workspace, stream=None):
+    """Synchronise and return the status that aqlm_gemv_multi calls with these
+    layers, token count and workspace recorded (AQLM_OK or AQLM_ERR_TIMEOUT)."""
+    lib = load_library()
+    wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return lib.aqlm_gemv_multi_check(_layers(layers, [None] * len(layers)), len(layers),
+                                     shape_of(layers[0]["codes"]), tokens, _p(workspace), wbytes, _stream(stream))
 
 
 def aqlm_gemv_check(codes, tokens, workspace, stream=None):

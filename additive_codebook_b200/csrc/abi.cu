@@ -44,6 +44,23 @@ aqlm_status check_layer(const void *codes, const uint16_t *codebooks, const uint
 
 inline aqlm_status from_cuda(cudaError_t e) { return e == cudaSuccess ? AQLM_OK : AQLM_ERR_CUDA; }
 
+// Synchronise cs, then read and clear the status word at byte `off` of the
+// workspace (off < 0: the path has no status word, AQLM_OK).
+aqlm_status read_status_word(long long off, void *workspace, size_t workspace_bytes, cudaStream_t cs) {
+    if (off < 0) return cudaStreamSynchronize(cs) == cudaSuccess ? AQLM_OK : AQLM_ERR_CUDA;
+    if (!workspace || workspace_bytes < (size_t)off + sizeof(int32_t) || !aligned(workspace, 16))
+        return AQLM_ERR_WORKSPACE;
+    int32_t *word = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + off);
+    int32_t h = 0;
+    if (cudaMemcpyAsync(&h, word, sizeof(h), cudaMemcpyDeviceToHost, cs) != cudaSuccess) return AQLM_ERR_CUDA;
+    if (cudaStreamSynchronize(cs) != cudaSuccess) return AQLM_ERR_CUDA;
+    if (h != 0) {
+        if (cudaMemsetAsync(word, 0, sizeof(int32_t), cs) != cudaSuccess) return AQLM_ERR_CUDA;
+        if (cudaStreamSynchronize(cs) != cudaSuccess) return AQLM_ERR_CUDA;
+    }
+    return h == 0 ? AQLM_OK : AQLM_ERR_TIMEOUT;
+}
+
 }  // namespace
 
 extern "C" {
@@ -114,7 +131,7 @@ size_t aqlm_gemv_multi_workspace_bytes(const aqlm_layer *layers, int32_t n_layer
     aqlm::RowLayerIn in[AQLM_MULTI_MAX_LAYERS];
     if (multi_layers(layers, n_layers, shape, in) != AQLM_OK) return 0;
     const Dims d = aqlm::make_dims(shape);
-    if (tokens < 1 || tokens > aqlm::gemv_row_tokens(d)) return 0;
+    if (tokens < 1 || tokens > AQLM_GEMV_MAX_TOKENS) return 0;
     return aqlm::gemv_multi_workspace_bytes(in, n_layers, d, tokens);
 }
 
@@ -134,32 +151,28 @@ aqlm_status aqlm_gemv_multi(const aqlm_layer *layers, int32_t n_layers, const ui
     if (!x || tokens < 1 || tokens > AQLM_GEMV_MAX_TOKENS) return AQLM_ERR_INVALID_ARG;
     if (!aligned(x, 16)) return AQLM_ERR_MISALIGNED;
     const Dims d = aqlm::make_dims(shape);
-    if (tokens > aqlm::gemv_row_tokens(d)) return AQLM_ERR_UNSUPPORTED;
     const size_t need = aqlm::gemv_multi_workspace_bytes(in, n_layers, d, tokens);
     if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16))) return AQLM_ERR_WORKSPACE;
     return from_cuda(aqlm::launch_gemv_multi(in, n_layers, x, tokens, d, need > 0 ? workspace : nullptr,
                                              to_cuda(stream)));
 }
 
+aqlm_status aqlm_gemv_multi_check(const aqlm_layer *layers, int32_t n_layers, aqlm_shape shape, int32_t tokens,
+                                  void *workspace, size_t workspace_bytes, aqlm_stream_t stream) {
+    aqlm::RowLayerIn in[AQLM_MULTI_MAX_LAYERS];
+    aqlm_status st = multi_layers(layers, n_layers, shape, in);
+    if (st != AQLM_OK) return st;
+    if (tokens < 1 || tokens > AQLM_GEMV_MAX_TOKENS) return AQLM_ERR_INVALID_ARG;
+    const long long off = aqlm::gemv_multi_status_offset(in, n_layers, aqlm::make_dims(shape), tokens);
+    return read_status_word(off, workspace, workspace_bytes, to_cuda(stream));
+}
+
 aqlm_status aqlm_gemv_check(aqlm_shape shape, int32_t tokens, void *workspace, size_t workspace_bytes,
                             aqlm_stream_t stream) {
     if (check_shape(shape) != AQLM_OK) return AQLM_ERR_UNSUPPORTED;
     if (tokens < 1 || tokens > AQLM_GEMV_MAX_TOKENS) return AQLM_ERR_INVALID_ARG;
-    const Dims d = aqlm::make_dims(shape);
-    const long long off = aqlm::gemv_status_offset(d, tokens);
-    const cudaStream_t cs = to_cuda(stream);
-    if (off < 0) return cudaStreamSynchronize(cs) == cudaSuccess ? AQLM_OK : AQLM_ERR_CUDA;
-    if (!workspace || workspace_bytes < (size_t)off + sizeof(int32_t) || !aligned(workspace, 16))
-        return AQLM_ERR_WORKSPACE;
-    int32_t *word = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + off);
-    int32_t h = 0;
-    if (cudaMemcpyAsync(&h, word, sizeof(h), cudaMemcpyDeviceToHost, cs) != cudaSuccess) return AQLM_ERR_CUDA;
-    if (cudaStreamSynchronize(cs) != cudaSuccess) return AQLM_ERR_CUDA;
-    if (h != 0) {
-        if (cudaMemsetAsync(word, 0, sizeof(int32_t), cs) != cudaSuccess) return AQLM_ERR_CUDA;
-        if (cudaStreamSynchronize(cs) != cudaSuccess) return AQLM_ERR_CUDA;
-    }
-    return h == 0 ? AQLM_OK : AQLM_ERR_TIMEOUT;
+    return read_status_word(aqlm::gemv_status_offset(aqlm::make_dims(shape), tokens), workspace, workspace_bytes,
+                            to_cuda(stream));
 }
 
 size_t aqlm_gemm_workspace_bytes(aqlm_shape shape, int32_t tokens) {

@@ -208,6 +208,7 @@ cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint
 int gemv_row_tokens(const Dims &d);
 size_t gemv_multi_workspace_bytes(const RowLayerIn *layers, int n, const Dims &d, int tokens);
 size_t gemv_multi_counter_offset(const RowLayerIn *layers, int n, const Dims &d, int tokens);
+long long gemv_multi_status_offset(const RowLayerIn *layers, int n, const Dims &d, int tokens);
 cudaError_t launch_gemv_multi(const RowLayerIn *layers, int n, const uint16_t *x, int tokens, const Dims &d,
                               void *workspace, cudaStream_t st);
 cudaError_t launch_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,

@@ -23,6 +23,11 @@ size_t gemv_tc_counter_offset(const Dims &d, int T, int sms);
 size_t gemv_tc_status_offset(const Dims &d, int T, int sms);
 cudaError_t launch_gemv_tc(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
                            uint16_t *y, int tokens, const Dims &d, void *workspace, int sms, cudaStream_t st);
+size_t gemv_tc_multi_counter_offset(const RowLayerIn *layers, int n, const Dims &d, int T, int sms);
+size_t gemv_tc_multi_workspace_bytes(const RowLayerIn *layers, int n, const Dims &d, int T, int sms);
+size_t gemv_tc_multi_status_offset(const RowLayerIn *layers, int n, const Dims &d, int T, int sms);
+cudaError_t launch_gemv_tc_multi(const RowLayerIn *layers, int n, const uint16_t *x, int tokens, const Dims &d,
+                                 void *workspace, int sms, cudaStream_t st);
 
 namespace {
 
@@ -68,21 +73,29 @@ cudaError_t launch_gemv(const void *codes, const uint16_t *codebooks, const uint
     return cudaErrorInvalidValue;
 }
 
-// Several layers that read the same activations, in one row-kernel launch
-// (the token counts of the row kernel only).
+// Several layers that read the same activations, in one launch of the
+// kernel their token count selects.
 int gemv_row_tokens(const Dims &d) { return rows_max_tokens(d); }
 
 size_t gemv_multi_workspace_bytes(const RowLayerIn *layers, int n, const Dims &d, int tokens) {
-    return gemv_rows_multi_workspace_bytes(layers, n, d, tokens);
+    if (gemv_rows_supported(d, tokens)) return gemv_rows_multi_workspace_bytes(layers, n, d, tokens);
+    return gemv_tc_multi_workspace_bytes(layers, n, d, tokens, device_sms());
 }
 
 size_t gemv_multi_counter_offset(const RowLayerIn *layers, int n, const Dims &d, int tokens) {
-    return gemv_rows_multi_counter_offset(layers, n, d, tokens);
+    if (gemv_rows_supported(d, tokens)) return gemv_rows_multi_counter_offset(layers, n, d, tokens);
+    return gemv_tc_multi_counter_offset(layers, n, d, tokens, device_sms());
+}
+
+long long gemv_multi_status_offset(const RowLayerIn *layers, int n, const Dims &d, int tokens) {
+    if (gemv_rows_supported(d, tokens) || !gemv_tc_supported(d, tokens)) return -1;
+    return (long long)gemv_tc_multi_status_offset(layers, n, d, tokens, device_sms());
 }
 
 cudaError_t launch_gemv_multi(const RowLayerIn *layers, int n, const uint16_t *x, int tokens, const Dims &d,
                               void *workspace, cudaStream_t st) {
-    return launch_gemv_rows_multi(layers, n, x, tokens, d, workspace, device_sms(), st);
+    if (gemv_rows_supported(d, tokens)) return launch_gemv_rows_multi(layers, n, x, tokens, d, workspace, device_sms(), st);
+    return launch_gemv_tc_multi(layers, n, x, tokens, d, workspace, device_sms(), st);
 }
 
 }  // namespace aqlm

@@ -93,25 +93,63 @@ struct TcBars {
     int last;
 };
 
-struct TcArgs {
+// One layer of a launch.  A launch runs the layers that read the same x (one
+// layer, or e.g. the q, k and v projections): their row tiles are numbered one
+// after the other, layer l owning tiles [tile0, tile0 + its tiles).
+struct TcLayer {
     const uint4 *codebooks;
     const __half *scales;
     __half *y;
+    int d_out;
+    int tile0;
+};
+
+template <int NL>
+struct TcArgs {
+    TcLayer layer[NL];
+    int n_layers;
     float *partial;      // [tiles][max_segs][T][128] partial sums of split tiles
     uint32_t *counters;  // [tiles], zero between calls
     int32_t *status;     // AQLM_ERR_TIMEOUT after a wait gave up
-    int d_out, G, T;
+    int G, T;
     int n_stages;        // stages of 64 inputs per row
     int max_segs;        // segments of one tile, at most
-    long long units;     // row tiles x n_stages
+    long long units;     // row tiles (all layers) x n_stages
 };
 
+// The code tensor maps of a launch's layers (layer l in m[l]).
+template <int NL>
+struct TcCodeMaps {
+    CUtensorMap m[NL];
+};
+
+// The layer of global row tile `tile` (static indices only, so the
+// descriptors stay in the kernel's parameter space).
+template <int NL>
+__device__ __forceinline__ int layer_of(int tile, const TcArgs<NL> &a) {
+    int l = 0;
+#pragma unroll
+    for (int i = 1; i < NL; ++i)
+        if (i < a.n_layers && tile >= a.layer[i].tile0) l = i;
+    return l;
+}
+template <int NL>
+__device__ __forceinline__ TcLayer layer_at(int l, const TcArgs<NL> &a) {
+    TcLayer L = a.layer[0];
+#pragma unroll
+    for (int i = 1; i < NL; ++i)
+        if (i == l) L = a.layer[i];
+    return L;
+}
+
 // CTA c works on units [unit_start(c), unit_start(c + 1)).
-__device__ __forceinline__ long long unit_start(int c, const TcArgs &a) {
+template <typename A>
+__device__ __forceinline__ long long unit_start(int c, const A &a) {
     return (long long)c * a.units / (long long)gridDim.x;
 }
 // The CTA whose range holds unit u.
-__device__ int cta_of_unit(long long u, const TcArgs &a) {
+template <typename A>
+__device__ int cta_of_unit(long long u, const A &a) {
     int c = (int)(u * (long long)gridDim.x / a.units);
     while (c + 1 < (int)gridDim.x && unit_start(c + 1, a) <= u) ++c;
     while (c > 0 && unit_start(c, a) > u) --c;
@@ -120,7 +158,8 @@ __device__ int cta_of_unit(long long u, const TcArgs &a) {
 struct Seg {
     int tile, k0, len;  // stages [k0, k0 + len) of row tile `tile`
 };
-__device__ __forceinline__ Seg seg_at(long long u, long long u_end, const TcArgs &a) {
+template <typename A>
+__device__ __forceinline__ Seg seg_at(long long u, long long u_end, const A &a) {
     Seg g;
     g.tile = (int)(u / a.n_stages);
     g.k0 = (int)(u - (long long)g.tile * a.n_stages);
@@ -254,10 +293,10 @@ __device__ __forceinline__ uint32_t tc_index(const uint4 (&c)[V], int q, int m) 
     }
 }
 
-template <int M, int B>
-__global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm) gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_codes,
-                                                               const __grid_constant__ CUtensorMap tmap_x,
-                                                               const TcArgs a) {
+template <int M, int B, int NL>
+__global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm)
+    gemv_tc_kernel(const __grid_constant__ TcCodeMaps<NL> maps, const __grid_constant__ CUtensorMap tmap_x,
+                   const TcArgs<NL> a) {
     using F = TcFmt<M, B>;
     constexpr int kCodeVecs = F::kStageCodeBytes / 16;  // 16-byte code pieces per row per stage
     extern __shared__ uint8_t smem_raw[];
@@ -284,16 +323,21 @@ __global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm) gemv_tc_k
         mbar_init(saddr(&bars->mma_done), 1);
         bars->abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_codes)) : "memory");
+#pragma unroll
+        for (int l = 0; l < NL; ++l)
+            if (l < a.n_layers)
+                asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.m[l])) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
     }
-    if (threadIdx.x == 32) {  // this CTA's share of the (usually cold) codebooks into L2
+    if (threadIdx.x == 32) {  // this CTA's share of each layer's (usually cold) codebooks into L2
         const uint32_t cb_bytes = (uint32_t)M * F::K * 16;
         const uint32_t share = ((cb_bytes + gridDim.x - 1) / gridDim.x + 255) & ~255u;
         const uint32_t off = blockIdx.x * share;
-        if (off < cb_bytes)
-            prefetch_l2_bulk(reinterpret_cast<const uint8_t *>(a.codebooks) + off, min(share, cb_bytes - off),
-                             policy_evict_last());
+#pragma unroll
+        for (int l = 0; l < NL; ++l)
+            if (l < a.n_layers && off < cb_bytes)
+                prefetch_l2_bulk(reinterpret_cast<const uint8_t *>(layer_at(l, a).codebooks) + off,
+                                 min(share, cb_bytes - off), policy_evict_last());
     }
     if (warp == 5) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(&bars->tmem_base)),
@@ -323,9 +367,14 @@ __global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm) gemv_tc_k
                 const uint32_t par = (uint32_t)((gb / kCodeSlots) & 1);
                 if (!tc_wait(saddr(&bars->code_empty[slot]), par ^ 1, bars, a.status)) return false;
                 const uint32_t full = saddr(&bars->code_full[slot]);
+                const int ly = layer_of(g.tile, a);
+                const CUtensorMap *map = &maps.m[0];
+#pragma unroll
+                for (int i = 1; i < NL; ++i)
+                    if (i == ly) map = &maps.m[i];
                 mbar_expect_tx(full, kTcRows * kCodeBoxBytes);
-                tma_load_2d(saddr(codes_s + (size_t)slot * kTcRows * kCodeBoxBytes), &tmap_codes,
-                            (g.k0 + bj * SPB) * F::kStageCodeBytes, g.tile * kTcRows, full);
+                tma_load_2d(saddr(codes_s + (size_t)slot * kTcRows * kCodeBoxBytes), map,
+                            (g.k0 + bj * SPB) * F::kStageCodeBytes, (g.tile - layer_at(ly, a).tile0) * kTcRows, full);
                 code_issued[slot] = (int)par;
                 slot_last[slot] = bgi + min(g.len, (bj + 1) * SPB) - 1;
                 ++gb;
@@ -415,7 +464,8 @@ __global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm) gemv_tc_k
         bool waited_grid = false;
         for (long long u = u_begin; u < u_end && ok; ++j) {
             const Seg g = seg_at(u, u_end, a);
-            const int row = g.tile * kTcRows + r;
+            const TcLayer L = layer_at(layer_of(g.tile, a), a);
+            const int row = (g.tile - L.tile0) * kTcRows + r;
             for (int l = 0; l < g.len; ++l) {
                 // the row's codes of local stage l, from its box
                 const int gbox = gb0 + l / SPB, slot = gbox % kCodeSlots;
@@ -448,7 +498,7 @@ __global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm) gemv_tc_k
                     for (int m = 0; m < M; ++m)
                         cp_async16_keep<B == 8>(
                             tile + (uint32_t)(m * kTileBytes) + (uint32_t)((q ^ (r & 7)) << 4),
-                            a.codebooks + (size_t)m * F::K + tc_index<M, B, kCodeVecs>(code, q, m), bytes, keep);
+                            L.codebooks + (size_t)m * F::K + tc_index<M, B, kCodeVecs>(code, q, m), bytes, keep);
                 }
                 cp_async_arrive_noinc(saddr(&bars->full[s]));
                 // the box's codes were read into registers and used above: its slot
@@ -472,10 +522,10 @@ __global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm) gemv_tc_k
             tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), v);
             tc_fence_before();  // the next segment's MMAs overwrite the accumulator
             if (g.len == a.n_stages) {
-                if (row < a.d_out) {
-                    const float sc = __half2float(a.scales[row]);
+                if (row < L.d_out) {
+                    const float sc = __half2float(L.scales[row]);
                     for (int t = 0; t < a.T; ++t)
-                        a.y[(size_t)t * a.d_out + row] = __float2half_rn(__uint_as_float(v[t]) * sc);
+                        L.y[(size_t)t * L.d_out + row] = __float2half_rn(__uint_as_float(v[t]) * sc);
                 }
             } else {
                 const long long t_u0 = (long long)g.tile * a.n_stages;
@@ -491,8 +541,8 @@ __global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm) gemv_tc_k
                 asm volatile("bar.sync 1, %0;" ::"n"(kDecoders) : "memory");
                 if (bars->last) {  // the last segment of the tile: add all of them in input order
                     __threadfence();
-                    if (row < a.d_out) {
-                        const float sc = __half2float(a.scales[row]);
+                    if (row < L.d_out) {
+                        const float sc = __half2float(L.scales[row]);
                         // segment by segment, every token's partial at once (up to 16
                         // loads in flight); each token's sum still runs in segment order
                         float sum[kTcN];
@@ -508,7 +558,7 @@ __global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm) gemv_tc_k
                         }
 #pragma unroll
                         for (int t = 0; t < kTcN; ++t)
-                            if (t < a.T) a.y[(size_t)t * a.d_out + row] = __float2half_rn(sum[t] * sc);
+                            if (t < a.T) L.y[(size_t)t * L.d_out + row] = __float2half_rn(sum[t] * sc);
                     }
                     if (threadIdx.x == 0) a.counters[g.tile] = 0u;
                 }
@@ -565,13 +615,13 @@ struct TcPlan {
     int max_segs;       // segments of one tile, at most
 };
 
-// Stream-K plan: as many CTAs as are resident at once (two per SM), each
-// with an equal contiguous range of at least 8 stage units (fewer CTAs for
-// small layers).
-TcPlan plan_tc(const Dims &d, int sms) {
+// Stream-K plan over `tiles` row tiles (all layers): as many CTAs as are
+// resident at once (two per SM), each with an equal contiguous range of at
+// least 8 stage units (fewer CTAs for small layers).
+TcPlan plan_tc(const Dims &d, long long tiles, int sms) {
     TcPlan p;
     const int per_sm = (d.M == 1) ? TcFmt<1, 16>::kCtasPerSm : TcFmt<2, 16>::kCtasPerSm;
-    p.tiles = (d.d_out + kTcRows - 1) / kTcRows;
+    p.tiles = (int)tiles;
     p.n_stages = (d.G + kStageGroups - 1) / kStageGroups;
     p.units = (long long)p.tiles * p.n_stages;
     constexpr long long kMinUnits = 8;
@@ -587,15 +637,73 @@ TcPlan plan_tc(const Dims &d, int sms) {
     return p;
 }
 
+long long tiles_of(const RowLayerIn *layers, int n) {
+    long long t = 0;
+    for (int l = 0; l < n; ++l) t += (layers[l].d_out + kTcRows - 1) / kTcRows;
+    return t;
+}
+
 inline size_t al16(size_t v) { return (v + 15) / 16 * 16; }
 
-template <int M, int B>
-cudaError_t launch_tc(const CUtensorMap &mc, const CUtensorMap &mx, const TcArgs &a, const TcPlan &p, cudaStream_t st) {
-    auto fn = gemv_tc_kernel<M, B>;
+// Workspace: [fp32 partials of split tiles][arrival counters][status word],
+// the last two zero before a call.
+size_t tc_counter_offset(const TcPlan &p, int T) {
+    return al16((size_t)p.tiles * p.max_segs * T * kTcRows * sizeof(float));
+}
+size_t tc_workspace_bytes(const TcPlan &p, int T) {
+    return tc_counter_offset(p, T) + al16((size_t)p.tiles * sizeof(uint32_t)) + 16;
+}
+
+template <int M, int B, int NL>
+cudaError_t launch_tc(const TcCodeMaps<NL> &mc, const CUtensorMap &mx, const TcArgs<NL> &a, const TcPlan &p,
+                      cudaStream_t st) {
+    auto fn = gemv_tc_kernel<M, B, NL>;
     const cudaError_t e = opt_in_dynamic_smem(fn, TcFmt<M, B>::kSmem);
     if (e != cudaSuccess) return e;
     return launch_kernel(fn, dim3(p.ctas), dim3(kTcThreads), TcFmt<M, B>::kSmem, st, true, mc, mx, a);
 }
+
+template <int NL>
+cudaError_t launch_tc_layers(const RowLayerIn *layers, int n, const uint16_t *x, int tokens, const Dims &d,
+                             void *workspace, int sms, cudaStream_t st) {
+    const TcPlan p = plan_tc(d, tiles_of(layers, n), sms);
+    TcCodeMaps<NL> mc;
+    CUtensorMap mx;
+    TcArgs<NL> a = {};
+    int tile0 = 0;
+    for (int l = 0; l < n; ++l) {
+        if (!encode_2d(&mc.m[l], CU_TENSOR_MAP_DATA_TYPE_UINT8, layers[l].codes, (uint64_t)d.row_bytes,
+                       (uint64_t)layers[l].d_out, (uint64_t)d.row_bytes, kCodeBoxBytes, kTcRows,
+                       CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+        TcLayer &L = a.layer[l];
+        L.codebooks = reinterpret_cast<const uint4 *>(layers[l].codebooks);
+        L.scales = reinterpret_cast<const __half *>(layers[l].scales);
+        L.y = reinterpret_cast<__half *>(layers[l].y);
+        L.d_out = layers[l].d_out;
+        L.tile0 = tile0;
+        tile0 += (layers[l].d_out + kTcRows - 1) / kTcRows;
+    }
+    for (int l = n; l < NL; ++l) mc.m[l] = mc.m[0];
+    if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, (uint64_t)d.d_in, (uint64_t)tokens, (uint64_t)d.d_in * 2,
+                   kStageK, kTcN, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    a.n_layers = n;
+    a.partial = reinterpret_cast<float *>(ws);
+    a.counters = reinterpret_cast<uint32_t *>(ws + tc_counter_offset(p, tokens));
+    a.status = reinterpret_cast<int32_t *>(ws + tc_workspace_bytes(p, tokens) - 16);
+    a.G = d.G;
+    a.T = tokens;
+    a.n_stages = p.n_stages;
+    a.max_segs = p.max_segs;
+    a.units = p.units;
+    if (d.M == 1) return launch_tc<1, 16, NL>(mc, mx, a, p, st);
+    if (d.B == 8) return launch_tc<2, 8, NL>(mc, mx, a, p, st);
+    return launch_tc<2, 16, NL>(mc, mx, a, p, st);
+}
+
+constexpr int kTcMaxLayers = AQLM_MULTI_MAX_LAYERS;
 
 }  // namespace
 
@@ -606,46 +714,38 @@ bool gemv_tc_supported(const Dims &d, int T) {
     return T >= 1 && T <= AQLM_GEMV_MAX_TOKENS;
 }
 
-// Workspace: [fp32 partials of split tiles][arrival counters][status word],
-// the last two zero before a call.
+size_t gemv_tc_multi_counter_offset(const RowLayerIn *layers, int n, const Dims &d, int T, int sms) {
+    return tc_counter_offset(plan_tc(d, tiles_of(layers, n), sms), T);
+}
+size_t gemv_tc_multi_workspace_bytes(const RowLayerIn *layers, int n, const Dims &d, int T, int sms) {
+    return tc_workspace_bytes(plan_tc(d, tiles_of(layers, n), sms), T);
+}
+size_t gemv_tc_multi_status_offset(const RowLayerIn *layers, int n, const Dims &d, int T, int sms) {
+    return gemv_tc_multi_workspace_bytes(layers, n, d, T, sms) - 16;
+}
+
+cudaError_t launch_gemv_tc_multi(const RowLayerIn *layers, int n, const uint16_t *x, int tokens, const Dims &d,
+                                 void *workspace, int sms, cudaStream_t st) {
+    if (n < 1 || n > kTcMaxLayers) return cudaErrorInvalidValue;
+    if (n == 1) return launch_tc_layers<1>(layers, n, x, tokens, d, workspace, sms, st);
+    return launch_tc_layers<kTcMaxLayers>(layers, n, x, tokens, d, workspace, sms, st);
+}
+
+// single layer: the same layout with one layer
 size_t gemv_tc_counter_offset(const Dims &d, int T, int sms) {
-    const TcPlan p = plan_tc(d, sms);
-    return al16((size_t)p.tiles * p.max_segs * T * kTcRows * sizeof(float));
+    const RowLayerIn one = {nullptr, nullptr, nullptr, nullptr, d.d_out};
+    return gemv_tc_multi_counter_offset(&one, 1, d, T, sms);
 }
-
 size_t gemv_tc_workspace_bytes(const Dims &d, int T, int sms) {
-    const TcPlan p = plan_tc(d, sms);
-    return gemv_tc_counter_offset(d, T, sms) + al16((size_t)p.tiles * sizeof(uint32_t)) + 16;
+    const RowLayerIn one = {nullptr, nullptr, nullptr, nullptr, d.d_out};
+    return gemv_tc_multi_workspace_bytes(&one, 1, d, T, sms);
 }
-
 size_t gemv_tc_status_offset(const Dims &d, int T, int sms) { return gemv_tc_workspace_bytes(d, T, sms) - 16; }
 
 cudaError_t launch_gemv_tc(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
                            uint16_t *y, int tokens, const Dims &d, void *workspace, int sms, cudaStream_t st) {
-    const TcPlan p = plan_tc(d, sms);
-    CUtensorMap mc, mx;
-    if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, (uint64_t)d.row_bytes, (uint64_t)d.d_out,
-                   (uint64_t)d.row_bytes, kCodeBoxBytes, kTcRows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, (uint64_t)d.d_in, (uint64_t)tokens,
-                   (uint64_t)d.d_in * 2, kStageK, kTcN, CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    TcArgs a;
-    a.codebooks = reinterpret_cast<const uint4 *>(codebooks);
-    a.scales = reinterpret_cast<const __half *>(scales);
-    a.y = reinterpret_cast<__half *>(y);
-    a.partial = reinterpret_cast<float *>(ws);
-    a.counters = reinterpret_cast<uint32_t *>(ws + gemv_tc_counter_offset(d, tokens, sms));
-    a.status = reinterpret_cast<int32_t *>(ws + gemv_tc_status_offset(d, tokens, sms));
-    a.d_out = d.d_out;
-    a.G = d.G;
-    a.T = tokens;
-    a.n_stages = p.n_stages;
-    a.max_segs = p.max_segs;
-    a.units = p.units;
-    if (d.M == 1) return launch_tc<1, 16>(mc, mx, a, p, st);
-    if (d.B == 8) return launch_tc<2, 8>(mc, mx, a, p, st);
-    return launch_tc<2, 16>(mc, mx, a, p, st);
+    const RowLayerIn one = {codes, codebooks, scales, y, d.d_out};
+    return launch_gemv_tc_multi(&one, 1, x, tokens, d, workspace, sms, st);
 }
 
 }  // namespace aqlm

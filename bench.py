@@ -264,8 +264,8 @@ def single_call_us(ac, bench, reps=50):
     return statistics.median(out)
 
 
-def bench_block(ac, fmt, steps, warmup, l2_bytes, fused=False):
-    """Llama-2-7B decoder block: its 7 linears back to back, batch 1.  fused:
+def bench_block(ac, fmt, steps, warmup, l2_bytes, fused=False, T=1):
+    """Llama-2-7B decoder block: its 7 linears back to back, T tokens.  fused:
     q/k/v in one aqlm_gemv_multi launch and gate/up in another (they read the
     same x), o and down alone -- 4 launches per block instead of 7."""
     import torch
@@ -273,19 +273,28 @@ def bench_block(ac, fmt, steps, warmup, l2_bytes, fused=False):
     specs = [LayerSpec(o, i, M, B) for _, o, i in LLAMA7B_SHAPES]
     per_block = sum(s.code_bytes() + s.codebook_bytes() + 2 * s.d_out for s in specs)
     R = max(2, int(np.ceil(3 * l2_bytes / per_block)))
-    blocks = [[Layers(s, 1, 1, seed=100 * r + k) for k, s in enumerate(specs)] for r in range(R)]
-    ys = [torch.empty((1, s.d_out), dtype=torch.float16, device="cuda") for s in specs]
+    blocks = [[Layers(s, 1, T, seed=100 * r + k) for k, s in enumerate(specs)] for r in range(R)]
+    ys = [torch.empty((T, s.d_out), dtype=torch.float16, device="cuda") for s in specs]
     x_in = {4096: blocks[0][0].x, 11008: blocks[0][6].x}
     groups = [[0, 1, 2], [3], [4, 5], [6]] if fused else [[k] for k in range(len(specs))]
 
+    # one zeroed workspace per launch group (the kernels leave it ready for the next call)
+    wss = []
+    for grp in groups:
+        if len(grp) == 1:
+            need = ac.gemv_workspace_bytes(ac.shape_of(blocks[0][grp[0]].copies[0]["codes"]), T)
+        else:
+            need = ac.gemv_multi_workspace_bytes([blocks[0][k].copies[0] for k in grp], T)
+        wss.append(torch.zeros(need, dtype=torch.uint8, device="cuda") if need else None)
+
     def block(blk):
-        for grp in groups:
+        for grp, ws in zip(groups, wss):
             x = x_in[specs[grp[0]].d_in]
             if len(grp) == 1:
                 d = blk[grp[0]].copies[0]
-                ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], x, y=ys[grp[0]])
+                ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], x, y=ys[grp[0]], workspace=ws)
             else:
-                ac.aqlm_gemv_multi([blk[k].copies[0] for k in grp], x, ys=[ys[k] for k in grp])
+                ac.aqlm_gemv_multi([blk[k].copies[0] for k in grp], x, ys=[ys[k] for k in grp], workspace=ws)
 
     g = torch.cuda.CUDAGraph()
     for blk in blocks:
@@ -296,7 +305,7 @@ def bench_block(ac, fmt, steps, warmup, l2_bytes, fused=False):
             block(blk)
     ms = time_replays(g, steps, warmup)
     us_block = ms * 1e3 / (steps * R)
-    return {"us_per_block": us_block, "bytes_per_block": sum(algo_bytes(s, 1) for s in specs), "copies": R,
+    return {"us_per_block": us_block, "bytes_per_block": sum(algo_bytes(s, T) for s in specs), "copies": R,
             "launches_per_block": len(groups)}
 
 
@@ -460,11 +469,11 @@ def run_gpu(args):
     if not args.quick:
         r = bench_gemv(ac, LayerSpec(4096, 4096, 2, 8), 1, max(3, args.steps // 2), args.warmup, l2)
         detail["2x8 4096x4096 T1"] = _gemv_detail(r, peaks)
-        for fmt in ((1, 16), (2, 8)):
+        for fmt, T in (((1, 16), 1), ((2, 8), 1), ((1, 16), 4)):
             for fused in (False, True):
-                b = bench_block(ac, fmt, max(3, args.steps // 2), args.warmup, l2, fused=fused)
+                b = bench_block(ac, fmt, max(3, args.steps // 2), args.warmup, l2, fused=fused, T=T)
                 gbs = b["bytes_per_block"] / (b["us_per_block"] * 1e-6) / 1e9
-                detail[f"llama2-7b block {fmt[0]}x{fmt[1]} T1" + (" fused qkv, gate+up" if fused else "")] = {
+                detail[f"llama2-7b block {fmt[0]}x{fmt[1]} T{T}" + (" fused qkv, gate+up" if fused else "")] = {
                     "us_per_block": round(b["us_per_block"], 3), "gbs": round(gbs, 1),
                     "hbm_frac": round(gbs / peaks["hbm_gbs"], 4), "launches": b["launches_per_block"]}
         for name, o, i in LLAMA70B_SHAPES:

@@ -136,9 +136,8 @@ AQLM_API aqlm_status aqlm_gemv(const void *codes, const uint16_t *codebooks, con
  * on the current device (0 if none); returns 0 for invalid arguments too. */
 AQLM_API size_t aqlm_gemv_workspace_bytes(aqlm_shape shape, int32_t tokens);
 
-/* Most tokens for which aqlm_gemv runs on the CUDA cores with no device waits
- * (1x16: 2, 2x16: 3, 2x8: 4), which is also the most aqlm_gemv_multi takes;
- * 0 for an unsupported shape.  The value belongs to this build of the library
+/* Most tokens for which aqlm_gemv and aqlm_gemv_multi run on the CUDA cores
+ * with no device waits (1x16: 2, 2x16: 3, 2x8: 4); 0 for an unsupported shape.  The value belongs to this build of the library
  * (it follows measurements of both kernels), so ask rather than hard-code it. */
 AQLM_API int32_t aqlm_gemv_row_tokens(aqlm_shape shape);
 
@@ -156,15 +155,17 @@ AQLM_API int32_t aqlm_gemv_row_tokens(aqlm_shape shape);
  *   (shape.d_in, group, num_codebooks, codebook_bits; shape.d_out is ignored)
  *   and its own codes, codebooks, scales, output and d_out >= 1.
  *   x: [tokens][d_in] fp16, read by every layer.
- *   tokens: 1 .. aqlm_gemv_row_tokens(shape); more -> AQLM_ERR_UNSUPPORTED
- *   (call aqlm_gemv per layer for those).
+ *   tokens: 1 .. 16.  Up to aqlm_gemv_row_tokens(shape) the row kernel runs
+ *   the layers with no device waits; past that the tensor-core kernel runs
+ *   them (its row tiles of all layers share one work split), with bounded
+ *   waits whose timeout status aqlm_gemv_multi_check() reads.
  *   workspace: as aqlm_gemv's, sized by aqlm_gemv_multi_workspace_bytes()
  *   (0 = none needed, NULL allowed); zero-filled before its first use, left
  *   ready for the next call; calls sharing it must not overlap on the GPU.
- * Errors: n_layers outside 1..AQLM_MULTI_MAX_LAYERS or a NULL pointer ->
- * AQLM_ERR_INVALID_ARG; alignment as aqlm_gemv (per layer) ->
- * AQLM_ERR_MISALIGNED; no launch happens on any error but AQLM_ERR_CUDA.
- * No device waits.  Launch: programmatic dependent launch, as aqlm_gemv.
+ * Errors: n_layers outside 1..AQLM_MULTI_MAX_LAYERS, a NULL pointer or tokens
+ * outside 1..16 -> AQLM_ERR_INVALID_ARG; alignment as aqlm_gemv (per layer)
+ * -> AQLM_ERR_MISALIGNED; no launch happens on any error but AQLM_ERR_CUDA.
+ * Launch: programmatic dependent launch, as aqlm_gemv.
  */
 AQLM_API aqlm_status aqlm_gemv_multi(const aqlm_layer *layers, int32_t n_layers, const uint16_t *x, int32_t tokens,
                                      aqlm_shape shape, void *workspace, size_t workspace_bytes,
@@ -175,6 +176,12 @@ AQLM_API aqlm_status aqlm_gemv_multi(const aqlm_layer *layers, int32_t n_layers,
  * none); returns 0 for invalid arguments too. */
 AQLM_API size_t aqlm_gemv_multi_workspace_bytes(const aqlm_layer *layers, int32_t n_layers, aqlm_shape shape,
                                                 int32_t tokens);
+
+/* aqlm_gemv_check for aqlm_gemv_multi calls with these layers (only their
+ * d_out is read), format, token count and workspace. */
+AQLM_API aqlm_status aqlm_gemv_multi_check(const aqlm_layer *layers, int32_t n_layers, aqlm_shape shape,
+                                           int32_t tokens, void *workspace, size_t workspace_bytes,
+                                           aqlm_stream_t stream);
 
 /*
  * aqlm_gemv_check -- synchronise `stream` and return the status that the

@@ -185,10 +185,10 @@ def test_gemv_multi_argument_errors():
     assert lib.aqlm_gemv_multi(q, 3, ODD, 1, s, NULL, 0, NULL) == ac.AQLM_ERR_MISALIGNED
     assert lib.aqlm_gemv_multi(q, 3, D16, 0, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
     assert lib.aqlm_gemv_multi(q, 3, D16, 17, s, NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
-    # past the row kernel's token count the call is refused (aqlm_gemv per layer instead)
-    assert lib.aqlm_gemv_multi(q, 3, D16, 5, s, NULL, 0, NULL) == ac.AQLM_ERR_UNSUPPORTED
+    # past the row kernel's token count: the tensor-core kernel, whose workspace holds a status word
     s16 = shape(d_out=0, d_in=4096, M=1, B=16)
-    assert lib.aqlm_gemv_multi(q, 3, D16, 3, s16, NULL, 0, NULL) == ac.AQLM_ERR_UNSUPPORTED
+    assert lib.aqlm_gemv_multi_workspace_bytes(q, 3, s16, 3) >= 16
+    assert lib.aqlm_gemv_multi(q, 3, D16, 3, s16, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
     assert lib.aqlm_gemv_multi(q, 3, D16, 1, shape(d_out=0, M=3), NULL, 0, NULL) == ac.AQLM_ERR_UNSUPPORTED
 
 
@@ -197,7 +197,8 @@ def test_gemv_multi_workspace_rules():
     s = shape(d_out=0, d_in=4096, M=1, B=16)
     q = _multi(4096, 1024, 1024)
     assert lib.aqlm_gemv_multi_workspace_bytes(q, 3, s, 1) == 0       # 8 KiB of activations: no split
-    assert lib.aqlm_gemv_multi_workspace_bytes(q, 3, s, 3) == 0       # past the row kernel: invalid
+    assert lib.aqlm_gemv_multi_workspace_bytes(q, 3, s, 3) >= 16      # tensor cores: status word at least
+    assert lib.aqlm_gemv_multi_workspace_bytes(q, 3, s, 17) == 0
     assert lib.aqlm_gemv_multi_workspace_bytes(q, 0, s, 1) == 0
     # 28672 inputs, 1 token: two activation slices; partials for all 6144
     # rows, then one counter per 8 rows of each layer
