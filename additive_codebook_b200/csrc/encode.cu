@@ -12,10 +12,13 @@
 //              the sum of squares in double, lane l of a warp summing inputs
 //              l, l+32, ... in order, then a butterfly of shuffles;
 //   groups     the row's inputs divided by its scale (binary32 division);
-//   distance   squared Euclidean in binary32: lanes 0,2,4,6 and 1,3,5,7 as two
-//              fused multiply-add chains (one packed fp32x2 chain), then e + o;
-//              the nearest codeword has the least distance, ties to the lowest
-//              index;
+//   nearest    least squared Euclidean distance |v - c|^2, ranked by the score
+//              |c|^2 - 2<v, c> (|v|^2 is common to every codeword), ties to
+//              the lowest index; in binary32 each of |c|^2 and <v, c> is lanes
+//              0,2,4,6 and 1,3,5,7 as two fused multiply-add chains (one packed
+//              fp32x2 chain), then e + o, and score = fma(-2, <v, c>, |c|^2);
+//              the distance reported for the winner is e + o of the squared
+//              differences in the same pattern;
 //   k-means    Lloyd updates: a centroid is the mean of its groups (sums in
 //              double), an empty one keeps its value; codebook m is k-means
 //              of the residuals left by codebooks 0..m-1, started from the
@@ -26,12 +29,12 @@
 // The nearest-codeword search is the expensive step (every group against
 // every codeword: 2^16 for 1x16) and runs on the CUDA cores in exact binary32
 // so that its integer results can be compared bit for bit.  Each thread keeps
-// four groups in registers and streams the codebook through shared memory
-// (stored negated, so a difference is one packed add); a CTA covers 1024
-// groups and a range of codewords, and the ranges' winners meet through a
-// 64-bit atomic minimum of (distance bits << 32 | index): distances are never
-// negative, so their bit patterns order like the values, and equal distances
-// fall to the lower index, exactly the tie rule.
+// four groups in registers and streams the codebook, with each codeword's
+// |c|^2, through shared memory; a CTA covers 1024 groups and a range of
+// codewords, and the ranges' winners meet through a 64-bit atomic minimum of
+// (key(score) << 32 | index), key the order-preserving map of a float onto
+// the unsigned integers: equal scores fall to the lower index, exactly the
+// tie rule.
 #include "common.cuh"
 
 namespace aqlm {
@@ -68,16 +71,33 @@ __global__ void __launch_bounds__(256) encode_scales_kernel(const float *__restr
 
 // ---- nearest codeword -------------------------------------------------------
 
-__device__ __forceinline__ unsigned long long pack_best(float d, int k) {
-    return ((unsigned long long)__float_as_uint(d) << 32) | (unsigned int)k;
+// Order-preserving key of a finite float: sign bit flipped for x >= 0, every
+// bit flipped for x < 0 (-0 is taken as +0, so equal values share a key).
+__device__ __forceinline__ unsigned long long pack_best(float s, int k) {
+    const uint32_t b = __float_as_uint(s == 0.0f ? 0.0f : s);
+    const uint32_t key = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return ((unsigned long long)key << 32) | (unsigned int)k;
 }
 
-// best[n] = min over codewords k in this CTA's range of pack(distance, k).
+// |c|^2 in the pattern of the score: even and odd lanes as fma chains, e + o.
+__device__ __forceinline__ float norm2(const float4 a, const float4 b) {
+    float e = __fmul_rn(a.x, a.x), o = __fmul_rn(a.y, a.y);
+    e = __fmaf_rn(a.z, a.z, e);
+    o = __fmaf_rn(a.w, a.w, o);
+    e = __fmaf_rn(b.x, b.x, e);
+    o = __fmaf_rn(b.y, b.y, o);
+    e = __fmaf_rn(b.z, b.z, e);
+    o = __fmaf_rn(b.w, b.w, o);
+    return __fadd_rn(e, o);
+}
+
+// best[n] = min over codewords k in this CTA's range of pack(score, k).
 // Codebook C [K][8] fp32; the CTA's range is [k_begin, k_end).
 __global__ void __launch_bounds__(kNearThreads) nearest_kernel(const float *__restrict__ V, long long N,
                                                                const float *__restrict__ C, int K, int k_per_cta,
                                                                unsigned long long *__restrict__ best) {
-    __shared__ float4 cs[kNearChunk][2];  // negated codewords
+    __shared__ float4 cs[kNearChunk][2];
+    __shared__ float cc[kNearChunk];  // |c|^2
     const long long n0 = (long long)blockIdx.x * kNearGroups + threadIdx.x;
     const int k_begin = blockIdx.y * k_per_cta;
     const int k_end = min(K, k_begin + k_per_cta);
@@ -102,29 +122,29 @@ __global__ void __launch_bounds__(kNearThreads) nearest_kernel(const float *__re
     for (int c0 = k_begin; c0 < k_end; c0 += kNearChunk) {
         const int cn = min(kNearChunk, k_end - c0);
         __syncthreads();
-        for (int i = threadIdx.x; i < cn * 2; i += kNearThreads) {
-            const float4 w = reinterpret_cast<const float4 *>(C)[2 * (long long)c0 + i];
-            cs[i >> 1][i & 1] = make_float4(-w.x, -w.y, -w.z, -w.w);
+        for (int i = threadIdx.x; i < cn; i += kNearThreads) {
+            const float4 a = reinterpret_cast<const float4 *>(C)[2 * ((long long)c0 + i)];
+            const float4 b = reinterpret_cast<const float4 *>(C)[2 * ((long long)c0 + i) + 1];
+            cs[i][0] = a;
+            cs[i][1] = b;
+            cc[i] = norm2(a, b);
         }
         __syncthreads();
         for (int j = 0; j < cn; ++j) {
             const float4 a = cs[j][0], b = cs[j][1];
+            const float n2 = cc[j];
             const float2 c01 = make_float2(a.x, a.y), c23 = make_float2(a.z, a.w);
             const float2 c45 = make_float2(b.x, b.y), c67 = make_float2(b.z, b.w);
 #pragma unroll
             for (int p = 0; p < kNearPerThread; ++p) {
-                // (even, odd) lanes of the squared differences, two fma chains
-                const float2 d01 = __fadd2_rn(v[p][0], c01);
-                const float2 d23 = __fadd2_rn(v[p][1], c23);
-                const float2 d45 = __fadd2_rn(v[p][2], c45);
-                const float2 d67 = __fadd2_rn(v[p][3], c67);
-                float2 eo = __fmul2_rn(d01, d01);
-                eo = __ffma2_rn(d23, d23, eo);
-                eo = __ffma2_rn(d45, d45, eo);
-                eo = __ffma2_rn(d67, d67, eo);
-                const float d = __fadd_rn(eo.x, eo.y);
-                if (d < bd[p]) {
-                    bd[p] = d;
+                // (even, odd) lanes of <v, c>, two fma chains
+                float2 eo = __fmul2_rn(v[p][0], c01);
+                eo = __ffma2_rn(v[p][1], c23, eo);
+                eo = __ffma2_rn(v[p][2], c45, eo);
+                eo = __ffma2_rn(v[p][3], c67, eo);
+                const float s = __fmaf_rn(-2.0f, __fadd_rn(eo.x, eo.y), n2);
+                if (s < bd[p]) {
+                    bd[p] = s;
                     bk[p] = c0 + j;
                 }
             }
@@ -142,13 +162,26 @@ __global__ void fill_u64_kernel(unsigned long long *p, long long n, unsigned lon
         p[i] = v;
 }
 
-// idx[n] (and dist[n]) from the packed winners.
-__global__ void unpack_best_kernel(const unsigned long long *__restrict__ best, long long N, int32_t *__restrict__ idx,
-                                   float *__restrict__ dist) {
+// idx[n] from the packed winners, and dist[n] = |v - c|^2 of the winner: the
+// squared differences' even and odd lanes as fma chains, then e + o.
+__global__ void unpack_best_kernel(const unsigned long long *__restrict__ best, long long N,
+                                   const float *__restrict__ V, const float *__restrict__ C,
+                                   int32_t *__restrict__ idx, float *__restrict__ dist) {
     for (long long n = blockIdx.x * (long long)blockDim.x + threadIdx.x; n < N; n += (long long)gridDim.x * blockDim.x) {
-        const unsigned long long b = best[n];
-        if (idx) idx[n] = (int32_t)(uint32_t)(b & 0xffffffffull);
-        if (dist) dist[n] = __uint_as_float((uint32_t)(b >> 32));
+        const uint32_t k = (uint32_t)(best[n] & 0xffffffffull);
+        if (idx) idx[n] = (int32_t)k;
+        if (dist) {
+            float d[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) d[t] = __fsub_rn(V[n * 8 + t], C[(long long)k * 8 + t]);
+            float e = __fmul_rn(d[0], d[0]), o = __fmul_rn(d[1], d[1]);
+#pragma unroll
+            for (int t = 2; t < 8; t += 2) {
+                e = __fmaf_rn(d[t], d[t], e);
+                o = __fmaf_rn(d[t + 1], d[t + 1], o);
+            }
+            dist[n] = __fadd_rn(e, o);
+        }
     }
 }
 
@@ -269,7 +302,7 @@ cudaError_t launch_nearest(const float *V, long long N, const float *C, int K, i
     auto *best = static_cast<unsigned long long *>(workspace);
     cudaError_t e = launch_nearest_packed(V, N, C, K, best, st);
     if (e != cudaSuccess || N == 0) return e;
-    unpack_best_kernel<<<elementwise_grid(N), 256, 0, st>>>(best, N, idx, dist);
+    unpack_best_kernel<<<elementwise_grid(N), 256, 0, st>>>(best, N, V, C, idx, dist);
     return cudaGetLastError();
 }
 

@@ -357,7 +357,7 @@ def bench_prefill(ac, spec, tokens, reps, warmup):
 
 # Lane operations of one distance evaluation: 8 differences, 8 squares
 # accumulated by multiply / fused multiply-add, 1 addition of the two chains.
-DIST_LANE_OPS = 17
+DIST_LANE_OPS = 10
 
 
 def bench_encode(ac, spec, reps=3):

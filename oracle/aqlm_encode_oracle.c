@@ -22,11 +22,14 @@
  *      pattern below) so that the binary16 result is reproducible;
  *   E2 the groups to encode are the row's inputs divided by the scale
  *      (binary32 division, correctly rounded);
- *   E3 distance between a group v and a codeword c: squared Euclidean,
- *      evaluated in binary32 as e + o with e the fused multiply-add chain of
- *      the squared differences of lanes 0, 2, 4, 6 and o that of lanes 1, 3,
- *      5, 7; the nearest codeword is the one of least distance, ties to the
- *      lowest index;
+ *   E3 nearest codeword: the one of least squared Euclidean distance
+ *      |v - c|^2 = |v|^2 + score(v, c), ranked by the score
+ *      score = |c|^2 - 2 <v, c> (|v|^2 is the same for every codeword), ties
+ *      to the lowest index.  In binary32: |c|^2 = e + o and <v, c> = e' + o',
+ *      each e the fused multiply-add chain of lanes 0, 2, 4, 6 (the first a
+ *      plain product) and o that of lanes 1, 3, 5, 7; score = fma(-2, <v, c>,
+ *      |c|^2).  The distance reported for the chosen codeword is e + o over
+ *      the squared differences (v_t - c_t)^2, in the same pattern;
  *   E4 k-means update (Lloyd): a centroid becomes the mean of the groups
  *      assigned to it (sums in double, one rounding to binary32); a centroid
  *      with no group keeps its value;
@@ -130,6 +133,27 @@ int aqlm_oracle_encode_scales(const float *W, int64_t d_out, int64_t d_in, uint1
 
 /* ---- E3: nearest codeword ------------------------------------------------ */
 
+/* Even lanes and odd lanes of a . b as two fused multiply-add chains. */
+static float dot8(const float *a, const float *b)
+{
+    float e = a[0] * b[0];
+    e = fmaf(a[2], b[2], e);
+    e = fmaf(a[4], b[4], e);
+    e = fmaf(a[6], b[6], e);
+    float o = a[1] * b[1];
+    o = fmaf(a[3], b[3], o);
+    o = fmaf(a[5], b[5], o);
+    o = fmaf(a[7], b[7], o);
+    return e + o;
+}
+
+/* The ranking score |c|^2 - 2 <v, c>, with |c|^2 given. */
+static float score(const float *v, const float *c, float cc)
+{
+    return fmaf(-2.0f, dot8(v, c), cc);
+}
+
+/* Squared distance of the chosen codeword (reported, not ranked). */
 static float distance(const float *v, const float *c)
 {
     float d[8];
@@ -145,23 +169,41 @@ static float distance(const float *v, const float *c)
     return e + o;
 }
 
+/* The nearest codeword of v: least score, ties to the lowest index. */
+static int64_t nearest_one(const float *v, const float *C, const float *cc, int64_t K)
+{
+    int64_t best = 0;
+    float bs = score(v, C, cc[0]);
+    for (int64_t k = 1; k < K; ++k) {
+        const float sk = score(v, C + k * 8, cc[k]);
+        if (sk < bs) {
+            bs = sk;
+            best = k;
+        }
+    }
+    return best;
+}
+
+static float *norms(const float *C, int64_t K)
+{
+    float *cc = (float *)malloc((size_t)K * sizeof(float));
+    if (cc)
+        for (int64_t k = 0; k < K; ++k) cc[k] = dot8(C + k * 8, C + k * 8);
+    return cc;
+}
+
 int aqlm_oracle_nearest(const float *V, int64_t N, const float *C, int64_t K, int32_t *idx, float *dist)
 {
     if (N < 0 || K < 1) return 1;
+    float *cc = norms(C, K);
+    if (!cc) return 2;
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; ++n) {
-        int64_t best = 0;
-        float bd = distance(V + n * 8, C);
-        for (int64_t k = 1; k < K; ++k) {
-            const float dk = distance(V + n * 8, C + k * 8);
-            if (dk < bd) {
-                bd = dk;
-                best = k;
-            }
-        }
+        const int64_t best = nearest_one(V + n * 8, C, cc, K);
         idx[n] = (int32_t)best;
-        if (dist) dist[n] = bd;
+        if (dist) dist[n] = distance(V + n * 8, C + best * 8);
     }
+    free(cc);
     return 0;
 }
 
@@ -238,25 +280,23 @@ int aqlm_oracle_encode_greedy(const float *V, int64_t N, const uint16_t *codeboo
     float *C = (float *)malloc((size_t)M * K * 8 * sizeof(float));
     if (!C) return 2;
     for (int64_t i = 0; i < (int64_t)M * K * 8; ++i) C[i] = half_to_float(codebooks[i]);
+    float *cc = norms(C, (int64_t)M * K);
+    if (!cc) {
+        free(C);
+        return 2;
+    }
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; ++n) {
         float r[8];
         memcpy(r, V + n * 8, sizeof(r));
         for (int m = 0; m < M; ++m) {
             const float *Cm = C + (int64_t)m * K * 8;
-            int64_t best = 0;
-            float bd = distance(r, Cm);
-            for (int64_t k = 1; k < K; ++k) {
-                const float dk = distance(r, Cm + k * 8);
-                if (dk < bd) {
-                    bd = dk;
-                    best = k;
-                }
-            }
+            const int64_t best = nearest_one(r, Cm, cc + (int64_t)m * K, K);
             codes[n * M + m] = (uint16_t)best;
             for (int t = 0; t < 8; ++t) r[t] = r[t] - Cm[best * 8 + t];
         }
     }
     free(C);
+    free(cc);
     return 0;
 }

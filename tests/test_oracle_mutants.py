@@ -43,9 +43,11 @@ MUTANTS = {
     # encoding
     "half_ties_away": (ENCODE, "double q = rint(ldexp(a, 11 - e));", "double q = round(ldexp(a, 11 - e));"),
     "scale_mean_abs": (ENCODE, "acc += (double)row[k] * (double)row[k];", "acc += fabs((double)row[k]);"),
-    "nearest_ties_high": (ENCODE, "const float dk = distance(V + n * 8, C + k * 8);\n            if (dk < bd) {",
-                          "const float dk = distance(V + n * 8, C + k * 8);\n            if (dk <= bd) {"),
+    "nearest_ties_high": (ENCODE, "if (sk < bs) {", "if (sk <= bs) {"),
     "distance_drops_lane": (ENCODE, "o = fmaf(d[7], d[7], o);", "o = o;"),
+    "score_drops_lane": (ENCODE, "o = fmaf(a[7], b[7], o);", "o = o;"),
+    "score_wrong_sign": (ENCODE, "return fmaf(-2.0f, dot8(v, c), cc);", "return fmaf(2.0f, dot8(v, c), cc);"),
+    "score_drops_norm": (ENCODE, "return fmaf(-2.0f, dot8(v, c), cc);", "return fmaf(-2.0f, dot8(v, c), 0.0f * cc);"),
     "update_off_by_one": (ENCODE, "(float)(sums[k * 8 + t] / (double)counts[k])",
                           "(float)(sums[k * 8 + t] / (double)(counts[k] + 1))"),
     "residual_not_subtracted": (ENCODE, "R[n * 8 + t] = R[n * 8 + t] - C[(int64_t)idx[n] * 8 + t];",
