@@ -27,10 +27,10 @@
 //     its slice of x); each writes fp32 row partials to the caller's workspace
 //     and the last CTA of a row range to arrive (an atomic counter, no waiting)
 //     adds them in split order, scales, rounds, and resets the counter.
-//   - Programmatic dependent launch: codebooks are prefetched into L2 and
-//     the first items' codes and codewords fetched before griddepcontrol.wait
-//     (weights are constant); x is read and y, the partials and the counters
-//     are written only after it.
+//   - Programmatic dependent launch: codebooks (and, for 2x8, x) are
+//     prefetched into L2 and the first items' codes and codewords fetched
+//     before griddepcontrol.wait (weights are constant); x is read and y, the
+//     partials and the counters are written only after it.
 #include "common.cuh"
 
 namespace aqlm {
@@ -153,6 +153,17 @@ __global__ void __launch_bounds__(RowFmt<M, B>::kThreads, 2) gemv_rows_kernel(co
         }
     } else {
         for (int c = threadIdx.x; c < M * F::K * kCbCopies; c += F::kThreads) cbs[c] = L.codebooks[c >> 3];
+        // 2x8 (whose CTA of the next launch is resident early): this CTA's
+        // slice of the activations into L2.  A prefetch returns no value, so
+        // it may precede the grid-dependency wait: what the previous grid
+        // writes to x lands in L2, where the loads after the wait read it.
+        // (1x16 / 2x16 CTAs start only as the previous launch's end, with no
+        // lead time for it; measured there, it cost 0.1 us per 4096x4096 layer.)
+        if (threadIdx.x == 32 && n_chunks > 0) {
+            for (int t = 0; t < T; ++t)
+                prefetch_l2_bulk(a.x + (size_t)t * a.d_in + (size_t)c0 * GPC * kGroup, (uint32_t)n_chunks * GPC * 16,
+                                 keep_pol);
+        }
     }
     // the scales of the warp's first 32 rows, lane j holding row j's (weights:
     // read before the grid-dependency wait, off the critical path)
