@@ -211,6 +211,9 @@ __global__ void __launch_bounds__(RowFmt<M, B>::kThreads, 2) gemv_rows_kernel(co
         gather(ch0, it0, cwA);
         gather(ch1, it1, cwB);
     }
+    // the next launch may be scheduled from here on (its own wait still
+    // holds it until this grid has completed)
+    grid_dep_launch();
     grid_dep_wait();
     {
         const int ng = n_chunks * GPC;  // groups of the slice
@@ -222,7 +225,6 @@ __global__ void __launch_bounds__(RowFmt<M, B>::kThreads, 2) gemv_rows_kernel(co
         }
         __syncthreads();
     }
-    grid_dep_launch();
 
     // two fp32 chains per token (even and odd lanes of the groups)
     float acc[T], acc2[T];
