@@ -54,16 +54,42 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def strip_c_comments(text):
+    """C/C++ source without its comments and blank lines (string and
+    character literals kept), so that editing documentation leaves the hash
+    of the code unchanged."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            while i < n and text[i] != "\n":
+                i += 1
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return "\n".join(l.rstrip() for l in "".join(out).splitlines() if l.strip())
+
+
 def kernel_source_hash(files):
-    """Hash of the sources a kernel is compiled from (names relative to the
-    package's csrc/ or to include/)."""
+    """Hash of the code (comments stripped) of the sources a kernel is
+    compiled from (names relative to the package's csrc/ or to include/)."""
     h = hashlib.sha256()
     for f in sorted(files):
         path = os.path.join(ROOT, "additive_codebook_b200", "csrc", f)
         if not os.path.exists(path):
             path = os.path.join(ROOT, "include", f)
         h.update(f.encode())
-        h.update(open(path, "rb").read())
+        h.update(strip_c_comments(open(path, encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -302,10 +302,14 @@ AQLM_API size_t aqlm_gemv_noalloc_max_scratch_bytes(void);
  *               l, l+32, ... in order, partial sums combined pairwise
  *               (l + (l ^ 16), then ^ 8, ^ 4, ^ 2, ^ 1); sqrt(sum / d_in);
  *   groups      v = W[i][8j .. 8j+7] / s_i (binary32 division), [d_out*d_in/8][8];
- *   distance    squared Euclidean in binary32: e = chain of fused multiply-adds
- *               of the squared differences of lanes 0, 2, 4, 6 (the first a plain
- *               product), o the same for lanes 1, 3, 5, 7, distance = e + o;
- *   nearest     least distance, ties to the lowest index;
+ *   nearest     least squared Euclidean distance |v - c|^2, ranked by the
+ *               score |c|^2 - 2<v, c> (|v|^2 is common to every codeword),
+ *               ties to the lowest index; in binary32 each of |c|^2 and <v, c>
+ *               is e + o, e the chain of fused multiply-adds of lanes 0, 2,
+ *               4, 6 (the first a plain product) and o that of lanes 1, 3, 5,
+ *               7, and score = fma(-2, <v, c>, |c|^2);
+ *   distance    (reported for the chosen codeword) e + o of the squared
+ *               differences (v_t - c_t)^2 in the same pattern;
  *   k-means     a centroid becomes the mean of its groups (sums in double, one
  *               rounding), one without groups keeps its value; codebook m is
  *               k-means of the residuals left by codebooks 0..m-1;
