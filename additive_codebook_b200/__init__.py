@@ -32,7 +32,7 @@ GEMV_MAX_TOKENS = 16
 # Every entry point declared in include/aqlm.h.
 EXPORTS = ["aqlm_gemv", "aqlm_gemv_workspace_bytes", "aqlm_gemv_row_tokens", "aqlm_gemv_multi",
            "aqlm_gemv_multi_workspace_bytes", "aqlm_gemv_multi_check", "aqlm_gemv_check", "aqlm_dequant", "aqlm_gemm",
-           "aqlm_gemm_workspace_bytes", "aqlm_gemm_check", "aqlm_bf16_gemm", "aqlm_decode_indices",
+           "aqlm_gemm_workspace_bytes", "aqlm_gemm_check", "aqlm_bf16_gemm", "aqlm_bf16_gemm_tile_n", "aqlm_decode_indices",
            "aqlm_test_gemm_timeout", "aqlm_gemv_noalloc", "aqlm_gemv_noalloc_max_scratch_bytes",
            "aqlm_status_string", "aqlm_version",
            "aqlm_encode_scales", "aqlm_nearest_workspace_bytes", "aqlm_nearest_codeword",
@@ -87,6 +87,7 @@ def load_library():
         "aqlm_gemm_workspace_bytes": ([Shape, i32], sz),
         "aqlm_gemm_check": ([vp, sz, vp], st),
         "aqlm_bf16_gemm": ([vp, vp, vp, i32, i32, i32, vp, vp], st),
+        "aqlm_bf16_gemm_tile_n": ([i32, i32, i32], i32),
         "aqlm_decode_indices": ([vp, vp, Shape, vp], st),
         "aqlm_test_gemm_timeout": ([vp, vp, vp, i32, i32, i32, vp, u64, vp], st),
         "aqlm_gemv_noalloc": ([vp, vp, vp, vp, vp, i32, Shape, vp], st),
@@ -295,6 +296,11 @@ def aqlm_gemm_check(workspace, stream=None):
     """Synchronise and return the status recorded in the GEMM workspace."""
     lib = load_library()
     return lib.aqlm_gemm_check(_p(workspace), workspace.numel(), _stream(stream))
+
+
+def bf16_gemm_tile_n(tokens, n, sms):
+    """Output tile width the tensor-core GEMM uses for tokens x n on `sms` SMs."""
+    return int(load_library().aqlm_bf16_gemm_tile_n(int(tokens), int(n), int(sms)))
 
 
 def aqlm_bf16_gemm(X, W, Y=None, status=None, stream=None):

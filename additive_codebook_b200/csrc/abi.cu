@@ -222,6 +222,11 @@ aqlm_status aqlm_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, in
     return from_cuda(aqlm::launch_bf16_gemm(X, W, Y, tokens, n, k, status, to_cuda(stream)));
 }
 
+int32_t aqlm_bf16_gemm_tile_n(int32_t tokens, int32_t n, int32_t sms) {
+    if (tokens < 1 || n < 1 || sms < 1) return 0;
+    return aqlm::gemm_tile_n(tokens, n, sms);
+}
+
 aqlm_status aqlm_test_gemm_timeout(const uint16_t *X, const uint16_t *W, uint16_t *Y, int32_t tokens, int32_t n,
                                    int32_t k, int32_t *status, uint64_t limit_ns, aqlm_stream_t stream) {
     if (!X || !W || !Y || !status || tokens < 1 || n < 1 || k < 1 || n % 8 || k % 8) return AQLM_ERR_INVALID_ARG;

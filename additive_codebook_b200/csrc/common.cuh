@@ -213,6 +213,7 @@ cudaError_t launch_gemv_multi(const RowLayerIn *layers, int n, const uint16_t *x
                               void *workspace, cudaStream_t st);
 cudaError_t launch_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                              int32_t *status, cudaStream_t st);
+int gemm_tile_n(int tokens, int n, int sms);
 // encoding (encode.cu)
 cudaError_t launch_encode_scales(const float *W, int d_out, int d_in, uint16_t *scales, float *V, cudaStream_t st);
 size_t nearest_workspace_bytes(long long N);

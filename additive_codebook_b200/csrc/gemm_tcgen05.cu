@@ -7,13 +7,14 @@
 // section "What is Multi-Codebook Quantization (MCQ)?" of "The AQLM
 // Quantization Algorithm, Explained".
 //
-// sm_100a design: a persistent kernel, one CTA per SM, 128x256 output tiles.
+// sm_100a design: a persistent kernel, one CTA per SM, 128 x BN output tiles.
 //   warp 0      one thread issues TMA tile loads (128-byte swizzle) into a
-//               4-stage shared-memory ring, each stage guarded by a pair of
-//               mbarriers (full: bytes landed; empty: MMAs done reading);
-//   warp 1      allocates all 512 tensor-memory columns (two 128x256 fp32
-//               accumulators) and one thread issues tcgen05.mma
-//               (cta_group::1, kind::f16, M=128 N=256 K=16), releasing each
+//               shared-memory ring (4 stages, 5 for BN = 192),
+//               each stage guarded by a pair of mbarriers (full: bytes
+//               landed; empty: MMAs done reading);
+//   warp 1      allocates the tensor memory of two 128 x BN fp32
+//               accumulators and one thread issues tcgen05.mma
+//               (cta_group::1, kind::f16, M=128 N=BN K=16), releasing each
 //               ring stage with tcgen05.commit;
 //   warps 2-5   epilogue: tcgen05.ld from the accumulator of the previous
 //               tile while the MMAs of the next tile run into the other one,
@@ -22,6 +23,16 @@
 // AQLM_ERR_TIMEOUT to the status word, raises a CTA-wide abort flag that the
 // other roles poll, waits (bounded) for its TMA loads and MMAs in flight and
 // frees its tensor memory before returning; nothing traps.
+//
+// The tile width BN is chosen per shape from {256, 240, 224, 192} so that the
+// tiles fill the waves of the SMs: with 2048 tokens, 11008 output columns are
+// 688 tiles of 128x256 (4.65 waves of 148 SMs, the last one 65% full) but 736
+// of 128x240 (4.97 waves).  A tile's time goes with the operand bytes it
+// streams, (128 + BN) x K (the ring is fed from L2 at close to its bandwidth),
+// so the estimate is waves x (128 + BN); measured on B200 it ranks the widths
+// as the clock does (2048 tokens: 11008x4096 141.3 / 135.2 us at BN 256 / 240,
+// 4096x11008 141.2 / 137.2, 8192x8192 204.8 / 200.7 / 196.6 at 256 / 240 / 224).
+// Narrower tiles lose: 128x112 ran at 60% of the 128x256 rate.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -29,30 +40,39 @@
 namespace aqlm {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 128, BK = 64;
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int ACC_COLS = BN;           // fp32 columns per accumulator
-constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
+constexpr int kMaxStages = 8;
 constexpr int kGemmThreads = 192;
 constexpr int kEpiWarps = 4;
-// bf16 x bf16 -> fp32, both operands K-major, M = 128, N = 256
-// (tcgen05 instruction descriptor: D format bits 4-5, A/B format bits 7-12,
-// N >> 3 at bits 17-22, M >> 4 at bits 24-28).
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
 
 struct Bars {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t mma_done;
     uint32_t tmem_base;
     int abort_flag;
 };
-constexpr size_t kGemmSmem = 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + sizeof(Bars);
+
+template <int BN>
+struct GemmCfg {
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M = 128");
+    static constexpr int B_BYTES = BN * BK * 2;                // a multiple of 1024: stages stay aligned
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = (200 * 1024) / STAGE_BYTES < kMaxStages ? (200 * 1024) / STAGE_BYTES : kMaxStages;
+    // each accumulator at a power-of-two column offset; the allocation is a power of two
+    static constexpr int ACC_STRIDE = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+    static constexpr uint32_t TMEM_COLS = 2 * ACC_STRIDE;
+    // bf16 x bf16 -> fp32, both operands K-major, M = 128, N = BN (tcgen05
+    // instruction descriptor: D format bits 4-5, A/B format bits 7-12, N >> 3
+    // at bits 17-22, M >> 4 at bits 24-28).
+    static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                      ((uint32_t)(BM >> 4) << 24);
+    static constexpr size_t SMEM = 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + sizeof(Bars);
+    static_assert(B_BYTES % 1024 == 0 && STAGES >= 2, "ring layout");
+};
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -142,11 +162,42 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
 
+// Columns [n0, n0 + 8 * V) of row m of Y from fp32 accumulator values r,
+// rounded to bf16, in 16-byte stores (columns past n_total skipped; n_total
+// is a multiple of 8).
+template <int V>
+__device__ __forceinline__ void store_bf16_row(__nv_bfloat16 *dst, const uint32_t *r, int n0, int n_total) {
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+        if (n0 + 8 * v < n_total) {
+            uint32_t p[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const __nv_bfloat162 b2 =
+                    __floats2bfloat162_rn(__uint_as_float(r[8 * v + 2 * h]), __uint_as_float(r[8 * v + 2 * h + 1]));
+                p[h] = *reinterpret_cast<const uint32_t *>(&b2);
+            }
+            *reinterpret_cast<uint4 *>(dst + 8 * v) = make_uint4(p[0], p[1], p[2], p[3]);
+        }
+    }
+}
+
+template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                   __nv_bfloat16 *__restrict__ Y, int m_total, int n_total, int k_total, int32_t *status,
                   unsigned long long limit_ns, int stall_test) {
+    using C = GemmCfg<BN>;
+    constexpr int STAGES = C::STAGES, STAGE_BYTES = C::STAGE_BYTES;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled tiles.
     const uint32_t raw = smem_addr(smem_raw);
@@ -177,7 +228,7 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_addr(&bars->tmem_base)),
-                     "r"(TMEM_COLS));
+                     "r"(C::TMEM_COLS));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     tc_fence_before();
@@ -202,7 +253,7 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
                     }
                     const uint32_t full = smem_addr(&bars->full[stage]);
                     const uint32_t dst = smem_addr(smem + (size_t)stage * STAGE_BYTES);
-                    mbar_expect_tx(full, STAGE_BYTES);
+                    mbar_expect_tx(full, (uint32_t)STAGE_BYTES);
                     tma_load_2d(dst, &tmap_x, kb * BK, mb * BM, full);
                     tma_load_2d(dst + A_BYTES, &tmap_w, kb * BK, nb * BN, full);
                     issued_parity[stage] = (int)phase;
@@ -237,7 +288,7 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)(acc * ACC_COLS);
+                const uint32_t d_tmem = tmem + (uint32_t)(acc * C::ACC_STRIDE);
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!wait_bounded(smem_addr(&bars->full[stage]), phase, bars, status, limit_ns)) {
                         ok = false;
@@ -249,7 +300,7 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
                         // K step of 16 bf16 = 32 bytes inside the 128-byte swizzled row.
-                        mma_bf16(d_tmem, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), kIdesc,
+                        mma_bf16(d_tmem, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), C::IDESC,
                                  (kb > 0 || k > 0) ? 1u : 0u);
                     }
                     mma_commit(smem_addr(&bars->empty[stage]));
@@ -285,28 +336,19 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
             if (!ok) break;
             tc_fence_after();
             const int m = mb * BM + row_in_tile;
-            const uint32_t t_base = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+            const uint32_t t_base = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * C::ACC_STRIDE);
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
                 tmem_ld32(t_base + (uint32_t)(c * 32), r);
                 const int n0 = nb * BN + c * 32;
-                if (m < m_total) {
-                    __nv_bfloat16 *dst = Y + (size_t)m * n_total + n0;
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        if (n0 + 8 * v < n_total) {
-                            uint32_t p[4];
-#pragma unroll
-                            for (int h = 0; h < 4; ++h) {
-                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(
-                                    __uint_as_float(r[8 * v + 2 * h]), __uint_as_float(r[8 * v + 2 * h + 1]));
-                                p[h] = *reinterpret_cast<const uint32_t *>(&b2);
-                            }
-                            *reinterpret_cast<uint4 *>(dst + 8 * v) = make_uint4(p[0], p[1], p[2], p[3]);
-                        }
-                    }
-                }
+                if (m < m_total) store_bf16_row<4>(Y + (size_t)m * n_total + n0, r, n0, n_total);
+            }
+            if constexpr (BN % 32 != 0) {  // the last 16 columns of the tile
+                uint32_t r[16];
+                tmem_ld16(t_base + (uint32_t)(BN / 32 * 32), r);
+                const int n0 = nb * BN + BN / 32 * 32;
+                if (m < m_total) store_bf16_row<2>(Y + (size_t)m * n_total + n0, r, n0, n_total);
             }
             tc_fence_before();
             __syncwarp();
@@ -322,7 +364,7 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
     __syncthreads();
     tc_fence_after();
     if (warp == 1) {
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS));
     }
 }
 
@@ -362,20 +404,58 @@ bool make_map(CUtensorMap *map, const void *base, int rows, int cols, int box_ro
 // Bound on any single wait of the GEMM (the whole GEMM takes well under this).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
-cudaError_t launch_bf16_gemm_ex(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
-                                int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test) {
+namespace {
+template <int BN>
+cudaError_t launch_gemm_bn(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
+                           int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test, int sms) {
+    using C = GemmCfg<BN>;
     CUtensorMap mx, mw;
     if (!make_map(&mx, X, tokens, k, BM) || !make_map(&mw, W, n, k, BN)) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kGemmSmem);
+    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::SMEM);
     if (e != cudaSuccess) return e;
+    const int tiles = ((tokens + BM - 1) / BM) * ((n + BN - 1) / BN);
+    const int grid = tiles < sms ? tiles : sms;
+    return launch_kernel(gemm_bf16_tcgen05<BN>, dim3(grid), dim3(kGemmThreads), C::SMEM, st, false, mx, mw,
+                         reinterpret_cast<__nv_bfloat16 *>(Y), tokens, n, k, status, limit_ns, stall_test);
+}
+}  // namespace
+
+// The tile width for a tokens x n product on `sms` SMs: the one whose tiles,
+// dealt round robin, give the least waves x (BM + BN) -- the busiest SM's
+// share of operand bytes; ties to the wider tile.
+int gemm_tile_n(int tokens, int n, int sms) {
+    constexpr int kCands[] = {256, 240, 224, 192};
+    const long long m_tiles = (tokens + BM - 1) / BM;
+    int best = kCands[0];
+    long long best_cost = -1;
+    for (int bn : kCands) {
+        const long long tiles = m_tiles * ((n + bn - 1) / bn);
+        const long long waves = (tiles + sms - 1) / sms;
+        const long long cost = waves * (BM + bn);
+        if (best_cost < 0 || cost < best_cost) {
+            best = bn;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
+cudaError_t launch_bf16_gemm_ex(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
+                                int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test) {
     int dev = 0;
     cudaGetDevice(&dev);
-    const int tiles = ((tokens + BM - 1) / BM) * ((n + BN - 1) / BN);
     const int sms = num_sms(dev);
-    const int grid = tiles < sms ? tiles : sms;
-    return launch_kernel(gemm_bf16_tcgen05, dim3(grid), dim3(kGemmThreads), kGemmSmem, st, false, mx, mw,
-                         reinterpret_cast<__nv_bfloat16 *>(Y), tokens, n, k, status, limit_ns, stall_test);
+    switch (gemm_tile_n(tokens, n, sms)) {
+        case 240:
+            return launch_gemm_bn<240>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms);
+        case 224:
+            return launch_gemm_bn<224>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms);
+        case 192:
+            return launch_gemm_bn<192>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms);
+        default:
+            return launch_gemm_bn<256>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms);
+    }
 }
 
 cudaError_t launch_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,

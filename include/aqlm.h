@@ -244,6 +244,15 @@ AQLM_API aqlm_status aqlm_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16
                            int32_t n, int32_t k, int32_t *status, aqlm_stream_t stream);
 
 /*
+ * aqlm_bf16_gemm_tile_n -- the output tile width (columns of W per tile:
+ * 256, 240, 224 or 192) that aqlm_bf16_gemm and aqlm_gemm use for `tokens`
+ * x `n` on a device with `sms` streaming multiprocessors: the width with the
+ * least waves x (128 + width), ties to the wider.  Host only; returns 0 if an
+ * argument is below 1.
+ */
+AQLM_API int32_t aqlm_bf16_gemm_tile_n(int32_t tokens, int32_t n, int32_t sms);
+
+/*
  * aqlm_decode_indices -- the code unpacking step on its own, for bit-exact
  * checks: idx_out[(i*G + j)*M + m] = index of codebook m for group j of row
  * i, as uint16 (G = d_in/8).  idx_out: d_out*G*M uint16, 2-byte aligned.

@@ -249,3 +249,23 @@ def test_encode_argument_errors():
     assert cws >= 4096 * 8 * 4 + 4096 * 8 + 2 * 256 * 8 * 4
     assert lib.aqlm_encode_codes(A16, B16, C16, s, D16, cws - 1, NULL) == ac.AQLM_ERR_WORKSPACE
     assert lib.aqlm_encode_codes(A16, B16, ODD, s, D16, cws, NULL) == ac.AQLM_ERR_MISALIGNED
+
+
+def test_gemm_tile_width_rule():
+    """The GEMM's tile width: least waves x (128 + width) over {256, 240, 224,
+    192}, ties to the wider, checked against the rule restated here over a
+    grid of shapes, and the prefill shapes on 148 SMs."""
+    def rule(tokens, n, sms):
+        best = None
+        for bn in (256, 240, 224, 192):
+            tiles = -(-tokens // 128) * -(-n // bn)
+            cost = -(-tiles // sms) * (128 + bn)
+            if best is None or cost < best[0]:
+                best = (cost, bn)
+        return best[1]
+    for tokens in (1, 127, 128, 300, 1000, 2048, 4096):
+        for n in (8, 256, 1000, 4096, 4608, 8192, 11008, 28672):
+            for sms in (1, 132, 148):
+                assert ac.bf16_gemm_tile_n(tokens, n, sms) == rule(tokens, n, sms)
+    assert [ac.bf16_gemm_tile_n(2048, n, 148) for n in (11008, 4096, 8192, 28672)] == [240, 240, 224, 240]
+    assert ac.bf16_gemm_tile_n(0, 8, 148) == 0 and ac.bf16_gemm_tile_n(8, 8, 0) == 0

@@ -268,6 +268,31 @@ def test_bf16_gemm_ragged_and_deep(tokens, n, k):
     assert bool(torch.all(err <= 2.0 ** -8 * ref.abs() + 2.0 ** -14 * absdot + 1e-6))
 
 
+# (tokens, n, k) whose tile width on 148 SMs is each of the four (ragged
+# tokens, n and k in every case)
+TILE_WIDTH_CASES = [(1000, 4608, 1032, 256), (2040, 4096, 520, 240), (1530, 4864, 520, 224), (300, 1000, 4104, 192)]
+
+
+@pytest.mark.parametrize("tokens,n,k,width", TILE_WIDTH_CASES, ids=[f"BN{c[3]}" for c in TILE_WIDTH_CASES])
+def test_bf16_gemm_every_tile_width(tokens, n, k, width):
+    """Each instantiation of the tile width (128x256, 128x240, 128x224,
+    128x192 output tiles) against torch (fp32 accumulation), including the
+    partial last column tile and the 16-column remainder of the 240 / 224
+    epilogue."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    if sms == 148:
+        assert ac.bf16_gemm_tile_n(tokens, n, sms) == width
+    g = torch.Generator(device="cpu").manual_seed(tokens + n + k)
+    X = (torch.randn(tokens, k, generator=g) / 4).to(torch.bfloat16).to(DEV)
+    W = (torch.randn(n, k, generator=g) / 4).to(torch.bfloat16).to(DEV)
+    Y, status = ac.aqlm_bf16_gemm(X, W)
+    assert int(status.item()) == 0
+    ref = X.float() @ W.float().T
+    absdot = X.float().abs() @ W.float().abs().T
+    err = (Y.float() - ref).abs()
+    assert bool(torch.all(err <= 2.0 ** -8 * ref.abs() + 2.0 ** -14 * absdot + 1e-6))
+
+
 def test_bf16_gemm_matches_torch():
     """The plain tensor-core GEMM against torch.matmul (fp32 accumulation) as a yardstick."""
     g = torch.Generator(device="cpu").manual_seed(7)
