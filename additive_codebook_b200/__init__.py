@@ -128,12 +128,19 @@ def _check(status, where):
 
 
 def _p(t):
-    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+    # an int (or None for NULL): ctypes converts it for a c_void_p argument
+    return t.data_ptr() if t is not None else None
 
 
-def _stream(stream):
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return ctypes.c_void_p(s.cuda_stream)
+_raw_stream = torch._C._cuda_getCurrentRawStream
+
+
+def _stream(stream, device=None):
+    """The cudaStream_t handle (an int) of `stream`, else of the current
+    stream of `device` (default: the current device)."""
+    if stream is not None:
+        return stream.cuda_stream
+    return _raw_stream(torch.cuda.current_device() if device is None else device)
 
 
 _shapes = {}
@@ -181,19 +188,21 @@ def gemm_workspace_bytes(shape, tokens):
 
 def aqlm_gemv(codes, codebooks, scales, x, y=None, workspace=None, stream=None):
     """y[T, d_out] = fp16(W^ . x) for x [T, d_in] float16, 1 <= T <= 16."""
-    lib = load_library()
+    lib = _lib if _lib is not None else load_library()
     shape = shape_of(codes)
     if x.dim() == 1:
         x = x.unsqueeze(0)
     T = x.shape[0]
+    dev = x.get_device()
     if y is None:
         y = torch.empty((T, shape.d_out), dtype=torch.float16, device=x.device)
-    need = _gemv_need(lib, shape, T, x.device.index)
+    need = _gemv_need(lib, shape, T, dev)
     if need and workspace is None:
         workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
     wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _check(lib.aqlm_gemv(_p(codes), _p(codebooks), _p(_flat_scales(scales)), _p(x), _p(y), T, shape,
-                         _p(workspace), wbytes, _stream(stream)), "aqlm_gemv")
+    _check(lib.aqlm_gemv(codes.data_ptr(), codebooks.data_ptr(), _flat_scales(scales).data_ptr(), x.data_ptr(),
+                         y.data_ptr(), T, shape, _p(workspace), wbytes, _stream(stream, dev if dev >= 0 else None)),
+           "aqlm_gemv")
     return y
 
 

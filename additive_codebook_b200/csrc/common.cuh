@@ -128,7 +128,30 @@ __device__ __forceinline__ void fma2_f16_f32(float &e, float &o, uint32_t c, uin
 template <typename... KArgs>
 cudaError_t opt_in_dynamic_smem(void (*kern)(KArgs...), size_t bytes) {
     if (bytes + 1024 <= 48 * 1024) return cudaSuccess;
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    // remember, per (kernel, device), the largest size already set, so that
+    // repeated launches skip the driver call
+    static std::mutex mu;
+    static std::vector<std::tuple<const void *, int, size_t>> done;
+    const void *key = reinterpret_cast<const void *>(kern);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (const auto &e : done)
+            if (std::get<0>(e) == key && std::get<1>(e) == dev && std::get<2>(e) >= bytes) return cudaSuccess;
+    }
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && dev >= 0) {
+        std::lock_guard<std::mutex> lock(mu);
+        bool found = false;
+        for (auto &d : done)
+            if (std::get<0>(d) == key && std::get<1>(d) == dev) {
+                if (std::get<2>(d) < bytes) std::get<2>(d) = bytes;
+                found = true;
+            }
+        if (!found && done.size() < 1024) done.emplace_back(key, dev, bytes);
+    }
+    return e;
 }
 
 // Launch through cudaLaunchKernelEx so that the returned error belongs to this
