@@ -132,7 +132,9 @@ def _p(t):
     return t.data_ptr() if t is not None else None
 
 
-_raw_stream = torch._C._cuda_getCurrentRawStream
+# the current stream's handle without building a torch.cuda.Stream object
+# (which costs microseconds per call); torch builds without it take the slow way
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
 
 
 def _stream(stream, device=None):
@@ -140,6 +142,8 @@ def _stream(stream, device=None):
     stream of `device` (default: the current device)."""
     if stream is not None:
         return stream.cuda_stream
+    if _raw_stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
     return _raw_stream(torch.cuda.current_device() if device is None else device)
 
 
