@@ -459,8 +459,26 @@ def pin_greedy_codes_recover_sums():
     assert np.array_equal(c1[clear], d.argmin(1)[clear])
 
 
+def pin_worked_encoding():
+    """A two-row layer encoded by hand (tests/golden/worked_example_encode.json):
+    binary16 scale bits (including the zero row's 1.0), the groups to within
+    one binary32 rounding of their exact quotients, the nearest codeword with
+    a tie, and the greedy codes."""
+    with open(os.path.join(GOLDEN, "worked_example_encode.json")) as fh:
+        ex = json.load(fh)
+    W = np.array(ex["W"], dtype=np.float32)
+    sc, V = oracle.encode_scales(W)
+    assert sc.view(np.uint16).tolist() == ex["expected_scale_bits"]
+    want = np.array([[n / d for n, d in row] for row in ex["expected_groups_num_den"]])
+    assert np.all(np.abs(V.astype(np.float64) - want) <= np.abs(want) * 2.0 ** -24)
+    cb = np.array(ex["codebooks"], dtype=np.float16)
+    idx, _ = oracle.nearest(V, cb[0].astype(np.float32))
+    assert idx.tolist() == ex["expected_nearest_codebook0"]
+    assert oracle.encode_greedy(V, cb).tolist() == ex["expected_codes"]
+
+
 ENCODE_PINS = [pin_double_to_half, pin_encode_scales, pin_nearest_codeword, pin_kmeans_update,
-               pin_residual_kmeans_recovers_clusters, pin_greedy_codes_recover_sums]
+               pin_residual_kmeans_recovers_clusters, pin_greedy_codes_recover_sums, pin_worked_encoding]
 
 ALL_PINS = [pin_half_conversion, pin_bf16_rounding, pin_decode_indices,
             pin_index_encoding_recovers_codes, pin_one_hot_activation, pin_linearity,
