@@ -29,7 +29,7 @@ def bf16_to_np_bits(t):
     return t.detach().cpu().view(torch.int16).numpy().view(np.uint16)
 
 
-def north_star_bound(W, x64):
+def stated_tolerance_bound(W, x64):
     """Per-token bound 2e-3 * ||x_tau||_2 * max_i ||(s . W)_i||_2 (norms in double)."""
     row = np.sqrt((W * W).sum(axis=1)).max()
     return 2e-3 * np.sqrt((x64 * x64).sum(axis=1)) * row          # [T]
@@ -42,7 +42,7 @@ def check_fp_output(y_gpu, y_ref, W, x64, out_rel, acc_rel):
       plus acc_rel * sum_k |W_ik x_k| (fp32 accumulation) plus a subnormal floor."""
     y_gpu = np.asarray(y_gpu, dtype=np.float64)
     err = np.abs(y_gpu - y_ref)
-    bound = north_star_bound(W, x64)
+    bound = stated_tolerance_bound(W, x64)
     worst = err.max(axis=1)
     assert np.all(worst <= bound), f"stated tolerance exceeded: {worst} > {bound}"
     absdot = x64.__abs__() @ np.abs(W).T                            # [T, d_out]
