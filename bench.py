@@ -13,7 +13,7 @@ scope: 2x8 4096^2, the Llama-2-7B decoder block (1x16 and 2x8), the
 Llama-2-70B layers (1x16 at 1/4/16 tokens, 2x16), and prefill (dequant +
 tcgen05 GEMM at 2048 tokens), each as us/layer and fraction of its roofline.
 
---impl reference times the CPU oracle (the baseline of this build) on the
+--impl reference times the CPU oracle (the reference arm) on the
 same workload and prints the same line with "impl": "reference".
 Inputs are synthetic (seeded numpy draws; see synth/), not trained weights.
 """

@@ -137,8 +137,9 @@ AQLM_API aqlm_status aqlm_gemv(const void *codes, const uint16_t *codebooks, con
 AQLM_API size_t aqlm_gemv_workspace_bytes(aqlm_shape shape, int32_t tokens);
 
 /* Most tokens for which aqlm_gemv and aqlm_gemv_multi run on the CUDA cores
- * with no device waits (1x16: 2, 2x16: 3, 2x8: 4); 0 for an unsupported shape.  The value belongs to this build of the library
- * (it follows measurements of both kernels), so ask rather than hard-code it. */
+ * with no device waits (1x16: 2, 2x16: 3, 2x8: 4); 0 for an unsupported
+ * shape.  The value may change between library versions (it follows
+ * measurements of both kernels), so ask rather than hard-code it. */
 AQLM_API int32_t aqlm_gemv_row_tokens(aqlm_shape shape);
 
 /*
