@@ -7,31 +7,40 @@
 // section "What is Multi-Codebook Quantization (MCQ)?": output channels are
 // scaled, cut into groups of 8 and each group approximated by the sum of M
 // codewords.  The pages give no loss, search or update rule beyond that, so
-// every step here is a stated reading (the same one the CPU oracle takes):
+// every step here is a stated reading of what is computed:
 //   scales     the row's root mean square rounded to fp16 (1.0 if that is 0);
-//              the sum of squares in double, lane l of a warp summing inputs
-//              l, l+32, ... in order, then a butterfly of shuffles;
 //   groups     the row's inputs divided by its scale (binary32 division);
-//   nearest    least squared Euclidean distance |v - c|^2, ranked by the score
-//              |c|^2 - 2<v, c> (|v|^2 is common to every codeword), ties to
-//              the lowest index; in binary32 each of |c|^2 and <v, c> is lanes
-//              0,2,4,6 and 1,3,5,7 as two fused multiply-add chains (one packed
-//              fp32x2 chain), then e + o, and score = fma(-2, <v, c>, |c|^2);
-//              the distance reported for the winner is e + o of the squared
-//              differences in the same pattern;
+//   nearest    least squared Euclidean distance |v - c|^2, ties to the lowest
+//              index;
 //   k-means    Lloyd updates: a centroid is the mean of its groups (sums in
 //              double), an empty one keeps its value; codebook m is k-means
 //              of the residuals left by codebooks 0..m-1, started from the
 //              residuals that init_idx names;
 //   codes      greedy, codebook by codebook: the nearest codeword of the
 //              residual, which then loses that codeword.
+// How each is evaluated here (any order meets the same error bounds):
+//   scales     the sum of squares in double, lane l of a warp summing inputs
+//              l, l+32, ... in order, then a butterfly of shuffles; the
+//              binary16 result can differ from a sequential sum's only where
+//              the root mean square lies within (d_in + 4) 2^-53 of a
+//              binary16 rounding boundary;
+//   nearest    ranked by the binary32 score |c|^2 - 2<v, c> (|v|^2 is common
+//              to every codeword): each of |c|^2 and <v, c> is the sum of two
+//              fused multiply-add chains (lanes 0,2,4,6 and 1,3,5,7, one packed
+//              fp32x2 chain), then score = fma(-2, <v, c>, |c|^2).  Its error
+//              is at most gamma_9 (|c|^2 + 2 sum_t |v_t c_t|) (u = 2^-24), so
+//              the chosen codeword is the exact nearest one unless another lies
+//              within twice that of it.  The distance reported for the winner
+//              is the same two-chain sum of the squared differences.
 //
 // The nearest-codeword search is the expensive step (every group against
-// every codeword: 2^16 for 1x16) and runs on the CUDA cores in exact binary32
-// so that its integer results can be compared bit for bit.  Each thread keeps
-// four groups in registers and streams the codebook, with each codeword's
-// |c|^2, through shared memory; a CTA covers 1024 groups and a range of
-// codewords, and the ranges' winners meet through a 64-bit atomic minimum of
+// every codeword: 2^16 for 1x16) and runs on the CUDA cores in binary32:
+// deterministic, with the error bound above.  (On the tensor cores the dot
+// products would be tf32 with an accumulation order the hardware does not
+// document, and the bound could not be stated.)  Each thread keeps four
+// groups in registers and streams the codebook, with each codeword's |c|^2,
+// through shared memory; a CTA covers 1024 groups and a range of codewords,
+// and the ranges' winners meet through a 64-bit atomic minimum of
 // (key(score) << 32 | index), key the order-preserving map of a float onto
 // the unsigned integers: equal scores fall to the lower index, exactly the
 // tie rule.

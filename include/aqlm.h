@@ -308,18 +308,19 @@ AQLM_API size_t aqlm_gemv_noalloc_max_scratch_bytes(void);
  * codebooks initialised "with a residual k-means approach".  The pages give
  * no loss, search or update rule beyond that; the readings taken here are:
  *   scale s_i   root mean square of row i rounded to fp16 (1.0 if it rounds to
- *               0): the sum of squares in double, lane l of 32 summing inputs
- *               l, l+32, ... in order, partial sums combined pairwise
- *               (l + (l ^ 16), then ^ 8, ^ 4, ^ 2, ^ 1); sqrt(sum / d_in);
+ *               0); the sum of squares is taken in double, so the result is
+ *               the correctly rounded one unless the root mean square lies
+ *               within (d_in + 4) 2^-53 (relative) of a rounding boundary;
  *   groups      v = W[i][8j .. 8j+7] / s_i (binary32 division), [d_out*d_in/8][8];
- *   nearest     least squared Euclidean distance |v - c|^2, ranked by the
- *               score |c|^2 - 2<v, c> (|v|^2 is common to every codeword),
- *               ties to the lowest index; in binary32 each of |c|^2 and <v, c>
- *               is e + o, e the chain of fused multiply-adds of lanes 0, 2,
- *               4, 6 (the first a plain product) and o that of lanes 1, 3, 5,
- *               7, and score = fma(-2, <v, c>, |c|^2);
- *   distance    (reported for the chosen codeword) e + o of the squared
- *               differences (v_t - c_t)^2 in the same pattern;
+ *   nearest     least squared Euclidean distance |v - c|^2, ties to the lowest
+ *               index.  Evaluated in binary32 as the score |c|^2 - 2<v, c>
+ *               (|v|^2 is common to every codeword), whose error is at most
+ *               beta(c) = gamma_9 (|c|^2 + 2 sum_t |v_t c_t|), gamma_n =
+ *               n u / (1 - n u), u = 2^-24: the chosen codeword k satisfies
+ *               |v - c_k|^2 <= min_c |v - c|^2 + beta(c_k) + beta(c_min), and is
+ *               the exact nearest wherever no other codeword lies that close;
+ *   distance    (reported for the chosen codeword) its squared distance in
+ *               binary32, within gamma_10 (relative) of the exact value;
  *   k-means     a centroid becomes the mean of its groups (sums in double, one
  *               rounding), one without groups keeps its value; codebook m is
  *               k-means of the residuals left by codebooks 0..m-1;

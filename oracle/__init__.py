@@ -48,7 +48,7 @@ def _configure(lib):
     lib.aqlm_oracle_double_to_half.argtypes = [ctypes.c_double]
     lib.aqlm_oracle_double_to_half.restype = ctypes.c_uint16
     lib.aqlm_oracle_encode_scales.argtypes = [vp, i64, i64, vp, vp]
-    lib.aqlm_oracle_nearest.argtypes = [vp, i64, vp, i64, vp, vp]
+    lib.aqlm_oracle_nearest.argtypes = [vp, i64, vp, i64, vp, vp, vp]
     lib.aqlm_oracle_kmeans_update.argtypes = [vp, vp, i64, i64, vp, vp, vp]
     lib.aqlm_oracle_residual_kmeans.argtypes = [vp, i64, i32, i64, vp, i32, vp]
     lib.aqlm_oracle_encode_greedy.argtypes = [vp, i64, vp, i32, i64, vp]
@@ -199,13 +199,16 @@ def encode_scales(W):
 
 
 def nearest(V, C):
-    """E3: (index int32 [N], distance float32 [N]) of each group's nearest codeword."""
+    """E3: (index int32 [N], distance float64 [N], runner-up distance float64
+    [N]) of each group's nearest codeword by the squared Euclidean distance in
+    double, ties to the lowest index."""
     V, C = _f32(V, 8), _f32(C, 8)
     N, K = V.size // 8, C.size // 8
     idx = np.empty(N, dtype=np.int32)
-    dist = np.empty(N, dtype=np.float32)
-    assert _load().aqlm_oracle_nearest(_ptr(V), N, _ptr(C), K, _ptr(idx), _ptr(dist)) == 0
-    return idx, dist
+    dist = np.empty(N, dtype=np.float64)
+    second = np.empty(N, dtype=np.float64)
+    assert _load().aqlm_oracle_nearest(_ptr(V), N, _ptr(C), K, _ptr(idx), _ptr(dist), _ptr(second)) == 0
+    return idx, dist, second
 
 
 def kmeans_update(V, idx, C_prev):

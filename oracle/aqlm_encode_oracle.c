@@ -17,19 +17,18 @@
  *
  * Readings where the pages are silent (each listed in the design notes):
  *   E1 scale of row i: the root mean square of the row, rounded to binary16
- *      (1.0 if that rounds to zero); the sum of squares is taken in double in
- *      a fixed order (32 interleaved partial sums combined by the butterfly
- *      pattern below) so that the binary16 result is reproducible;
+ *      (1.0 if that rounds to zero); the sum of squares is a plain
+ *      left-to-right sum in double of the exact squares (double holds the
+ *      square of every binary32 value exactly);
  *   E2 the groups to encode are the row's inputs divided by the scale
  *      (binary32 division, correctly rounded);
  *   E3 nearest codeword: the one of least squared Euclidean distance
- *      |v - c|^2 = |v|^2 + score(v, c), ranked by the score
- *      score = |c|^2 - 2 <v, c> (|v|^2 is the same for every codeword), ties
- *      to the lowest index.  In binary32: |c|^2 = e + o and <v, c> = e' + o',
- *      each e the fused multiply-add chain of lanes 0, 2, 4, 6 (the first a
- *      plain product) and o that of lanes 1, 3, 5, 7; score = fma(-2, <v, c>,
- *      |c|^2).  The distance reported for the chosen codeword is e + o over
- *      the squared differences (v_t - c_t)^2, in the same pattern;
+ *      |v - c|^2 = sum_t (v_t - c_t)^2, evaluated here in double for every
+ *      codeword, ties to the lowest index.  Any evaluation of the distance
+ *      carries rounding error, so another implementation (in binary32, in
+ *      any order) may pick a different codeword only where two distances
+ *      lie within its error bound of each other; the tests check exactly
+ *      that, with the bound stated there;
  *   E4 k-means update (Lloyd): a centroid becomes the mean of the groups
  *      assigned to it (sums in double, one rounding to binary32); a centroid
  *      with no group keeps its value;
@@ -96,23 +95,12 @@ static float half_to_float(uint16_t h)
 
 /* ---- E1, E2: row scales and the groups to encode ------------------------ */
 
-/* Sum of squares of one row: 32 interleaved partial sums in double (partial
- * l takes inputs l, l+32, ... in order), combined pairwise by the butterfly
- * pattern (partial l gets partial l ^ o added, o = 16, 8, 4, 2, 1). */
+/* Sum of squares of one row, left to right, in double. */
 static double row_sum_squares(const float *row, int64_t n)
 {
-    double p[32];
-    for (int l = 0; l < 32; ++l) {
-        double acc = 0.0;
-        for (int64_t k = l; k < n; k += 32) acc += (double)row[k] * (double)row[k];
-        p[l] = acc;
-    }
-    for (int o = 16; o > 0; o >>= 1) {
-        double q[32];
-        for (int l = 0; l < 32; ++l) q[l] = p[l] + p[l ^ o];
-        memcpy(p, q, sizeof(p));
-    }
-    return p[0];
+    double acc = 0.0;
+    for (int64_t k = 0; k < n; ++k) acc += (double)row[k] * (double)row[k];
+    return acc;
 }
 
 int aqlm_oracle_encode_scales(const float *W, int64_t d_out, int64_t d_in, uint16_t *scales, float *V)
@@ -133,77 +121,52 @@ int aqlm_oracle_encode_scales(const float *W, int64_t d_out, int64_t d_in, uint1
 
 /* ---- E3: nearest codeword ------------------------------------------------ */
 
-/* Even lanes and odd lanes of a . b as two fused multiply-add chains. */
-static float dot8(const float *a, const float *b)
+/* Squared Euclidean distance of two groups, in double. */
+static double distance(const float *v, const float *c)
 {
-    float e = a[0] * b[0];
-    e = fmaf(a[2], b[2], e);
-    e = fmaf(a[4], b[4], e);
-    e = fmaf(a[6], b[6], e);
-    float o = a[1] * b[1];
-    o = fmaf(a[3], b[3], o);
-    o = fmaf(a[5], b[5], o);
-    o = fmaf(a[7], b[7], o);
-    return e + o;
+    double d = 0.0;
+    for (int t = 0; t < 8; ++t) {
+        const double e = (double)v[t] - (double)c[t];
+        d += e * e;
+    }
+    return d;
 }
 
-/* The ranking score |c|^2 - 2 <v, c>, with |c|^2 given. */
-static float score(const float *v, const float *c, float cc)
-{
-    return fmaf(-2.0f, dot8(v, c), cc);
-}
-
-/* Squared distance of the chosen codeword (reported, not ranked). */
-static float distance(const float *v, const float *c)
-{
-    float d[8];
-    for (int t = 0; t < 8; ++t) d[t] = v[t] - c[t];
-    float e = d[0] * d[0];
-    e = fmaf(d[2], d[2], e);
-    e = fmaf(d[4], d[4], e);
-    e = fmaf(d[6], d[6], e);
-    float o = d[1] * d[1];
-    o = fmaf(d[3], d[3], o);
-    o = fmaf(d[5], d[5], o);
-    o = fmaf(d[7], d[7], o);
-    return e + o;
-}
-
-/* The nearest codeword of v: least score, ties to the lowest index. */
-static int64_t nearest_one(const float *v, const float *C, const float *cc, int64_t K)
+/* The nearest codeword of v (least distance, ties to the lowest index);
+ * *best_d receives its distance and *second_d the least distance over the
+ * other codewords (+inf when K = 1). */
+static int64_t nearest_one(const float *v, const float *C, int64_t K, double *best_d, double *second_d)
 {
     int64_t best = 0;
-    float bs = score(v, C, cc[0]);
+    double bd = distance(v, C), sd = INFINITY;
     for (int64_t k = 1; k < K; ++k) {
-        const float sk = score(v, C + k * 8, cc[k]);
-        if (sk < bs) {
-            bs = sk;
+        const double dk = distance(v, C + k * 8);
+        if (dk < bd) {
+            sd = bd;
+            bd = dk;
             best = k;
+        } else if (dk < sd) {
+            sd = dk;
         }
     }
+    if (best_d) *best_d = bd;
+    if (second_d) *second_d = sd;
     return best;
 }
 
-static float *norms(const float *C, int64_t K)
-{
-    float *cc = (float *)malloc((size_t)K * sizeof(float));
-    if (cc)
-        for (int64_t k = 0; k < K; ++k) cc[k] = dot8(C + k * 8, C + k * 8);
-    return cc;
-}
-
-int aqlm_oracle_nearest(const float *V, int64_t N, const float *C, int64_t K, int32_t *idx, float *dist)
+/* idx[n], dist[n] (its distance) and second[n] (the runner-up's distance) of
+ * each of the N groups of V; dist and second may be NULL. */
+int aqlm_oracle_nearest(const float *V, int64_t N, const float *C, int64_t K, int32_t *idx, double *dist,
+                        double *second)
 {
     if (N < 0 || K < 1) return 1;
-    float *cc = norms(C, K);
-    if (!cc) return 2;
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; ++n) {
-        const int64_t best = nearest_one(V + n * 8, C, cc, K);
-        idx[n] = (int32_t)best;
-        if (dist) dist[n] = distance(V + n * 8, C + best * 8);
+        double bd, sd;
+        idx[n] = (int32_t)nearest_one(V + n * 8, C, K, &bd, &sd);
+        if (dist) dist[n] = bd;
+        if (second) second[n] = sd;
     }
-    free(cc);
     return 0;
 }
 
@@ -257,12 +220,12 @@ int aqlm_oracle_residual_kmeans(const float *V, int64_t N, int M, int64_t K, con
             memcpy(C + k * 8, R + n * 8, 8 * sizeof(float));
         }
         for (int it = 0; it < iters && !rc; ++it) {
-            aqlm_oracle_nearest(R, N, C, K, idx, NULL);
+            aqlm_oracle_nearest(R, N, C, K, idx, NULL, NULL);
             rc = aqlm_oracle_kmeans_update(R, idx, N, K, C, tmp, counts);
             memcpy(C, tmp, (size_t)K * 8 * sizeof(float));
         }
         if (rc) break;
-        aqlm_oracle_nearest(R, N, C, K, idx, NULL);
+        aqlm_oracle_nearest(R, N, C, K, idx, NULL, NULL);
         for (int64_t n = 0; n < N; ++n)
             for (int t = 0; t < 8; ++t) R[n * 8 + t] = R[n * 8 + t] - C[(int64_t)idx[n] * 8 + t];
     }
@@ -280,23 +243,17 @@ int aqlm_oracle_encode_greedy(const float *V, int64_t N, const uint16_t *codeboo
     float *C = (float *)malloc((size_t)M * K * 8 * sizeof(float));
     if (!C) return 2;
     for (int64_t i = 0; i < (int64_t)M * K * 8; ++i) C[i] = half_to_float(codebooks[i]);
-    float *cc = norms(C, (int64_t)M * K);
-    if (!cc) {
-        free(C);
-        return 2;
-    }
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; ++n) {
         float r[8];
         memcpy(r, V + n * 8, sizeof(r));
         for (int m = 0; m < M; ++m) {
             const float *Cm = C + (int64_t)m * K * 8;
-            const int64_t best = nearest_one(r, Cm, cc + (int64_t)m * K, K);
+            const int64_t best = nearest_one(r, Cm, K, NULL, NULL);
             codes[n * M + m] = (uint16_t)best;
             for (int t = 0; t < 8; ++t) r[t] = r[t] - Cm[best * 8 + t];
         }
     }
     free(C);
-    free(cc);
     return 0;
 }

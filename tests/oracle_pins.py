@@ -355,31 +355,44 @@ def _brute_nearest(V, C):
 
 
 def pin_nearest_codeword():
-    """E3: the chosen codeword is the nearest by the float64 distance (brute
-    force), exactly so wherever the two nearest are not within rounding of
-    each other; a group equal to a codeword gets that codeword at distance 0;
-    duplicated codewords resolve to the lowest index."""
+    """E3 against float64 brute force on small inputs: the chosen codeword's
+    distance is the least one (to within double rounding), the index is the
+    brute-force argmin wherever the two nearest differ by more than double
+    rounding, and the reported distance and runner-up distance are the
+    brute-force smallest and second smallest; a group equal to a codeword gets
+    it at distance 0; a group exactly midway between two codewords (dyadic
+    values, so both distances are exact) and duplicated codewords resolve to
+    the lowest index."""
     rng = _rng(22)
     C = rng.standard_normal((300, 8)).astype(np.float32)
     V = rng.standard_normal((500, 8)).astype(np.float32)
     V[:50] = C[rng.integers(0, 300, 50)]
-    idx, dist = oracle.nearest(V, C)
+    idx, dist, second = oracle.nearest(V, C)
     d = _brute_nearest(V, C)
-    best = d.min(axis=1)
-    chosen = d[np.arange(len(V)), idx]
-    assert np.all(chosen <= best * (1 + 1e-5) + 1e-12)
     srt = np.sort(d, axis=1)
-    clear = srt[:, 1] > srt[:, 0] * (1 + 1e-4) + 1e-9
+    rows = np.arange(len(V))
+    assert np.all(d[rows, idx] <= srt[:, 0] * (1 + 1e-12))
+    clear = srt[:, 1] - srt[:, 0] > 1e-9 * srt[:, 1]
+    assert clear.mean() > 0.99
     assert np.array_equal(idx[clear], d.argmin(axis=1)[clear])
-    assert np.allclose(dist, chosen, rtol=1e-5, atol=1e-12)
+    assert np.allclose(dist, srt[:, 0], rtol=1e-12, atol=0)
+    assert np.allclose(second, srt[:, 1], rtol=1e-12, atol=0)
     assert np.all(dist[:50] == 0)
     # duplicates: codewords 10 and 20 equal, a group equal to them -> 10
     C2 = C.copy()
     C2[20] = C2[10]
-    i2, _ = oracle.nearest(C2[10:11] + np.float32(0), C2)
-    assert i2[0] == 10
-    i3, _ = oracle.nearest(C2[20:21], C2[::-1].copy())
+    i2, d2, s2 = oracle.nearest(C2[10:11] + np.float32(0), C2)
+    assert i2[0] == 10 and d2[0] == 0 and s2[0] == 0
+    i3, _, _ = oracle.nearest(C2[20:21], C2[::-1].copy())
     assert i3[0] == 300 - 1 - 20
+    # exact midpoint: v = 0.25 * (1, -1, 0, ...), codewords v + e at 7 and v - e at 3 (e dyadic)
+    v = np.zeros((1, 8), dtype=np.float32)
+    v[0, :2] = [0.25, -0.25]
+    e = np.array([0.5, 0.25, -0.125, 0, 0, 0, 0.0625, 0], dtype=np.float32)
+    C3 = np.full((9, 8), 4.0, dtype=np.float32)
+    C3[7], C3[3] = v[0] + e, v[0] - e
+    i4, d4, s4 = oracle.nearest(v, C3)
+    assert i4[0] == 3 and d4[0] == s4[0] == float((e.astype(np.float64) ** 2).sum())
 
 
 def pin_kmeans_update():
@@ -472,7 +485,7 @@ def pin_worked_encoding():
     want = np.array([[n / d for n, d in row] for row in ex["expected_groups_num_den"]])
     assert np.all(np.abs(V.astype(np.float64) - want) <= np.abs(want) * 2.0 ** -24)
     cb = np.array(ex["codebooks"], dtype=np.float16)
-    idx, _ = oracle.nearest(V, cb[0].astype(np.float32))
+    idx, _, _ = oracle.nearest(V, cb[0].astype(np.float32))
     assert idx.tolist() == ex["expected_nearest_codebook0"]
     assert oracle.encode_greedy(V, cb).tolist() == ex["expected_codes"]
 

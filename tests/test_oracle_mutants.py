@@ -43,11 +43,12 @@ MUTANTS = {
     # encoding
     "half_ties_away": (ENCODE, "double q = rint(ldexp(a, 11 - e));", "double q = round(ldexp(a, 11 - e));"),
     "scale_mean_abs": (ENCODE, "acc += (double)row[k] * (double)row[k];", "acc += fabs((double)row[k]);"),
-    "nearest_ties_high": (ENCODE, "if (sk < bs) {", "if (sk <= bs) {"),
-    "distance_drops_lane": (ENCODE, "o = fmaf(d[7], d[7], o);", "o = o;"),
-    "score_drops_lane": (ENCODE, "o = fmaf(a[7], b[7], o);", "o = o;"),
-    "score_wrong_sign": (ENCODE, "return fmaf(-2.0f, dot8(v, c), cc);", "return fmaf(2.0f, dot8(v, c), cc);"),
-    "score_drops_norm": (ENCODE, "return fmaf(-2.0f, dot8(v, c), cc);", "return fmaf(-2.0f, dot8(v, c), 0.0f * cc);"),
+    "nearest_ties_high": (ENCODE, "if (dk < bd) {", "if (dk <= bd) {"),
+    "distance_drops_lane": (ENCODE, "for (int t = 0; t < 8; ++t) {\n        const double e",
+                            "for (int t = 0; t < 7; ++t) {\n        const double e"),
+    "distance_wrong_sign": (ENCODE, "(double)v[t] - (double)c[t]", "(double)v[t] + (double)c[t]"),
+    "distance_not_squared": (ENCODE, "d += e * e;", "d += fabs(e);"),
+    "runner_up_lost": (ENCODE, "            sd = bd;\n            bd = dk;", "            bd = dk;"),
     "update_off_by_one": (ENCODE, "(float)(sums[k * 8 + t] / (double)counts[k])",
                           "(float)(sums[k * 8 + t] / (double)(counts[k] + 1))"),
     "residual_not_subtracted": (ENCODE, "R[n * 8 + t] = R[n * 8 + t] - C[(int64_t)idx[n] * 8 + t];",
