@@ -34,6 +34,7 @@ EXPORTS = ["aqlm_gemv", "aqlm_gemv_workspace_bytes", "aqlm_gemv_row_tokens", "aq
            "aqlm_gemv_multi_workspace_bytes", "aqlm_gemv_multi_check", "aqlm_gemv_check", "aqlm_dequant", "aqlm_gemm",
            "aqlm_gemm_workspace_bytes", "aqlm_gemm_check", "aqlm_bf16_gemm", "aqlm_bf16_gemm_tile_n", "aqlm_decode_indices",
            "aqlm_test_gemm_timeout", "aqlm_gemv_noalloc", "aqlm_gemv_noalloc_max_scratch_bytes",
+           "aqlm_gemv_noalloc_check", "aqlm_test_gemv_noalloc_set_status",
            "aqlm_status_string", "aqlm_version",
            "aqlm_encode_scales", "aqlm_nearest_workspace_bytes", "aqlm_nearest_codeword",
            "aqlm_kmeans_workspace_bytes", "aqlm_kmeans_update", "aqlm_residual_kmeans_workspace_bytes",
@@ -92,6 +93,8 @@ def load_library():
         "aqlm_test_gemm_timeout": ([vp, vp, vp, i32, i32, i32, vp, u64, vp], st),
         "aqlm_gemv_noalloc": ([vp, vp, vp, vp, vp, i32, Shape, vp], st),
         "aqlm_gemv_noalloc_max_scratch_bytes": ([], sz),
+        "aqlm_gemv_noalloc_check": ([Shape, i32, vp], st),
+        "aqlm_test_gemv_noalloc_set_status": ([Shape, i32, i32, vp], st),
         "aqlm_encode_scales": ([vp, i32, i32, vp, vp, vp], st),
         "aqlm_nearest_workspace_bytes": ([i64], sz),
         "aqlm_nearest_codeword": ([vp, i64, vp, i32, vp, vp, vp, sz, vp], st),
@@ -278,6 +281,12 @@ def aqlm_gemv_noalloc(codes, codebooks, scales, x, y=None, stream=None):
     _check(lib.aqlm_gemv_noalloc(_p(codes), _p(codebooks), _p(_flat_scales(scales)), _p(x), _p(y), T, shape,
                                  _stream(stream)), "aqlm_gemv_noalloc")
     return y
+
+
+def aqlm_gemv_noalloc_check(codes, tokens, stream=None):
+    """Synchronise and return the status the last aqlm_gemv_noalloc call of
+    this layer shape and token count recorded (AQLM_OK or AQLM_ERR_TIMEOUT)."""
+    return load_library().aqlm_gemv_noalloc_check(shape_of(codes), tokens, _stream(stream))
 
 
 def aqlm_dequant(codes, codebooks, scales, out=None, stream=None):

@@ -63,6 +63,20 @@ aqlm_status read_status_word(long long off, void *workspace, size_t workspace_by
 
 }  // namespace
 
+namespace aqlm {
+
+// The argument checks of aqlm_gemv other than the workspace's.
+aqlm_status check_gemv_args(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
+                            const uint16_t *y, int32_t tokens, const aqlm_shape &shape) {
+    const aqlm_status st = check_layer(codes, codebooks, scales, shape);
+    if (st != AQLM_OK) return st;
+    if (!x || !y || tokens < 1 || tokens > AQLM_GEMV_MAX_TOKENS) return AQLM_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(y, 2)) return AQLM_ERR_MISALIGNED;
+    return AQLM_OK;
+}
+
+}  // namespace aqlm
+
 extern "C" {
 
 aqlm_status aqlm_decode_indices(const void *codes, uint16_t *idx_out, aqlm_shape shape, aqlm_stream_t stream) {
@@ -90,10 +104,8 @@ size_t aqlm_gemv_workspace_bytes(aqlm_shape shape, int32_t tokens) {
 aqlm_status aqlm_gemv(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
                       uint16_t *y, int32_t tokens, aqlm_shape shape, void *workspace, size_t workspace_bytes,
                       aqlm_stream_t stream) {
-    aqlm_status st = check_layer(codes, codebooks, scales, shape);
+    const aqlm_status st = aqlm::check_gemv_args(codes, codebooks, scales, x, y, tokens, shape);
     if (st != AQLM_OK) return st;
-    if (!x || !y || tokens < 1 || tokens > AQLM_GEMV_MAX_TOKENS) return AQLM_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(y, 2)) return AQLM_ERR_MISALIGNED;
     const Dims d = aqlm::make_dims(shape);
     const size_t need = aqlm::gemv_workspace_bytes(d, tokens);
     if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16))) return AQLM_ERR_WORKSPACE;

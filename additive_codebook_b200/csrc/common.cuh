@@ -222,6 +222,8 @@ namespace aqlm {
 cudaError_t launch_decode_indices(const void *codes, uint16_t *idx, const Dims &d, cudaStream_t st);
 cudaError_t launch_dequant(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                            uint16_t *W, const Dims &d, cudaStream_t st);
+aqlm_status check_gemv_args(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
+                            const uint16_t *y, int32_t tokens, const aqlm_shape &shape);
 size_t gemv_workspace_bytes(const Dims &d, int tokens);
 size_t gemv_workspace_counter_offset(const Dims &d, int tokens);
 long long gemv_status_offset(const Dims &d, int tokens);

@@ -284,14 +284,19 @@ AQLM_API aqlm_status aqlm_test_gemm_timeout(const uint16_t *X, const uint16_t *W
  * GPU (aqlm_gemv_noalloc_max_scratch_bytes()), held by every GPU that loads
  * the library until the process exits.  A shape and token count whose
  * scratch (aqlm_gemv_workspace_bytes) exceeds that is rejected with
- * AQLM_ERR_WORKSPACE.  The first call on a device looks up the array's
+ * AQLM_ERR_WORKSPACE.  Arguments are checked as aqlm_gemv checks them before
+ * anything is enqueued.  The first call on a device looks up the array's
  * device address there (cudaGetSymbolAddress); make that first call before
- * any stream capture.  The part of the array that must start at zero is
- * cleared on `stream` at every call.  All calls on a device share the one
+ * any stream capture (a lookup that fails is not kept: the next call tries
+ * again).  Each call clears the array's arrival counters on `stream`; the
+ * status word is left alone, so a bounded wait that gave up (4 tokens and
+ * more, see aqlm_gemv) stays recorded until aqlm_gemv_noalloc_check reads
+ * it -- check before the next call of another shape or token count, whose
+ * layout may reuse that word's bytes.  All calls on a device share the one
  * array and it keeps the last call's contents: calls that overlap on the GPU
  * (other streams, other host threads) race and must be avoided.  No
- * cudaMalloc, cudaFree or other allocating routine is called.  Arguments,
- * results and errors otherwise as aqlm_gemv.
+ * cudaMalloc, cudaFree or other allocating routine is called.  Results and
+ * errors otherwise as aqlm_gemv.
  */
 AQLM_API aqlm_status aqlm_gemv_noalloc(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                                        const uint16_t *x, uint16_t *y, int32_t tokens, aqlm_shape shape,
@@ -299,6 +304,20 @@ AQLM_API aqlm_status aqlm_gemv_noalloc(const void *codes, const uint16_t *codebo
 
 /* Size of aqlm_gemv_noalloc's built-in scratch array, in bytes. */
 AQLM_API size_t aqlm_gemv_noalloc_max_scratch_bytes(void);
+
+/* aqlm_gemv_check for aqlm_gemv_noalloc: synchronise `stream`, then read and
+ * clear the status word that the last aqlm_gemv_noalloc call of this shape
+ * and token count left in the built-in array: AQLM_OK, or AQLM_ERR_TIMEOUT
+ * (y of that call is then not valid).  Paths without device waits: AQLM_OK
+ * after the synchronisation.  No counterpart on the pages. */
+AQLM_API aqlm_status aqlm_gemv_noalloc_check(aqlm_shape shape, int32_t tokens, aqlm_stream_t stream);
+
+/* Test only: write `value` into the status word of (shape, tokens)'s layout
+ * in aqlm_gemv_noalloc's array and synchronise (AQLM_ERR_UNSUPPORTED where
+ * that path has no status word), so that tests can check the reporting
+ * without making a device wait run out. */
+AQLM_API aqlm_status aqlm_test_gemv_noalloc_set_status(aqlm_shape shape, int32_t tokens, int32_t value,
+                                                       aqlm_stream_t stream);
 
 /* ===========================================================================
  * Encoding: scales, codebooks and codes of a layer from its weights.

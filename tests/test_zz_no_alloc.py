@@ -5,8 +5,10 @@ call it -- a plugin that its host engine hands only input and output
 pointers, or an engine that fixes its device memory at start-up.  For them
 aqlm_gemv_noalloc keeps its scratch in an array built into the library
 instead of a caller-provided workspace.  These tests call it through the C
-ABI, twice in a row on the same shape, and hold its output to the tolerance
-of the other parity tests against aqlm_gemv's output on the same inputs.
+ABI, twice in a row on the same shape, and hold its output to the oracle
+(the tolerance of the other parity tests) and bit for bit to aqlm_gemv's
+output on the same inputs (the same kernels on the same scratch layout); its
+status word must survive later calls until aqlm_gemv_noalloc_check reads it.
 
 This file is named so that pytest collects it last: a run that stops at the
 first failure has then already run every other test.
@@ -31,43 +33,83 @@ pytestmark = pytest.mark.gpu
 CASES = [(1024, 28672, 2, 8, 3), (2048, 4096, 2, 8, 6), (1024, 4096, 1, 16, 16), (512, 4160, 2, 16, 8)]
 
 
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
 def _call_noalloc(lib, d, x, y):
     shape = ac.shape_of(d["codes"])
-    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     return lib.aqlm_gemv_noalloc(ctypes.c_void_p(d["codes"].data_ptr()), ctypes.c_void_p(d["codebooks"].data_ptr()),
                                  ctypes.c_void_p(d["scales"].data_ptr()), ctypes.c_void_p(x.data_ptr()),
-                                 ctypes.c_void_p(y.data_ptr()), x.shape[0], shape, stream)
+                                 ctypes.c_void_p(y.data_ptr()), x.shape[0], shape, _stream())
 
 
 @pytest.mark.parametrize("d_out,d_in,M,B,T", CASES)
-def test_noalloc_matches_gemv_on_two_calls(cuda_device, d_out, d_in, M, B, T):
+def test_noalloc_matches_oracle_and_gemv_on_two_calls(cuda_device, d_out, d_in, M, B, T):
     lib = ac.load_library()
     spec = LayerSpec(d_out, d_in, M, B)
     L = make_layer(spec, seed=77 + T, tokens=T)
     d = to_dev(L)
     shape = ac.shape_of(d["codes"])
     assert 0 < lib.aqlm_gemv_workspace_bytes(shape, T) <= lib.aqlm_gemv_noalloc_max_scratch_bytes()
-    y_ref = ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], d["x"]).cpu().numpy().astype(np.float64)
+    y_gemv = ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], d["x"]).cpu().numpy()
     W = oracle_W(L, spec)
     x64 = L["x"].astype(np.float64)
+    y_ref = W @ x64.T
     for _ in range(2):
         y = torch.full((T, d_out), float("nan"), dtype=torch.float16, device=DEV)
         assert _call_noalloc(lib, d, d["x"], y) == ac.AQLM_OK
-        torch.cuda.synchronize()
-        check_fp_output(y.cpu().numpy(), y_ref, W, x64, out_rel=2.0 ** -10, acc_rel=2.0 ** -14)
+        assert lib.aqlm_gemv_noalloc_check(shape, T, _stream()) == ac.AQLM_OK
+        y = y.cpu().numpy()
+        check_fp_output(y, y_ref.T, W, x64, out_rel=2.0 ** -10, acc_rel=2.0 ** -14)
+        assert np.array_equal(y.view(np.uint16), y_gemv.view(np.uint16))
 
 
-def test_noalloc_rejects_scratch_beyond_its_maximum(cuda_device):
+def test_noalloc_status_survives_until_checked(cuda_device):
+    """A status word set in the built-in array (as a bounded wait that gave up
+    would set it) is reported by aqlm_gemv_noalloc_check even after another
+    call of the same shape, then cleared."""
     lib = ac.load_library()
+    d_out, d_in, M, B, T = CASES[2]
+    spec = LayerSpec(d_out, d_in, M, B)
+    L = make_layer(spec, seed=5, tokens=T)
+    d = to_dev(L)
+    shape = ac.shape_of(d["codes"])
+    y = torch.empty((T, d_out), dtype=torch.float16, device=DEV)
+    assert _call_noalloc(lib, d, d["x"], y) == ac.AQLM_OK
+    assert lib.aqlm_gemv_noalloc_check(shape, T, _stream()) == ac.AQLM_OK
+    assert lib.aqlm_test_gemv_noalloc_set_status(shape, T, ac.AQLM_ERR_TIMEOUT, _stream()) == ac.AQLM_OK
+    assert _call_noalloc(lib, d, d["x"], y) == ac.AQLM_OK
+    assert lib.aqlm_gemv_noalloc_check(shape, T, _stream()) == ac.AQLM_ERR_TIMEOUT
+    assert lib.aqlm_gemv_noalloc_check(shape, T, _stream()) == ac.AQLM_OK
+    # the row-kernel path has no status word
+    row = ac.Shape(1024, 28672, 8, 2, 8)
+    assert lib.aqlm_test_gemv_noalloc_set_status(row, 3, 1, _stream()) == ac.AQLM_ERR_UNSUPPORTED
+    assert lib.aqlm_gemv_noalloc_check(row, 3, _stream()) == ac.AQLM_OK
+
+
+def test_noalloc_checks_arguments_before_touching_the_array(cuda_device):
+    """A call rejected for its arguments enqueues nothing: a recorded status
+    stays, and sizes beyond the array are rejected with AQLM_ERR_WORKSPACE."""
+    lib = ac.load_library()
+    d_out, d_in, M, B, T = CASES[2]
+    shape = ac.Shape(d_out, d_in, 8, M, B)
+    x = torch.zeros((T, d_in), dtype=torch.float16, device=DEV)
+    y = torch.zeros((T, d_out), dtype=torch.float16, device=DEV)
+    codes = torch.zeros(16, dtype=torch.uint8, device=DEV)
+    p = ctypes.c_void_p(codes.data_ptr())
+    assert lib.aqlm_test_gemv_noalloc_set_status(shape, T, ac.AQLM_ERR_TIMEOUT, _stream()) == ac.AQLM_OK
+    st = lib.aqlm_gemv_noalloc(p, p, p, ctypes.c_void_p(x.data_ptr()), None, T, shape, _stream())
+    assert st == ac.AQLM_ERR_INVALID_ARG
+    st = lib.aqlm_gemv_noalloc(p, p, p, ctypes.c_void_p(x.data_ptr() + 2), ctypes.c_void_p(y.data_ptr()), T, shape,
+                               _stream())
+    assert st == ac.AQLM_ERR_MISALIGNED
+    assert lib.aqlm_gemv_noalloc_check(shape, T, _stream()) == ac.AQLM_ERR_TIMEOUT
     # 3 tokens of 28672 inputs on the row kernel (2x8): seven activation
     # slices, 7 x 3 x 131072 fp32 partial sums (11 MB), more than the 8 MiB
     # built in
-    shape = ac.Shape(131072, 28672, 8, 2, 8)
-    assert lib.aqlm_gemv_workspace_bytes(shape, 3) > lib.aqlm_gemv_noalloc_max_scratch_bytes()
-    codes = torch.zeros(16, dtype=torch.uint8, device=DEV)   # never read: the call is rejected first
-    x = torch.zeros(16, 16, dtype=torch.float16, device=DEV)
-    y = torch.zeros(16, 16, dtype=torch.float16, device=DEV)
-    p = ctypes.c_void_p(codes.data_ptr())
-    st = lib.aqlm_gemv_noalloc(p, p, p, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()), 3, shape,
-                               ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    big = ac.Shape(131072, 28672, 8, 2, 8)
+    assert lib.aqlm_gemv_workspace_bytes(big, 3) > lib.aqlm_gemv_noalloc_max_scratch_bytes()
+    st = lib.aqlm_gemv_noalloc(p, p, p, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()), 3, big,
+                               _stream())
     assert st == ac.AQLM_ERR_WORKSPACE
