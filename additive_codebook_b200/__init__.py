@@ -34,7 +34,8 @@ EXPORTS = ["aqlm_gemv", "aqlm_gemv_workspace_bytes", "aqlm_gemv_row_tokens", "aq
            "aqlm_gemv_multi_workspace_bytes", "aqlm_gemv_multi_check", "aqlm_gemv_check", "aqlm_dequant", "aqlm_gemm",
            "aqlm_gemm_workspace_bytes", "aqlm_gemm_check", "aqlm_bf16_gemm", "aqlm_bf16_gemm_tile_n", "aqlm_decode_indices",
            "aqlm_test_gemm_timeout", "aqlm_gemv_noalloc", "aqlm_gemv_noalloc_max_scratch_bytes",
-           "aqlm_gemv_noalloc_check", "aqlm_test_gemv_noalloc_set_status",
+           "aqlm_gemv_noalloc_check", "aqlm_test_gemv_noalloc_set_status", "aqlm_probe_gather_sink_bytes",
+           "aqlm_probe_gather",
            "aqlm_status_string", "aqlm_version",
            "aqlm_encode_scales", "aqlm_nearest_workspace_bytes", "aqlm_nearest_codeword",
            "aqlm_kmeans_workspace_bytes", "aqlm_kmeans_update", "aqlm_residual_kmeans_workspace_bytes",
@@ -93,8 +94,10 @@ def load_library():
         "aqlm_test_gemm_timeout": ([vp, vp, vp, i32, i32, i32, vp, u64, vp], st),
         "aqlm_gemv_noalloc": ([vp, vp, vp, vp, vp, i32, Shape, vp], st),
         "aqlm_gemv_noalloc_max_scratch_bytes": ([], sz),
-        "aqlm_gemv_noalloc_check": ([Shape, i32, vp], st),
-        "aqlm_test_gemv_noalloc_set_status": ([Shape, i32, i32, vp], st),
+        "aqlm_gemv_noalloc_check": ([vp], st),
+        "aqlm_test_gemv_noalloc_set_status": ([i32, vp], st),
+        "aqlm_probe_gather_sink_bytes": ([i32], sz),
+        "aqlm_probe_gather": ([vp, sz, i32, i32, i32, vp, sz, ctypes.POINTER(u64), vp], st),
         "aqlm_encode_scales": ([vp, i32, i32, vp, vp, vp], st),
         "aqlm_nearest_workspace_bytes": ([i64], sz),
         "aqlm_nearest_codeword": ([vp, i64, vp, i32, vp, vp, vp, sz, vp], st),
@@ -283,10 +286,24 @@ def aqlm_gemv_noalloc(codes, codebooks, scales, x, y=None, stream=None):
     return y
 
 
-def aqlm_gemv_noalloc_check(codes, tokens, stream=None):
-    """Synchronise and return the status the last aqlm_gemv_noalloc call of
-    this layer shape and token count recorded (AQLM_OK or AQLM_ERR_TIMEOUT)."""
-    return load_library().aqlm_gemv_noalloc_check(shape_of(codes), tokens, _stream(stream))
+def aqlm_gemv_noalloc_check(stream=None):
+    """Synchronise and return the status that aqlm_gemv_noalloc calls since the
+    last check recorded (AQLM_OK or AQLM_ERR_TIMEOUT); clears it."""
+    return load_library().aqlm_gemv_noalloc_check(_stream(stream))
+
+
+def probe_gather(table, source, ctas_per_sm=8, iters=64, sink=None, stream=None):
+    """Launch the random 16-byte gather probe on `table` (a device tensor);
+    returns (gathers made, sink).  source 0: through L1/L2 like the 1x16 and
+    2x16 codeword loads; 1: from a shared-memory copy (table <= 64 KiB)."""
+    lib = load_library()
+    nbytes = table.numel() * table.element_size()
+    if sink is None:
+        sink = torch.empty(lib.aqlm_probe_gather_sink_bytes(ctas_per_sm), dtype=torch.uint8, device=table.device)
+    n = ctypes.c_uint64(0)
+    _check(lib.aqlm_probe_gather(_p(table), nbytes, source, ctas_per_sm, iters, _p(sink), sink.numel(),
+                                 ctypes.byref(n), _stream(stream)), "aqlm_probe_gather")
+    return n.value, sink
 
 
 def aqlm_dequant(codes, codebooks, scales, out=None, stream=None):

@@ -17,9 +17,14 @@
 // successful lookup is kept: a failed one (say, attempted during a stream
 // capture) is retried by the next call.
 //
-// Every call clears the arrival counters of its layout on the stream, but not
-// the status word: a bounded wait that gave up stays recorded there until
-// aqlm_gemv_noalloc_check reads and clears it.
+// Status word.  From 4 tokens up the product runs on the tensor cores with
+// bounded waits, and a wait that gives up records AQLM_ERR_TIMEOUT in the
+// workspace's last 16 bytes.  Here every such workspace is placed at the END
+// of the array, so that word is always the array's last 16 bytes, whatever
+// the shape; the layouts without a status word are placed at the start and
+// kept clear of those bytes.  No call's partial sums or counters ever land on
+// the word, each call clears only its own counters, and a recorded timeout
+// therefore stays until aqlm_gemv_noalloc_check reads and clears it.
 #include <atomic>
 #include <mutex>
 
@@ -55,10 +60,15 @@ cudaError_t scratch_on_current_device(unsigned char **out) {
     return cudaSuccess;
 }
 
-// Byte offset of the status word of (shape, tokens)'s layout, or -1 if that
-// path has none; the shape and token count must be valid.
-long long status_offset(const aqlm_shape &shape, int32_t tokens) {
-    return aqlm::gemv_status_offset(aqlm::make_dims(shape), tokens);
+constexpr size_t kStatusBytes = 16;  // the array's last 16 bytes: the status word
+
+// Where the workspace of (d, tokens) starts inside the array: at the end for
+// layouts with a status word (which then falls on the array's last 16 bytes),
+// at the start otherwise.
+bool has_status_word(const aqlm::Dims &d, int32_t tokens) { return aqlm::gemv_status_offset(d, tokens) >= 0; }
+
+size_t usable_bytes(const aqlm::Dims &d, int32_t tokens) {
+    return has_status_word(d, tokens) ? kNoAllocScratchBytes : kNoAllocScratchBytes - kStatusBytes;
 }
 
 }  // namespace
@@ -74,43 +84,44 @@ aqlm_status aqlm_gemv_noalloc(const void *codes, const uint16_t *codebooks, cons
     if (st != AQLM_OK) return st;
     const aqlm::Dims d = aqlm::make_dims(shape);
     const size_t need = aqlm::gemv_workspace_bytes(d, tokens);
-    if (need > kNoAllocScratchBytes) return AQLM_ERR_WORKSPACE;
-    unsigned char *scratch = nullptr;
+    if (need > usable_bytes(d, tokens)) return AQLM_ERR_WORKSPACE;
+    unsigned char *ws = nullptr;
     if (need > 0) {
+        unsigned char *scratch = nullptr;
         if (scratch_on_current_device(&scratch) != cudaSuccess) return AQLM_ERR_CUDA;
-        // Clear the arrival counters on the stream (an earlier call of another
-        // shape may have left partial sums there), up to the status word.
+        const bool status = has_status_word(d, tokens);
+        ws = status ? scratch + (kNoAllocScratchBytes - need) : scratch;  // need is a multiple of 16 there
+        // Clear this layout's arrival counters on the stream (an earlier call of
+        // another shape may have left partial sums there), not the status word.
         const size_t off = aqlm::gemv_workspace_counter_offset(d, tokens);
-        const long long so = status_offset(shape, tokens);
-        const size_t end = so >= 0 ? (size_t)so : need;
+        const size_t end = status ? need - kStatusBytes : need;
         if (end > off &&
-            cudaMemsetAsync(scratch + off, 0, end - off, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+            cudaMemsetAsync(ws + off, 0, end - off, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
             return AQLM_ERR_CUDA;
     }
-    return aqlm_gemv(codes, codebooks, scales, x, y, tokens, shape, scratch, need, stream);
+    return aqlm_gemv(codes, codebooks, scales, x, y, tokens, shape, ws, need, stream);
 }
 
-aqlm_status aqlm_gemv_noalloc_check(aqlm_shape shape, int32_t tokens, aqlm_stream_t stream) {
-    if (aqlm_gemv_row_tokens(shape) < 1) return AQLM_ERR_UNSUPPORTED;  // the shape checks of aqlm_gemv_check
-    if (tokens < 1 || tokens > AQLM_GEMV_MAX_TOKENS) return AQLM_ERR_INVALID_ARG;
+aqlm_status aqlm_gemv_noalloc_check(aqlm_stream_t stream) {
     const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    if (status_offset(shape, tokens) < 0) return cudaStreamSynchronize(cs) == cudaSuccess ? AQLM_OK : AQLM_ERR_CUDA;
-    const size_t need = aqlm_gemv_workspace_bytes(shape, tokens);
-    if (need > kNoAllocScratchBytes) return AQLM_ERR_WORKSPACE;
     unsigned char *scratch = nullptr;
     if (scratch_on_current_device(&scratch) != cudaSuccess) return AQLM_ERR_CUDA;
-    return aqlm_gemv_check(shape, tokens, scratch, need, stream);
+    int32_t *word = reinterpret_cast<int32_t *>(scratch + kNoAllocScratchBytes - kStatusBytes);
+    int32_t h = 0;
+    if (cudaMemcpyAsync(&h, word, sizeof(h), cudaMemcpyDeviceToHost, cs) != cudaSuccess) return AQLM_ERR_CUDA;
+    if (cudaStreamSynchronize(cs) != cudaSuccess) return AQLM_ERR_CUDA;
+    if (h == 0) return AQLM_OK;
+    if (cudaMemsetAsync(word, 0, sizeof(int32_t), cs) != cudaSuccess) return AQLM_ERR_CUDA;
+    if (cudaStreamSynchronize(cs) != cudaSuccess) return AQLM_ERR_CUDA;
+    return AQLM_ERR_TIMEOUT;
 }
 
-aqlm_status aqlm_test_gemv_noalloc_set_status(aqlm_shape shape, int32_t tokens, int32_t value, aqlm_stream_t stream) {
-    if (aqlm_gemv_workspace_bytes(shape, tokens) > kNoAllocScratchBytes) return AQLM_ERR_WORKSPACE;
-    if (aqlm_gemv_row_tokens(shape) < 1 || tokens < 1 || tokens > AQLM_GEMV_MAX_TOKENS) return AQLM_ERR_INVALID_ARG;
-    const long long so = status_offset(shape, tokens);
-    if (so < 0) return AQLM_ERR_UNSUPPORTED;
+aqlm_status aqlm_test_gemv_noalloc_set_status(int32_t value, aqlm_stream_t stream) {
     unsigned char *scratch = nullptr;
     if (scratch_on_current_device(&scratch) != cudaSuccess) return AQLM_ERR_CUDA;
     const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaMemcpyAsync(scratch + so, &value, sizeof(value), cudaMemcpyHostToDevice, cs) != cudaSuccess)
+    if (cudaMemcpyAsync(scratch + kNoAllocScratchBytes - kStatusBytes, &value, sizeof(value), cudaMemcpyHostToDevice,
+                        cs) != cudaSuccess)
         return AQLM_ERR_CUDA;
     return cudaStreamSynchronize(cs) == cudaSuccess ? AQLM_OK : AQLM_ERR_CUDA;
 }

@@ -269,15 +269,22 @@ def bench_gemv(ac, spec, T, steps, warmup, l2_bytes, n_launch=STEP_LAYERS, dist=
             "launches": steps * n_launch, "ms": ms, "layers": layers, "ws": ws}
 
 
-def single_call_us(ac, bench, reps=50):
-    """Latency of one aqlm_gemv call on its own (not in a graph, no neighbour to
-    overlap with): CUDA events around each call, median over `reps` calls that
-    cycle over the layer copies."""
+def call_latency(ac, bench, reps=200):
+    """Latency of one aqlm_gemv call on its own, split into its parts:
+    - device_us: CUDA events around each isolated call (median; no graph, no
+      neighbour to overlap with);
+    - host_c_us: host time of the C entry point alone (validation, kernel
+      choice, launch), called through ctypes with pre-marshalled arguments,
+      mean over `reps` calls that return without synchronising;
+    - host_python_us: the same through the Python binding (argument
+      marshalling included)."""
+    import ctypes
     import torch
     layers, ws = bench["layers"], bench["ws"]
-    y = torch.empty((layers.T, layers.spec.d_out), dtype=torch.float16, device="cuda")
-    out = []
-    for i in range(reps + 5):
+    T, spec = layers.T, layers.spec
+    y = torch.empty((T, spec.d_out), dtype=torch.float16, device="cuda")
+    dev = []
+    for i in range(55):
         d = layers.copies[i % layers.R]
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
@@ -286,8 +293,30 @@ def single_call_us(ac, bench, reps=50):
         e1.record()
         torch.cuda.synchronize()
         if i >= 5:
-            out.append(e0.elapsed_time(e1) * 1e3)
-    return statistics.median(out)
+            dev.append(e0.elapsed_time(e1) * 1e3)
+    lib = ac.load_library()
+    shape = ac.shape_of(layers.copies[0]["codes"])
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    wsp, wsb = (ctypes.c_void_p(ws.data_ptr()), ws.numel()) if ws is not None else (None, 0)
+    args = [(ctypes.c_void_p(d["codes"].data_ptr()), ctypes.c_void_p(d["codebooks"].data_ptr()),
+             ctypes.c_void_p(d["scales"].data_ptr())) for d in layers.copies[:8]]
+    xp, yp = ctypes.c_void_p(layers.x.data_ptr()), ctypes.c_void_p(y.data_ptr())
+    fn = lib.aqlm_gemv
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(reps):
+        c, cb, sc = args[i & 7]
+        fn(c, cb, sc, xp, yp, T, shape, wsp, wsb, stream)
+    t_c = (time.perf_counter() - t0) / reps
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(reps):
+        d = layers.copies[i % layers.R]
+        ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], layers.x, y=y, workspace=ws)
+    t_py = (time.perf_counter() - t0) / reps
+    torch.cuda.synchronize()
+    return {"device_us": round(statistics.median(dev), 3), "host_c_us": round(t_c * 1e6, 3),
+            "host_python_us": round(t_py * 1e6, 3)}
 
 
 def bench_block(ac, fmt, steps, warmup, l2_bytes, fused=False, T=1):
@@ -467,6 +496,47 @@ def cpu_oracle_sample(spec, T, budget_s=10.0):
             "kind": "oracle", "sample": f"{n} full {spec.name} layer products, T={T}, {el:.1f} s"}
 
 
+def cpu_oracle_block(fmt, budget_s=4.0):
+    """The oracle on whole Llama-2-7B decoder blocks (its 7 layer products,
+    one token), repeated for about budget_s; us per block and GB/s."""
+    import oracle
+    M, B = fmt
+    specs = [LayerSpec(o, i, M, B) for _, o, i in LLAMA7B_SHAPES]
+    Ls = [make_layer(sp, seed=k, tokens=1) for k, sp in enumerate(specs)]
+    n, t0 = 0, time.perf_counter()
+    while True:
+        for sp, L in zip(specs, Ls):
+            oracle.gemv_f64(L["codes"], L["codebooks"], L["scales"], L["x"], sp.d_out, sp.d_in, 8, M, B)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    bytes_block = sum(algo_bytes(sp, 1) for sp in specs)
+    return {"us_per_block": round(el / n * 1e6, 1), "value": round(n * bytes_block / el / 1e9, 4), "unit": "GB/s",
+            "cores": oracle.num_threads(), "kind": "oracle", "sample": f"{n} full blocks, {el:.1f} s"}
+
+
+def cpu_oracle_prefill(spec, tokens, subset=128):
+    """The oracle's prefill on the host cores: its double-precision
+    dequantisation of the layer once, and its matmul on a subset of `subset`
+    tokens, scaled to `tokens` (the full product would take minutes)."""
+    import oracle
+    L = make_layer(spec, seed=0, tokens=subset, x_dtype="bf16")
+    t0 = time.perf_counter()
+    W = oracle.dequant_f64(L["codes"], L["codebooks"], L["scales"], spec.d_out, spec.d_in, 8, spec.M, spec.B)
+    t_deq = time.perf_counter() - t0
+    X = oracle.bf16_bits_to_f64(L["x"])
+    t0 = time.perf_counter()
+    oracle.matmul_f64(W, X)
+    t_mm = time.perf_counter() - t0
+    t_full = t_deq + t_mm * tokens / subset
+    flops = 2.0 * tokens * spec.d_out * spec.d_in
+    return {"us_per_layer": round(t_full * 1e6, 1), "value": round(flops / t_full / 1e12, 5), "unit": "TFLOP/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": (f"dequant of the layer ({t_deq:.2f} s) + matmul of {subset} of the {tokens} tokens "
+                       f"({t_mm:.2f} s), matmul time scaled by {tokens // subset}")}
+
+
 def run_gpu(args):
     import torch
     import additive_codebook_b200 as ac
@@ -491,23 +561,30 @@ def run_gpu(args):
     n_launch = max(STEP_LAYERS, head["copies"])
     value = whole_job_gbs(world, args.steps, n_launch, head["bytes_per_layer"], head["ms"])
     achieved = head["bytes_per_layer"] / (head["us_per_layer"] * 1e-6) / 1e9
+    rate = measure_gather_rates(ac)
+    cpu_ok = rank == 0 and world == 1 and not args.quick
     detail = {}
     if not args.quick:
-        r = bench_gemv(ac, LayerSpec(4096, 4096, 2, 8), 1, max(3, args.steps // 2), args.warmup, l2)
-        detail["2x8 4096x4096 T1"] = _gemv_detail(r, peaks)
+        for (o, i) in ((256, 512), (4096, 4096)):
+            r = bench_gemv(ac, LayerSpec(o, i, 2, 8), 1, max(3, args.steps // 2), args.warmup, l2)
+            detail[f"2x8 {o}x{i} T1"] = _gemv_detail(r, peaks, rate)
+            detail[f"2x8 {o}x{i} T1"]["copies"] = r["copies"]
+            del r
         for fmt, T in (((1, 16), 1), ((2, 8), 1), ((1, 16), 4)):
             for fused in (False, True):
                 b = bench_block(ac, fmt, max(3, args.steps // 2), args.warmup, l2, fused=fused, T=T)
                 gbs = b["bytes_per_block"] / (b["us_per_block"] * 1e-6) / 1e9
-                detail[f"llama2-7b block {fmt[0]}x{fmt[1]} T{T}" + (" fused qkv, gate+up" if fused else "")] = {
-                    "us_per_block": round(b["us_per_block"], 3), "gbs": round(gbs, 1),
-                    "hbm_frac": round(gbs / peaks["hbm_gbs"], 4), "launches": b["launches_per_block"]}
+                key = f"llama2-7b block {fmt[0]}x{fmt[1]} T{T}" + (" fused qkv, gate+up" if fused else "")
+                detail[key] = {"us_per_block": round(b["us_per_block"], 3), "gbs": round(gbs, 1),
+                               "hbm_frac": round(gbs / peaks["hbm_gbs"], 4), "launches": b["launches_per_block"]}
+                if cpu_ok and T == 1 and not fused:
+                    detail[key]["cpu_oracle"] = cpu_oracle_block(fmt)
         for name, o, i in LLAMA70B_SHAPES:
-            for (M, B), Ts in (((1, 16), (1, 4, 16)), ((2, 16), (1,))):
+            for (M, B), Ts in (((1, 16), (1, 4, 16)), ((2, 16), (1,)), ((2, 8), (1,))):
                 for T in Ts:
                     r = bench_gemv(ac, LayerSpec(o, i, M, B), T, 3, 2, l2, n_launch=64)
                     detail[f"llama2-70b {name} {o}x{i} {M}x{B} T{T}"] = _gemv_detail(
-                        r, peaks, T=T, row_tokens=ac.gemv_row_tokens(ac.Shape(o, i, 8, M, B)))
+                        r, peaks, rate, T=T, row_tokens=ac.gemv_row_tokens(ac.Shape(o, i, 8, M, B)))
                     del r
                     torch.cuda.empty_cache()
         for M, B in ((1, 16), (2, 8)):
@@ -516,18 +593,21 @@ def run_gpu(args):
         for o, i in PREFILL_SHAPES:
             for M, B in ((1, 16), (2, 8)):
                 p = bench_prefill(ac, LayerSpec(o, i, M, B), 2048, reps=5, warmup=3)
-                detail[f"prefill {M}x{B} {o}x{i} T2048"] = {
+                key = f"prefill {M}x{B} {o}x{i} T2048"
+                detail[key] = {
                     "us_per_layer": round(p["us_total"], 2), "tflops": round(p["tflops"], 1),
                     "tensor_frac": round(p["tflops"] / peaks["bf16_tflops"], 4),
                     "us_dequant": round(p["us_dequant"], 2), "dequant_gbs": round(p["dequant_gbs"], 1),
                     "us_gemm": round(p["us_gemm"], 2), "gemm_tflops": round(p["gemm_tflops"], 1)}
+                if cpu_ok and (o, i) == PREFILL_SHAPES[0]:
+                    detail[key]["cpu_oracle"] = cpu_oracle_prefill(LayerSpec(o, i, M, B), 2048)
                 torch.cuda.empty_cache()
     e2e = e2e_gemv(ac, head, max(3, args.steps // 4), 2)
-    single_us = single_call_us(ac, head)
+    latency = call_latency(ac, head)
     sampler.__exit__(None, None, None)
     clocks = sampler.summary()
 
-    cpu = cpu_oracle_sample(HEADLINE, 1) if (rank == 0 and world == 1 and not args.quick) else None
+    cpu = cpu_oracle_sample(HEADLINE, 1) if cpu_ok else None
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(head["ms"] / args.steps, 4), "higher_is_better": True,
@@ -538,7 +618,9 @@ def run_gpu(args):
                    "l2_policy": "inputs larger than L2: each step cycles over copies totalling > 3x L2",
                    "parallelism": f"replicas x{world}"},
         "us_per_layer": round(head["us_per_layer"], 4),
-        "single_call_us": round(single_us, 3),
+        "single_call_us": latency["device_us"],
+        "single_call": latency,
+        "gather_rates": rate,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4),
                      "traffic": recorded_traffic("gemv 1x16 4096x4096 T1"),
@@ -547,7 +629,7 @@ def run_gpu(args):
                      "algorithmic_bytes_per_launch": head["bytes_per_layer"],
                      # the roofline that actually binds a batch-1 1x16 layer: one random 16-byte
                      # codeword gather from L2 per group
-                     "gather_bound": gather_roofline(HEADLINE, head["us_per_layer"])},
+                     "gather_bound": gather_roofline(HEADLINE, head["us_per_layer"], rate)},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": head["launches"],
@@ -561,35 +643,55 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
-# Random 16-byte gathers from an L2-resident 1-2 MiB table, measured on this
-# B200 with a microbenchmark (indices generated in registers): 304 G/s at 8
-# warps per SM and 315 G/s at 16 to 64, with 4, 8 or 16 gathers in flight per
-# thread alike -- about one 32-byte sector per SM clock.
-L2_GATHER_PEAK_G_PER_S = 315.0
 # fp32 FMA peak: 148 SMs x 128 FMA/clock x the 1965 MHz maximum clock.
 FMA_PEAK_TERA_PER_S = 148 * 128 * 1.965e9 / 1e12
 
 
-def gather_roofline(spec, us):
-    """Codeword gathers per second against the measured L2 gather rate (1x16 and
-    2x16 gather M codewords per group; 2x8 uses shared-memory tables instead)."""
-    if spec.B != 16:
-        return None
+def measure_gather_rates(ac, reps=5):
+    """Random 16-byte gathers per second, measured now on this GPU with the
+    library's probe (aqlm_probe_gather): from a 1 MiB table through the load
+    path of the 1x16 / 2x16 codeword gathers (L1 + L2 evict-last), and from an
+    8 KiB table in shared memory (the 2x8 kernels' path).  CUDA events on the
+    current stream around `reps` back-to-back launches after one warm-up."""
+    import torch
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(0)
+    table = torch.randint(-32768, 32767, (1 << 19,), dtype=torch.int16, device="cuda", generator=gen)   # 1 MiB
+    out = {}
+    for key, src, tab, cps in (("l2_1mib_g_per_s", 0, table, 8), ("smem_8kib_g_per_s", 1, table[:4096], 4)):
+        n, sink = ac.probe_gather(tab, src, ctas_per_sm=cps, iters=64)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            ac.probe_gather(tab, src, ctas_per_sm=cps, iters=64, sink=sink)
+        e1.record()
+        torch.cuda.synchronize()
+        out[key] = round(reps * n / (e0.elapsed_time(e1) * 1e-3) / 1e9, 1)
+    out["how"] = ("aqlm_probe_gather: 8 (L2) / 4 (shared memory) CTAs of 256 threads per SM, 8 random 16-byte "
+                  "reads in flight per thread, indices from a register LCG; G gathers/s over 5 launches")
+    return out
+
+
+def gather_roofline(spec, us, rate):
+    """Codeword gathers per second against the gather rate measured in this
+    run (1x16 and 2x16 gather M codewords per group from L2; 2x8 reads its
+    codewords from shared memory, reported against that rate)."""
     gathers = spec.d_out * spec.groups * spec.M
     achieved = gathers / (us * 1e-6) / 1e9
-    return {"achieved": round(achieved, 1), "peak": L2_GATHER_PEAK_G_PER_S, "unit": "G gathers/s",
-            "frac": round(achieved / L2_GATHER_PEAK_G_PER_S, 4),
-            "peak_source": "random 16-byte gather microbenchmark on this B200"}
+    peak = rate["l2_1mib_g_per_s"] if spec.B == 16 else rate["smem_8kib_g_per_s"]
+    return {"achieved": round(achieved, 1), "peak": peak, "unit": "G gathers/s",
+            "frac": round(achieved / peak, 4),
+            "peak_source": "aqlm_probe_gather in this run (" + ("1 MiB table via L1/L2" if spec.B == 16
+                                                                else "8 KiB table in shared memory") + ")"}
 
 
-def _gemv_detail(r, peaks, T=1, row_tokens=None):
+def _gemv_detail(r, peaks, rate, T=1, row_tokens=None):
     gbs = r["bytes_per_layer"] / (r["us_per_layer"] * 1e-6) / 1e9
     spec = r["layers"].spec
     out = {"us_per_layer": round(r["us_per_layer"], 3), "gbs": round(gbs, 1),
            "hbm_frac": round(gbs / peaks["hbm_gbs"], 4)}
-    gr = gather_roofline(spec, r["us_per_layer"])
-    if gr is not None:
-        out["gather_frac"] = gr["frac"]
+    out["gather_frac"] = gather_roofline(spec, r["us_per_layer"], rate)["frac"]
     if T > 1:
         # multiply-adds of the product per second; up to the format's row-kernel
         # token count (aqlm_gemv_row_tokens) they run on the CUDA cores (fraction

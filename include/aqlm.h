@@ -282,17 +282,18 @@ AQLM_API aqlm_status aqlm_test_gemm_timeout(const uint16_t *X, const uint16_t *W
  *
  * The scratch it needs lives in a fixed array inside the library, 8 MiB per
  * GPU (aqlm_gemv_noalloc_max_scratch_bytes()), held by every GPU that loads
- * the library until the process exits.  A shape and token count whose
- * scratch (aqlm_gemv_workspace_bytes) exceeds that is rejected with
- * AQLM_ERR_WORKSPACE.  Arguments are checked as aqlm_gemv checks them before
- * anything is enqueued.  The first call on a device looks up the array's
+ * the library until the process exits.  Arguments are checked as aqlm_gemv
+ * checks them before anything is enqueued.  The first call on a device looks
+ * up the array's
  * device address there (cudaGetSymbolAddress); make that first call before
  * any stream capture (a lookup that fails is not kept: the next call tries
  * again).  Each call clears the array's arrival counters on `stream`; the
- * status word is left alone, so a bounded wait that gave up (4 tokens and
- * more, see aqlm_gemv) stays recorded until aqlm_gemv_noalloc_check reads
- * it -- check before the next call of another shape or token count, whose
- * layout may reuse that word's bytes.  All calls on a device share the one
+ * status word (the array's last 16 bytes, which no call's other data ever
+ * reaches) is left alone, so a bounded wait that gave up (4 tokens and more,
+ * see aqlm_gemv) stays recorded, whatever calls follow, until
+ * aqlm_gemv_noalloc_check reads it.  A shape and token count whose scratch
+ * exceeds the array (less those 16 bytes where the path has no status word)
+ * is rejected with AQLM_ERR_WORKSPACE.  All calls on a device share the one
  * array and it keeps the last call's contents: calls that overlap on the GPU
  * (other streams, other host threads) race and must be avoided.  No
  * cudaMalloc, cudaFree or other allocating routine is called.  Results and
@@ -306,18 +307,15 @@ AQLM_API aqlm_status aqlm_gemv_noalloc(const void *codes, const uint16_t *codebo
 AQLM_API size_t aqlm_gemv_noalloc_max_scratch_bytes(void);
 
 /* aqlm_gemv_check for aqlm_gemv_noalloc: synchronise `stream`, then read and
- * clear the status word that the last aqlm_gemv_noalloc call of this shape
- * and token count left in the built-in array: AQLM_OK, or AQLM_ERR_TIMEOUT
- * (y of that call is then not valid).  Paths without device waits: AQLM_OK
- * after the synchronisation.  No counterpart on the pages. */
-AQLM_API aqlm_status aqlm_gemv_noalloc_check(aqlm_shape shape, int32_t tokens, aqlm_stream_t stream);
+ * clear the status word of the current device's built-in array: AQLM_OK, or
+ * AQLM_ERR_TIMEOUT if a bounded wait of any aqlm_gemv_noalloc call since the
+ * last check gave up (that call's y is not valid).  No counterpart on the
+ * pages. */
+AQLM_API aqlm_status aqlm_gemv_noalloc_check(aqlm_stream_t stream);
 
-/* Test only: write `value` into the status word of (shape, tokens)'s layout
- * in aqlm_gemv_noalloc's array and synchronise (AQLM_ERR_UNSUPPORTED where
- * that path has no status word), so that tests can check the reporting
- * without making a device wait run out. */
-AQLM_API aqlm_status aqlm_test_gemv_noalloc_set_status(aqlm_shape shape, int32_t tokens, int32_t value,
-                                                       aqlm_stream_t stream);
+/* Test only: write `value` into that status word and synchronise, so that
+ * tests can check the reporting without making a device wait run out. */
+AQLM_API aqlm_status aqlm_test_gemv_noalloc_set_status(int32_t value, aqlm_stream_t stream);
 
 /* ===========================================================================
  * Encoding: scales, codebooks and codes of a layer from its weights.
@@ -398,6 +396,27 @@ AQLM_API size_t aqlm_encode_layer_workspace_bytes(aqlm_shape shape);
 AQLM_API aqlm_status aqlm_encode_layer(const float *W, aqlm_shape shape, const int32_t *init_idx, int32_t iters,
                                        void *codes, uint16_t *codebooks, uint16_t *scales, void *workspace,
                                        size_t workspace_bytes, aqlm_stream_t stream);
+
+/* ===========================================================================
+ * Measurement: the random 16-byte gather rate.
+ *
+ * Not part of the method.  At one token a decode product gathers one random
+ * 16-byte codeword per group and codebook ("The AQLM Quantization Algorithm,
+ * Explained", section "Key AQLM quantization parameters": more codewords make
+ * decoding slower); aqlm_probe_gather launches ctas_per_sm (1..8) CTAs of
+ * 256 threads per SM that each make `iters` x 8 random 16-byte reads of
+ * `table` (table_bytes, a multiple of 16), through the load the 1x16 / 2x16
+ * decode kernels use for codewords (L1 evict-last, L2 evict-last; source 0)
+ * or from a copy of the table in shared memory (source 1, table_bytes <=
+ * 64 KiB; the 2x8 kernels' path).  *gathers (host) receives the number of
+ * reads the launch makes; time it with events on `stream`.  `sink` (device,
+ * aqlm_probe_gather_sink_bytes(ctas_per_sm) bytes, 16-byte aligned) receives
+ * one word per thread so the reads are not optimised away.
+ * ======================================================================== */
+AQLM_API size_t aqlm_probe_gather_sink_bytes(int32_t ctas_per_sm);
+AQLM_API aqlm_status aqlm_probe_gather(const void *table, size_t table_bytes, int32_t source, int32_t ctas_per_sm,
+                                       int32_t iters, void *sink, size_t sink_bytes, uint64_t *gathers,
+                                       aqlm_stream_t stream);
 
 /* A static, human-readable name of a status code. */
 AQLM_API const char *aqlm_status_string(aqlm_status status);

@@ -59,7 +59,7 @@ def test_noalloc_matches_oracle_and_gemv_on_two_calls(cuda_device, d_out, d_in, 
     for _ in range(2):
         y = torch.full((T, d_out), float("nan"), dtype=torch.float16, device=DEV)
         assert _call_noalloc(lib, d, d["x"], y) == ac.AQLM_OK
-        assert lib.aqlm_gemv_noalloc_check(shape, T, _stream()) == ac.AQLM_OK
+        assert lib.aqlm_gemv_noalloc_check(_stream()) == ac.AQLM_OK
         y = y.cpu().numpy()
         check_fp_output(y, y_ref.T, W, x64, out_rel=2.0 ** -10, acc_rel=2.0 ** -14)
         assert np.array_equal(y.view(np.uint16), y_gemv.view(np.uint16))
@@ -67,30 +67,24 @@ def test_noalloc_matches_oracle_and_gemv_on_two_calls(cuda_device, d_out, d_in, 
 
 def test_noalloc_status_survives_until_checked(cuda_device):
     """A status word set in the built-in array (as a bounded wait that gave up
-    would set it) is reported by aqlm_gemv_noalloc_check even after another
-    call of the same shape, then cleared."""
+    would set it) is reported by aqlm_gemv_noalloc_check even after further
+    calls of other shapes and token counts, then cleared; a call rejected for
+    its arguments enqueues nothing."""
     lib = ac.load_library()
-    d_out, d_in, M, B, T = CASES[2]
-    spec = LayerSpec(d_out, d_in, M, B)
-    L = make_layer(spec, seed=5, tokens=T)
-    d = to_dev(L)
-    shape = ac.shape_of(d["codes"])
-    y = torch.empty((T, d_out), dtype=torch.float16, device=DEV)
-    assert _call_noalloc(lib, d, d["x"], y) == ac.AQLM_OK
-    assert lib.aqlm_gemv_noalloc_check(shape, T, _stream()) == ac.AQLM_OK
-    assert lib.aqlm_test_gemv_noalloc_set_status(shape, T, ac.AQLM_ERR_TIMEOUT, _stream()) == ac.AQLM_OK
-    assert _call_noalloc(lib, d, d["x"], y) == ac.AQLM_OK
-    assert lib.aqlm_gemv_noalloc_check(shape, T, _stream()) == ac.AQLM_ERR_TIMEOUT
-    assert lib.aqlm_gemv_noalloc_check(shape, T, _stream()) == ac.AQLM_OK
-    # the row-kernel path has no status word
-    row = ac.Shape(1024, 28672, 8, 2, 8)
-    assert lib.aqlm_test_gemv_noalloc_set_status(row, 3, 1, _stream()) == ac.AQLM_ERR_UNSUPPORTED
-    assert lib.aqlm_gemv_noalloc_check(row, 3, _stream()) == ac.AQLM_OK
+    assert lib.aqlm_gemv_noalloc_check(_stream()) == ac.AQLM_OK
+    assert lib.aqlm_test_gemv_noalloc_set_status(ac.AQLM_ERR_TIMEOUT, _stream()) == ac.AQLM_OK
+    for d_out, d_in, M, B, T in CASES:
+        L = make_layer(LayerSpec(d_out, d_in, M, B), seed=5, tokens=T)
+        d = to_dev(L)
+        y = torch.empty((T, d_out), dtype=torch.float16, device=DEV)
+        assert _call_noalloc(lib, d, d["x"], y) == ac.AQLM_OK
+    assert lib.aqlm_gemv_noalloc_check(_stream()) == ac.AQLM_ERR_TIMEOUT
+    assert lib.aqlm_gemv_noalloc_check(_stream()) == ac.AQLM_OK
 
 
-def test_noalloc_checks_arguments_before_touching_the_array(cuda_device):
-    """A call rejected for its arguments enqueues nothing: a recorded status
-    stays, and sizes beyond the array are rejected with AQLM_ERR_WORKSPACE."""
+def test_noalloc_checks_arguments_first(cuda_device):
+    """Bad pointers and sizes beyond the array are rejected before anything is
+    enqueued (AQLM_ERR_INVALID_ARG, _MISALIGNED, _WORKSPACE)."""
     lib = ac.load_library()
     d_out, d_in, M, B, T = CASES[2]
     shape = ac.Shape(d_out, d_in, 8, M, B)
@@ -98,13 +92,11 @@ def test_noalloc_checks_arguments_before_touching_the_array(cuda_device):
     y = torch.zeros((T, d_out), dtype=torch.float16, device=DEV)
     codes = torch.zeros(16, dtype=torch.uint8, device=DEV)
     p = ctypes.c_void_p(codes.data_ptr())
-    assert lib.aqlm_test_gemv_noalloc_set_status(shape, T, ac.AQLM_ERR_TIMEOUT, _stream()) == ac.AQLM_OK
     st = lib.aqlm_gemv_noalloc(p, p, p, ctypes.c_void_p(x.data_ptr()), None, T, shape, _stream())
     assert st == ac.AQLM_ERR_INVALID_ARG
     st = lib.aqlm_gemv_noalloc(p, p, p, ctypes.c_void_p(x.data_ptr() + 2), ctypes.c_void_p(y.data_ptr()), T, shape,
                                _stream())
     assert st == ac.AQLM_ERR_MISALIGNED
-    assert lib.aqlm_gemv_noalloc_check(shape, T, _stream()) == ac.AQLM_ERR_TIMEOUT
     # 3 tokens of 28672 inputs on the row kernel (2x8): seven activation
     # slices, 7 x 3 x 131072 fp32 partial sums (11 MB), more than the 8 MiB
     # built in
@@ -113,3 +105,4 @@ def test_noalloc_checks_arguments_before_touching_the_array(cuda_device):
     st = lib.aqlm_gemv_noalloc(p, p, p, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()), 3, big,
                                _stream())
     assert st == ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_gemv_noalloc_check(_stream()) == ac.AQLM_OK
