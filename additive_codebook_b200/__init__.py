@@ -35,7 +35,7 @@ EXPORTS = ["aqlm_gemv", "aqlm_gemv_workspace_bytes", "aqlm_gemv_row_tokens", "aq
            "aqlm_gemm_workspace_bytes", "aqlm_gemm_check", "aqlm_bf16_gemm", "aqlm_bf16_gemm_tile_n", "aqlm_decode_indices",
            "aqlm_test_gemm_timeout", "aqlm_gemv_noalloc", "aqlm_gemv_noalloc_max_scratch_bytes",
            "aqlm_gemv_noalloc_check", "aqlm_test_gemv_noalloc_set_status", "aqlm_probe_gather_sink_bytes",
-           "aqlm_probe_gather",
+           "aqlm_probe_gather", "aqlm_gemv_lut", "aqlm_gemv_lut_workspace_bytes",
            "aqlm_status_string", "aqlm_version",
            "aqlm_encode_scales", "aqlm_nearest_workspace_bytes", "aqlm_nearest_codeword",
            "aqlm_kmeans_workspace_bytes", "aqlm_kmeans_update", "aqlm_residual_kmeans_workspace_bytes",
@@ -97,6 +97,8 @@ def load_library():
         "aqlm_gemv_noalloc_check": ([vp], st),
         "aqlm_test_gemv_noalloc_set_status": ([i32, vp], st),
         "aqlm_probe_gather_sink_bytes": ([i32], sz),
+        "aqlm_gemv_lut": ([vp, vp, vp, vp, vp, Shape, vp, sz, vp], st),
+        "aqlm_gemv_lut_workspace_bytes": ([Shape], sz),
         "aqlm_probe_gather": ([vp, sz, i32, i32, i32, vp, sz, ctypes.POINTER(u64), vp], st),
         "aqlm_encode_scales": ([vp, i32, i32, vp, vp, vp], st),
         "aqlm_nearest_workspace_bytes": ([i64], sz),
@@ -214,6 +216,27 @@ def aqlm_gemv(codes, codebooks, scales, x, y=None, workspace=None, stream=None):
                          y.data_ptr(), T, shape, _p(workspace), wbytes, _stream(stream, dev if dev >= 0 else None)),
            "aqlm_gemv")
     return y
+
+
+def aqlm_gemv_lut(codes, codebooks, scales, x, y=None, workspace=None, stream=None):
+    """2x8, one token: y[1, d_out] = fp16(W^ . x) through per-slab lookup tables."""
+    lib = load_library()
+    shape = shape_of(codes)
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    if y is None:
+        y = torch.empty((1, shape.d_out), dtype=torch.float16, device=x.device)
+    need = lib.aqlm_gemv_lut_workspace_bytes(shape)
+    if need and workspace is None:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=x.device)
+    wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib.aqlm_gemv_lut(_p(codes), _p(codebooks), _p(_flat_scales(scales)), _p(x), _p(y), shape, _p(workspace),
+                             wbytes, _stream(stream)), "aqlm_gemv_lut")
+    return y
+
+
+def gemv_lut_workspace_bytes(shape):
+    return int(load_library().aqlm_gemv_lut_workspace_bytes(shape))
 
 
 def gemv_row_tokens(shape):

@@ -14,8 +14,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libaqlm_b200.so")
-SOURCES = ["abi.cu", "dequant.cu", "encode.cu", "gemv.cu", "gemm_tcgen05.cu", "gemv_noalloc.cu", "gemv_rows.cu",
-           "gemv_tc.cu", "probe.cu"]
+SOURCES = ["abi.cu", "dequant.cu", "encode.cu", "gemv.cu", "gemm_tcgen05.cu", "gemv_noalloc.cu", "gemv_lut.cu",
+           "gemv_rows.cu", "gemv_tc.cu", "probe.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -113,6 +113,28 @@ aqlm_status aqlm_gemv(const void *codes, const uint16_t *codebooks, const uint16
                                        to_cuda(stream)));
 }
 
+size_t aqlm_gemv_lut_workspace_bytes(aqlm_shape shape) {
+    if (check_shape(shape) != AQLM_OK || !aqlm::gemv_lut_supported(aqlm::make_dims(shape), 1)) return 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    return aqlm::gemv_lut_workspace_bytes(aqlm::make_dims(shape), aqlm::num_sms(dev));
+}
+
+aqlm_status aqlm_gemv_lut(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
+                          uint16_t *y, aqlm_shape shape, void *workspace, size_t workspace_bytes, aqlm_stream_t stream) {
+    const aqlm_status st = aqlm::check_gemv_args(codes, codebooks, scales, x, y, 1, shape);
+    if (st != AQLM_OK) return st;
+    const Dims d = aqlm::make_dims(shape);
+    if (!aqlm::gemv_lut_supported(d, 1)) return AQLM_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;   // the launch below then reports the error
+    const int sms = aqlm::num_sms(dev);
+    const size_t need = aqlm::gemv_lut_workspace_bytes(d, sms);
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16))) return AQLM_ERR_WORKSPACE;
+    return from_cuda(aqlm::launch_gemv_lut(codes, codebooks, scales, x, y, d, need > 0 ? workspace : nullptr, sms,
+                                           to_cuda(stream)));
+}
+
 int32_t aqlm_gemv_row_tokens(aqlm_shape shape) {
     if (check_shape(shape) != AQLM_OK) return 0;
     return aqlm::gemv_row_tokens(aqlm::make_dims(shape));

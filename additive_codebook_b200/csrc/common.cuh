@@ -236,6 +236,10 @@ size_t gemv_multi_counter_offset(const RowLayerIn *layers, int n, const Dims &d,
 long long gemv_multi_status_offset(const RowLayerIn *layers, int n, const Dims &d, int tokens);
 cudaError_t launch_gemv_multi(const RowLayerIn *layers, int n, const uint16_t *x, int tokens, const Dims &d,
                               void *workspace, cudaStream_t st);
+bool gemv_lut_supported(const Dims &d, int T);
+size_t gemv_lut_workspace_bytes(const Dims &d, int sms);
+cudaError_t launch_gemv_lut(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *x,
+                            uint16_t *y, const Dims &d, void *workspace, int sms, cudaStream_t st);
 cudaError_t launch_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                              int32_t *status, cudaStream_t st);
 int gemm_tile_n(int tokens, int n, int sms);

@@ -2,7 +2,10 @@
 // workspace layout.  Few tokens: gemv_rows.cu (coalesced row streaming on the
 // CUDA cores, the input range split when the activations do not fit on chip).
 // More tokens: gemv_tc.cu (the weights decoded into shared memory for tcgen05
-// tensor-core MMAs).  Both launch with programmatic dependent launch.
+// tensor-core MMAs).  Both launch with programmatic dependent launch.  The
+// lookup-table kernel of gemv_lut.cu (2x8, one token) has its own entry point,
+// aqlm_gemv_lut: measured on B200 it does not beat the row kernel, so
+// aqlm_gemv does not choose it.
 #include "common.cuh"
 
 namespace aqlm {

@@ -193,8 +193,9 @@ def copies_for(spec, T, l2_bytes, min_copies=2):
     return max(min_copies, int(np.ceil(3 * l2_bytes / per)))
 
 
-def gemv_graph(ac, layers, n_launch, ys, workspaces):
-    """Capture n_launch aqlm_gemv calls cycling over the copies in one graph."""
+def gemv_graph(ac, layers, n_launch, ys, workspaces, call=None):
+    """Capture n_launch aqlm_gemv (or `call`) calls cycling over the copies in one graph."""
+    call = call or ac.aqlm_gemv
     import torch
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
@@ -202,15 +203,13 @@ def gemv_graph(ac, layers, n_launch, ys, workspaces):
     with torch.cuda.stream(s):
         for i in range(min(n_launch, layers.R)):   # warm-up outside capture (sets kernel attributes)
             d = layers.copies[i]
-            ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], layers.x, y=ys[i % len(ys)],
-                         workspace=workspaces)
+            call(d["codes"], d["codebooks"], d["scales"], layers.x, y=ys[i % len(ys)], workspace=workspaces)
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
     with torch.cuda.graph(g, capture_error_mode="relaxed"):
         for i in range(n_launch):
             d = layers.copies[i % layers.R]
-            ac.aqlm_gemv(d["codes"], d["codebooks"], d["scales"], layers.x, y=ys[i % len(ys)],
-                         workspace=workspaces)
+            call(d["codes"], d["codebooks"], d["scales"], layers.x, y=ys[i % len(ys)], workspace=workspaces)
     return g
 
 
@@ -252,15 +251,18 @@ def whole_job_gbs(world, steps, launches_per_step, bytes_per_launch, max_ms):
     return world * steps * launches_per_step * bytes_per_launch / (max_ms * 1e-3) / 1e9
 
 
-def bench_gemv(ac, spec, T, steps, warmup, l2_bytes, n_launch=STEP_LAYERS, dist=None):
+def bench_gemv(ac, spec, T, steps, warmup, l2_bytes, n_launch=STEP_LAYERS, dist=None, lut=False):
+    """aqlm_gemv (lut=True: aqlm_gemv_lut, 2x8 one token) over R layer copies
+    larger than L2, n_launch launches per graph replay."""
     import torch
     R = copies_for(spec, T, l2_bytes)
     layers = Layers(spec, R, T)
     ys = [torch.empty((T, spec.d_out), dtype=torch.float16, device="cuda") for _ in range(4)]
-    need = ac.gemv_workspace_bytes(ac.shape_of(layers.copies[0]["codes"]), T)
+    shape = ac.shape_of(layers.copies[0]["codes"])
+    need = ac.gemv_lut_workspace_bytes(shape) if lut else ac.gemv_workspace_bytes(shape, T)
     ws = torch.zeros(need, dtype=torch.uint8, device="cuda") if need else None
     n_launch = max(n_launch, R)
-    g = gemv_graph(ac, layers, n_launch, ys, ws)
+    g = gemv_graph(ac, layers, n_launch, ys, ws, call=ac.aqlm_gemv_lut if lut else None)
     ms = time_replays(g, steps, warmup, dist)
     us_layer = ms * 1e3 / (steps * n_launch)
     del g
@@ -587,6 +589,16 @@ def run_gpu(args):
                         r, peaks, rate, T=T, row_tokens=ac.gemv_row_tokens(ac.Shape(o, i, 8, M, B)))
                     del r
                     torch.cuda.empty_cache()
+        # the lookup-table kernel (aqlm_gemv_lut), beside the row kernel's figures above
+        for o, i in ((4096, 4096), (8192, 8192), (28672, 8192), (8192, 28672)):
+            r = bench_gemv(ac, LayerSpec(o, i, 2, 8), 1, 3, 2, l2, n_launch=64 if o * i > 4096 * 4096 else 1024,
+                           lut=True)
+            det = _gemv_detail(r, peaks, rate)
+            det.pop("gather_frac", None)
+            det["lookups_g_per_s"] = round(o * (i // 8) * 2 / (r["us_per_layer"] * 1e-6) / 1e9, 1)
+            detail[f"2x8 lookup tables {o}x{i} T1"] = det
+            del r
+            torch.cuda.empty_cache()
         for M, B in ((1, 16), (2, 8)):
             detail[f"encode codes {M}x{B} 4096x4096"] = bench_encode(ac, LayerSpec(4096, 4096, M, B))
             torch.cuda.empty_cache()
@@ -744,6 +756,7 @@ PROFILE_CASES = {
     # name: (kind, d_out, d_in, M, B, tokens)
     "gemv-1x16-4096": ("gemv", 4096, 4096, 1, 16, 1),
     "gemv-2x8-4096": ("gemv", 4096, 4096, 2, 8, 1),
+    "gemv-2x8-28672x8192": ("gemv", 28672, 8192, 2, 8, 1),
     "gemv-1x16-8192-t16": ("gemv", 8192, 8192, 1, 16, 16),
     "gemv-1x16-8192-t4": ("gemv", 8192, 8192, 1, 16, 4),
     "gemv-1x16-28672x8192-t4": ("gemv", 28672, 8192, 1, 16, 4),

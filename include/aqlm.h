@@ -143,6 +143,31 @@ AQLM_API size_t aqlm_gemv_workspace_bytes(aqlm_shape shape, int32_t tokens);
 AQLM_API int32_t aqlm_gemv_row_tokens(aqlm_shape shape);
 
 /*
+ * aqlm_gemv_lut -- the 2x8 decode product for one token through lookup
+ * tables: y = W^ . x computed as y_i = s_i * sum_j (L_0[j][b(i,j,0)] +
+ * L_1[j][b(i,j,1)]) with L_m[j][k] = <C_m[k], x_j>, which equals the product
+ * of section "What is Multi-Codebook Quantization (MCQ)?" because it is
+ * linear in the codewords.  Each table entry is an fp32 sum of eight exact
+ * fp16 products, each row the fp32 sum of its entries in a fixed order, y
+ * rounded once to fp16: reproducible bit for bit, within the stated tolerance
+ * of the exact product (not bit-identical to aqlm_gemv, whose summation order
+ * differs).  Only shape 2x8 (else AQLM_ERR_UNSUPPORTED); x [1][d_in], y
+ * [1][d_out]; workspace as aqlm_gemv's (size from
+ * aqlm_gemv_lut_workspace_bytes, zero-filled before its first use, left ready
+ * for the next call; calls sharing one must not overlap).  Launch with
+ * programmatic dependent launch as aqlm_gemv; no device waits.  aqlm_gemv
+ * does not use this kernel: on B200 it measured slower than the row kernel
+ * at every tested shape.
+ */
+AQLM_API aqlm_status aqlm_gemv_lut(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                                   const uint16_t *x, uint16_t *y, aqlm_shape shape, void *workspace,
+                                   size_t workspace_bytes, aqlm_stream_t stream);
+
+/* Bytes of workspace aqlm_gemv_lut needs on the current device (0 if none,
+ * or for a shape it does not take). */
+AQLM_API size_t aqlm_gemv_lut_workspace_bytes(aqlm_shape shape);
+
+/*
  * aqlm_gemv_multi -- the products y_l = W^_l . x of 1 to AQLM_MULTI_MAX_LAYERS
  * layers that read the SAME activations x, in one launch: e.g. the query, key
  * and value projections of an attention block, or the gate and up

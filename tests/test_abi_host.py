@@ -89,6 +89,16 @@ def test_gemv_workspace_rules():
     assert lib.aqlm_gemv_workspace_bytes(big, 1) == 0          # enough row tiles: no split
     assert lib.aqlm_gemv_workspace_bytes(shape(M=1, B=16), 1) == 0   # one token: whole rows per warp
     assert lib.aqlm_gemv_workspace_bytes(shape(), 1) == 0      # 2x8, one token: 2 KiB of activations
+    # aqlm_gemv_lut keeps one fp32 sum per row and group of slabs that a CTA
+    # covers (plus a counter per row range); a 4096x4096 layer takes one slab
+    # of 32 groups per CTA (16 sums per row); rows of one slab need none
+    assert lib.aqlm_gemv_lut_workspace_bytes(shape(d_out=4096, d_in=4096)) >= 16 * 4096 * 4
+    assert lib.aqlm_gemv_lut_workspace_bytes(shape(d_in=256)) == 0
+    assert lib.aqlm_gemv_lut_workspace_bytes(shape(M=1, B=16)) == 0
+    assert lib.aqlm_gemv_lut(A16, B16, C16, D16, E16, shape(M=1, B=16), NULL, 0, NULL) == ac.AQLM_ERR_UNSUPPORTED
+    assert lib.aqlm_gemv_lut(A16, B16, C16, D16, E16, shape(d_out=4096, d_in=4096), NULL, 0, NULL) == \
+        ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_gemv_lut(NULL, B16, C16, D16, E16, shape(), NULL, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
     wide = shape(d_in=4096)                                    # 8 tokens, 2 row tiles: split to fill the SMs
     assert lib.aqlm_gemv_workspace_bytes(shape(d_in=4096, M=1, B=16), 2) == 0   # 16 KiB of activations: one slice
     small = lib.aqlm_gemv_workspace_bytes(wide, 8)

@@ -122,6 +122,42 @@ def test_gemv_rows_split_input_range(M, B, T, d_in):
     _gemv_case(M, B, 100, d_in, T, seed=30 + T)
 
 
+LUT_SHAPES = [(1, 64), (17, 192), (300, 1600), (4100, 2560), (33, 65536), (4096, 4096), (2000, 28672), (28672, 8192)]
+
+
+@pytest.mark.parametrize("d_out,d_in", LUT_SHAPES)
+def test_gemv_lut_shapes(d_out, d_in):
+    # aqlm_gemv_lut (2x8, one token; slabs of 32 groups, rows in batches of 16
+    # per warp, chunks of 256 rows): last slabs of 8, 24, 8, 0 and 0 groups,
+    # row ranges that are not multiples of 16, a single row, 256 slabs (more
+    # than SMs), several slabs per CTA (28672 inputs; 28672 rows); each output
+    # also bit-identical on a second call through the same workspace
+    spec = LayerSpec(d_out, d_in, 2, 8)
+    L = make_layer(spec, seed=80 + d_out, tokens=1)
+    d = to_dev(L)
+    ws = torch.zeros(max(16, ac.gemv_lut_workspace_bytes(ac.shape_of(d["codes"]))), dtype=torch.uint8, device=DEV)
+    y = ac.aqlm_gemv_lut(d["codes"], d["codebooks"], d["scales"], d["x"], workspace=ws)
+    y2 = ac.aqlm_gemv_lut(d["codes"], d["codebooks"], d["scales"], d["x"], workspace=ws)
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+    rows = np.arange(d_out)
+    if d_out > 4096:      # sampled rows, computed one by one by the oracle
+        rng = np.random.Generator(np.random.PCG64(7))
+        rows = np.unique(np.concatenate([rng.choice(d_out, 512, replace=False), [0, d_out - 1]]))
+    codes = np.ascontiguousarray(L["codes"][rows])
+    sc = np.ascontiguousarray(L["scales"][rows])
+    y_ref = oracle.gemv_f64(codes, L["codebooks"], sc, L["x"], len(rows), d_in, 8, 2, 8)
+    W = oracle.dequant_f64(codes, L["codebooks"], sc, len(rows), d_in, 8, 2, 8)
+    check_fp_output(y.cpu().numpy()[:, rows], y_ref, W, L["x"].astype(np.float64), out_rel=2.0 ** -10,
+                    acc_rel=2.0 ** -14)
+
+
+def test_gemv_lut_rejects_other_formats():
+    for M, B in ((1, 16), (2, 16)):
+        d = to_dev(make_layer(LayerSpec(64, 512, M, B), seed=1, tokens=1))
+        with pytest.raises(ac.AqlmError):
+            ac.aqlm_gemv_lut(d["codes"], d["codebooks"], d["scales"], d["x"])
+
+
 @pytest.mark.parametrize("T", [4, 5, 16])
 def test_gemv_tensor_core_ragged_stage(T):
     # 2x16 with 516 groups: the last 8-group stage of the tensor-core path holds
