@@ -31,7 +31,7 @@
 //              after the last stage they are the epilogue (tcgen05.ld of their
 //              TMEM lane quarter, scale, fp16 store or fp32 partials);
 //   warp 4     one thread issues the TMA loads: code tiles (64 bytes x 128
-//              rows, two slots) and the activation tiles of every stage (64
+//              rows in the 64-byte swizzle, two slots) and the activation tiles of every stage (64
 //              inputs x 16 tokens, tokens past T read as zeros);
 //   warp 5     allocates 32 TMEM columns; one thread issues
 //              tcgen05.mma.cta_group::1.kind::f16 (M = 128, N = 16, K = 16)
@@ -474,12 +474,17 @@ __global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm)
                     ok = false;
                     break;
                 }
+                // the code tile arrives in the 64-byte swizzle: 16-byte piece c of row r
+                // sits at piece c ^ ((r >> 1) & 3), so the 8 rows of a quarter warp read
+                // 8 different bank quads (unswizzled, rows 64 bytes apart hit only
+                // quads 0 and 4: four-way conflicts)
                 uint4 code[kCodeVecs];
-                const uint4 *src = reinterpret_cast<const uint4 *>(codes_s + (size_t)slot * kTcRows * kCodeBoxBytes +
-                                                                   (size_t)r * kCodeBoxBytes +
-                                                                   (size_t)(l % SPB) * F::kStageCodeBytes);
+                const uint8_t *rowp = codes_s + (size_t)slot * kTcRows * kCodeBoxBytes + (size_t)r * kCodeBoxBytes;
 #pragma unroll
-                for (int v = 0; v < kCodeVecs; ++v) code[v] = src[v];
+                for (int v = 0; v < kCodeVecs; ++v) {
+                    const int piece = (l % SPB) * kCodeVecs + v;
+                    code[v] = *reinterpret_cast<const uint4 *>(rowp + ((piece ^ ((r >> 1) & 3)) << 4));
+                }
                 // the stage's A tiles are free once the MMAs of its previous use are done
                 const int gi = gi0 + l, s = gi % F::kStages;
                 if (!tc_wait(saddr(&bars->empty[s]), (uint32_t)(((gi / F::kStages) & 1) ^ 1), bars, a.status)) {
@@ -674,7 +679,7 @@ cudaError_t launch_tc_layers(const RowLayerIn *layers, int n, const uint16_t *x,
     for (int l = 0; l < n; ++l) {
         if (!encode_2d(&mc.m[l], CU_TENSOR_MAP_DATA_TYPE_UINT8, layers[l].codes, (uint64_t)d.row_bytes,
                        (uint64_t)layers[l].d_out, (uint64_t)d.row_bytes, kCodeBoxBytes, kTcRows,
-                       CU_TENSOR_MAP_SWIZZLE_NONE))
+                       CU_TENSOR_MAP_SWIZZLE_64B))
             return cudaErrorInvalidValue;
         TcLayer &L = a.layer[l];
         L.codebooks = reinterpret_cast<const uint4 *>(layers[l].codebooks);
