@@ -35,7 +35,8 @@ EXPORTS = ["aqlm_gemv", "aqlm_gemv_workspace_bytes", "aqlm_gemv_row_tokens", "aq
            "aqlm_gemm_workspace_bytes", "aqlm_gemm_check", "aqlm_bf16_gemm", "aqlm_bf16_gemm_tile_n", "aqlm_decode_indices",
            "aqlm_test_gemm_timeout", "aqlm_gemv_noalloc", "aqlm_gemv_noalloc_max_scratch_bytes",
            "aqlm_gemv_noalloc_check", "aqlm_test_gemv_noalloc_set_status", "aqlm_probe_gather_sink_bytes",
-           "aqlm_probe_gather", "aqlm_gemv_lut", "aqlm_gemv_lut_workspace_bytes",
+           "aqlm_probe_gather", "aqlm_gemv_lut", "aqlm_gemv_lut_workspace_bytes", "aqlm_gemm_fused",
+           "aqlm_gemm_fused_workspace_bytes",
            "aqlm_status_string", "aqlm_version",
            "aqlm_encode_scales", "aqlm_nearest_workspace_bytes", "aqlm_nearest_codeword",
            "aqlm_kmeans_workspace_bytes", "aqlm_kmeans_update", "aqlm_residual_kmeans_workspace_bytes",
@@ -99,6 +100,8 @@ def load_library():
         "aqlm_probe_gather_sink_bytes": ([i32], sz),
         "aqlm_gemv_lut": ([vp, vp, vp, vp, vp, Shape, vp, sz, vp], st),
         "aqlm_gemv_lut_workspace_bytes": ([Shape], sz),
+        "aqlm_gemm_fused": ([vp, vp, vp, vp, vp, i32, Shape, vp, sz, vp], st),
+        "aqlm_gemm_fused_workspace_bytes": ([Shape, i32], sz),
         "aqlm_probe_gather": ([vp, sz, i32, i32, i32, vp, sz, ctypes.POINTER(u64), vp], st),
         "aqlm_encode_scales": ([vp, i32, i32, vp, vp, vp], st),
         "aqlm_nearest_workspace_bytes": ([i64], sz),
@@ -351,6 +354,20 @@ def aqlm_gemm(codes, codebooks, scales, X, Y=None, workspace=None, stream=None):
         workspace = torch.empty(lib.aqlm_gemm_workspace_bytes(shape, T), dtype=torch.uint8, device=X.device)
     _check(lib.aqlm_gemm(_p(codes), _p(codebooks), _p(_flat_scales(scales)), _p(X), _p(Y), T, shape,
                          _p(workspace), workspace.numel(), _stream(stream)), "aqlm_gemm")
+    return Y, workspace
+
+
+def aqlm_gemm_fused(codes, codebooks, scales, X, Y=None, workspace=None, stream=None):
+    """Y[T, d_out] = bf16(X . W^T) with the dequantisation inside the GEMM (no W^ buffer)."""
+    lib = load_library()
+    shape = shape_of(codes)
+    T = X.shape[0]
+    if Y is None:
+        Y = torch.empty((T, shape.d_out), dtype=torch.bfloat16, device=X.device)
+    if workspace is None:
+        workspace = torch.empty(lib.aqlm_gemm_fused_workspace_bytes(shape, T), dtype=torch.uint8, device=X.device)
+    _check(lib.aqlm_gemm_fused(_p(codes), _p(codebooks), _p(_flat_scales(scales)), _p(X), _p(Y), T, shape,
+                               _p(workspace), workspace.numel(), _stream(stream)), "aqlm_gemm_fused")
     return Y, workspace
 
 

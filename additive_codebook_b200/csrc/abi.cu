@@ -8,6 +8,9 @@
 namespace aqlm {
 cudaError_t launch_bf16_gemm_ex(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                                 int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test);
+cudaError_t launch_fused_gemm(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                              const uint16_t *X, uint16_t *Y, int tokens, const Dims &d, int32_t *status,
+                              cudaStream_t st);
 }
 
 namespace {
@@ -232,6 +235,27 @@ aqlm_status aqlm_gemm(const void *codes, const uint16_t *codebooks, const uint16
     e = aqlm::launch_dequant(codes, codebooks, scales, W, aqlm::make_dims(shape), cs);
     if (e != cudaSuccess) return AQLM_ERR_CUDA;
     return from_cuda(aqlm::launch_bf16_gemm(X, W, Y, tokens, shape.d_out, shape.d_in, status, cs));
+}
+
+size_t aqlm_gemm_fused_workspace_bytes(aqlm_shape shape, int32_t tokens) {
+    if (check_shape(shape) != AQLM_OK || tokens < 1) return 0;
+    return kStatusBytes;
+}
+
+aqlm_status aqlm_gemm_fused(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *X,
+                            uint16_t *Y, int32_t tokens, aqlm_shape shape, void *workspace, size_t workspace_bytes,
+                            aqlm_stream_t stream) {
+    aqlm_status st = check_layer(codes, codebooks, scales, shape);
+    if (st != AQLM_OK) return st;
+    if (!X || !Y || tokens < 1) return AQLM_ERR_INVALID_ARG;
+    if (shape.d_out % 8) return AQLM_ERR_UNSUPPORTED;
+    if (!aligned(X, 16) || !aligned(Y, 16)) return AQLM_ERR_MISALIGNED;
+    if (!workspace || workspace_bytes < kStatusBytes || !aligned(workspace, 16)) return AQLM_ERR_WORKSPACE;
+    const cudaStream_t cs = to_cuda(stream);
+    int32_t *status = static_cast<int32_t *>(workspace);
+    if (cudaMemsetAsync(status, 0, sizeof(int32_t), cs) != cudaSuccess) return AQLM_ERR_CUDA;
+    return from_cuda(
+        aqlm::launch_fused_gemm(codes, codebooks, scales, X, Y, tokens, aqlm::make_dims(shape), status, cs));
 }
 
 aqlm_status aqlm_gemm_check(void *workspace, size_t workspace_bytes, aqlm_stream_t stream) {

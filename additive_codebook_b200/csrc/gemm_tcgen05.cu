@@ -56,12 +56,15 @@ struct Bars {
     int abort_flag;
 };
 
-template <int BN>
+// RESERVE: shared memory the fused decoders keep for their codebook copies.
+template <int BN, int RESERVE = 0>
 struct GemmCfg {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M = 128");
     static constexpr int B_BYTES = BN * BK * 2;                // a multiple of 1024: stages stay aligned
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES = (200 * 1024) / STAGE_BYTES < kMaxStages ? (200 * 1024) / STAGE_BYTES : kMaxStages;
+    // the ring gets 200 KiB; a fused kernel with codebook copies 220 KiB less the copies
+    static constexpr int BUDGET = RESERVE ? 220 * 1024 - RESERVE : 200 * 1024;
+    static constexpr int STAGES = BUDGET / STAGE_BYTES < kMaxStages ? BUDGET / STAGE_BYTES : kMaxStages;
     // each accumulator at a power-of-two column offset; the allocation is a power of two
     static constexpr int ACC_STRIDE = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
     static constexpr uint32_t TMEM_COLS = 2 * ACC_STRIDE;
@@ -70,9 +73,36 @@ struct GemmCfg {
     // at bits 17-22, M >> 4 at bits 24-28).
     static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                       ((uint32_t)(BM >> 4) << 24);
-    static constexpr size_t SMEM = 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + sizeof(Bars);
+    static constexpr size_t SMEM = 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + sizeof(Bars) + 16 + RESERVE;
     static_assert(B_BYTES % 1024 == 0 && STAGES >= 2, "ring layout");
 };
+
+// ---- fused dequantisation: the B tiles decoded in shared memory -------------
+// With FM > 0 (the codebook count of the layer, FB its code bits) the kernel
+// reads no W^: eight more warps decode each stage's B tile -- BN rows of W^ x
+// 64 inputs -- from the codes, codebooks and scales, with the binary32 steps
+// of aqlm_dequant (codewords added in codebook order, times the row's scale,
+// rounded to bf16), straight into the 128-byte-swizzled K-major layout the
+// MMA reads, then order their stores before the tensor cores' reads (proxy
+// fence) and arrive on the stage's full barrier, which the X tile's TMA bytes
+// complete.  Every CTA decodes the W^ rows of its own tiles; a row block is
+// decoded once per 128-token tile that uses it, and nothing is written to or
+// read from a W^ buffer in global memory.
+constexpr int kDecWarps = 8;
+constexpr int kDecThreads = 32 * kDecWarps;
+constexpr int kCbCopies = 8;   // 2x8: the codebooks in shared memory, copy p in bank quad p
+
+struct DecodeArgs {
+    const uint8_t *codes;      // [d_out][G][M]
+    const uint4 *codebooks;    // [M][2^B] codewords of 8 fp16
+    const __half *scales;      // [d_out]
+    int G, row_bytes;
+};
+
+template <int FM, int FB>
+constexpr int decode_reserve() {
+    return (FM > 0 && FB == 8) ? FM * 256 * 16 * kCbCopies : 0;
+}
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -191,18 +221,39 @@ __device__ __forceinline__ void store_bf16_row(__nv_bfloat16 *dst, const uint32_
     }
 }
 
-template <int BN>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+// Code index of codebook m of group q (0..7) of a stage from a row's code bytes.
+template <int FM, int FB, int V>
+__device__ __forceinline__ uint32_t stage_code(const uint4 (&c)[V], int q, int m) {
+    if constexpr (FM == 1) {
+        const uint32_t w[4] = {c[0].x, c[0].y, c[0].z, c[0].w};
+        return (w[q >> 1] >> (16 * (q & 1))) & 0xffffu;
+    } else if constexpr (FB == 8) {  // byte 0 codebook 0, byte 1 codebook 1
+        const uint32_t w[4] = {c[0].x, c[0].y, c[0].z, c[0].w};
+        return (w[q >> 1] >> (16 * (q & 1) + 8 * m)) & 0xffu;
+    } else {  // 2x16: 4 bytes per group, codebook 0 in the low half
+        const uint32_t w[8] = {c[0].x, c[0].y, c[0].z, c[0].w, c[V - 1].x, c[V - 1].y, c[V - 1].z, c[V - 1].w};
+        return (w[q] >> (16 * m)) & 0xffffu;
+    }
+}
+
+template <int BN, int FM, int FB>
+__global__ void __launch_bounds__(kGemmThreads + (FM > 0 ? kDecThreads : 0), 1)
 gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                   __nv_bfloat16 *__restrict__ Y, int m_total, int n_total, int k_total, int32_t *status,
-                  unsigned long long limit_ns, int stall_test) {
-    using C = GemmCfg<BN>;
+                  unsigned long long limit_ns, int stall_test, const DecodeArgs da) {
+    constexpr int RESERVE = decode_reserve<FM, FB>();
+    using C = GemmCfg<BN, RESERVE>;
     constexpr int STAGES = C::STAGES, STAGE_BYTES = C::STAGE_BYTES;
+    constexpr bool kFused = FM > 0;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled tiles.
     const uint32_t raw = smem_addr(smem_raw);
     uint8_t *smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
     Bars *bars = reinterpret_cast<Bars *>(smem + (size_t)STAGES * STAGE_BYTES);
+    uint4 *cbs = reinterpret_cast<uint4 *>(smem + (size_t)STAGES * STAGE_BYTES + ((sizeof(Bars) + 15) & ~size_t(15)));
+    if constexpr (kFused && FB == 8) {  // 2x8 codebooks: kCbCopies copies, codeword e of copy p at word 8e + p
+        for (int i = threadIdx.x; i < FM * 256 * kCbCopies; i += blockDim.x) cbs[i] = da.codebooks[i >> 3];
+    }
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m_tiles = (m_total + BM - 1) / BM;
@@ -212,7 +263,8 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_addr(&bars->full[s]), 1);
+            // full: the X tile's TMA (one arrival with its bytes) and, fused, each decoder warp
+            mbar_init(smem_addr(&bars->full[s]), kFused ? 1 + kDecWarps : 1);
             mbar_init(smem_addr(&bars->empty[s]), 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -253,9 +305,9 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
                     }
                     const uint32_t full = smem_addr(&bars->full[stage]);
                     const uint32_t dst = smem_addr(smem + (size_t)stage * STAGE_BYTES);
-                    mbar_expect_tx(full, (uint32_t)STAGE_BYTES);
+                    mbar_expect_tx(full, (uint32_t)(kFused ? A_BYTES : STAGE_BYTES));
                     tma_load_2d(dst, &tmap_x, kb * BK, mb * BM, full);
-                    tma_load_2d(dst + A_BYTES, &tmap_w, kb * BK, nb * BN, full);
+                    if constexpr (!kFused) tma_load_2d(dst + A_BYTES, &tmap_w, kb * BK, nb * BN, full);
                     issued_parity[stage] = (int)phase;
                     if (++stage == STAGES) {
                         stage = 0;
@@ -320,6 +372,107 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
             mma_commit(smem_addr(&bars->mma_done));
             const uint64_t t0 = now_ns();
             while (!mbar_try_wait(smem_addr(&bars->mma_done), 0) && now_ns() - t0 < limit_ns) {
+            }
+        }
+        __syncwarp();
+    } else if (kFused && warp >= 2 + kEpiWarps) {
+        // ---- decoders (fused): thread dt owns row dt of every B tile ----
+        // (FM = 0, the plain GEMM, never runs this branch; the constants stay valid for it)
+        constexpr int kCodeVecs = FM * FB >= 16 ? (FM * FB) / 16 : 1;        // 16-byte code pieces per row and stage
+        constexpr int kGroupsPerVec = FM * FB > 0 ? 16 * 8 / (FM * FB) : 8;  // groups per 16-byte piece
+        constexpr int kCodeDepth = 4;                                          // stages of codes held ahead
+        const int dt = threadIdx.x - kGemmThreads;
+        const int copy = lane & (kCbCopies - 1);
+        const uint64_t keep = policy_evict_last();
+        const uint64_t stream_pol = policy_evict_first();
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            const int nb = tile / m_tiles;
+            const int n = nb * BN + dt;
+            const bool mine = dt < BN;                   // a row of the tile
+            const bool live = mine && n < n_total;       // a row of W^ (past it: zeros)
+            const float s = live ? __half2float(da.scales[n]) : 0.f;
+            const uint8_t *crow = da.codes + (size_t)(live ? n : 0) * da.row_bytes;
+            auto load_codes = [&](int kb, uint4 (&c)[kCodeVecs]) {
+#pragma unroll
+                for (int v = 0; v < kCodeVecs; ++v) {
+                    c[v] = make_uint4(0, 0, 0, 0);
+                    if (live && kb < num_kb && kb * 8 + v * kGroupsPerVec < da.G)
+                        c[v] = ld_stream_u4(crow + (size_t)kb * 8 * (FM * FB / 8) + 16 * v, stream_pol);
+                }
+            };
+            // the row's codes of the tile: an L2 prefetch of all of them (each 128-byte
+            // line once), then register copies kCodeDepth stages ahead of their use
+            if (live) {
+                const size_t row_code_bytes = (size_t)da.G * (FM * FB / 8);
+                for (size_t off = 0; off < row_code_bytes; off += 128)
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(crow + off));
+            }
+            uint4 ring[kCodeDepth][kCodeVecs];
+#pragma unroll
+            for (int u = 0; u < kCodeDepth; ++u) load_codes(u, ring[u]);
+            for (int kb0 = 0; kb0 < num_kb && ok; kb0 += kCodeDepth) {
+#pragma unroll
+                for (int u = 0; u < kCodeDepth; ++u) {
+                    const int kb = kb0 + u;
+                    if (kb >= num_kb) break;
+                    uint4 code[kCodeVecs];
+#pragma unroll
+                    for (int v = 0; v < kCodeVecs; ++v) code[v] = ring[u][v];
+                    load_codes(kb + kCodeDepth, ring[u]);
+                    bool w = true;
+                    if (lane == 0)
+                        w = wait_bounded(smem_addr(&bars->empty[stage]), phase ^ 1, bars, status, limit_ns);
+                    if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
+                        ok = false;
+                        break;
+                    }
+                    if (mine) {
+                        uint8_t *brow = smem + (size_t)stage * STAGE_BYTES + A_BYTES + (size_t)(dt >> 3) * 1024 +
+                                        (size_t)(dt & 7) * 128;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            uint4 out = make_uint4(0, 0, 0, 0);
+                            if (live && kb * 8 + q < da.G) {
+                                // W^ = bf16_rn(s * (C_0[b0] + ... )), binary32 steps, as aqlm_dequant
+                                // (each lane of the packed pair operations rounds on its own)
+                                float2 acc[4];
+#pragma unroll
+                                for (int m = 0; m < FM; ++m) {
+                                    const uint32_t k = stage_code<FM, FB, kCodeVecs>(code, q, m);
+                                    const uint4 cw = FB == 8
+                                                         ? cbs[((m * 256 + k) << 3) | copy]
+                                                         : ld_keep_u4(da.codebooks + (size_t)m * (1u << FB) + k, keep);
+                                    const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+                                    for (int h = 0; h < 4; ++h) {
+                                        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&wv[h]));
+                                        acc[h] = m == 0 ? f : __fadd2_rn(acc[h], f);
+                                    }
+                                }
+                                const float2 s2 = make_float2(s, s);
+                                uint32_t o[4];
+#pragma unroll
+                                for (int h = 0; h < 4; ++h) {
+                                    const __nv_bfloat162 b2 = __float22bfloat162_rn(__fmul2_rn(acc[h], s2));
+                                    o[h] = *reinterpret_cast<const uint32_t *>(&b2);
+                                }
+                                out = make_uint4(o[0], o[1], o[2], o[3]);
+                            }
+                            *reinterpret_cast<uint4 *>(brow + ((q ^ (dt & 7)) << 4)) = out;
+                        }
+                    }
+                    // generic-proxy stores before the tensor cores' (async-proxy) reads
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(&bars->full[stage]));
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
             }
         }
         __syncwarp();
@@ -405,19 +558,22 @@ bool make_map(CUtensorMap *map, const void *base, int rows, int cols, int box_ro
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 namespace {
-template <int BN>
+template <int BN, int FM, int FB>
 cudaError_t launch_gemm_bn(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
-                           int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test, int sms) {
-    using C = GemmCfg<BN>;
+                           int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test, int sms,
+                           const DecodeArgs &da) {
+    using C = GemmCfg<BN, decode_reserve<FM, FB>()>;
     CUtensorMap mx, mw;
-    if (!make_map(&mx, X, tokens, k, BM) || !make_map(&mw, W, n, k, BN)) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tcgen05<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::SMEM);
+    if (!make_map(&mx, X, tokens, k, BM)) return cudaErrorInvalidValue;
+    if (FM == 0 && !make_map(&mw, W, n, k, BN)) return cudaErrorInvalidValue;
+    if (FM > 0) mw = mx;   // unused by the fused kernel
+    auto fn = gemm_bf16_tcgen05<BN, FM, FB>;
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
     if (e != cudaSuccess) return e;
     const int tiles = ((tokens + BM - 1) / BM) * ((n + BN - 1) / BN);
     const int grid = tiles < sms ? tiles : sms;
-    return launch_kernel(gemm_bf16_tcgen05<BN>, dim3(grid), dim3(kGemmThreads), C::SMEM, st, false, mx, mw,
-                         reinterpret_cast<__nv_bfloat16 *>(Y), tokens, n, k, status, limit_ns, stall_test);
+    return launch_kernel(fn, dim3(grid), dim3(kGemmThreads + (FM > 0 ? kDecThreads : 0)), C::SMEM, st, false, mx,
+                         mw, reinterpret_cast<__nv_bfloat16 *>(Y), tokens, n, k, status, limit_ns, stall_test, da);
 }
 }  // namespace
 
@@ -441,21 +597,46 @@ int gemm_tile_n(int tokens, int n, int sms) {
     return best;
 }
 
-cudaError_t launch_bf16_gemm_ex(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
-                                int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test) {
+namespace {
+template <int FM, int FB>
+cudaError_t launch_by_width(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
+                            int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test,
+                            const DecodeArgs &da) {
     int dev = 0;
     cudaGetDevice(&dev);
     const int sms = num_sms(dev);
     switch (gemm_tile_n(tokens, n, sms)) {
         case 240:
-            return launch_gemm_bn<240>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms);
+            return launch_gemm_bn<240, FM, FB>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, da);
         case 224:
-            return launch_gemm_bn<224>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms);
+            return launch_gemm_bn<224, FM, FB>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, da);
         case 192:
-            return launch_gemm_bn<192>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms);
+            return launch_gemm_bn<192, FM, FB>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, da);
         default:
-            return launch_gemm_bn<256>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms);
+            return launch_gemm_bn<256, FM, FB>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, da);
     }
+}
+}  // namespace
+
+cudaError_t launch_bf16_gemm_ex(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
+                                int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test) {
+    const DecodeArgs none = {};
+    return launch_by_width<0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, none);
+}
+
+// Prefill with the dequantisation fused into the GEMM (no W^ in global memory).
+cudaError_t launch_fused_gemm(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                              const uint16_t *X, uint16_t *Y, int tokens, const Dims &d, int32_t *status,
+                              cudaStream_t st) {
+    DecodeArgs da;
+    da.codes = static_cast<const uint8_t *>(codes);
+    da.codebooks = reinterpret_cast<const uint4 *>(codebooks);
+    da.scales = reinterpret_cast<const __half *>(scales);
+    da.G = d.G;
+    da.row_bytes = d.row_bytes;
+    if (d.M == 1) return launch_by_width<1, 16>(X, nullptr, Y, tokens, d.d_out, d.d_in, status, st, kWaitLimitNs, 0, da);
+    if (d.B == 8) return launch_by_width<2, 8>(X, nullptr, Y, tokens, d.d_out, d.d_in, status, st, kWaitLimitNs, 0, da);
+    return launch_by_width<2, 16>(X, nullptr, Y, tokens, d.d_out, d.d_in, status, st, kWaitLimitNs, 0, da);
 }
 
 cudaError_t launch_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,

@@ -406,9 +406,14 @@ def bench_prefill(ac, spec, tokens, reps, warmup):
     t_deq = timed(lambda: ac.aqlm_dequant(d["codes"], d["codebooks"], d["scales"], out=W))
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     t_gemm = timed(lambda: ac.aqlm_bf16_gemm(X, W, Y=Y, status=status))
+    ws_f = torch.empty(ac.load_library().aqlm_gemm_fused_workspace_bytes(ac.shape_of(d["codes"]), tokens),
+                       dtype=torch.uint8, device="cuda")
+    t_fused = timed(lambda: ac.aqlm_gemm_fused(d["codes"], d["codebooks"], d["scales"], X, Y=Y, workspace=ws_f))
+    assert ac.aqlm_gemm_check(ws_f) == ac.AQLM_OK
     flops = 2.0 * tokens * spec.d_out * spec.d_in
     deq_bytes = spec.code_bytes() + 2 * spec.d_out + 2 * spec.d_out * spec.d_in
-    return {"us_total": t_total, "us_dequant": t_deq, "us_gemm": t_gemm, "tflops": flops / t_total / 1e6,
+    return {"us_total": t_total, "us_dequant": t_deq, "us_gemm": t_gemm, "us_fused": t_fused,
+            "fused_tflops": flops / t_fused / 1e6, "tflops": flops / t_total / 1e6,
             "gemm_tflops": flops / t_gemm / 1e6, "dequant_gbs": deq_bytes / t_deq / 1e3}
 
 
@@ -610,7 +615,10 @@ def run_gpu(args):
                     "us_per_layer": round(p["us_total"], 2), "tflops": round(p["tflops"], 1),
                     "tensor_frac": round(p["tflops"] / peaks["bf16_tflops"], 4),
                     "us_dequant": round(p["us_dequant"], 2), "dequant_gbs": round(p["dequant_gbs"], 1),
-                    "us_gemm": round(p["us_gemm"], 2), "gemm_tflops": round(p["gemm_tflops"], 1)}
+                    "us_gemm": round(p["us_gemm"], 2), "gemm_tflops": round(p["gemm_tflops"], 1),
+                    "fused_no_workspace": {"us_per_layer": round(p["us_fused"], 2),
+                                           "tflops": round(p["fused_tflops"], 1),
+                                           "tensor_frac": round(p["fused_tflops"] / peaks["bf16_tflops"], 4)}}
                 if cpu_ok and (o, i) == PREFILL_SHAPES[0]:
                     detail[key]["cpu_oracle"] = cpu_oracle_prefill(LayerSpec(o, i, M, B), 2048)
                 torch.cuda.empty_cache()

@@ -253,6 +253,29 @@ AQLM_API aqlm_status aqlm_gemm(const void *codes, const uint16_t *codebooks, con
 AQLM_API size_t aqlm_gemm_workspace_bytes(aqlm_shape shape, int32_t tokens);
 
 /*
+ * aqlm_gemm_fused -- the prefill product of aqlm_gemm, Y = bf16(X . W^T),
+ * with the dequantisation fused into the GEMM: extra warps of every GEMM CTA
+ * decode the W^ rows of its own output tiles, 64 inputs at a time, straight
+ * into the tensor cores' shared-memory operand tiles, with the same binary32
+ * steps as aqlm_dequant (so Y equals aqlm_gemm's, bit for bit).  No W^ is
+ * written to global memory: the workspace is only the 256-byte status word
+ * (aqlm_gemm_fused_workspace_bytes), for callers that cannot hold the bf16
+ * copy of a layer (90 MB for 11008 x 4096).  The page this follows, "The
+ * AQLM Quantization Algorithm, Explained", section "Why and what do we
+ * quantize?": weights are fetched compressed and dequantised at runtime.
+ * Each 128-token tile decodes its W^ rows again (16 times for 2048 tokens),
+ * so on B200 it is slower than aqlm_gemm (the decoding competes with the
+ * tensor cores for shared-memory bandwidth; 1x16 and 2x16 also gather their
+ * codewords from L2).  Arguments, alignment, waits and aqlm_gemm_check as for
+ * aqlm_gemm.
+ */
+AQLM_API aqlm_status aqlm_gemm_fused(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                                     const uint16_t *X, uint16_t *Y, int32_t tokens, aqlm_shape shape,
+                                     void *workspace, size_t workspace_bytes, aqlm_stream_t stream);
+
+AQLM_API size_t aqlm_gemm_fused_workspace_bytes(aqlm_shape shape, int32_t tokens);
+
+/*
  * aqlm_gemm_check -- synchronises `stream`, reads and clears the status word
  * that aqlm_gemm calls with this workspace recorded.  Returns AQLM_OK,
  * AQLM_ERR_TIMEOUT, or AQLM_ERR_CUDA if the stream itself reports an error.

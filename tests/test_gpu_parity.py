@@ -359,6 +359,62 @@ def test_gemm_full_size_sampled_tokens(d_out, d_in, M, B):
     _gemm_check(bf16_to_np_bits(Y), L, spec, L["x"], tokens_idx=toks)
 
 
+@pytest.mark.parametrize("M,B", FORMATS)
+@pytest.mark.parametrize("tokens,d_out,d_in", [(200, 520, 576), (256, 512, 1024), (130, 264, 64), (128, 256, 160)])
+def test_gemm_fused_small(M, B, tokens, d_out, d_in):
+    """The fused prefill (W^ decoded inside the GEMM) against the oracle, and
+    bit for bit against aqlm_gemm (the same binary32 decoding, the same MMAs);
+    160 inputs in 2x16 end on a stage of 4 groups."""
+    if (d_in // 8 * M * B // 8) % 16:
+        pytest.skip("row of codes not 16-byte aligned")
+    spec = LayerSpec(d_out, d_in, M, B)
+    L = make_layer(spec, seed=40 + tokens, tokens=tokens, x_dtype="bf16")
+    d = to_dev(L)
+    Y, ws = ac.aqlm_gemm_fused(d["codes"], d["codebooks"], d["scales"], d["x"])
+    assert ws.numel() == 256 and ac.aqlm_gemm_check(ws) == ac.AQLM_OK
+    Y2, ws2 = ac.aqlm_gemm(d["codes"], d["codebooks"], d["scales"], d["x"])
+    assert ac.aqlm_gemm_check(ws2) == ac.AQLM_OK
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+    _gemm_check(bf16_to_np_bits(Y), L, spec, L["x"])
+
+
+# (tokens, d_out) whose tile width on 148 SMs is each of the four
+FUSED_WIDTH_CASES = [(1000, 4608, 256), (2040, 4096, 240), (1530, 4864, 224), (300, 1000, 192)]
+
+
+@pytest.mark.parametrize("tokens,d_out,width", FUSED_WIDTH_CASES, ids=[f"BN{c[2]}" for c in FUSED_WIDTH_CASES])
+@pytest.mark.parametrize("M,B", [(2, 8), (1, 16)])
+def test_gemm_fused_every_tile_width(tokens, d_out, width, M, B):
+    """Each tile width of the fused kernel (its decoders fill 256, 240, 224 or
+    192 rows of every B tile) equals aqlm_gemm bit for bit; sampled tokens
+    against the oracle."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    if sms == 148:
+        assert ac.bf16_gemm_tile_n(tokens, d_out, sms) == width
+    spec = LayerSpec(d_out, 512, M, B)
+    L = make_layer(spec, seed=50 + tokens, tokens=tokens, x_dtype="bf16")
+    d = to_dev(L)
+    Y, ws = ac.aqlm_gemm_fused(d["codes"], d["codebooks"], d["scales"], d["x"])
+    assert ac.aqlm_gemm_check(ws) == ac.AQLM_OK
+    Y2, ws2 = ac.aqlm_gemm(d["codes"], d["codebooks"], d["scales"], d["x"])
+    assert ac.aqlm_gemm_check(ws2) == ac.AQLM_OK
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+    toks = np.array([0, 1, tokens // 2, tokens - 1])
+    _gemm_check(bf16_to_np_bits(Y), L, spec, L["x"], tokens_idx=toks)
+
+
+@pytest.mark.parametrize("d_out,d_in,M,B", [(11008, 4096, 2, 8), (4096, 11008, 1, 16)], ids=["2x8", "1x16"])
+def test_gemm_fused_full_size_sampled_tokens(d_out, d_in, M, B):
+    spec = LayerSpec(d_out, d_in, M, B)
+    L = make_layer(spec, seed=0, tokens=2048, x_dtype="bf16")
+    d = to_dev(L)
+    Y, ws = ac.aqlm_gemm_fused(d["codes"], d["codebooks"], d["scales"], d["x"])
+    assert ac.aqlm_gemm_check(ws) == ac.AQLM_OK
+    rng = np.random.Generator(np.random.PCG64(321))
+    toks = np.unique(np.concatenate([rng.choice(2048, size=12, replace=False), [0, 127, 128, 2047]]))
+    _gemm_check(bf16_to_np_bits(Y), L, spec, L["x"], tokens_idx=toks)
+
+
 def test_gemm_bounded_wait_reports_timeout():
     """Loads withheld on purpose: the first wait runs out, the kernel records
     AQLM_ERR_TIMEOUT, frees its tensor memory and returns; the context stays usable."""
