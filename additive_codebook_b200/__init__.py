@@ -19,6 +19,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libaqlm_b200.so")
+DEBUG_BOUNDS_LIB_PATH = os.path.join(_HERE, "libaqlm_b200_debug_bounds.so")
 
 AQLM_OK = 0
 AQLM_ERR_INVALID_ARG = 1
@@ -36,7 +37,7 @@ EXPORTS = ["aqlm_gemv", "aqlm_gemv_workspace_bytes", "aqlm_gemv_row_tokens", "aq
            "aqlm_test_gemm_timeout", "aqlm_gemv_noalloc", "aqlm_gemv_noalloc_max_scratch_bytes",
            "aqlm_gemv_noalloc_check", "aqlm_test_gemv_noalloc_set_status", "aqlm_probe_gather_sink_bytes",
            "aqlm_probe_gather", "aqlm_gemv_lut", "aqlm_gemv_lut_workspace_bytes", "aqlm_gemm_fused",
-           "aqlm_gemm_fused_workspace_bytes",
+           "aqlm_gemm_fused_workspace_bytes", "aqlm_debug_bounds_read", "aqlm_test_debug_bounds_trip",
            "aqlm_status_string", "aqlm_version",
            "aqlm_encode_scales", "aqlm_nearest_workspace_bytes", "aqlm_nearest_codeword",
            "aqlm_kmeans_workspace_bytes", "aqlm_kmeans_update", "aqlm_residual_kmeans_workspace_bytes",
@@ -72,9 +73,21 @@ def load_library():
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m additive_codebook_b200.build`")
-    lib = ctypes.CDLL(LIB_PATH)
+    _lib = _open(LIB_PATH, "python -m additive_codebook_b200.build")
+    return _lib
+
+
+def load_debug_bounds_library():
+    """The library built with device bounds checks (libaqlm_b200_debug_bounds.so),
+    with the same C signatures; the module's functions keep using the product
+    library unless a caller swaps it in."""
+    return _open(DEBUG_BOUNDS_LIB_PATH, "python -m additive_codebook_b200.build --debug-bounds")
+
+
+def _open(path, how):
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `{how}`")
+    lib = ctypes.CDLL(path)
     vp, i32, sz, u64, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_uint64, ctypes.c_int64
     st = ctypes.c_int
     sig = {
@@ -102,6 +115,8 @@ def load_library():
         "aqlm_gemv_lut_workspace_bytes": ([Shape], sz),
         "aqlm_gemm_fused": ([vp, vp, vp, vp, vp, i32, Shape, vp, sz, vp], st),
         "aqlm_gemm_fused_workspace_bytes": ([Shape, i32], sz),
+        "aqlm_debug_bounds_read": ([ctypes.POINTER(u64), i32], st),
+        "aqlm_test_debug_bounds_trip": ([u64, vp], st),
         "aqlm_probe_gather": ([vp, sz, i32, i32, i32, vp, sz, ctypes.POINTER(u64), vp], st),
         "aqlm_encode_scales": ([vp, i32, i32, vp, vp, vp], st),
         "aqlm_nearest_workspace_bytes": ([i64], sz),
@@ -121,7 +136,6 @@ def load_library():
         fn = getattr(lib, name)
         fn.argtypes = args
         fn.restype = res
-    _lib = lib
     return lib
 
 

@@ -47,6 +47,59 @@ struct RowLayerIn {
     int d_out;
 };
 
+// ---- debug bounds checks ------------------------------------------------------
+// Built with -DAQLM_DEBUG_BOUNDS (the debug variant of the library), the
+// kernels test the index of every computed global or shared-memory access
+// before making it: an index out of range is recorded -- the first one, as
+// (site << 48 | index) -- in a device word of its source file, and the access
+// is skipped.  Nothing traps.  aqlm_debug_bounds_read() collects the words of
+// all files.  In the product build AQLM_IN_BOUNDS is `true` and costs nothing.
+enum BoundsSite : uint32_t {
+    kSiteRowsCodes = 1, kSiteRowsX, kSiteRowsY, kSiteRowsPartial, kSiteRowsSmem,
+    kSiteTcCodes, kSiteTcY, kSiteTcPartial, kSiteTcA,
+    kSiteLutRing, kSiteLutTable, kSiteLutY, kSiteLutPartial,
+    kSiteDequantCodes, kSiteDequantW,
+    kSiteGemmY, kSiteGemmB, kSiteGemmCodebook,
+    kSiteNearest, kSiteKmeans, kSiteEncode,
+    kSiteProbe, kSiteTest
+};
+#ifdef AQLM_DEBUG_BOUNDS
+namespace {
+__device__ unsigned long long g_bounds_word;
+}  // namespace
+__device__ __forceinline__ bool in_bounds(bool ok, uint32_t site, uint64_t index) {
+    if (!ok) atomicCAS(&g_bounds_word, 0ull, ((unsigned long long)site << 48) | (index & 0xffffffffffffull));
+    return ok;
+}
+#define AQLM_IN_BOUNDS(cond, site, index) ::aqlm::in_bounds((cond), (site), (uint64_t)(index))
+// Host: this file's word (and clear it); cudaErrorNotSupported never.
+#define AQLM_DEFINE_BOUNDS_READER(fn)                                                              \
+    cudaError_t fn(unsigned long long *word, bool clear) {                                         \
+        cudaError_t e = cudaMemcpyFromSymbol(word, g_bounds_word, sizeof(*word));                  \
+        if (e == cudaSuccess && clear && *word) {                                                  \
+            const unsigned long long z = 0;                                                         \
+            e = cudaMemcpyToSymbol(g_bounds_word, &z, sizeof(z));                                   \
+        }                                                                                           \
+        return e;                                                                                   \
+    }
+#else
+#define AQLM_IN_BOUNDS(cond, site, index) true
+#define AQLM_DEFINE_BOUNDS_READER(fn)                                                              \
+    cudaError_t fn(unsigned long long *word, bool) {                                               \
+        *word = 0;                                                                                  \
+        return cudaErrorNotSupported;                                                               \
+    }
+#endif
+// one reader per source file that has device code (defined at its end)
+cudaError_t bounds_word_abi(unsigned long long *, bool);
+cudaError_t bounds_word_dequant(unsigned long long *, bool);
+cudaError_t bounds_word_encode(unsigned long long *, bool);
+cudaError_t bounds_word_gemm(unsigned long long *, bool);
+cudaError_t bounds_word_lut(unsigned long long *, bool);
+cudaError_t bounds_word_rows(unsigned long long *, bool);
+cudaError_t bounds_word_tc(unsigned long long *, bool);
+cudaError_t bounds_word_probe(unsigned long long *, bool);
+
 // ---- cache-hinted global loads (PTX ISA: ld with L1/L2 eviction priority) ----
 
 // L2 eviction policies (PTX createpolicy), passed to cache-hinted loads.

@@ -142,7 +142,9 @@ __global__ void __launch_bounds__(256, 3) dequant_kernel(const uint8_t *__restri
         for (int i = 0; i < kPerLane; ++i) {
             const int64_t g = gt + 32 * i;
             if (g >= n_groups) break;
-            const float s = __half2float(scales[row_of(g, rd)]);
+            const int64_t row = row_of(g, rd);   // the division by G through the reciprocal: checked in debug builds
+            if (!AQLM_IN_BOUNDS(row * rd.G <= g && g < (row + 1) * rd.G, kSiteDequantW, g)) continue;
+            const float s = __half2float(scales[row]);
             float acc[kGroup];
             half8_to_float8(cw[i][0], acc);
 #pragma unroll
@@ -230,5 +232,7 @@ cudaError_t launch_dequant(const void *codes, const uint16_t *codebooks, const u
     auto k = dequant_kernel<2, 16>;
     return launch_kernel(k, one_wave_grid(k, n), 256, 0, st, false, c, cb, s, w, rd, n);
 }
+
+AQLM_DEFINE_BOUNDS_READER(bounds_word_dequant)
 
 }  // namespace aqlm

@@ -174,10 +174,11 @@ __global__ void fill_u64_kernel(unsigned long long *p, long long n, unsigned lon
 // idx[n] from the packed winners, and dist[n] = |v - c|^2 of the winner: the
 // squared differences' even and odd lanes as fma chains, then e + o.
 __global__ void unpack_best_kernel(const unsigned long long *__restrict__ best, long long N,
-                                   const float *__restrict__ V, const float *__restrict__ C,
+                                   const float *__restrict__ V, const float *__restrict__ C, int K,
                                    int32_t *__restrict__ idx, float *__restrict__ dist) {
     for (long long n = blockIdx.x * (long long)blockDim.x + threadIdx.x; n < N; n += (long long)gridDim.x * blockDim.x) {
         const uint32_t k = (uint32_t)(best[n] & 0xffffffffull);
+        if (!AQLM_IN_BOUNDS(k < (uint32_t)K, kSiteNearest, n)) continue;
         if (idx) idx[n] = (int32_t)k;
         if (dist) {
             float d[8];
@@ -204,7 +205,8 @@ __global__ void kmeans_accumulate_kernel(const float *__restrict__ V, const int3
         const long long n = i >> 3;
         const int t = (int)(i & 7);
         const int k = idx[n];
-        if (k < 0 || k >= K) continue;  // the host validates nothing on the device: skip bad indices
+        if (k < 0 || k >= K) continue;  // the host validates nothing on the device: skip bad indices (by design,
+                                        // not a bounds error: aqlm_kmeans_update documents that they are ignored)
         atomicAdd(&sums[(long long)k * 8 + t], (double)V[i]);
         if (t == 0) atomicAdd(&counts[k], 1u);
     }
@@ -228,18 +230,19 @@ __global__ void gather_rows_kernel(const float *__restrict__ R, const int32_t *_
                                    float *__restrict__ C) {
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < (long long)K * 8;
          i += (long long)gridDim.x * blockDim.x)
-        C[i] = R[(long long)init[i >> 3] * 8 + (i & 7)];
+        if (AQLM_IN_BOUNDS(init[i >> 3] >= 0, kSiteKmeans, i)) C[i] = R[(long long)init[i >> 3] * 8 + (i & 7)];
 }
 
 // R[n] -= C[best index of n]; optionally the index as the n-th code of codebook m.
 __global__ void subtract_nearest_kernel(float *__restrict__ R, const unsigned long long *__restrict__ best,
-                                        long long N, const float *__restrict__ C, void *__restrict__ codes, int M,
-                                        int m, int code_bytes) {
+                                        long long N, const float *__restrict__ C, int K, void *__restrict__ codes,
+                                        int M, int m, int code_bytes) {
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < N * 8;
          i += (long long)gridDim.x * blockDim.x) {
         const long long n = i >> 3;
         const int t = (int)(i & 7);
         const uint32_t k = (uint32_t)(best[n] & 0xffffffffull);
+        if (!AQLM_IN_BOUNDS(k < (uint32_t)K, kSiteEncode, n)) continue;
         R[i] = __fsub_rn(R[i], C[(long long)k * 8 + t]);
         if (codes && t == 0) {
             if (code_bytes == 1) {
@@ -311,7 +314,7 @@ cudaError_t launch_nearest(const float *V, long long N, const float *C, int K, i
     auto *best = static_cast<unsigned long long *>(workspace);
     cudaError_t e = launch_nearest_packed(V, N, C, K, best, st);
     if (e != cudaSuccess || N == 0) return e;
-    unpack_best_kernel<<<elementwise_grid(N), 256, 0, st>>>(best, N, V, C, idx, dist);
+    unpack_best_kernel<<<elementwise_grid(N), 256, 0, st>>>(best, N, V, C, K, idx, dist);
     return cudaGetLastError();
 }
 
@@ -364,7 +367,7 @@ cudaError_t launch_residual_kmeans(const float *V, long long N, int M, int K, co
                 return e;
         }
         if ((e = launch_nearest_packed(R, N, C, K, best, st)) != cudaSuccess) return e;
-        subtract_nearest_kernel<<<elementwise_grid(N * 8), 256, 0, st>>>(R, best, N, C, nullptr, 1, 0, 2);
+        subtract_nearest_kernel<<<elementwise_grid(N * 8), 256, 0, st>>>(R, best, N, C, K, nullptr, 1, 0, 2);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -390,7 +393,7 @@ cudaError_t launch_encode_codes(const float *V, long long N, const uint16_t *cod
     for (int m = 0; m < M; ++m) {
         const float *Cm = C + (size_t)m * K * 8;
         if ((e = launch_nearest_packed(R, N, Cm, K, best, st)) != cudaSuccess) return e;
-        subtract_nearest_kernel<<<elementwise_grid(N * 8), 256, 0, st>>>(R, best, N, Cm, codes, M, m, code_bytes);
+        subtract_nearest_kernel<<<elementwise_grid(N * 8), 256, 0, st>>>(R, best, N, Cm, K, codes, M, m, code_bytes);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -400,5 +403,7 @@ cudaError_t launch_round_codebooks(const float *C, long long n, uint16_t *C16, c
     float_to_half_kernel<<<elementwise_grid(n), 256, 0, st>>>(C, n, reinterpret_cast<__half *>(C16));
     return cudaGetLastError();
 }
+
+AQLM_DEFINE_BOUNDS_READER(bounds_word_encode)
 
 }  // namespace aqlm

@@ -442,7 +442,9 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
 #pragma unroll
                                 for (int m = 0; m < FM; ++m) {
                                     const uint32_t k = stage_code<FM, FB, kCodeVecs>(code, q, m);
-                                    const uint4 cw = FB == 8
+                                    const uint4 cw = !AQLM_IN_BOUNDS(k < (1u << FB), kSiteGemmCodebook, k)
+                                                         ? make_uint4(0, 0, 0, 0)
+                                                         : FB == 8
                                                          ? cbs[((m * 256 + k) << 3) | copy]
                                                          : ld_keep_u4(da.codebooks + (size_t)m * (1u << FB) + k, keep);
                                     const uint32_t wv[4] = {cw.x, cw.y, cw.z, cw.w};
@@ -461,7 +463,8 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
                                 }
                                 out = make_uint4(o[0], o[1], o[2], o[3]);
                             }
-                            *reinterpret_cast<uint4 *>(brow + ((q ^ (dt & 7)) << 4)) = out;
+                            if (AQLM_IN_BOUNDS(dt < BN, kSiteGemmB, dt))
+                                *reinterpret_cast<uint4 *>(brow + ((q ^ (dt & 7)) << 4)) = out;
                         }
                     }
                     // generic-proxy stores before the tensor cores' (async-proxy) reads
@@ -495,13 +498,15 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
                 uint32_t r[32];
                 tmem_ld32(t_base + (uint32_t)(c * 32), r);
                 const int n0 = nb * BN + c * 32;
-                if (m < m_total) store_bf16_row<4>(Y + (size_t)m * n_total + n0, r, n0, n_total);
+                if (m < m_total && AQLM_IN_BOUNDS(nb < n_tiles && mb < m_tiles, kSiteGemmY, (size_t)m * n_total + n0))
+                    store_bf16_row<4>(Y + (size_t)m * n_total + n0, r, n0, n_total);
             }
             if constexpr (BN % 32 != 0) {  // the last 16 columns of the tile
                 uint32_t r[16];
                 tmem_ld16(t_base + (uint32_t)(BN / 32 * 32), r);
                 const int n0 = nb * BN + BN / 32 * 32;
-                if (m < m_total) store_bf16_row<2>(Y + (size_t)m * n_total + n0, r, n0, n_total);
+                if (m < m_total && AQLM_IN_BOUNDS(nb < n_tiles && mb < m_tiles, kSiteGemmY, (size_t)m * n_total + n0))
+                    store_bf16_row<2>(Y + (size_t)m * n_total + n0, r, n0, n_total);
             }
             tc_fence_before();
             __syncwarp();
@@ -643,5 +648,7 @@ cudaError_t launch_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, 
                              int32_t *status, cudaStream_t st) {
     return launch_bf16_gemm_ex(X, W, Y, tokens, n, k, status, st, kWaitLimitNs, 0);
 }
+
+AQLM_DEFINE_BOUNDS_READER(bounds_word_gemm)
 
 }  // namespace aqlm

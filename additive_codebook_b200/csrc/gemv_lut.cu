@@ -118,8 +118,10 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const LutArgs 
                 const int r = r0 + ic * kChunkRows + (piece >> 2);
                 const int g = is * kSlab + (piece & 3) * 8;      // first group of this 16-byte piece
                 const bool in = r < r1 && g < a.G;
-                cp_async16(ring_s + (uint32_t)(islot * kChunkBytes + piece * 16),
-                           in ? a.codes + (size_t)r * a.row_bytes + (size_t)g * 2 : a.codes, in ? 16u : 0u);
+                const bool ok = AQLM_IN_BOUNDS(islot < kRing && piece * 16 < kChunkBytes && (!in || r < a.d_out),
+                                               kSiteLutRing, piece);
+                cp_async16(ring_s + (uint32_t)((ok ? islot : 0) * kChunkBytes + (ok ? piece : 0) * 16),
+                           in && ok ? a.codes + (size_t)r * a.row_bytes + (size_t)g * 2 : a.codes, in && ok ? 16u : 0u);
             }
             if (++ic == n_chunks) {
                 ic = 0;
@@ -175,7 +177,9 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const LutArgs 
 #pragma unroll
             for (int i = 0; i < kBatch; ++i) {
                 const uint32_t code = codes_s[i * kSlab];
-                v[i] = lut0[(code & 0xffu) * kSlab] + lut1[(code >> 8) * kSlab];
+                v[i] = AQLM_IN_BOUNDS(code < 65536u, kSiteLutTable, code)
+                           ? lut0[(code & 0xffu) * kSlab] + lut1[(code >> 8) * kSlab]
+                           : 0.f;
             }
             // butterfly over the 16 rows: after the step of offset o, v[0..o) hold
             // rows (lane & o ? o..2o : 0..o) of the current half, summed over the lane pair
@@ -191,7 +195,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const LutArgs 
             }
             v[0] += __shfl_xor_sync(0xffffffffu, v[0], 16);   // lanes l and l ^ 16 hold row l & 15
             const int rr = c * kChunkRows + warp * kBatch + lane;   // row from r0; lanes 0..15 write
-            if (lane < kBatch && r0 + rr < r1) {
+            if (lane < kBatch && r0 + rr < r1 && AQLM_IN_BOUNDS(r1 <= a.d_out && grp < a.n_groups, kSiteLutY, r0 + rr)) {
                 if (multi) {
                     rowacc[rr] = (s == slab0 ? 0.f : rowacc[rr]) + v[0];
                 } else if (a.n_groups == 1) {
@@ -322,5 +326,7 @@ cudaError_t launch_gemv_lut(const void *codes, const uint16_t *codebooks, const 
     if (e != cudaSuccess) return e;
     return launch_kernel(gemv_lut_kernel, dim3(p.n_groups, p.n_ranges), dim3(kLutThreads), p.smem, st, true, a);
 }
+
+AQLM_DEFINE_BOUNDS_READER(bounds_word_lut)
 
 }  // namespace aqlm

@@ -182,10 +182,11 @@ __global__ void __launch_bounds__(RowFmt<M, B>::kThreads, 2) gemv_rows_kernel(co
     };
     auto lane_live = [&](Item it) { return it.j < n_rows && lane + 32 * it.s < n_chunks; };
     auto load_code = [&](Item it) -> uint4 {
-        if (lane_live(it))
-            return ld_stream_u4(L.codes + (size_t)(r0 + warp + F::kWarps * it.j) * a.row_bytes +
-                                    (size_t)(c0 + lane + 32 * it.s) * 16,
-                                stream_pol);
+        if (lane_live(it)) {
+            const int row = r0 + warp + F::kWarps * it.j, chunk = c0 + lane + 32 * it.s;
+            if (AQLM_IN_BOUNDS(row < L.d_out && chunk * 16 < a.row_bytes, kSiteRowsCodes, (size_t)row * a.row_bytes))
+                return ld_stream_u4(L.codes + (size_t)row * a.row_bytes + (size_t)chunk * 16, stream_pol);
+        }
         return make_uint4(0, 0, 0, 0);
     };
     auto gather = [&](const uint4 &ch, Item it, uint4 (&cw)[GPC][M]) {
@@ -220,8 +221,9 @@ __global__ void __launch_bounds__(RowFmt<M, B>::kThreads, 2) gemv_rows_kernel(co
         for (int i = threadIdx.x; i < T * ng; i += F::kThreads) {  // stage x, transposed by chunk
             const int t = i / ng, g = i - t * ng;
             const int c = g / GPC, q = g - c * GPC;
-            xs[((size_t)t * GPC + q) * xstride + c] =
-                *reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.d_in + (size_t)(c0 * GPC + g) * kGroup);
+            if (AQLM_IN_BOUNDS((c0 * GPC + g + 1) * kGroup <= a.d_in && c < xstride, kSiteRowsX, c0 * GPC + g))
+                xs[((size_t)t * GPC + q) * xstride + c] =
+                    *reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.d_in + (size_t)(c0 * GPC + g) * kGroup);
         }
         __syncthreads();
     }
@@ -243,9 +245,10 @@ __global__ void __launch_bounds__(RowFmt<M, B>::kThreads, 2) gemv_rows_kernel(co
             if (lane == 0) {
                 if (splits == 1) {
                     const float s_r = it.j < 32 ? sc : __half2float(L.scales[r]);
-                    L.y[(size_t)t * L.d_out + r] = __float2half_rn(v * s_r);
+                    if (AQLM_IN_BOUNDS(r < L.d_out, kSiteRowsY, r)) L.y[(size_t)t * L.d_out + r] = __float2half_rn(v * s_r);
                 } else {
-                    a.partial[((size_t)split * T + t) * a.total_rows + row0 + r] = v;
+                    if (AQLM_IN_BOUNDS(row0 + r < a.total_rows, kSiteRowsPartial, row0 + r))
+                        a.partial[((size_t)split * T + t) * a.total_rows + row0 + r] = v;
                 }
             }
             acc[t] = acc2[t] = 0.f;
@@ -256,7 +259,8 @@ __global__ void __launch_bounds__(RowFmt<M, B>::kThreads, 2) gemv_rows_kernel(co
     auto dot_group = [&](const uint4 &cw0, const uint4 &cw1, int q, int c) {
 #pragma unroll
         for (int t = 0; t < T; ++t) {
-            const uint4 xv = xs[((size_t)t * GPC + q) * xstride + c];
+            const uint4 xv = AQLM_IN_BOUNDS(c < xstride, kSiteRowsSmem, c) ? xs[((size_t)t * GPC + q) * xstride + c]
+                                                                           : make_uint4(0, 0, 0, 0);
             fma2_f16_f32(acc[t], acc2[t], cw0.x, xv.x);
             fma2_f16_f32(acc[t], acc2[t], cw0.y, xv.y);
             fma2_f16_f32(acc[t], acc2[t], cw0.z, xv.z);
@@ -341,7 +345,8 @@ __global__ void __launch_bounds__(RowFmt<M, B>::kThreads, 2) gemv_rows_kernel(co
 #pragma unroll
             for (int u = 0; u < 4; ++u) sum += v[u];
         }
-        L.y[(size_t)t * L.d_out + r] = __float2half_rn(sum * __half2float(L.scales[r]));
+        if (AQLM_IN_BOUNDS(r < L.d_out, kSiteRowsY, r))
+            L.y[(size_t)t * L.d_out + r] = __float2half_rn(sum * __half2float(L.scales[r]));
     }
     if (threadIdx.x == 0) a.counters[blockIdx.x] = 0u;
 }
@@ -552,5 +557,7 @@ cudaError_t launch_gemv_rows(const void *codes, const uint16_t *codebooks, const
     const RowLayerIn layer = {codes, codebooks, scales, y, d.d_out};
     return launch_gemv_rows_multi(&layer, 1, x, tokens, d, workspace, sms, st);
 }
+
+AQLM_DEFINE_BOUNDS_READER(bounds_word_rows)
 
 }  // namespace aqlm

@@ -483,7 +483,9 @@ __global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm)
 #pragma unroll
                 for (int v = 0; v < kCodeVecs; ++v) {
                     const int piece = (l % SPB) * kCodeVecs + v;
-                    code[v] = *reinterpret_cast<const uint4 *>(rowp + ((piece ^ ((r >> 1) & 3)) << 4));
+                    code[v] = AQLM_IN_BOUNDS(piece < kCodeBoxBytes / 16, kSiteTcCodes, piece)
+                                  ? *reinterpret_cast<const uint4 *>(rowp + ((piece ^ ((r >> 1) & 3)) << 4))
+                                  : make_uint4(0, 0, 0, 0);
                 }
                 // the stage's A tiles are free once the MMAs of its previous use are done
                 const int gi = gi0 + l, s = gi % F::kStages;
@@ -500,10 +502,12 @@ __global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm)
                 for (int q = 0; q < kStageGroups; ++q) {
                     const uint32_t bytes = (grp0 + q < a.G) ? 16u : 0u;
 #pragma unroll
-                    for (int m = 0; m < M; ++m)
-                        cp_async16_keep<B == 8>(
-                            tile + (uint32_t)(m * kTileBytes) + (uint32_t)((q ^ (r & 7)) << 4),
-                            L.codebooks + (size_t)m * F::K + tc_index<M, B, kCodeVecs>(code, q, m), bytes, keep);
+                    for (int m = 0; m < M; ++m) {
+                        const uint32_t k = tc_index<M, B, kCodeVecs>(code, q, m);
+                        const bool in = AQLM_IN_BOUNDS(k < (uint32_t)F::K && r * 128 + 128 <= kTileBytes, kSiteTcA, r);
+                        cp_async16_keep<B == 8>(tile + (uint32_t)(m * kTileBytes) + (uint32_t)((q ^ (r & 7)) << 4),
+                                                L.codebooks + (size_t)m * F::K + (in ? k : 0u), in ? bytes : 0u, keep);
+                    }
                 }
                 cp_async_arrive_noinc(saddr(&bars->full[s]));
                 // the box's codes were read into registers and used above: its slot
@@ -530,15 +534,18 @@ __global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm)
                 if (row < L.d_out) {
                     const float sc = __half2float(L.scales[row]);
                     for (int t = 0; t < a.T; ++t)
-                        L.y[(size_t)t * L.d_out + row] = __float2half_rn(__uint_as_float(v[t]) * sc);
+                        if (AQLM_IN_BOUNDS(row < L.d_out, kSiteTcY, row))
+                            L.y[(size_t)t * L.d_out + row] = __float2half_rn(__uint_as_float(v[t]) * sc);
                 }
             } else {
                 const long long t_u0 = (long long)g.tile * a.n_stages;
                 const int c_lo = cta_of_unit(t_u0, a);
                 const int n_seg = cta_of_unit(t_u0 + a.n_stages - 1, a) - c_lo + 1;
                 float *part = a.partial + (size_t)g.tile * a.max_segs * a.T * kTcRows;
-                for (int t = 0; t < a.T; ++t)
-                    part[((size_t)(blockIdx.x - c_lo) * a.T + t) * kTcRows + r] = __uint_as_float(v[t]);
+                if (AQLM_IN_BOUNDS((int)blockIdx.x - c_lo < a.max_segs && n_seg <= a.max_segs, kSiteTcPartial,
+                                   (int)blockIdx.x - c_lo))
+                    for (int t = 0; t < a.T; ++t)
+                        part[((size_t)(blockIdx.x - c_lo) * a.T + t) * kTcRows + r] = __uint_as_float(v[t]);
                 __threadfence();
                 asm volatile("bar.sync 1, %0;" ::"n"(kDecoders) : "memory");
                 if (threadIdx.x == 0)
@@ -563,7 +570,8 @@ __global__ void __launch_bounds__(kTcThreads, TcFmt<M, B>::kCtasPerSm)
                         }
 #pragma unroll
                         for (int t = 0; t < kTcN; ++t)
-                            if (t < a.T) L.y[(size_t)t * L.d_out + row] = __float2half_rn(sum[t] * sc);
+                            if (t < a.T && AQLM_IN_BOUNDS(row < L.d_out, kSiteTcY, row))
+                                L.y[(size_t)t * L.d_out + row] = __float2half_rn(sum[t] * sc);
                     }
                     if (threadIdx.x == 0) a.counters[g.tile] = 0u;
                 }
@@ -752,5 +760,7 @@ cudaError_t launch_gemv_tc(const void *codes, const uint16_t *codebooks, const u
     const RowLayerIn one = {codes, codebooks, scales, y, d.d_out};
     return launch_gemv_tc_multi(&one, 1, x, tokens, d, workspace, sms, st);
 }
+
+AQLM_DEFINE_BOUNDS_READER(bounds_word_tc)
 
 }  // namespace aqlm

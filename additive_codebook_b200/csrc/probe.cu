@@ -38,7 +38,9 @@ __global__ void __launch_bounds__(kProbeThreads) probe_gather_kernel(const uint4
         for (int u = 0; u < kProbeUnroll; ++u) {
             h = h * 1664525u + 1013904223u;
             const uint32_t i = __umulhi(h, entries);
-            v[u] = SRC == 0 ? ld_keep_u4(table + i, pol) : stab[i];
+            v[u] = !AQLM_IN_BOUNDS(i < entries, kSiteProbe, i) ? make_uint4(0, 0, 0, 0)
+                   : SRC == 0                                          ? ld_keep_u4(table + i, pol)
+                                                                       : stab[i];
         }
 #pragma unroll
         for (int u = 0; u < kProbeUnroll; ++u) acc ^= v[u].x + v[u].y + v[u].z + v[u].w;
@@ -46,10 +48,47 @@ __global__ void __launch_bounds__(kProbeThreads) probe_gather_kernel(const uint4
     sink[blockIdx.x * blockDim.x + threadIdx.x] = acc;
 }
 
+// Records a bounds violation on purpose (site kSiteTest, index `index`) and
+// touches no memory: the test of the debug-bounds mechanism itself.
+__global__ void bounds_trip_kernel(uint64_t index) { (void)AQLM_IN_BOUNDS(false, kSiteTest, index); }
+
 }  // namespace
+
+AQLM_DEFINE_BOUNDS_READER(bounds_word_probe)
+
 }  // namespace aqlm
 
 extern "C" {
+
+aqlm_status aqlm_debug_bounds_read(uint64_t *word, int32_t clear) {
+    if (!word) return AQLM_ERR_INVALID_ARG;
+    cudaError_t (*readers[])(unsigned long long *, bool) = {
+        aqlm::bounds_word_dequant, aqlm::bounds_word_encode, aqlm::bounds_word_gemm, aqlm::bounds_word_lut,
+        aqlm::bounds_word_rows,    aqlm::bounds_word_tc,     aqlm::bounds_word_probe};
+    *word = 0;
+    for (auto rd : readers) {
+        unsigned long long w = 0;
+        const cudaError_t e = rd(&w, clear != 0);
+        if (e == cudaErrorNotSupported) return AQLM_ERR_UNSUPPORTED;
+        if (e != cudaSuccess) return AQLM_ERR_CUDA;
+        if (w && !*word) *word = w;
+    }
+    return AQLM_OK;
+}
+
+aqlm_status aqlm_test_debug_bounds_trip(uint64_t index, aqlm_stream_t stream) {
+#ifdef AQLM_DEBUG_BOUNDS
+    return aqlm::launch_kernel(aqlm::bounds_trip_kernel, dim3(1), dim3(1), 0, reinterpret_cast<cudaStream_t>(stream),
+                               false, index) == cudaSuccess
+               ? AQLM_OK
+               : AQLM_ERR_CUDA;
+#else
+    (void)index;
+    (void)stream;
+    return AQLM_ERR_UNSUPPORTED;
+#endif
+}
+
 
 size_t aqlm_probe_gather_sink_bytes(int32_t ctas_per_sm) {
     int dev = 0;

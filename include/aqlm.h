@@ -466,6 +466,25 @@ AQLM_API aqlm_status aqlm_probe_gather(const void *table, size_t table_bytes, in
                                        int32_t iters, void *sink, size_t sink_bytes, uint64_t *gathers,
                                        aqlm_stream_t stream);
 
+/* ===========================================================================
+ * Debug bounds checks.
+ *
+ * Not part of the method.  The library built with -DAQLM_DEBUG_BOUNDS
+ * (libaqlm_b200_debug_bounds.so, `python -m additive_codebook_b200.build
+ * --debug-bounds`) tests, in every kernel, the computed indices of its global
+ * and shared-memory accesses before making them; an index out of range is
+ * recorded -- the first one, as (site << 48 | index), the sites numbered in
+ * csrc/common.cuh -- in a device word, and the access is skipped.  Nothing
+ * traps.  aqlm_debug_bounds_read stores that word (0: no violation since the
+ * last clear) in *word (host memory), clearing it if `clear`; it
+ * synchronises the device.  The product build returns AQLM_ERR_UNSUPPORTED.
+ * aqlm_test_debug_bounds_trip records a violation at site 23 with `index` on
+ * purpose, touching no memory (a test of the mechanism; AQLM_ERR_UNSUPPORTED
+ * in the product build).
+ * ======================================================================== */
+AQLM_API aqlm_status aqlm_debug_bounds_read(uint64_t *word, int32_t clear);
+AQLM_API aqlm_status aqlm_test_debug_bounds_trip(uint64_t index, aqlm_stream_t stream);
+
 /* A static, human-readable name of a status code. */
 AQLM_API const char *aqlm_status_string(aqlm_status status);
 

@@ -279,3 +279,24 @@ def test_gemm_tile_width_rule():
                 assert ac.bf16_gemm_tile_n(tokens, n, sms) == rule(tokens, n, sms)
     assert [ac.bf16_gemm_tile_n(2048, n, 148) for n in (11008, 4096, 8192, 28672)] == [240, 240, 224, 240]
     assert ac.bf16_gemm_tile_n(0, 8, 148) == 0 and ac.bf16_gemm_tile_n(8, 8, 0) == 0
+
+
+def test_debug_bounds_entry_points_in_the_product_build():
+    """The product library answers the debug-bounds calls with
+    AQLM_ERR_UNSUPPORTED (no device checks are compiled in); no CUDA call."""
+    lib = ac.load_library()
+    w = ctypes.c_uint64(1)
+    assert lib.aqlm_debug_bounds_read(ctypes.byref(w), 1) == ac.AQLM_ERR_UNSUPPORTED and w.value == 0
+    assert lib.aqlm_test_debug_bounds_trip(1, NULL) == ac.AQLM_ERR_UNSUPPORTED
+    assert lib.aqlm_debug_bounds_read(None, 0) == ac.AQLM_ERR_INVALID_ARG
+
+
+def test_library_builds_with_debug_bounds(tmp_path):
+    """-DAQLM_DEBUG_BOUNDS still compiles and links every source, and the
+    result exports every declared entry point."""
+    from additive_codebook_b200 import build as cuda_build
+    lib_path = cuda_build.build(force=True, debug_bounds=True, out_lib=str(tmp_path / "libdbg.so"),
+                                objdir=str(tmp_path / "obj"))
+    lib = ctypes.CDLL(lib_path)
+    for name in ac.EXPORTS:
+        assert hasattr(lib, name), name
