@@ -207,6 +207,32 @@ cudaError_t opt_in_dynamic_smem(void (*kern)(KArgs...), size_t bytes) {
     return e;
 }
 
+// Ask for the largest shared-memory carveout for `kern` (once per kernel and
+// device).  An SM runs CTAs of different kernels side by side only under one
+// L1 / shared-memory split; a kernel whose launches leave room for the next
+// launch's CTA keeps that overlap across layers of different shapes only if
+// every launch asks for the same split.
+template <typename... KArgs>
+cudaError_t prefer_max_shared_carveout(void (*kern)(KArgs...)) {
+    static std::mutex mu;
+    static std::vector<std::pair<const void *, int>> done;
+    const void *key = reinterpret_cast<const void *>(kern);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (const auto &e : done)
+            if (e.first == key && e.second == dev) return cudaSuccess;
+    }
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess && dev >= 0) {
+        std::lock_guard<std::mutex> lock(mu);
+        if (done.size() < 1024) done.emplace_back(key, dev);
+    }
+    return e;
+}
+
 // Launch through cudaLaunchKernelEx so that the returned error belongs to this
 // launch only.  `pdl` allows programmatic dependent launch: the kernel may
 // start while the previous kernel in the stream finishes, and must execute

@@ -508,6 +508,10 @@ cudaError_t launch_rows(const RowLayerIn *layers, int n, const uint16_t *x, int 
         fn = rows_fn<2, 16, NL>(tokens);
     }
     if (!fn) return cudaErrorInvalidValue;
+    if (d.B == 8) {  // one CTA per SM and launch, the next launch's CTA beside it: one carveout for all shapes
+        const cudaError_t e = prefer_max_shared_carveout(fn);
+        if (e != cudaSuccess) return e;
+    }
     const int threads = row_warps(d) * 32;
     const int occ = resident_ctas(reinterpret_cast<const void *>(fn), threads, p.smem);
     int d_outs[kRowMaxLayers], ctas[kRowMaxLayers];

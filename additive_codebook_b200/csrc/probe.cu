@@ -48,9 +48,11 @@ __global__ void __launch_bounds__(kProbeThreads) probe_gather_kernel(const uint4
     sink[blockIdx.x * blockDim.x + threadIdx.x] = acc;
 }
 
+#ifdef AQLM_DEBUG_BOUNDS
 // Records a bounds violation on purpose (site kSiteTest, index `index`) and
 // touches no memory: the test of the debug-bounds mechanism itself.
 __global__ void bounds_trip_kernel(uint64_t index) { (void)AQLM_IN_BOUNDS(false, kSiteTest, index); }
+#endif
 
 }  // namespace
 
