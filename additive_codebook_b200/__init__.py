@@ -33,7 +33,7 @@ GEMV_MAX_TOKENS = 16
 # Every entry point declared in include/aqlm.h.
 EXPORTS = ["aqlm_gemv", "aqlm_gemv_workspace_bytes", "aqlm_gemv_row_tokens", "aqlm_gemv_multi",
            "aqlm_gemv_multi_workspace_bytes", "aqlm_gemv_multi_check", "aqlm_gemv_check", "aqlm_dequant", "aqlm_gemm",
-           "aqlm_gemm_workspace_bytes", "aqlm_gemm_check", "aqlm_bf16_gemm", "aqlm_bf16_gemm_tile_n", "aqlm_decode_indices",
+           "aqlm_gemm_workspace_bytes", "aqlm_gemm_check", "aqlm_bf16_gemm", "aqlm_bf16_gemm_tile_n", "aqlm_bf16_gemm_plan", "aqlm_bf16_gemm_config", "aqlm_decode_indices",
            "aqlm_test_gemm_timeout", "aqlm_gemv_noalloc", "aqlm_gemv_noalloc_max_scratch_bytes",
            "aqlm_gemv_noalloc_check", "aqlm_test_gemv_noalloc_set_status", "aqlm_probe_gather_sink_bytes",
            "aqlm_probe_gather", "aqlm_gemv_lut", "aqlm_gemv_lut_workspace_bytes", "aqlm_gemm_fused",
@@ -105,7 +105,9 @@ def _open(path, how):
         "aqlm_bf16_gemm": ([vp, vp, vp, i32, i32, i32, vp, vp], st),
         "aqlm_bf16_gemm_tile_n": ([i32, i32, i32], i32),
         "aqlm_decode_indices": ([vp, vp, Shape, vp], st),
-        "aqlm_test_gemm_timeout": ([vp, vp, vp, i32, i32, i32, vp, u64, vp], st),
+        "aqlm_bf16_gemm_plan": ([i32, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)], st),
+        "aqlm_bf16_gemm_config": ([vp, vp, vp, i32, i32, i32, vp, i32, i32, vp], st),
+        "aqlm_test_gemm_timeout": ([vp, vp, vp, i32, i32, i32, vp, u64, i32, vp], st),
         "aqlm_gemv_noalloc": ([vp, vp, vp, vp, vp, i32, Shape, vp], st),
         "aqlm_gemv_noalloc_max_scratch_bytes": ([], sz),
         "aqlm_gemv_noalloc_check": ([vp], st),
@@ -396,6 +398,28 @@ def bf16_gemm_tile_n(tokens, n, sms):
     return int(load_library().aqlm_bf16_gemm_tile_n(int(tokens), int(n), int(sms)))
 
 
+def bf16_gemm_plan(tokens, n, sms):
+    """(cta_pair, tile_n): the GEMM kernel chosen for tokens x n on `sms` SMs."""
+    pair, width = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(load_library().aqlm_bf16_gemm_plan(int(tokens), int(n), int(sms), ctypes.byref(pair),
+                                              ctypes.byref(width)), "aqlm_bf16_gemm_plan")
+    return int(pair.value), int(width.value)
+
+
+def aqlm_bf16_gemm_config(X, W, cta_pair, tile_n, Y=None, status=None, stream=None):
+    """aqlm_bf16_gemm with the kernel variant chosen by the caller."""
+    lib = load_library()
+    T, k = X.shape
+    n = W.shape[0]
+    if Y is None:
+        Y = torch.empty((T, n), dtype=torch.bfloat16, device=X.device)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=X.device)
+    _check(lib.aqlm_bf16_gemm_config(_p(X), _p(W), _p(Y), T, n, k, _p(status), int(cta_pair), int(tile_n),
+                                     _stream(stream)), "aqlm_bf16_gemm_config")
+    return Y, status
+
+
 def aqlm_bf16_gemm(X, W, Y=None, status=None, stream=None):
     """Y[T, n] = bf16(X[T, k] . W[n, k]^T) on the tensor cores."""
     lib = load_library()
@@ -419,11 +443,12 @@ def aqlm_decode_indices(codes, out=None, stream=None):
     return out
 
 
-def aqlm_test_gemm_timeout(X, W, Y, status, limit_ns, stream=None):
+def aqlm_test_gemm_timeout(X, W, Y, status, limit_ns, cta_pair=0, stream=None):
     lib = load_library()
     T, k = X.shape
     n = W.shape[0]
-    return lib.aqlm_test_gemm_timeout(_p(X), _p(W), _p(Y), T, n, k, _p(status), limit_ns, _stream(stream))
+    return lib.aqlm_test_gemm_timeout(_p(X), _p(W), _p(Y), T, n, k, _p(status), limit_ns, int(cta_pair),
+                                      _stream(stream))
 
 
 # --------------------------------------------------------------------------- encoding

@@ -8,6 +8,9 @@
 namespace aqlm {
 cudaError_t launch_bf16_gemm_ex(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                                 int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test);
+cudaError_t launch_bf16_gemm_cfg(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
+                                 int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test,
+                                 int cta_pair, int tile_n);
 cudaError_t launch_fused_gemm(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                               const uint16_t *X, uint16_t *Y, int tokens, const Dims &d, int32_t *status,
                               cudaStream_t st);
@@ -285,12 +288,41 @@ int32_t aqlm_bf16_gemm_tile_n(int32_t tokens, int32_t n, int32_t sms) {
     return aqlm::gemm_tile_n(tokens, n, sms);
 }
 
-aqlm_status aqlm_test_gemm_timeout(const uint16_t *X, const uint16_t *W, uint16_t *Y, int32_t tokens, int32_t n,
-                                   int32_t k, int32_t *status, uint64_t limit_ns, aqlm_stream_t stream) {
-    if (!X || !W || !Y || !status || tokens < 1 || n < 1 || k < 1 || n % 8 || k % 8) return AQLM_ERR_INVALID_ARG;
-    if (limit_ns == 0 || limit_ns > 1000000000ull) return AQLM_ERR_INVALID_ARG;
+aqlm_status aqlm_bf16_gemm_plan(int32_t tokens, int32_t n, int32_t sms, int32_t *cta_pair, int32_t *tile_n) {
+    if (!cta_pair || !tile_n) return AQLM_ERR_INVALID_ARG;
+    *cta_pair = 0;
+    *tile_n = 0;
+    if (tokens < 1 || n < 1 || sms < 2) return AQLM_ERR_INVALID_ARG;
+    const bool pair = aqlm::gemm_uses_pair(tokens);
+    *cta_pair = pair ? 1 : 0;
+    *tile_n = pair ? aqlm::gemm_pair_tile_n(tokens, n, sms / 2) : aqlm::gemm_tile_n(tokens, n, sms);
+    return AQLM_OK;
+}
+
+static bool known_tile_n(int32_t tile_n) {
+    return tile_n == 0 || tile_n == 256 || tile_n == 240 || tile_n == 224 || tile_n == 192;
+}
+
+aqlm_status aqlm_bf16_gemm_config(const uint16_t *X, const uint16_t *W, uint16_t *Y, int32_t tokens, int32_t n,
+                                  int32_t k, int32_t *status, int32_t cta_pair, int32_t tile_n,
+                                  aqlm_stream_t stream) {
+    if (!X || !W || !Y || !status || tokens < 1 || n < 1 || k < 1) return AQLM_ERR_INVALID_ARG;
+    if (n > kMaxDim || k > kMaxDim || tokens > kMaxDim) return AQLM_ERR_INVALID_ARG;
+    if (cta_pair < -1 || cta_pair > 1 || !known_tile_n(tile_n)) return AQLM_ERR_INVALID_ARG;
+    if (n % 8 || k % 8) return AQLM_ERR_UNSUPPORTED;
     if (!aligned(X, 16) || !aligned(W, 16) || !aligned(Y, 16) || !aligned(status, 4)) return AQLM_ERR_MISALIGNED;
-    return from_cuda(aqlm::launch_bf16_gemm_ex(X, W, Y, tokens, n, k, status, to_cuda(stream), limit_ns, 1));
+    return from_cuda(aqlm::launch_bf16_gemm_cfg(X, W, Y, tokens, n, k, status, to_cuda(stream),
+                                                aqlm::kGemmWaitLimitNs, 0, cta_pair, tile_n));
+}
+
+aqlm_status aqlm_test_gemm_timeout(const uint16_t *X, const uint16_t *W, uint16_t *Y, int32_t tokens, int32_t n,
+                                   int32_t k, int32_t *status, uint64_t limit_ns, int32_t cta_pair,
+                                   aqlm_stream_t stream) {
+    if (!X || !W || !Y || !status || tokens < 1 || n < 1 || k < 1 || n % 8 || k % 8) return AQLM_ERR_INVALID_ARG;
+    if (limit_ns == 0 || limit_ns > 1000000000ull || cta_pair < -1 || cta_pair > 1) return AQLM_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(W, 16) || !aligned(Y, 16) || !aligned(status, 4)) return AQLM_ERR_MISALIGNED;
+    return from_cuda(aqlm::launch_bf16_gemm_cfg(X, W, Y, tokens, n, k, status, to_cuda(stream), limit_ns, 1,
+                                                cta_pair, 0));
 }
 
 // ---- encoding ----

@@ -321,7 +321,11 @@ cudaError_t launch_gemv_lut(const void *codes, const uint16_t *codebooks, const 
                             uint16_t *y, const Dims &d, void *workspace, int sms, cudaStream_t st);
 cudaError_t launch_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                              int32_t *status, cudaStream_t st);
+// Bound on any single wait of the GEMM kernels (a whole GEMM takes well under this).
+constexpr unsigned long long kGemmWaitLimitNs = 2000000000ull;
 int gemm_tile_n(int tokens, int n, int sms);
+int gemm_pair_tile_n(int tokens, int n, int pairs);
+bool gemm_uses_pair(int tokens);
 // encoding (encode.cu)
 cudaError_t launch_encode_scales(const float *W, int d_out, int d_in, uint16_t *scales, float *V, cudaStream_t st);
 size_t nearest_workspace_bytes(long long N);

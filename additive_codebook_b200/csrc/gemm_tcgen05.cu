@@ -526,6 +526,337 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
     }
 }
 
+// ---- the CTA-pair GEMM: 256 x BN tiles on two SMs ---------------------------
+// tcgen05.mma.cta_group::2 (M = 256) runs one MMA on the tensor cores of a
+// pair of SMs, a cluster of two CTAs: CTA r of the pair stages rows
+// [128 r, 128 r + 128) of the X tile and rows [r BN/2, (r + 1) BN/2) of the W
+// tile in its own shared memory (at the same offsets in both CTAs), the MMA
+// reads both CTAs' tiles, and CTA r's tensor memory receives output rows
+// [128 r, 128 r + 128) x all BN columns.  Per SM a stage is 128 + BN/2 rows of
+// 128 bytes instead of 128 + BN, so each SM streams a third less operand data
+// for the same MMA work, and six stages fit where four did.
+//   both CTAs   warp 0 lane 0 loads its own halves with TMA; the bytes of both
+//               complete the leader's (rank 0) full barrier, which the
+//               leader's producer armed with the bytes of the two CTAs;
+//   leader      warp 1 lane 0 issues the MMAs and commits to the empty and
+//               tfull barriers of both CTAs (tcgen05.commit with a CTA mask);
+//   both CTAs   warps 2-5 read their own accumulator rows and arrive on the
+//               leader's tempty barrier (4 + 4 arrivals free an accumulator).
+// Tensor memory is allocated and freed by warp 1 of both CTAs together
+// (.cta_group::2).  Every wait is bounded; a wait that gives up raises the
+// abort flag of both CTAs.  Before exiting, each CTA waits (bounded) for the
+// arrivals the other CTA or the tensor cores still owe its barriers, and the
+// two meet at a cluster barrier that every thread reaches, so that neither
+// leaves while the other may still touch its shared or tensor memory.
+constexpr int kPairRows = 2 * BM;   // output rows of a pair tile
+
+template <int BN>
+struct PairCfg {
+    static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "MMA N for M = 256");
+    static constexpr int B_HALF = BN / 2;                   // rows of W each CTA stages (a multiple of 8)
+    static constexpr int B_BYTES = B_HALF * BK * 2;         // a multiple of 1024: stages stay aligned
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = 200 * 1024 / STAGE_BYTES < kMaxStages ? 200 * 1024 / STAGE_BYTES : kMaxStages;
+    static constexpr int ACC_STRIDE = BN <= 128 ? 128 : 256;
+    static constexpr uint32_t TMEM_COLS = 2 * ACC_STRIDE;
+    // as GemmCfg::IDESC with M = 256
+    static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                      ((uint32_t)(kPairRows >> 4) << 24);
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Bars) + 16;
+    static_assert(B_BYTES % 1024 == 0 && STAGES >= 2, "ring layout");
+};
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_count_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+// The shared::cluster address of the variable at shared address `saddr` in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_shared(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cl_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
+}
+__device__ __forceinline__ void st_remote_u32(uint32_t cl_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cl_addr), "r"(v) : "memory");
+}
+// TMA tile load into this CTA's shared memory whose bytes complete the
+// barrier at shared::cluster address `bar` in either CTA of the pair.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+// Arrive on the barrier at shared address `bar` of both CTAs (mask 0b11) once
+// the MMAs issued before have completed.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+    const uint16_t both = 3;
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            bar),
+        "h"(both)
+        : "memory");
+}
+
+// wait_bounded for a CTA of a pair: a wait that gives up also raises the
+// other CTA's abort flag (at shared::cluster address peer_abort).
+__device__ bool wait_bounded_pair(uint32_t bar, uint32_t parity, Bars *bars, uint32_t peer_abort, int32_t *status,
+                                  uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = now_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15) == 0) {
+            if (*reinterpret_cast<volatile int *>(&bars->abort_flag)) return false;
+            if (now_ns() - t0 > limit_ns) {
+                *reinterpret_cast<volatile int *>(&bars->abort_flag) = 1;
+                st_remote_u32(peer_abort, 1u);
+                atomicExch(status, (int32_t)AQLM_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_bf16_tcgen05_pair(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                       __nv_bfloat16 *__restrict__ Y, int m_total, int n_total, int k_total, int32_t *status,
+                       unsigned long long limit_ns, int stall_test) {
+    using C = PairCfg<BN>;
+    constexpr int STAGES = C::STAGES, STAGE_BYTES = C::STAGE_BYTES;
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte alignment for the swizzled tiles (the same offsets in both CTAs)
+    const uint32_t raw = smem_addr(smem_raw);
+    uint8_t *smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
+    Bars *bars = reinterpret_cast<Bars *>(smem + (size_t)STAGES * STAGE_BYTES);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();           // 0: the leader, which issues the MMAs
+    const int pair_id = (int)cluster_id_x(), pairs = (int)cluster_count_x();
+    const int m_tiles = (m_total + kPairRows - 1) / kPairRows;
+    const int n_tiles = (n_total + BN - 1) / BN;
+    const int num_tiles = m_tiles * n_tiles;
+    const int num_kb = (k_total + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_addr(&bars->full[s]), 1);    // leader: its producer's arrival with both CTAs' bytes
+            mbar_init(smem_addr(&bars->empty[s]), 1);   // the leader's MMA commit
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_addr(&bars->tfull[a]), 1);
+            mbar_init(smem_addr(&bars->tempty[a]), 2 * kEpiWarps);   // leader: the epilogue warps of both CTAs
+        }
+        mbar_init(smem_addr(&bars->mma_done), 1);
+        bars->abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(&bars->tmem_base)),
+                     "r"(C::TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
+    // the barriers of both CTAs initialised before either CTA uses the other's
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    const uint32_t peer_abort = map_shared(smem_addr(&bars->abort_flag), rank ^ 1u);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---- TMA producer (both CTAs) ----
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued_parity[STAGES];
+            for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
+            bool ok = true;
+            for (int tile = pair_id; tile < num_tiles && ok && !stall_test; tile += pairs) {
+                const int mb = tile % m_tiles, nb = tile / m_tiles;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!wait_bounded_pair(smem_addr(&bars->empty[stage]), phase ^ 1, bars, peer_abort, status,
+                                           limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t full_local = smem_addr(&bars->full[stage]);
+                    const uint32_t full_leader = map_shared(full_local, 0);
+                    const uint32_t dst = smem_addr(smem + (size_t)stage * STAGE_BYTES);
+                    if (rank == 0) mbar_expect_tx(full_local, (uint32_t)(2 * STAGE_BYTES));
+                    tma_load_2d_pair(dst, &tmap_x, kb * BK, mb * kPairRows + (int)rank * BM, full_leader);
+                    tma_load_2d_pair(dst + A_BYTES, &tmap_w, kb * BK, nb * BN + (int)rank * C::B_HALF, full_leader);
+                    issued_parity[stage] = (int)phase;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            // Every stage released by the MMAs: the commits owed to this CTA's empty barriers have landed.
+            for (int s = 0; s < STAGES; ++s) {
+                if (!wait_bounded_pair(smem_addr(&bars->empty[stage]), phase ^ 1, bars, peer_abort, status, limit_ns))
+                    break;
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+            // The leader's full barriers count the copies of both CTAs: none may still be landing.
+            if (rank == 0) {
+                for (int s = 0; s < STAGES; ++s) {
+                    if (issued_parity[s] >= 0) {
+                        const uint32_t full = smem_addr(&bars->full[s]);
+                        const uint64_t t0 = now_ns();
+                        while (!mbar_try_wait(full, (uint32_t)issued_parity[s]) && now_ns() - t0 < limit_ns) {
+                        }
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            if (rank == 0) {
+                // ---- MMA issuer (leader) ----
+                int stage = 0;
+                uint32_t phase = 0;
+                int acc = 0;
+                uint32_t acc_phase = 0;
+                bool ok = true;
+                for (int tile = pair_id; tile < num_tiles && ok; tile += pairs) {
+                    if (!wait_bounded_pair(smem_addr(&bars->tempty[acc]), acc_phase ^ 1, bars, peer_abort, status,
+                                           limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem + (uint32_t)(acc * C::ACC_STRIDE);
+                    for (int kb = 0; kb < num_kb; ++kb) {
+                        if (!wait_bounded_pair(smem_addr(&bars->full[stage]), phase, bars, peer_abort, status,
+                                               limit_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t a0 = smem_addr(smem + (size_t)stage * STAGE_BYTES);
+                        const uint32_t b0 = a0 + A_BYTES;
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k) {
+                            mma_bf16_pair(d_tmem, sw128_desc(a0 + 32 * k), sw128_desc(b0 + 32 * k), C::IDESC,
+                                          (kb > 0 || k > 0) ? 1u : 0u);
+                        }
+                        mma_commit_pair(smem_addr(&bars->empty[stage]));
+                        if (++stage == STAGES) {
+                            stage = 0;
+                            phase ^= 1;
+                        }
+                    }
+                    if (!ok) break;
+                    mma_commit_pair(smem_addr(&bars->tfull[acc]));
+                    if (++acc == 2) {
+                        acc = 0;
+                        acc_phase ^= 1;
+                    }
+                }
+                mma_commit_pair(smem_addr(&bars->mma_done));
+                // Both accumulators released by the epilogues of both CTAs: the
+                // peer's arrivals on this CTA's tempty barriers have landed.
+                for (int a = 0; a < 2; ++a) {
+                    if (!wait_bounded_pair(smem_addr(&bars->tempty[acc]), acc_phase ^ 1, bars, peer_abort, status,
+                                           limit_ns))
+                        break;
+                    if (++acc == 2) {
+                        acc = 0;
+                        acc_phase ^= 1;
+                    }
+                }
+            }
+            // Tensor memory is freed below only after every issued MMA completed
+            // (the leader's last commit reaches both CTAs).
+            const uint64_t t0 = now_ns();
+            while (!mbar_try_wait(smem_addr(&bars->mma_done), 0) && now_ns() - t0 < limit_ns) {
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue (both CTAs): warps 2..5, TMEM lane quarter = warp % 4 ----
+        const int quarter = warp & 3;
+        const int row_in_tile = (int)rank * BM + quarter * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = pair_id; tile < num_tiles; tile += pairs) {
+            const int mb = tile % m_tiles, nb = tile / m_tiles;
+            bool ok = wait_bounded_pair(smem_addr(&bars->tfull[acc]), acc_phase, bars, peer_abort, status, limit_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            const int m = mb * kPairRows + row_in_tile;
+            const uint32_t t_base = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * C::ACC_STRIDE);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(t_base + (uint32_t)(c * 32), r);
+                const int n0 = nb * BN + c * 32;
+                if (m < m_total && AQLM_IN_BOUNDS(nb < n_tiles && mb < m_tiles, kSiteGemmY, (size_t)m * n_total + n0))
+                    store_bf16_row<4>(Y + (size_t)m * n_total + n0, r, n0, n_total);
+            }
+            if constexpr (BN % 32 != 0) {  // the last 16 columns of the tile
+                uint32_t r[16];
+                tmem_ld16(t_base + (uint32_t)(BN / 32 * 32), r);
+                const int n0 = nb * BN + BN / 32 * 32;
+                if (m < m_total && AQLM_IN_BOUNDS(nb < n_tiles && mb < m_tiles, kSiteGemmY, (size_t)m * n_total + n0))
+                    store_bf16_row<2>(Y + (size_t)m * n_total + n0, r, n0, n_total);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(map_shared(smem_addr(&bars->tempty[acc]), 0));
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1;
+            }
+        }
+    }
+
+    // Neither CTA leaves (or frees the pair's tensor memory) while the other
+    // may still read its shared memory or signal its barriers.
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    tc_fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS));
+    }
+}
+
 // ---- host side: tensor maps through the driver entry point ----
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -559,8 +890,6 @@ bool make_map(CUtensorMap *map, const void *base, int rows, int cols, int box_ro
 
 }  // namespace
 
-// Bound on any single wait of the GEMM (the whole GEMM takes well under this).
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 namespace {
 template <int BN, int FM, int FB>
@@ -623,10 +952,133 @@ cudaError_t launch_by_width(const uint16_t *X, const uint16_t *W, uint16_t *Y, i
 }
 }  // namespace
 
+namespace {
+// Pairs of SMs that can hold a CTA pair of the BN kernel at once (0 if the
+// device cannot), queried once per device.
+template <int BN>
+int pair_slots(int dev) {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> cached[kMaxDevices];
+    if (dev >= 0 && dev < kMaxDevices) {
+        const int c = cached[dev].load(std::memory_order_relaxed);
+        if (c != 0) return c > 0 ? c : 0;
+    }
+    using C = PairCfg<BN>;
+    auto fn = gemm_bf16_tcgen05_pair<BN>;
+    int count = 0;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM) == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * num_sms(dev));
+        cfg.blockDim = dim3(kGemmThreads);
+        cfg.dynamicSmemBytes = C::SMEM;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&count, fn, &cfg) != cudaSuccess) count = 0;
+    }
+    if (dev >= 0 && dev < kMaxDevices) cached[dev].store(count > 0 ? count : -1, std::memory_order_relaxed);
+    return count > 0 ? count : 0;
+}
+
+template <int BN>
+cudaError_t launch_gemm_pair_bn(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
+                                int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test,
+                                int dev) {
+    using C = PairCfg<BN>;
+    const int slots = pair_slots<BN>(dev);
+    if (slots < 1) return cudaErrorNotSupported;
+    CUtensorMap mx, mw;
+    if (!make_map(&mx, X, tokens, k, BM)) return cudaErrorInvalidValue;
+    if (!make_map(&mw, W, n, k, C::B_HALF)) return cudaErrorInvalidValue;
+    auto fn = gemm_bf16_tcgen05_pair<BN>;
+    const int tiles = ((tokens + kPairRows - 1) / kPairRows) * ((n + BN - 1) / BN);
+    const int pairs = tiles < slots ? tiles : slots;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fn, mx, mw, reinterpret_cast<__nv_bfloat16 *>(Y), tokens, n, k, status, limit_ns,
+                              stall_test);
+}
+}  // namespace
+
+// The tile width of the CTA-pair kernel for a tokens x n product on `pairs`
+// SM pairs: a pair tile costs its SMs MMA time in proportion to its width
+// (each SM computes 128 x width per k step), so the rule takes the least
+// waves x width, ties to the wider tile.
+int gemm_pair_tile_n(int tokens, int n, int pairs) {
+    constexpr int kCands[] = {256, 240, 224, 192};
+    const long long m_tiles = (tokens + kPairRows - 1) / kPairRows;
+    int best = kCands[0];
+    long long best_cost = -1;
+    for (int bn : kCands) {
+        const long long tiles = m_tiles * ((n + bn - 1) / bn);
+        const long long waves = (tiles + pairs - 1) / pairs;
+        const long long cost = waves * bn;
+        if (best_cost < 0 || cost < best_cost) {
+            best = bn;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
+// The pair kernel serves products of more than one 128-token tile.
+bool gemm_uses_pair(int tokens) { return tokens > BM; }
+
+cudaError_t launch_bf16_gemm_cfg(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
+                                 int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test,
+                                 int cta_pair, int tile_n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const bool pair = cta_pair < 0 ? gemm_uses_pair(tokens) : cta_pair != 0;
+    if (!pair) {
+        const DecodeArgs none = {};
+        if (tile_n == 0) return launch_by_width<0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, none);
+        const int sms = num_sms(dev);
+        switch (tile_n) {
+            case 256:
+                return launch_gemm_bn<256, 0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, none);
+            case 240:
+                return launch_gemm_bn<240, 0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, none);
+            case 224:
+                return launch_gemm_bn<224, 0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, none);
+            case 192:
+                return launch_gemm_bn<192, 0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, none);
+            default:
+                return cudaErrorInvalidValue;
+        }
+    }
+    if (tile_n == 0) tile_n = gemm_pair_tile_n(tokens, n, pair_slots<256>(dev) > 0 ? pair_slots<256>(dev) : 1);
+    switch (tile_n) {
+        case 256:
+            return launch_gemm_pair_bn<256>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, dev);
+        case 240:
+            return launch_gemm_pair_bn<240>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, dev);
+        case 224:
+            return launch_gemm_pair_bn<224>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, dev);
+        case 192:
+            return launch_gemm_pair_bn<192>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, dev);
+        default:
+            return cudaErrorInvalidValue;
+    }
+}
+
 cudaError_t launch_bf16_gemm_ex(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                                 int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test) {
-    const DecodeArgs none = {};
-    return launch_by_width<0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, none);
+    return launch_bf16_gemm_cfg(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, -1, 0);
 }
 
 // Prefill with the dequantisation fused into the GEMM (no W^ in global memory).
@@ -639,14 +1091,14 @@ cudaError_t launch_fused_gemm(const void *codes, const uint16_t *codebooks, cons
     da.scales = reinterpret_cast<const __half *>(scales);
     da.G = d.G;
     da.row_bytes = d.row_bytes;
-    if (d.M == 1) return launch_by_width<1, 16>(X, nullptr, Y, tokens, d.d_out, d.d_in, status, st, kWaitLimitNs, 0, da);
-    if (d.B == 8) return launch_by_width<2, 8>(X, nullptr, Y, tokens, d.d_out, d.d_in, status, st, kWaitLimitNs, 0, da);
-    return launch_by_width<2, 16>(X, nullptr, Y, tokens, d.d_out, d.d_in, status, st, kWaitLimitNs, 0, da);
+    if (d.M == 1) return launch_by_width<1, 16>(X, nullptr, Y, tokens, d.d_out, d.d_in, status, st, kGemmWaitLimitNs, 0, da);
+    if (d.B == 8) return launch_by_width<2, 8>(X, nullptr, Y, tokens, d.d_out, d.d_in, status, st, kGemmWaitLimitNs, 0, da);
+    return launch_by_width<2, 16>(X, nullptr, Y, tokens, d.d_out, d.d_in, status, st, kGemmWaitLimitNs, 0, da);
 }
 
 cudaError_t launch_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                              int32_t *status, cudaStream_t st) {
-    return launch_bf16_gemm_ex(X, W, Y, tokens, n, k, status, st, kWaitLimitNs, 0);
+    return launch_bf16_gemm_ex(X, W, Y, tokens, n, k, status, st, kGemmWaitLimitNs, 0);
 }
 
 AQLM_DEFINE_BOUNDS_READER(bounds_word_gemm)

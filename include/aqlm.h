@@ -302,6 +302,37 @@ AQLM_API aqlm_status aqlm_bf16_gemm(const uint16_t *X, const uint16_t *W, uint16
 AQLM_API int32_t aqlm_bf16_gemm_tile_n(int32_t tokens, int32_t n, int32_t sms);
 
 /*
+ * aqlm_bf16_gemm_plan -- the kernel aqlm_bf16_gemm and aqlm_gemm choose for
+ * `tokens` x `n` on a device with `sms` streaming multiprocessors, written to
+ * *cta_pair and *tile_n.  More than 128 tokens: the CTA-pair kernel
+ * (*cta_pair = 1; one MMA of 256 x tile_n on the tensor cores of two SMs, a
+ * cluster of two CTAs), whose width is the one with the least waves x width
+ * over sms / 2 pairs, ties to the wider.  Otherwise the single-CTA kernel
+ * (*cta_pair = 0) with the width of aqlm_bf16_gemm_tile_n.  The launch uses
+ * the pair count the device reports for the kernel, which on a device whose
+ * SMs all pair up is sms / 2.  Host only.  Errors: AQLM_ERR_INVALID_ARG
+ * (null pointer, tokens or n below 1, sms below 2; both outputs then 0).
+ */
+AQLM_API aqlm_status aqlm_bf16_gemm_plan(int32_t tokens, int32_t n, int32_t sms, int32_t *cta_pair,
+                                         int32_t *tile_n);
+
+/*
+ * aqlm_bf16_gemm_config -- aqlm_bf16_gemm with the kernel chosen by the
+ * caller, for measurements and tests of each variant: cta_pair 1 = the
+ * CTA-pair kernel (256-token tiles), 0 = the single-CTA kernel (128-token
+ * tiles), -1 = the rule of aqlm_bf16_gemm_plan; tile_n one of 256, 240, 224,
+ * 192, or 0 for the rule's width.  Every variant computes the same products
+ * with the same fp32 accumulation order within a tile column (16 k values
+ * per MMA step, k steps in order), so the results agree bit for bit.
+ * Arguments and errors as aqlm_bf16_gemm, plus AQLM_ERR_INVALID_ARG for
+ * another cta_pair or tile_n, and AQLM_ERR_CUDA when the device cannot
+ * hold a CTA pair.
+ */
+AQLM_API aqlm_status aqlm_bf16_gemm_config(const uint16_t *X, const uint16_t *W, uint16_t *Y, int32_t tokens,
+                                           int32_t n, int32_t k, int32_t *status, int32_t cta_pair,
+                                           int32_t tile_n, aqlm_stream_t stream);
+
+/*
  * aqlm_decode_indices -- the code unpacking step on its own, for bit-exact
  * checks: idx_out[(i*G + j)*M + m] = index of codebook m for group j of row
  * i, as uint16 (G = d_in/8).  idx_out: d_out*G*M uint16, 2-byte aligned.
@@ -316,10 +347,14 @@ AQLM_API aqlm_status aqlm_decode_indices(const void *codes, uint16_t *idx_out, a
  * the kernel of aqlm_bf16_gemm with its loads withheld, so that the first
  * bounded wait runs out after `limit_ns` nanoseconds (1 ns .. 1 s).  The
  * kernel must then write AQLM_ERR_TIMEOUT to *status, free its tensor
- * memory and return; nothing faults or hangs.  Arguments as aqlm_bf16_gemm.
+ * memory and return; nothing faults or hangs.  cta_pair selects the kernel
+ * as in aqlm_bf16_gemm_config (with the CTA pair, the timeout of the
+ * leader's wait also ends the other CTA's waits).  Other arguments as
+ * aqlm_bf16_gemm.
  */
 AQLM_API aqlm_status aqlm_test_gemm_timeout(const uint16_t *X, const uint16_t *W, uint16_t *Y, int32_t tokens, int32_t n,
-                                   int32_t k, int32_t *status, uint64_t limit_ns, aqlm_stream_t stream);
+                                   int32_t k, int32_t *status, uint64_t limit_ns, int32_t cta_pair,
+                                   aqlm_stream_t stream);
 
 /*
  * aqlm_gemv_noalloc -- aqlm_gemv without a caller-provided workspace, for

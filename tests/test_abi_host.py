@@ -143,6 +143,11 @@ def test_gemm_argument_errors():
     assert lib.aqlm_bf16_gemm(A16, B16, C16, 16, 100, 64, D16, NULL) == ac.AQLM_ERR_UNSUPPORTED
     assert lib.aqlm_bf16_gemm(A16, B16, C16, 16, 128, 64, NULL, NULL) == ac.AQLM_ERR_INVALID_ARG
     assert lib.aqlm_gemm_check(NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
+    # the variant chooser: unknown kernels and widths are refused before any launch
+    for pair, width in ((2, 0), (-2, 0), (1, 128), (0, 250), (0, 512)):
+        assert lib.aqlm_bf16_gemm_config(A16, B16, C16, 256, 128, 64, D16, pair, width, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_bf16_gemm_config(A16, B16, C16, 256, 100, 64, D16, 1, 0, NULL) == ac.AQLM_ERR_UNSUPPORTED
+    assert lib.aqlm_bf16_gemm_config(ODD, B16, C16, 256, 128, 64, D16, 1, 0, NULL) == ac.AQLM_ERR_MISALIGNED
 
 
 def test_dequant_and_decode_argument_errors():
@@ -152,7 +157,8 @@ def test_dequant_and_decode_argument_errors():
     assert lib.aqlm_dequant(A16, B16, C16, ODD, s, NULL) == ac.AQLM_ERR_MISALIGNED
     assert lib.aqlm_decode_indices(NULL, A16, s, NULL) == ac.AQLM_ERR_INVALID_ARG
     assert lib.aqlm_decode_indices(A16, ctypes.c_void_p(0x10001), s, NULL) == ac.AQLM_ERR_MISALIGNED
-    assert lib.aqlm_test_gemm_timeout(A16, B16, C16, 16, 128, 64, D16, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_test_gemm_timeout(A16, B16, C16, 16, 128, 64, D16, 0, 0, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_test_gemm_timeout(A16, B16, C16, 16, 128, 64, D16, 1000, 2, NULL) == ac.AQLM_ERR_INVALID_ARG
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
@@ -279,6 +285,35 @@ def test_gemm_tile_width_rule():
                 assert ac.bf16_gemm_tile_n(tokens, n, sms) == rule(tokens, n, sms)
     assert [ac.bf16_gemm_tile_n(2048, n, 148) for n in (11008, 4096, 8192, 28672)] == [240, 240, 224, 240]
     assert ac.bf16_gemm_tile_n(0, 8, 148) == 0 and ac.bf16_gemm_tile_n(8, 8, 0) == 0
+
+
+def test_gemm_plan_rule():
+    """The GEMM kernel choice: the CTA pair past 128 tokens, with the least
+    waves x width over sms / 2 pairs of 256-token tiles (ties to the wider),
+    the single-CTA kernel and its own rule up to 128 tokens; checked against
+    the rule restated here over a grid of shapes."""
+    def pair_rule(tokens, n, pairs):
+        best = None
+        for bn in (256, 240, 224, 192):
+            tiles = -(-tokens // 256) * -(-n // bn)
+            cost = -(-tiles // pairs) * bn
+            if best is None or cost < best[0]:
+                best = (cost, bn)
+        return best[1]
+    for tokens in (1, 128, 129, 300, 1000, 2048, 4096):
+        for n in (8, 256, 1000, 4096, 4608, 8192, 11008, 28672):
+            for sms in (2, 132, 148):
+                pair, width = ac.bf16_gemm_plan(tokens, n, sms)
+                if tokens <= 128:
+                    assert (pair, width) == (0, ac.bf16_gemm_tile_n(tokens, n, sms))
+                else:
+                    assert (pair, width) == (1, pair_rule(tokens, n, sms // 2))
+    assert [ac.bf16_gemm_plan(2048, n, 148) for n in (11008, 4096, 8192, 28672)] == [(1, 240), (1, 240), (1, 224), (1, 240)]
+    lib = ac.load_library()
+    p, w = ctypes.c_int32(7), ctypes.c_int32(7)
+    assert lib.aqlm_bf16_gemm_plan(2048, 4096, 1, ctypes.byref(p), ctypes.byref(w)) == ac.AQLM_ERR_INVALID_ARG
+    assert (p.value, w.value) == (0, 0)
+    assert lib.aqlm_bf16_gemm_plan(2048, 4096, 148, None, ctypes.byref(w)) == ac.AQLM_ERR_INVALID_ARG
 
 
 def test_debug_bounds_entry_points_in_the_product_build():

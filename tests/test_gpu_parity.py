@@ -311,22 +311,49 @@ TILE_WIDTH_CASES = [(1000, 4608, 1032, 256), (2040, 4096, 520, 240), (1530, 4864
 
 @pytest.mark.parametrize("tokens,n,k,width", TILE_WIDTH_CASES, ids=[f"BN{c[3]}" for c in TILE_WIDTH_CASES])
 def test_bf16_gemm_every_tile_width(tokens, n, k, width):
-    """Each instantiation of the tile width (128x256, 128x240, 128x224,
-    128x192 output tiles) against torch (fp32 accumulation), including the
-    partial last column tile and the 16-column remainder of the 240 / 224
-    epilogue."""
+    """Each instantiation of the tile width of the single-CTA kernel (128x256,
+    128x240, 128x224, 128x192 output tiles) against torch (fp32
+    accumulation), including the partial last column tile and the 16-column
+    remainder of the 240 / 224 epilogue."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     if sms == 148:
         assert ac.bf16_gemm_tile_n(tokens, n, sms) == width
     g = torch.Generator(device="cpu").manual_seed(tokens + n + k)
     X = (torch.randn(tokens, k, generator=g) / 4).to(torch.bfloat16).to(DEV)
     W = (torch.randn(n, k, generator=g) / 4).to(torch.bfloat16).to(DEV)
-    Y, status = ac.aqlm_bf16_gemm(X, W)
+    Y, status = ac.aqlm_bf16_gemm_config(X, W, 0, 0)
     assert int(status.item()) == 0
     ref = X.float() @ W.float().T
     absdot = X.float().abs() @ W.float().abs().T
     err = (Y.float() - ref).abs()
     assert bool(torch.all(err <= 2.0 ** -8 * ref.abs() + 2.0 ** -14 * absdot + 1e-6))
+
+
+# (tokens, n, k): one pair tile; ragged tokens (the second CTA's rows partly
+# and wholly past the end), n and k; a long k loop
+PAIR_CASES = [(256, 256, 64), (200, 520, 576), (130, 264, 1032), (1000, 4608, 1032), (300, 1000, 4104),
+              (2040, 4096, 520), (384, 512, 16384)]
+
+
+@pytest.mark.parametrize("width", [256, 240, 224, 192])
+@pytest.mark.parametrize("tokens,n,k", PAIR_CASES, ids=[f"{t}x{n}x{k}" for t, n, k in PAIR_CASES])
+def test_bf16_gemm_cta_pair_every_width(tokens, n, k, width):
+    """The CTA-pair kernel (256 x width tiles, one MMA on the tensor cores of
+    two SMs) at each width: against torch (fp32 accumulation), and bit for
+    bit against the single-CTA kernel at the same width (the same MMA k
+    steps in the same order for every output element)."""
+    g = torch.Generator(device="cpu").manual_seed(3 * tokens + n + k)
+    X = (torch.randn(tokens, k, generator=g) / 4).to(torch.bfloat16).to(DEV)
+    W = (torch.randn(n, k, generator=g) / 4).to(torch.bfloat16).to(DEV)
+    Y, status = ac.aqlm_bf16_gemm_config(X, W, 1, width)
+    Y1, status1 = ac.aqlm_bf16_gemm_config(X, W, 0, width)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0 and int(status1.item()) == 0
+    ref = X.float() @ W.float().T
+    absdot = X.float().abs() @ W.float().abs().T
+    err = (Y.float() - ref).abs()
+    assert bool(torch.all(err <= 2.0 ** -8 * ref.abs() + 2.0 ** -14 * absdot + 1e-6))
+    assert torch.equal(Y.view(torch.int16), Y1.view(torch.int16))
 
 
 def test_bf16_gemm_matches_torch():
@@ -415,19 +442,22 @@ def test_gemm_fused_full_size_sampled_tokens(d_out, d_in, M, B):
     _gemm_check(bf16_to_np_bits(Y), L, spec, L["x"], tokens_idx=toks)
 
 
-def test_gemm_bounded_wait_reports_timeout():
+@pytest.mark.parametrize("cta_pair", [0, 1], ids=["single", "pair"])
+def test_gemm_bounded_wait_reports_timeout(cta_pair):
     """Loads withheld on purpose: the first wait runs out, the kernel records
-    AQLM_ERR_TIMEOUT, frees its tensor memory and returns; the context stays usable."""
-    X = torch.zeros(128, 64, dtype=torch.bfloat16, device=DEV)
+    AQLM_ERR_TIMEOUT, frees its tensor memory and returns (with the CTA pair,
+    the other CTA's waits end on the abort flag the leader raises in it); the
+    context stays usable."""
+    X = torch.zeros(256, 64, dtype=torch.bfloat16, device=DEV)
     W = torch.zeros(256, 64, dtype=torch.bfloat16, device=DEV)
-    Y = torch.empty(128, 256, dtype=torch.bfloat16, device=DEV)
+    Y = torch.empty(256, 256, dtype=torch.bfloat16, device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
-    assert ac.aqlm_test_gemm_timeout(X, W, Y, status, 20_000_000) == ac.AQLM_OK
+    assert ac.aqlm_test_gemm_timeout(X, W, Y, status, 20_000_000, cta_pair) == ac.AQLM_OK
     torch.cuda.synchronize()
     assert int(status.item()) == ac.AQLM_ERR_TIMEOUT
     # the device still works, and a normal GEMM afterwards is correct
-    Y2, st2 = ac.aqlm_bf16_gemm(torch.ones(128, 64, dtype=torch.bfloat16, device=DEV),
-                                torch.ones(256, 64, dtype=torch.bfloat16, device=DEV))
+    Y2, st2 = ac.aqlm_bf16_gemm_config(torch.ones(256, 64, dtype=torch.bfloat16, device=DEV),
+                                       torch.ones(256, 64, dtype=torch.bfloat16, device=DEV), cta_pair, 0)
     torch.cuda.synchronize()
     assert int(st2.item()) == 0 and torch.all(Y2.float() == 64.0)
 
