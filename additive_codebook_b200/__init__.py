@@ -33,7 +33,7 @@ GEMV_MAX_TOKENS = 16
 # Every entry point declared in include/aqlm.h.
 EXPORTS = ["aqlm_gemv", "aqlm_gemv_workspace_bytes", "aqlm_gemv_row_tokens", "aqlm_gemv_multi",
            "aqlm_gemv_multi_workspace_bytes", "aqlm_gemv_multi_check", "aqlm_gemv_check", "aqlm_dequant", "aqlm_gemm",
-           "aqlm_gemm_workspace_bytes", "aqlm_gemm_check", "aqlm_bf16_gemm", "aqlm_bf16_gemm_tile_n", "aqlm_bf16_gemm_plan", "aqlm_bf16_gemm_config", "aqlm_decode_indices",
+           "aqlm_gemm_workspace_bytes", "aqlm_gemm_check", "aqlm_gemm_overlap", "aqlm_bf16_gemm", "aqlm_bf16_gemm_tile_n", "aqlm_bf16_gemm_plan", "aqlm_bf16_gemm_config", "aqlm_decode_indices",
            "aqlm_test_gemm_timeout", "aqlm_gemv_noalloc", "aqlm_gemv_noalloc_max_scratch_bytes",
            "aqlm_gemv_noalloc_check", "aqlm_test_gemv_noalloc_set_status", "aqlm_probe_gather_sink_bytes",
            "aqlm_probe_gather", "aqlm_gemv_lut", "aqlm_gemv_lut_workspace_bytes", "aqlm_gemm_fused",
@@ -116,6 +116,7 @@ def _open(path, how):
         "aqlm_gemv_lut": ([vp, vp, vp, vp, vp, Shape, vp, sz, vp], st),
         "aqlm_gemv_lut_workspace_bytes": ([Shape], sz),
         "aqlm_gemm_fused": ([vp, vp, vp, vp, vp, i32, Shape, vp, sz, vp], st),
+        "aqlm_gemm_overlap": ([vp, vp, vp, vp, vp, i32, Shape, vp, sz, vp], st),
         "aqlm_gemm_fused_workspace_bytes": ([Shape, i32], sz),
         "aqlm_debug_bounds_read": ([ctypes.POINTER(u64), i32], st),
         "aqlm_test_debug_bounds_trip": ([u64, vp], st),
@@ -360,7 +361,8 @@ def aqlm_dequant(codes, codebooks, scales, out=None, stream=None):
 
 
 def aqlm_gemm(codes, codebooks, scales, X, Y=None, workspace=None, stream=None):
-    """Y[T, d_out] = bf16(X . W^T): dequant into the workspace + tcgen05 GEMM."""
+    """Y[T, d_out] = bf16(X . W^T): aqlm_dequant into the workspace (W^ in its
+    last 2 * d_out * d_in bytes), then the tcgen05 GEMM."""
     lib = load_library()
     shape = shape_of(codes)
     T = X.shape[0]
@@ -370,6 +372,21 @@ def aqlm_gemm(codes, codebooks, scales, X, Y=None, workspace=None, stream=None):
         workspace = torch.empty(lib.aqlm_gemm_workspace_bytes(shape, T), dtype=torch.uint8, device=X.device)
     _check(lib.aqlm_gemm(_p(codes), _p(codebooks), _p(_flat_scales(scales)), _p(X), _p(Y), T, shape,
                          _p(workspace), workspace.numel(), _stream(stream)), "aqlm_gemm")
+    return Y, workspace
+
+
+def aqlm_gemm_overlap(codes, codebooks, scales, X, Y=None, workspace=None, stream=None):
+    """aqlm_gemm in one kernel: W^ decoded into the workspace by the GEMM's own
+    decoder warps, overlapped with the MMAs."""
+    lib = load_library()
+    shape = shape_of(codes)
+    T = X.shape[0]
+    if Y is None:
+        Y = torch.empty((T, shape.d_out), dtype=torch.bfloat16, device=X.device)
+    if workspace is None:
+        workspace = torch.empty(lib.aqlm_gemm_workspace_bytes(shape, T), dtype=torch.uint8, device=X.device)
+    _check(lib.aqlm_gemm_overlap(_p(codes), _p(codebooks), _p(_flat_scales(scales)), _p(X), _p(Y), T, shape,
+                                 _p(workspace), workspace.numel(), _stream(stream)), "aqlm_gemm_overlap")
     return Y, workspace
 
 

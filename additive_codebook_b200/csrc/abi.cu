@@ -10,7 +10,9 @@ cudaError_t launch_bf16_gemm_ex(const uint16_t *X, const uint16_t *W, uint16_t *
                                 int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test);
 cudaError_t launch_bf16_gemm_cfg(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                                  int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test,
-                                 int cta_pair, int tile_n);
+                                 int cta_pair, int tile_n, bool pdl);
+cudaError_t launch_bf16_gemm_after_dequant(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n,
+                                          int k, int32_t *status, cudaStream_t st);
 cudaError_t launch_fused_gemm(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
                               const uint16_t *X, uint16_t *Y, int tokens, const Dims &d, int32_t *status,
                               cudaStream_t st);
@@ -217,7 +219,7 @@ aqlm_status aqlm_gemv_check(aqlm_shape shape, int32_t tokens, void *workspace, s
 
 size_t aqlm_gemm_workspace_bytes(aqlm_shape shape, int32_t tokens) {
     if (check_shape(shape) != AQLM_OK || tokens < 1) return 0;
-    return kStatusBytes + (size_t)shape.d_out * shape.d_in * 2;
+    return kStatusBytes + aqlm::overlap_counter_bytes(shape.d_out, shape.d_in) + (size_t)shape.d_out * shape.d_in * 2;
 }
 
 aqlm_status aqlm_gemm(const void *codes, const uint16_t *codebooks, const uint16_t *scales, const uint16_t *X,
@@ -232,12 +234,33 @@ aqlm_status aqlm_gemm(const void *codes, const uint16_t *codebooks, const uint16
     if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return AQLM_ERR_WORKSPACE;
     const cudaStream_t cs = to_cuda(stream);
     int32_t *status = static_cast<int32_t *>(workspace);
-    uint16_t *W = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(workspace) + kStatusBytes);
+    uint8_t *counters = static_cast<uint8_t *>(workspace) + kStatusBytes;
+    uint16_t *W = reinterpret_cast<uint16_t *>(counters + aqlm::overlap_counter_bytes(shape.d_out, shape.d_in));
+    (void)counters;   // used by aqlm_gemm_overlap only
     cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), cs);
     if (e != cudaSuccess) return AQLM_ERR_CUDA;
     e = aqlm::launch_dequant(codes, codebooks, scales, W, aqlm::make_dims(shape), cs);
     if (e != cudaSuccess) return AQLM_ERR_CUDA;
-    return from_cuda(aqlm::launch_bf16_gemm(X, W, Y, tokens, shape.d_out, shape.d_in, status, cs));
+    return from_cuda(aqlm::launch_bf16_gemm_after_dequant(X, W, Y, tokens, shape.d_out, shape.d_in, status, cs));
+}
+
+aqlm_status aqlm_gemm_overlap(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                              const uint16_t *X, uint16_t *Y, int32_t tokens, aqlm_shape shape, void *workspace,
+                              size_t workspace_bytes, aqlm_stream_t stream) {
+    aqlm_status st = check_layer(codes, codebooks, scales, shape);
+    if (st != AQLM_OK) return st;
+    if (!X || !Y || tokens < 1) return AQLM_ERR_INVALID_ARG;
+    if (shape.d_out % 8) return AQLM_ERR_UNSUPPORTED;
+    if (!aligned(X, 16) || !aligned(Y, 16)) return AQLM_ERR_MISALIGNED;
+    const size_t need = aqlm_gemm_workspace_bytes(shape, tokens);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return AQLM_ERR_WORKSPACE;
+    const cudaStream_t cs = to_cuda(stream);
+    int32_t *status = static_cast<int32_t *>(workspace);
+    uint8_t *counters = static_cast<uint8_t *>(workspace) + kStatusBytes;
+    uint16_t *W = reinterpret_cast<uint16_t *>(counters + aqlm::overlap_counter_bytes(shape.d_out, shape.d_in));
+    if (cudaMemsetAsync(status, 0, sizeof(int32_t), cs) != cudaSuccess) return AQLM_ERR_CUDA;
+    return from_cuda(aqlm::launch_overlap_gemm(codes, codebooks, scales, X, W, Y, tokens, aqlm::make_dims(shape),
+                                               status, counters, cs));
 }
 
 size_t aqlm_gemm_fused_workspace_bytes(aqlm_shape shape, int32_t tokens) {
@@ -312,7 +335,7 @@ aqlm_status aqlm_bf16_gemm_config(const uint16_t *X, const uint16_t *W, uint16_t
     if (n % 8 || k % 8) return AQLM_ERR_UNSUPPORTED;
     if (!aligned(X, 16) || !aligned(W, 16) || !aligned(Y, 16) || !aligned(status, 4)) return AQLM_ERR_MISALIGNED;
     return from_cuda(aqlm::launch_bf16_gemm_cfg(X, W, Y, tokens, n, k, status, to_cuda(stream),
-                                                aqlm::kGemmWaitLimitNs, 0, cta_pair, tile_n));
+                                                aqlm::kGemmWaitLimitNs, 0, cta_pair, tile_n, false));
 }
 
 aqlm_status aqlm_test_gemm_timeout(const uint16_t *X, const uint16_t *W, uint16_t *Y, int32_t tokens, int32_t n,
@@ -322,7 +345,7 @@ aqlm_status aqlm_test_gemm_timeout(const uint16_t *X, const uint16_t *W, uint16_
     if (limit_ns == 0 || limit_ns > 1000000000ull || cta_pair < -1 || cta_pair > 1) return AQLM_ERR_INVALID_ARG;
     if (!aligned(X, 16) || !aligned(W, 16) || !aligned(Y, 16) || !aligned(status, 4)) return AQLM_ERR_MISALIGNED;
     return from_cuda(aqlm::launch_bf16_gemm_cfg(X, W, Y, tokens, n, k, status, to_cuda(stream), limit_ns, 1,
-                                                cta_pair, 0));
+                                                cta_pair, 0, false));
 }
 
 // ---- encoding ----

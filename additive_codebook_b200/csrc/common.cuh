@@ -326,6 +326,10 @@ constexpr unsigned long long kGemmWaitLimitNs = 2000000000ull;
 int gemm_tile_n(int tokens, int n, int sms);
 int gemm_pair_tile_n(int tokens, int n, int pairs);
 bool gemm_uses_pair(int tokens);
+size_t overlap_counter_bytes(int d_out, int d_in);
+cudaError_t launch_overlap_gemm(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                                const uint16_t *X, uint16_t *W, uint16_t *Y, int tokens, const Dims &d,
+                                int32_t *status, void *counters, cudaStream_t st);
 // encoding (encode.cu)
 cudaError_t launch_encode_scales(const float *W, int d_out, int d_in, uint16_t *scales, float *V, cudaStream_t st);
 size_t nearest_workspace_bytes(long long N);

@@ -105,6 +105,9 @@ __global__ void __launch_bounds__(256, 3) dequant_kernel(const uint8_t *__restri
                                                       const __half *__restrict__ scales,
                                                       uint4 *__restrict__ W, const RowDivider rd, int64_t n_groups) {
     constexpr int K = 1 << B;
+    // the GEMM that reads W^ may launch now: its CTAs fit beside these, set up
+    // their barriers and tensor memory, and wait for this grid before loading
+    grid_dep_launch();
     // 2x8: both codebooks (2 x 256 codewords x 16 B = 8 KiB) live in shared memory.
     __shared__ uint4 cb_smem[B == 8 ? M * K : 1];
     if constexpr (B == 8) {

@@ -291,6 +291,7 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
     if (warp == 0) {
         if (lane == 0 && !stall_test) {
             // ---- TMA producer ----
+            grid_dep_wait();   // launched early after the kernel writing W (a no-op otherwise)
             int stage = 0;
             uint32_t phase = 0;
             int issued_parity[STAGES];
@@ -550,21 +551,24 @@ gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
 // leaves while the other may still touch its shared or tensor memory.
 constexpr int kPairRows = 2 * BM;   // output rows of a pair tile
 
-template <int BN>
+// RESERVE: shared memory the decoder warps keep for 8-bit codebooks.
+template <int BN, int RESERVE = 0>
 struct PairCfg {
     static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "MMA N for M = 256");
     static constexpr int B_HALF = BN / 2;                   // rows of W each CTA stages (a multiple of 8)
     static constexpr int B_BYTES = B_HALF * BK * 2;         // a multiple of 1024: stages stay aligned
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES = 200 * 1024 / STAGE_BYTES < kMaxStages ? 200 * 1024 / STAGE_BYTES : kMaxStages;
+    static constexpr int BUDGET = 216 * 1024 - RESERVE;   // of the 227 KiB a CTA may hold
+    static constexpr int STAGES = BUDGET / STAGE_BYTES < kMaxStages ? BUDGET / STAGE_BYTES : kMaxStages;
     static constexpr int ACC_STRIDE = BN <= 128 ? 128 : 256;
     static constexpr uint32_t TMEM_COLS = 2 * ACC_STRIDE;
     // as GemmCfg::IDESC with M = 256
     static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                       ((uint32_t)(kPairRows >> 4) << 24);
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Bars) + 16;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Bars) + 16 + RESERVE;
     static_assert(B_BYTES % 1024 == 0 && STAGES >= 2, "ring layout");
 };
+
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
@@ -642,18 +646,424 @@ __device__ bool wait_bounded_pair(uint32_t bar, uint32_t parity, Bars *bars, uin
     }
 }
 
-template <int BN>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+// ---- overlapped dequantisation: W^ decoded once, in the order the MMAs need it
+// With FM > 0 the pair kernel also decodes the layer: eight decoder warps per
+// CTA turn codes into W^ rows in global memory (the workspace), with the
+// binary32 steps of aqlm_dequant, while the tensor cores run; each CTA's TMA
+// producer loads a W tile only once the units that write it are complete.
+// The work is cut into units of 16 rows x 64 inputs (one k block of a 16-row
+// slice of a band of BN rows).  Units are numbered in the order the tiles
+// need them -- bands in groups of about one wave's worth (GB bands, whose
+// first tiles fall in the same wave), k blocks in order within a group -- and
+// decoder warps claim the next ones from global counters, so the whole GPU
+// decodes what the first wave needs first, and no CTA ever waits for a CTA
+// that is not running (whoever claims a unit is running and finishes it).
+// Claims (U consecutive units) are dealt over kClaimStreams counters: decoder
+// warp w of a CTA takes claims w, w + 8, w + 16, ... from counter w, which
+// keeps the need order while spreading the atomics over eight L2 lines.  A finished unit adds 1 to its panel's counter
+// (release, GPU scope, after a proxy fence that orders the generic stores
+// before asynchronous-proxy reads); the producer reads the counters of 8 k
+// blocks at a time and loads when a panel holds all BN/16 of its units.
+// Division of x < 2^31 by an invariant d as a multiply and a shift (the
+// scheme of Granlund and Montgomery, "Division by invariant integers using
+// multiplication", 1994): s = ceil(log2 d), m = floor(2^(31+s) / d) + 1 < 2^32,
+// x / d = floor(x m / 2^(31+s)).
+struct FastDiv {
+    uint32_t d, m;
+    int shift;
+    __device__ __forceinline__ uint32_t div(uint32_t x) const { return (uint32_t)(((uint64_t)x * m) >> shift); }
+};
+inline FastDiv make_fast_div(uint32_t d) {
+    int s = 0;
+    while ((1ull << s) < d) ++s;
+    FastDiv f;
+    f.d = d;
+    f.m = (uint32_t)((1ull << (31 + s)) / d + 1);
+    f.shift = 31 + s;
+    return f;
+}
+
+constexpr int kClaimStreams = 8;   // = the decoder warps of a CTA
+constexpr int kClaimBytes = 128 * kClaimStreams;
+static_assert(kClaimStreams == kDecWarps, "one claim stream per decoder warp");
+
+struct OverlapArgs {
+    const uint8_t *codes;       // [d_out][G] groups of M*B/8 bytes
+    const uint4 *codebooks;     // [M][2^B] codewords of 8 fp16
+    const __half *scales;       // [d_out]
+    uint4 *W;                   // W^ [d_out][d_in] bf16, 8 per uint4 (G per row)
+    uint32_t *next_claim;       // kClaimStreams claim counters, 128 bytes apart, zero at launch
+    uint32_t *panel_done;       // [n_bands][kb_pad] finished units, zero at launch
+    int d_out, G, row_bytes;
+    int n_bands, num_kb, kb_pad, GB;
+    uint32_t total_units;       // n_bands * (BN / 16) * num_kb (< 2^31)
+    FastDiv per_group;          // units of a group of GB bands
+    FastDiv per_kb, per_kb_last;   // units of one k block of a full group, of the last group
+};
+
+// Decoder warps hand their finished units to one publisher warp of the CTA
+// through shared memory (a ring of kMailSlots per decoder warp, written with
+// CTA-scope release), so that no decoder warp ever waits for a GPU-scope
+// fence -- which would drain its loads and gathers in flight.  The publisher,
+// with no memory traffic of its own, reads the rings (acquire, CTA scope),
+// issues one fence.acq_rel.gpu for everything it read and then adds the
+// units to their panel counters: the decoders' stores happen before the
+// fence (CTA-scope release/acquire), so every SM that sees a count also
+// sees the stores.
+constexpr int kMailSlots = 32;
+struct Mailbox {
+    uint32_t head[kDecWarps];                 // entries written by decoder warp w
+    uint32_t tail[kDecWarps];                 // entries of warp w the publisher has counted
+    uint32_t finished[kDecWarps];             // decoder warp w is done
+    uint32_t entry[kDecWarps][kMailSlots];    // packed units
+};
+constexpr int kMailBytes = (int)((sizeof(Mailbox) + 127) / 128 * 128);
+constexpr int kOverlapThreads = kGemmThreads + kDecThreads + 32;   // + the publisher warp
+
+template <int FM, int FB>
+constexpr int overlap_reserve() {
+    return FM > 0 ? (FB == 8 ? FM * 256 * 16 : 0) + kMailBytes : 0;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_shared(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_shared(uint32_t *p, uint32_t v) {
+    asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_addr(p)), "r"(v) : "memory");
+}
+
+// Unit u in need order -> band nb, k block kb and 16-row slice r of the band.
+template <int CHUNKS>
+__device__ __forceinline__ bool unit_coords(uint32_t u, const OverlapArgs &oa, int &nb, int &kb, int &r) {
+    if (u >= oa.total_units) return false;
+    const uint32_t g = oa.per_group.div(u);
+    const uint32_t rem = u - g * oa.per_group.d;
+    const int b_lo = (int)g * oa.GB;
+    const FastDiv &fk = oa.n_bands - b_lo < oa.GB ? oa.per_kb_last : oa.per_kb;
+    kb = (int)fk.div(rem);
+    const uint32_t rem2 = rem - (uint32_t)kb * fk.d;
+    nb = b_lo + (int)(rem2 / CHUNKS);
+    r = (int)(rem2 % CHUNKS);
+    return true;
+}
+
+__device__ __forceinline__ void red_relaxed_add(uint32_t *p, uint32_t v) {
+    asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint4 ld_relaxed_u4(const uint32_t *p) {
+    uint4 v;
+    asm volatile("ld.relaxed.gpu.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+
+// A claimed unit packed in one word: band << 18 | k block << 4 | slice
+// (0xffffffff: no unit, past the last one).
+__device__ __forceinline__ uint32_t pack_unit(int nb, int kb, int r) {
+    return ((uint32_t)nb << 18) | ((uint32_t)kb << 4) | (uint32_t)r;
+}
+
+// The decoder warps' loop.  A claim is U consecutive units; lane l of a
+// unit's step s (0..3) handles row 4 s + l / 8 of the 16-row slice and group
+// l % 8 of the k block, so each 16-byte store of the warp fills four 128-byte
+// lines.  Three claims are in flight at once, one phase apart: the codes of
+// the newest are loading, the codewords of the next are being gathered, and
+// the oldest is converted, stored and counted -- so a phase waits for one
+// memory latency, whose loads, gathers and stores overlap; the ticket of the
+// next claim (a global atomic) is taken one phase before it is used.
+template <int BN, int FM, int FB>
+__device__ void decode_units(const OverlapArgs &oa, const uint4 *cbs, Mailbox *mbx, int stream, int lane,
+                             int32_t *status, uint64_t limit_ns) {
+    constexpr int CHUNKS = BN / 16;
+    constexpr int CB = FM * FB / 8;                       // code bytes per group
+    constexpr int U = FM == 2 ? 1 : 2;                    // units per claim (registers: M codewords per group)
+    constexpr int S = 4 * U;                              // groups per lane per claim
+    const uint64_t keep = policy_evict_last();
+    struct Claim {
+        uint32_t u0;
+        uint32_t pk[U];
+    };
+    auto claim_of = [&](uint32_t ticket, Claim &c) {
+        c.u0 = __shfl_sync(0xffffffffu, ticket, 0);
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+            int nb, kb, r;
+            c.pk[j] = unit_coords<CHUNKS>(c.u0 + j, oa, nb, kb, r) ? pack_unit(nb, kb, r) : 0xffffffffu;
+        }
+    };
+    uint32_t *counter = oa.next_claim + 32 * stream;
+    // the first unit of the next claim of this stream (lane 0; shuffled when used)
+    auto ticket = [&]() -> uint32_t {
+        return lane == 0 ? (atomicAdd(counter, 1u) * kClaimStreams + (uint32_t)stream) * (uint32_t)U : 0u;
+    };
+    // this lane's first row (step 0) and group in unit j of c; false: no work in the unit
+    auto unit_base = [&](const Claim &c, int j, int &row0, int &grp) -> bool {
+        const uint32_t pk = c.pk[j];
+        row0 = (int)(pk >> 18) * BN + (int)(pk & 15) * 16 + (lane >> 3);
+        grp = (int)((pk >> 4) & 0x3fff) * 8 + (lane & 7);
+        return pk != 0xffffffffu && grp < oa.G;
+    };
+    auto load = [&](const Claim &c, uint32_t (&code)[S]) {
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+            int row0, grp;
+            const bool ok = unit_base(c, j, row0, grp);
+            const uint8_t *p = oa.codes + (size_t)row0 * oa.row_bytes + (size_t)grp * CB;
+            const size_t step = (size_t)4 * oa.row_bytes;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                code[4 * j + t] = 0;
+                if (ok && row0 + 4 * t < oa.d_out)
+                    code[4 * j + t] = CB == 2 ? (uint32_t)__ldcs(reinterpret_cast<const uint16_t *>(p + t * step))
+                                              : __ldcs(reinterpret_cast<const uint32_t *>(p + t * step));
+            }
+        }
+    };
+    auto gather = [&](const Claim &c, const uint32_t (&code)[S], uint4 (&cw)[S][FM], float (&sc)[S]) {
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            int row0, grp;
+            const bool in = unit_base(c, s >> 2, row0, grp) && row0 + 4 * (s & 3) < oa.d_out;
+            sc[s] = in ? __half2float(oa.scales[row0 + 4 * (s & 3)]) : 0.f;
+#pragma unroll
+            for (int m = 0; m < FM; ++m) {
+                const uint32_t k = FM == 1 ? (code[s] & 0xffffu)
+                                           : FB == 8 ? (code[s] >> (8 * m)) & 0xffu : (code[s] >> (16 * m)) & 0xffffu;
+                cw[s][m] = make_uint4(0, 0, 0, 0);
+                if (in && AQLM_IN_BOUNDS(k < (1u << FB), kSiteGemmCodebook, k))
+                    cw[s][m] = FB == 8 ? cbs[m * 256 + k] : ld_keep_u4(oa.codebooks + ((size_t)m << FB) + k, keep);
+            }
+        }
+    };
+    auto emit = [&](const Claim &c, const uint4 (&cw)[S][FM], const float (&sc)[S]) {
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            int row0, grp;
+            if (!unit_base(c, s >> 2, row0, grp)) continue;
+            const int row = row0 + 4 * (s & 3);
+            if (row >= oa.d_out) continue;
+            // W^ = bf16_rn(s * (C_0[b0] + ...)), binary32 steps in codebook order, as aqlm_dequant
+            float acc[kGroup];
+            half8_to_float8(cw[s][0], acc);
+#pragma unroll
+            for (int m = 1; m < FM; ++m) {
+                float f[kGroup];
+                half8_to_float8(cw[s][m], f);
+#pragma unroll
+                for (int t = 0; t < kGroup; ++t) acc[t] = __fadd_rn(acc[t], f[t]);
+            }
+            uint32_t out[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const __nv_bfloat16 lo = __float2bfloat16_rn(__fmul_rn(acc[2 * h], sc[s]));
+                const __nv_bfloat16 hi = __float2bfloat16_rn(__fmul_rn(acc[2 * h + 1], sc[s]));
+                out[h] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+            }
+            const size_t w = (size_t)row * oa.G + grp;
+            if (AQLM_IN_BOUNDS(w < (size_t)oa.d_out * oa.G, kSiteGemmB, w)) oa.W[w] = make_uint4(out[0], out[1], out[2], out[3]);
+        }
+    };
+    // Hand the units of claim c to the publisher: the stores ordered before
+    // the async-proxy reads of any SM that later sees the counts (proxy
+    // fence), then the ring entries, released at CTA scope with the new head.
+    uint32_t head = 0;   // lane 0: entries written to this warp's ring
+    auto publish = [&](const Claim &c) {
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+            for (int j = 0; j < U; ++j) {
+                const uint32_t pk = c.pk[j];
+                if (pk == 0xffffffffu) continue;
+                // a free slot (the publisher empties the ring within microseconds)
+                uint64_t t0 = 0;
+                while (head - ld_acquire_shared(&mbx->tail[stream]) >= (uint32_t)kMailSlots) {
+                    const uint64_t t = now_ns();
+                    if (t0 == 0) t0 = t;
+                    else if (t - t0 > limit_ns) {
+                        atomicExch(status, (int32_t)AQLM_ERR_TIMEOUT);
+                        break;
+                    }
+                }
+                mbx->entry[stream][head % kMailSlots] = pk;
+                ++head;
+            }
+            st_release_shared(&mbx->head[stream], head);
+        }
+    };
+
+    Claim a, b, c, n;
+    uint32_t code[S];
+    uint4 cwA[S][FM], cwB[S][FM];
+    float scA[S], scB[S];
+    // prologue: a's codewords being gathered, b's codes loading, the ticket of the third taken
+    claim_of(ticket(), a);
+    load(a, code);
+    gather(a, code, cwA, scA);
+    claim_of(ticket(), b);
+    load(b, code);
+    uint32_t tk = ticket();
+    while (a.u0 < oa.total_units) {
+        gather(b, code, cwB, scB);
+        claim_of(tk, c);
+        tk = ticket();
+        load(c, code);
+        emit(a, cwA, scA);
+        publish(a);
+        if (b.u0 >= oa.total_units) break;
+        gather(c, code, cwA, scA);
+        claim_of(tk, n);
+        tk = ticket();
+        load(n, code);
+        emit(b, cwB, scB);
+        publish(b);
+        // c's codewords in cwA, n's codes loading: the loop's entry state again
+        a = c;
+        b = n;
+    }
+    __syncwarp();
+    if (lane == 0) st_release_shared(&mbx->finished[stream], 1u);
+}
+
+// The publisher warp's loop (one lane): count the units the decoder warps
+// handed over, one GPU-scope fence per batch, until every decoder warp is
+// done.  Bounded: gives up (status AQLM_ERR_TIMEOUT) after limit_ns without
+// a new entry.
+__device__ void publish_units(const OverlapArgs &oa, Mailbox *mbx, int32_t *status, uint64_t limit_ns) {
+    uint32_t seen[kDecWarps];
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) seen[w] = 0;
+    uint64_t idle_since = now_ns();
+    for (;;) {
+        uint32_t h[kDecWarps];
+        bool all_done = true, any = false;
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) {
+            all_done &= ld_acquire_shared(&mbx->finished[w]) != 0;   // before the head: a done warp's last head is seen
+            h[w] = ld_acquire_shared(&mbx->head[w]);
+            any |= h[w] != seen[w];
+        }
+        if (any) {
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");
+#pragma unroll
+            for (int w = 0; w < kDecWarps; ++w) {
+                for (uint32_t i = seen[w]; i != h[w]; ++i) {
+                    const uint32_t pk = *reinterpret_cast<volatile uint32_t *>(&mbx->entry[w][i % kMailSlots]);
+                    red_relaxed_add(oa.panel_done + (size_t)(pk >> 18) * oa.kb_pad + ((pk >> 4) & 0x3fff), 1u);
+                }
+                if (h[w] != seen[w]) st_release_shared(&mbx->tail[w], h[w]);
+                seen[w] = h[w];
+            }
+            idle_since = now_ns();
+        } else if (all_done) {
+            break;
+        } else {
+            __nanosleep(64);
+            if (now_ns() - idle_since > limit_ns) {
+                atomicExch(status, (int32_t)AQLM_ERR_TIMEOUT);
+                break;
+            }
+        }
+    }
+}
+
+// The producer's view of the panel counters: windows of 32 k blocks of one
+// band (kb_pad is a multiple of 32), read with 8 relaxed 16-byte loads.  A
+// window's loads are issued ahead of need (issue) and evaluated when the
+// producer gets there (scan); a panel found incomplete is waited for with
+// bounded polling (wait_window).  A successful evaluation is followed by an
+// acquire fence (GPU scope) and a proxy fence, so the TMA loads issued after
+// it see the decoders' stores.
+constexpr int kWindow = 32;
+
+struct PanelWindow {
+    uint4 v[kWindow / 4];
+    int nb = -1, w = -1;   // band and window index whose counters v holds (or is loading)
+    __device__ void issue(const OverlapArgs &oa, int band, int window) {
+        const uint32_t *row = oa.panel_done + (size_t)band * oa.kb_pad + window * kWindow;
+#pragma unroll
+        for (int i = 0; i < kWindow / 4; ++i) v[i] = ld_relaxed_u4(row + 4 * i);
+        nb = band;
+        w = window;
+    }
+    // If panel kb of the window is complete: the last k block d >= kb such that
+    // kb..d are complete (within the window and the band), else -1.
+    template <int CHUNKS>
+    __device__ int scan(const OverlapArgs &oa, int kb) const {
+        uint32_t done = 0;   // bit i: panel base + i complete
+#pragma unroll
+        for (int i = 0; i < kWindow / 4; ++i) {
+            done |= (uint32_t)(v[i].x >= (uint32_t)CHUNKS) << (4 * i);
+            done |= (uint32_t)(v[i].y >= (uint32_t)CHUNKS) << (4 * i + 1);
+            done |= (uint32_t)(v[i].z >= (uint32_t)CHUNKS) << (4 * i + 2);
+            done |= (uint32_t)(v[i].w >= (uint32_t)CHUNKS) << (4 * i + 3);
+        }
+        const int base = w * kWindow;
+        const uint32_t run = ~(done >> (kb - base));   // first set bit: the first incomplete panel from kb on
+        if (run & 1u) return -1;
+        const int d = kb + (run ? __ffs((int)run) - 1 : kWindow) - 1;
+        const int last = (base + kWindow < oa.num_kb ? base + kWindow : oa.num_kb) - 1;
+        return d < last ? d : last;
+    }
+};
+
+// Bounded wait until panel (nb, kb) is complete; returns the last complete k
+// block from kb on (as scan), or -1 after a timeout or an abort.
+template <int CHUNKS>
+__device__ int wait_window(const OverlapArgs &oa, PanelWindow &pw, int nb, int kb, Bars *bars, uint32_t peer_abort,
+                           int32_t *status, uint64_t limit_ns) {
+    uint64_t t0 = 0;
+    for (;;) {
+        pw.issue(oa, nb, kb / kWindow);
+        const int d = pw.template scan<CHUNKS>(oa, kb);
+        if (d >= 0) return d;
+        if (*reinterpret_cast<volatile int *>(&bars->abort_flag)) return -1;
+        const uint64_t t = now_ns();
+        if (t0 == 0) {
+            t0 = t;
+        } else if (t - t0 > limit_ns) {
+            *reinterpret_cast<volatile int *>(&bars->abort_flag) = 1;
+            st_remote_u32(peer_abort, 1u);
+            atomicExch(status, (int32_t)AQLM_ERR_TIMEOUT);
+            return -1;
+        }
+    }
+}
+
+template <int BN, int FM, int FB>
+__global__ void __launch_bounds__(FM > 0 ? kOverlapThreads : kGemmThreads, 1)
 gemm_bf16_tcgen05_pair(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                        __nv_bfloat16 *__restrict__ Y, int m_total, int n_total, int k_total, int32_t *status,
-                       unsigned long long limit_ns, int stall_test) {
-    using C = PairCfg<BN>;
+                       unsigned long long limit_ns, int stall_test, const OverlapArgs oa) {
+    using C = PairCfg<BN, overlap_reserve<FM, FB>()>;
     constexpr int STAGES = C::STAGES, STAGE_BYTES = C::STAGE_BYTES;
+    constexpr bool kDecode = FM > 0;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled tiles (the same offsets in both CTAs)
     const uint32_t raw = smem_addr(smem_raw);
     uint8_t *smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
     Bars *bars = reinterpret_cast<Bars *>(smem + (size_t)STAGES * STAGE_BYTES);
+    uint4 *cbs = reinterpret_cast<uint4 *>(smem + (size_t)STAGES * STAGE_BYTES + ((sizeof(Bars) + 15) & ~size_t(15)));
+    Mailbox *mbx = reinterpret_cast<Mailbox *>(reinterpret_cast<uint8_t *>(cbs) + (FB == 8 ? FM * 256 * 16 : 0));
+    if constexpr (kDecode) {
+        if constexpr (FB == 8) {  // 8-bit codebooks in shared memory
+            for (int i = threadIdx.x; i < FM * 256; i += blockDim.x) cbs[i] = oa.codebooks[i];
+        } else if (threadIdx.x == 0) {
+            // 16-bit codebooks (1-2 MiB, usually cold): each CTA asks L2 for its share
+            const uint32_t cb_bytes = (uint32_t)FM * (1u << FB) * 16;
+            const uint32_t share = ((cb_bytes + gridDim.x - 1) / gridDim.x + 255) & ~255u;
+            const uint32_t off = blockIdx.x * share;
+            if (off < cb_bytes)
+                prefetch_l2_bulk(reinterpret_cast<const uint8_t *>(oa.codebooks) + off, min(share, cb_bytes - off),
+                                 policy_evict_last());
+        }
+        for (int i = threadIdx.x; i < (int)(sizeof(Mailbox) / 4); i += blockDim.x)
+            reinterpret_cast<uint32_t *>(mbx)[i] = 0;
+    }
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();           // 0: the leader, which issues the MMAs
@@ -695,11 +1105,14 @@ gemm_bf16_tcgen05_pair(const __grid_constant__ CUtensorMap tmap_x, const __grid_
     if (warp == 0) {
         if (lane == 0) {
             // ---- TMA producer (both CTAs) ----
+            grid_dep_wait();   // launched early after the kernel writing W (a no-op otherwise)
             int stage = 0;
             uint32_t phase = 0;
             int issued_parity[STAGES];
             for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
             bool ok = true;
+            int poll_nb = -1, done_kb = -1;   // decoded panels known complete: band poll_nb, k blocks <= done_kb
+            PanelWindow ahead;                // counters loading ahead of need
             for (int tile = pair_id; tile < num_tiles && ok && !stall_test; tile += pairs) {
                 const int mb = tile % m_tiles, nb = tile / m_tiles;
                 for (int kb = 0; kb < num_kb; ++kb) {
@@ -707,6 +1120,33 @@ gemm_bf16_tcgen05_pair(const __grid_constant__ CUtensorMap tmap_x, const __grid_
                                            limit_ns)) {
                         ok = false;
                         break;
+                    }
+                    if constexpr (kDecode) {
+                        constexpr int CHUNKS = BN / 16;
+                        if (nb != poll_nb || kb > done_kb) {
+                            int d = -1;
+                            if (ahead.nb == nb && ahead.w == kb / kWindow) d = ahead.template scan<CHUNKS>(oa, kb);
+                            if (d < 0) d = wait_window<CHUNKS>(oa, ahead, nb, kb, bars, peer_abort, status, limit_ns);
+                            if (d < 0) {
+                                ok = false;
+                                break;
+                            }
+                            asm volatile("fence.acq_rel.gpu;" ::: "memory");
+                            asm volatile("fence.proxy.async.global;" ::: "memory");
+                            poll_nb = nb;
+                            done_kb = d;
+                            ahead.nb = -1;
+                        }
+                        // 8 stages before the known-complete panels run out, load the
+                        // counters that come next: this band's, or the next tile's band's
+                        if (ahead.nb < 0 && kb + 8 >= done_kb) {
+                            if (done_kb + 1 < num_kb) {
+                                ahead.issue(oa, nb, (done_kb + 1) / kWindow);
+                            } else if (tile + pairs < num_tiles) {
+                                const int nb_next = (tile + pairs) / m_tiles;
+                                if (nb_next != nb) ahead.issue(oa, nb_next, 0);
+                            }
+                        }
                     }
                     const uint32_t full_local = smem_addr(&bars->full[stage]);
                     const uint32_t full_leader = map_shared(full_local, 0);
@@ -807,6 +1247,17 @@ gemm_bf16_tcgen05_pair(const __grid_constant__ CUtensorMap tmap_x, const __grid_
             }
         }
         __syncwarp();
+    } else if (kDecode && warp >= 2 + kEpiWarps + kDecWarps) {
+        // ---- publisher (both CTAs): the decoders' units to the panel counters ----
+        if constexpr (kDecode) {
+            if (lane == 0) publish_units(oa, mbx, status, limit_ns);
+        }
+        __syncwarp();
+    } else if (kDecode && warp >= 2 + kEpiWarps) {
+        // ---- decoders (both CTAs): W^ for every CTA of the grid ----
+        if constexpr (kDecode)
+            decode_units<BN, FM, FB>(oa, cbs, mbx, warp - (2 + kEpiWarps), lane, status, limit_ns);
+        __syncwarp();
     } else {
         // ---- epilogue (both CTAs): warps 2..5, TMEM lane quarter = warp % 4 ----
         const int quarter = warp & 3;
@@ -895,7 +1346,7 @@ namespace {
 template <int BN, int FM, int FB>
 cudaError_t launch_gemm_bn(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                            int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test, int sms,
-                           const DecodeArgs &da) {
+                           const DecodeArgs &da, bool pdl = false) {
     using C = GemmCfg<BN, decode_reserve<FM, FB>()>;
     CUtensorMap mx, mw;
     if (!make_map(&mx, X, tokens, k, BM)) return cudaErrorInvalidValue;
@@ -906,7 +1357,7 @@ cudaError_t launch_gemm_bn(const uint16_t *X, const uint16_t *W, uint16_t *Y, in
     if (e != cudaSuccess) return e;
     const int tiles = ((tokens + BM - 1) / BM) * ((n + BN - 1) / BN);
     const int grid = tiles < sms ? tiles : sms;
-    return launch_kernel(fn, dim3(grid), dim3(kGemmThreads + (FM > 0 ? kDecThreads : 0)), C::SMEM, st, false, mx,
+    return launch_kernel(fn, dim3(grid), dim3(kGemmThreads + (FM > 0 ? kDecThreads : 0)), C::SMEM, st, pdl, mx,
                          mw, reinterpret_cast<__nv_bfloat16 *>(Y), tokens, n, k, status, limit_ns, stall_test, da);
 }
 }  // namespace
@@ -935,27 +1386,27 @@ namespace {
 template <int FM, int FB>
 cudaError_t launch_by_width(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                             int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test,
-                            const DecodeArgs &da) {
+                            const DecodeArgs &da, bool pdl = false) {
     int dev = 0;
     cudaGetDevice(&dev);
     const int sms = num_sms(dev);
     switch (gemm_tile_n(tokens, n, sms)) {
         case 240:
-            return launch_gemm_bn<240, FM, FB>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, da);
+            return launch_gemm_bn<240, FM, FB>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, da, pdl);
         case 224:
-            return launch_gemm_bn<224, FM, FB>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, da);
+            return launch_gemm_bn<224, FM, FB>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, da, pdl);
         case 192:
-            return launch_gemm_bn<192, FM, FB>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, da);
+            return launch_gemm_bn<192, FM, FB>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, da, pdl);
         default:
-            return launch_gemm_bn<256, FM, FB>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, da);
+            return launch_gemm_bn<256, FM, FB>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, da, pdl);
     }
 }
 }  // namespace
 
 namespace {
-// Pairs of SMs that can hold a CTA pair of the BN kernel at once (0 if the
+// Pairs of SMs that can hold a CTA pair of the kernel at once (0 if the
 // device cannot), queried once per device.
-template <int BN>
+template <int BN, int FM, int FB>
 int pair_slots(int dev) {
     constexpr int kMaxDevices = 64;
     static std::atomic<int> cached[kMaxDevices];
@@ -963,13 +1414,13 @@ int pair_slots(int dev) {
         const int c = cached[dev].load(std::memory_order_relaxed);
         if (c != 0) return c > 0 ? c : 0;
     }
-    using C = PairCfg<BN>;
-    auto fn = gemm_bf16_tcgen05_pair<BN>;
+    using C = PairCfg<BN, overlap_reserve<FM, FB>()>;
+    auto fn = gemm_bf16_tcgen05_pair<BN, FM, FB>;
     int count = 0;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM) == cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * num_sms(dev));
-        cfg.blockDim = dim3(kGemmThreads);
+        cfg.blockDim = dim3(FM > 0 ? kOverlapThreads : kGemmThreads);
         cfg.dynamicSmemBytes = C::SMEM;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -984,33 +1435,50 @@ int pair_slots(int dev) {
     return count > 0 ? count : 0;
 }
 
-template <int BN>
+// Tiles of a tokens x n product in 256 x BN pair tiles.
+long long pair_tiles(int tokens, int n, int bn) {
+    return (long long)((tokens + kPairRows - 1) / kPairRows) * ((n + bn - 1) / bn);
+}
+
+// oa: the decoding work (FM > 0); its pair-dependent field GB is set here.
+template <int BN, int FM, int FB>
 cudaError_t launch_gemm_pair_bn(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                                 int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test,
-                                int dev) {
-    using C = PairCfg<BN>;
-    const int slots = pair_slots<BN>(dev);
+                                int dev, OverlapArgs oa, bool pdl = false) {
+    using C = PairCfg<BN, overlap_reserve<FM, FB>()>;
+    const int slots = pair_slots<BN, FM, FB>(dev);
     if (slots < 1) return cudaErrorNotSupported;
     CUtensorMap mx, mw;
     if (!make_map(&mx, X, tokens, k, BM)) return cudaErrorInvalidValue;
     if (!make_map(&mw, W, n, k, C::B_HALF)) return cudaErrorInvalidValue;
-    auto fn = gemm_bf16_tcgen05_pair<BN>;
-    const int tiles = ((tokens + kPairRows - 1) / kPairRows) * ((n + BN - 1) / BN);
-    const int pairs = tiles < slots ? tiles : slots;
+    auto fn = gemm_bf16_tcgen05_pair<BN, FM, FB>;
+    const long long tiles = pair_tiles(tokens, n, BN);
+    const int pairs = tiles < slots ? (int)tiles : slots;
+    const int m_tiles = (tokens + kPairRows - 1) / kPairRows;
+    oa.GB = (pairs + m_tiles - 1) / m_tiles;   // bands whose first tiles share a wave
+    if (oa.n_bands > 0) {
+        constexpr uint32_t CHUNKS = BN / 16;
+        const int last = oa.n_bands - (oa.n_bands - 1) / oa.GB * oa.GB;   // bands of the last group
+        oa.per_group = make_fast_div((uint32_t)oa.GB * CHUNKS * (uint32_t)oa.num_kb);
+        oa.per_kb = make_fast_div((uint32_t)oa.GB * CHUNKS);
+        oa.per_kb_last = make_fast_div((uint32_t)last * CHUNKS);
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs);
-    cfg.blockDim = dim3(kGemmThreads);
+    cfg.blockDim = dim3(FM > 0 ? kOverlapThreads : kGemmThreads);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, fn, mx, mw, reinterpret_cast<__nv_bfloat16 *>(Y), tokens, n, k, status, limit_ns,
-                              stall_test);
+                              stall_test, oa);
 }
 }  // namespace
 
@@ -1040,37 +1508,50 @@ bool gemm_uses_pair(int tokens) { return tokens > BM; }
 
 cudaError_t launch_bf16_gemm_cfg(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                                  int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test,
-                                 int cta_pair, int tile_n) {
+                                 int cta_pair, int tile_n, bool pdl) {
     int dev = 0;
     cudaGetDevice(&dev);
     const bool pair = cta_pair < 0 ? gemm_uses_pair(tokens) : cta_pair != 0;
     if (!pair) {
         const DecodeArgs none = {};
-        if (tile_n == 0) return launch_by_width<0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, none);
+        if (tile_n == 0)
+            return launch_by_width<0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, none, pdl);
         const int sms = num_sms(dev);
         switch (tile_n) {
             case 256:
-                return launch_gemm_bn<256, 0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, none);
+                return launch_gemm_bn<256, 0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, none,
+                                                 pdl);
             case 240:
-                return launch_gemm_bn<240, 0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, none);
+                return launch_gemm_bn<240, 0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, none,
+                                                 pdl);
             case 224:
-                return launch_gemm_bn<224, 0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, none);
+                return launch_gemm_bn<224, 0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, none,
+                                                 pdl);
             case 192:
-                return launch_gemm_bn<192, 0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, none);
+                return launch_gemm_bn<192, 0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, sms, none,
+                                                 pdl);
             default:
                 return cudaErrorInvalidValue;
         }
     }
-    if (tile_n == 0) tile_n = gemm_pair_tile_n(tokens, n, pair_slots<256>(dev) > 0 ? pair_slots<256>(dev) : 1);
+    if (tile_n == 0) {
+        const int slots = pair_slots<256, 0, 0>(dev);
+        tile_n = gemm_pair_tile_n(tokens, n, slots > 0 ? slots : 1);
+    }
+    const OverlapArgs none = {};
     switch (tile_n) {
         case 256:
-            return launch_gemm_pair_bn<256>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, dev);
+            return launch_gemm_pair_bn<256, 0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, dev, none,
+                                                  pdl);
         case 240:
-            return launch_gemm_pair_bn<240>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, dev);
+            return launch_gemm_pair_bn<240, 0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, dev, none,
+                                                  pdl);
         case 224:
-            return launch_gemm_pair_bn<224>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, dev);
+            return launch_gemm_pair_bn<224, 0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, dev, none,
+                                                  pdl);
         case 192:
-            return launch_gemm_pair_bn<192>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, dev);
+            return launch_gemm_pair_bn<192, 0, 0>(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, dev, none,
+                                                  pdl);
         default:
             return cudaErrorInvalidValue;
     }
@@ -1078,7 +1559,79 @@ cudaError_t launch_bf16_gemm_cfg(const uint16_t *X, const uint16_t *W, uint16_t 
 
 cudaError_t launch_bf16_gemm_ex(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                                 int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test) {
-    return launch_bf16_gemm_cfg(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, -1, 0);
+    return launch_bf16_gemm_cfg(X, W, Y, tokens, n, k, status, st, limit_ns, stall_test, -1, 0, false);
+}
+
+// The GEMM of aqlm_gemm, launched while the dequantisation before it in the
+// stream still runs (programmatic dependent launch): its CTAs set up beside
+// the dequantisation's, and its TMA producer waits for that grid before the
+// first load.
+cudaError_t launch_bf16_gemm_after_dequant(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n,
+                                          int k, int32_t *status, cudaStream_t st) {
+    return launch_bf16_gemm_cfg(X, W, Y, tokens, n, k, status, st, kGemmWaitLimitNs, 0, -1, 0, true);
+}
+
+// ---- prefill with the dequantisation overlapped (CTA pairs) ----
+size_t overlap_counter_bytes(int d_out, int d_in) {
+    const long long bands = (d_out + 191) / 192;               // the narrowest tile has the most bands
+    const long long kb_pad = ((d_in + BK - 1) / BK + 31) / 32 * 32;
+    return kClaimBytes + (size_t)((bands * kb_pad * 4 + 255) / 256 * 256);
+}
+
+namespace {
+template <int BN, int FM, int FB>
+cudaError_t launch_overlap_bn(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                              const uint16_t *X, uint16_t *W, uint16_t *Y, int tokens, const Dims &d,
+                              int32_t *status, void *counters, cudaStream_t st, int dev) {
+    OverlapArgs oa = {};
+    oa.codes = static_cast<const uint8_t *>(codes);
+    oa.codebooks = reinterpret_cast<const uint4 *>(codebooks);
+    oa.scales = reinterpret_cast<const __half *>(scales);
+    oa.W = reinterpret_cast<uint4 *>(W);
+    oa.next_claim = static_cast<uint32_t *>(counters);
+    oa.panel_done = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(counters) + kClaimBytes);
+    oa.d_out = d.d_out;
+    oa.G = d.G;
+    oa.row_bytes = d.row_bytes;
+    oa.n_bands = (d.d_out + BN - 1) / BN;
+    oa.num_kb = (d.d_in + BK - 1) / BK;
+    oa.kb_pad = (oa.num_kb + kWindow - 1) / kWindow * kWindow;
+    oa.total_units = (uint32_t)oa.n_bands * (BN / 16) * (uint32_t)oa.num_kb;   // < 2^31 for any layer of 2^20 x 2^20
+    const size_t bytes = kClaimBytes + (size_t)oa.n_bands * oa.kb_pad * 4;
+    const cudaError_t e = cudaMemsetAsync(counters, 0, bytes, st);
+    if (e != cudaSuccess) return e;
+    return launch_gemm_pair_bn<BN, FM, FB>(X, W, Y, tokens, d.d_out, d.d_in, status, st, kGemmWaitLimitNs, 0, dev,
+                                           oa);
+}
+
+template <int FM, int FB>
+cudaError_t launch_overlap_fmt(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                               const uint16_t *X, uint16_t *W, uint16_t *Y, int tokens, const Dims &d,
+                               int32_t *status, void *counters, cudaStream_t st) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int slots = pair_slots<240, FM, FB>(dev);
+    switch (gemm_pair_tile_n(tokens, d.d_out, slots > 0 ? slots : 1)) {
+        case 240:
+            return launch_overlap_bn<240, FM, FB>(codes, codebooks, scales, X, W, Y, tokens, d, status, counters, st, dev);
+        case 224:
+            return launch_overlap_bn<224, FM, FB>(codes, codebooks, scales, X, W, Y, tokens, d, status, counters, st, dev);
+        case 192:
+            return launch_overlap_bn<192, FM, FB>(codes, codebooks, scales, X, W, Y, tokens, d, status, counters, st, dev);
+        default:
+            return launch_overlap_bn<256, FM, FB>(codes, codebooks, scales, X, W, Y, tokens, d, status, counters, st, dev);
+    }
+}
+}  // namespace
+
+// Y = X . W^T with W^ decoded into W (d_out x d_in bf16) by the GEMM's own
+// decoder warps; counters: overlap_counter_bytes(d_out, d_in) bytes.
+cudaError_t launch_overlap_gemm(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                                const uint16_t *X, uint16_t *W, uint16_t *Y, int tokens, const Dims &d,
+                                int32_t *status, void *counters, cudaStream_t st) {
+    if (d.M == 1) return launch_overlap_fmt<1, 16>(codes, codebooks, scales, X, W, Y, tokens, d, status, counters, st);
+    if (d.B == 8) return launch_overlap_fmt<2, 8>(codes, codebooks, scales, X, W, Y, tokens, d, status, counters, st);
+    return launch_overlap_fmt<2, 16>(codes, codebooks, scales, X, W, Y, tokens, d, status, counters, st);
 }
 
 // Prefill with the dequantisation fused into the GEMM (no W^ in global memory).

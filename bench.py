@@ -410,9 +410,11 @@ def bench_prefill(ac, spec, tokens, reps, warmup):
                        dtype=torch.uint8, device="cuda")
     t_fused = timed(lambda: ac.aqlm_gemm_fused(d["codes"], d["codebooks"], d["scales"], X, Y=Y, workspace=ws_f))
     assert ac.aqlm_gemm_check(ws_f) == ac.AQLM_OK
+    t_overlap = timed(lambda: ac.aqlm_gemm_overlap(d["codes"], d["codebooks"], d["scales"], X, Y=Y, workspace=ws))
+    assert ac.aqlm_gemm_check(ws) == ac.AQLM_OK
     flops = 2.0 * tokens * spec.d_out * spec.d_in
     deq_bytes = spec.code_bytes() + 2 * spec.d_out + 2 * spec.d_out * spec.d_in
-    return {"us_total": t_total, "us_dequant": t_deq, "us_gemm": t_gemm, "us_fused": t_fused,
+    return {"us_total": t_total, "us_dequant": t_deq, "us_gemm": t_gemm, "us_fused": t_fused, "us_overlap": t_overlap,
             "fused_tflops": flops / t_fused / 1e6, "tflops": flops / t_total / 1e6,
             "gemm_tflops": flops / t_gemm / 1e6, "dequant_gbs": deq_bytes / t_deq / 1e3}
 
@@ -618,7 +620,9 @@ def run_gpu(args):
                     "us_gemm": round(p["us_gemm"], 2), "gemm_tflops": round(p["gemm_tflops"], 1),
                     "fused_no_workspace": {"us_per_layer": round(p["us_fused"], 2),
                                            "tflops": round(p["fused_tflops"], 1),
-                                           "tensor_frac": round(p["fused_tflops"] / peaks["bf16_tflops"], 4)}}
+                                           "tensor_frac": round(p["fused_tflops"] / peaks["bf16_tflops"], 4)},
+                    "overlap_one_kernel": {"us_per_layer": round(p["us_overlap"], 2),
+                                           "tflops": round(2.0 * 2048 * o * i / p["us_overlap"] / 1e6, 1)}}
                 if cpu_ok and (o, i) == PREFILL_SHAPES[0]:
                     detail[key]["cpu_oracle"] = cpu_oracle_prefill(LayerSpec(o, i, M, B), 2048)
                 torch.cuda.empty_cache()

@@ -236,11 +236,14 @@ AQLM_API aqlm_status aqlm_dequant(const void *codes, const uint16_t *codebooks, 
 
 /*
  * aqlm_gemm -- prefill product Y = X . W^T for many tokens: aqlm_dequant into
- * the workspace, then a tcgen05 tensor-core GEMM (bf16 operands, fp32
- * accumulation in tensor memory, bf16 output rounded to nearest even).
+ * the workspace (W^, bf16), then the tcgen05 tensor-core GEMM of
+ * aqlm_bf16_gemm (bf16 operands, fp32 accumulation in tensor memory, bf16
+ * output rounded to nearest even; CTA pairs past 128 tokens, see
+ * aqlm_bf16_gemm_plan).  Y equals aqlm_bf16_gemm on aqlm_dequant's W^.
  *   X: [tokens][d_in] bf16.  Y: [tokens][d_out] bf16 (written).  tokens >= 1.
  *   workspace: at least aqlm_gemm_workspace_bytes(shape, tokens) bytes,
- *   16-byte aligned; it holds the dequantised weight and a status word.
+ *   16-byte aligned: a 256-byte status word, the counters aqlm_gemm_overlap
+ *   uses, and W^ in the last 2 * d_out * d_in bytes.
  *   Every device-side wait of the GEMM is bounded; a wait that gives up
  *   records AQLM_ERR_TIMEOUT in the workspace's status word (read it with
  *   aqlm_gemm_check) and the kernel returns without trapping.
@@ -251,6 +254,31 @@ AQLM_API aqlm_status aqlm_gemm(const void *codes, const uint16_t *codebooks, con
                       void *workspace, size_t workspace_bytes, aqlm_stream_t stream);
 
 AQLM_API size_t aqlm_gemm_workspace_bytes(aqlm_shape shape, int32_t tokens);
+
+/*
+ * aqlm_gemm_overlap -- the product of aqlm_gemm in ONE kernel that decodes
+ * each W^ block once and overlaps the decoding with the MMAs: the CTA-pair
+ * GEMM (aqlm_bf16_gemm_plan's width for more than 128 tokens; the same
+ * kernel with half-empty pair tiles below) with eight decoder warps and a
+ * publisher warp in every CTA.  The decoders write W^ into the workspace in
+ * the order the tiles need it (units of 16 rows x 64 inputs, claimed from
+ * global counters) with the binary32 steps of aqlm_dequant; a CTA's TMA load
+ * of a W^ tile waits (bounded) until the counters say every unit that writes
+ * it is done.  The page this follows, "The AQLM Quantization Algorithm,
+ * Explained", section "Why and what do we quantize?": the weights are
+ * fetched compressed and dequantised at runtime before the matmul.  W^ left
+ * in the workspace equals aqlm_dequant's output and Y equals
+ * aqlm_bf16_gemm_config on it with the CTA pair at the same width, bit for
+ * bit.  Arguments, workspace (aqlm_gemm_workspace_bytes) and errors as
+ * aqlm_gemm; a bounded wait that gives up records AQLM_ERR_TIMEOUT in the
+ * status word (aqlm_gemm_check).  Every CTA of the grid must be resident
+ * for the decoding to be shared: the grid is the device's co-resident pair
+ * count at most, and a unit is always claimed by a running warp.  On B200 it
+ * runs as fast as aqlm_gemm's two kernels, within a few per cent either way.
+ */
+AQLM_API aqlm_status aqlm_gemm_overlap(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
+                                       const uint16_t *X, uint16_t *Y, int32_t tokens, aqlm_shape shape,
+                                       void *workspace, size_t workspace_bytes, aqlm_stream_t stream);
 
 /*
  * aqlm_gemm_fused -- the prefill product of aqlm_gemm, Y = bf16(X . W^T),

@@ -133,7 +133,11 @@ def test_gemm_argument_errors():
     lib = ac.load_library()
     s = ac.Shape(4096, 4096, 8, 1, 16)
     need = lib.aqlm_gemm_workspace_bytes(s, 2048)
-    assert need == 256 + 4096 * 4096 * 2
+    # status word, the overlapped decoding's counters (8 claim words on their
+    # own 128-byte lines + one per 192-row band and k block, k blocks padded
+    # to a multiple of 32), the bf16 W^
+    counters = 1024 + -(-(-(-4096 // 192) * 64 * 4) // 256) * 256
+    assert need == 256 + counters + 4096 * 4096 * 2
     assert lib.aqlm_gemm(A16, B16, C16, D16, E16, 2048, s, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
     assert lib.aqlm_gemm(A16, B16, C16, D16, E16, 2048, s, A16, need - 1, NULL) == ac.AQLM_ERR_WORKSPACE
     assert lib.aqlm_gemm(A16, B16, C16, D16, E16, 0, s, A16, need, NULL) == ac.AQLM_ERR_INVALID_ARG

@@ -285,6 +285,44 @@ def test_gemm_small(M, B, tokens, d_out, d_in):
     _gemm_check(bf16_to_np_bits(Y), L, spec, L["x"])
 
 
+# (tokens, d_out, d_in): bands (256 / 240 / 224 / 192 rows) with a ragged last
+# band, k blocks with a ragged last one, one and several pair tiles, widths
+# chosen by the rule on 148 SMs (so 4608 outputs take 256-wide tiles)
+OVERLAP_CASES = [(200, 520, 576), (256, 512, 1024), (130, 264, 64), (1000, 4608, 1032), (2040, 4096, 520),
+                 (1530, 4864, 520), (300, 1000, 4104), (100, 264, 576), (2048, 11008, 4096)]
+
+
+@pytest.mark.parametrize("M,B", FORMATS)
+@pytest.mark.parametrize("tokens,d_out,d_in", OVERLAP_CASES, ids=[f"{t}x{o}x{i}" for t, o, i in OVERLAP_CASES])
+def test_gemm_overlapped_decode_equals_two_kernels(M, B, tokens, d_out, d_in):
+    """aqlm_gemm_overlap decodes W^ inside the CTA-pair GEMM (decoder warps of
+    every CTA, loads gated by per-panel counters).  The W^ it leaves in the
+    workspace equals aqlm_dequant's bit for bit, and Y equals the CTA-pair
+    GEMM of that W^ at the same width bit for bit, and aqlm_gemm's Y;
+    sampled tokens against the oracle."""
+    if (d_in // 8 * M * B // 8) % 16:
+        pytest.skip("row of codes not 16-byte aligned")
+    spec = LayerSpec(d_out, d_in, M, B)
+    L = make_layer(spec, seed=60 + tokens + d_in, tokens=tokens, x_dtype="bf16")
+    d = to_dev(L)
+    Y, ws = ac.aqlm_gemm_overlap(d["codes"], d["codebooks"], d["scales"], d["x"])
+    assert ac.aqlm_gemm_check(ws) == ac.AQLM_OK
+    W_ws = ws[ws.numel() - 2 * d_out * d_in:].view(torch.int16).view(d_out, d_in)
+    W_ref = ac.aqlm_dequant(d["codes"], d["codebooks"], d["scales"])
+    torch.cuda.synchronize()
+    assert torch.equal(W_ws, W_ref.view(torch.int16))
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    width = ac.bf16_gemm_plan(max(tokens, 129), d_out, sms)[1]   # the pair rule's width, at any token count
+    Y2, st2 = ac.aqlm_bf16_gemm_config(d["x"], W_ref, 1, width)
+    Y3, ws3 = ac.aqlm_gemm(d["codes"], d["codebooks"], d["scales"], d["x"])
+    torch.cuda.synchronize()
+    assert int(st2.item()) == 0 and ac.aqlm_gemm_check(ws3) == ac.AQLM_OK
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+    assert torch.equal(Y.view(torch.int16), Y3.view(torch.int16))
+    toks = np.unique(np.array([0, 1, tokens // 2, tokens - 1]))
+    _gemm_check(bf16_to_np_bits(Y), L, spec, L["x"], tokens_idx=toks)
+
+
 @pytest.mark.parametrize("tokens,n,k", [(200, 520, 576), (128, 256, 65536), (130, 264, 64)])
 def test_bf16_gemm_ragged_and_deep(tokens, n, k):
     """Ragged tiles in every dimension (200 x 520 x 576), one tile with a long
