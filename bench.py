@@ -777,6 +777,7 @@ PROFILE_CASES = {
     "dequant-1x16-11008x4096": ("dequant", 11008, 4096, 1, 16, 0),
     "dequant-2x8-11008x4096": ("dequant", 11008, 4096, 2, 8, 0),
     "gemm-2048x11008x4096": ("gemm", 11008, 4096, 2, 8, 2048),
+    "overlap-1x16-2048x11008x4096": ("overlap", 11008, 4096, 1, 16, 2048),
     "encode-1x16-256x4096": ("encode", 256, 4096, 1, 16, 0),
 }
 
@@ -814,8 +815,9 @@ def run_profile_case(name, launches=12):
         layers = Layers(spec, 1, T, x_dtype="bf16")
         d = layers.copies[0]
         ws = torch.empty(ac.gemm_workspace_bytes(ac.shape_of(d["codes"]), T), dtype=torch.uint8, device="cuda")
+        call = ac.aqlm_gemm_overlap if kind == "overlap" else ac.aqlm_gemm
         for _ in range(max(2, launches // 4)):
-            ac.aqlm_gemm(d["codes"], d["codebooks"], d["scales"], layers.x, workspace=ws)
+            call(d["codes"], d["codebooks"], d["scales"], layers.x, workspace=ws)
         assert ac.aqlm_gemm_check(ws) == ac.AQLM_OK
     torch.cuda.synchronize()
     print(json.dumps({"profile_case": name, "launches": launches}))
