@@ -144,6 +144,12 @@ def test_gemm_argument_errors():
     assert lib.aqlm_gemm(A16, B16, C16, ODD, E16, 16, s, A16, need, NULL) == ac.AQLM_ERR_MISALIGNED
     s_odd = ac.Shape(4100, 4096, 8, 1, 16)
     assert lib.aqlm_gemm(A16, B16, C16, D16, E16, 16, s_odd, A16, 1 << 40, NULL) == ac.AQLM_ERR_UNSUPPORTED
+    # the one-kernel prefill validates exactly as aqlm_gemm, with the same workspace
+    assert lib.aqlm_gemm_overlap(A16, B16, C16, D16, E16, 2048, s, NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_gemm_overlap(A16, B16, C16, D16, E16, 2048, s, A16, need - 1, NULL) == ac.AQLM_ERR_WORKSPACE
+    assert lib.aqlm_gemm_overlap(A16, B16, C16, D16, E16, 0, s, A16, need, NULL) == ac.AQLM_ERR_INVALID_ARG
+    assert lib.aqlm_gemm_overlap(A16, B16, C16, ODD, E16, 16, s, A16, need, NULL) == ac.AQLM_ERR_MISALIGNED
+    assert lib.aqlm_gemm_overlap(A16, B16, C16, D16, E16, 16, s_odd, A16, 1 << 40, NULL) == ac.AQLM_ERR_UNSUPPORTED
     assert lib.aqlm_bf16_gemm(A16, B16, C16, 16, 100, 64, D16, NULL) == ac.AQLM_ERR_UNSUPPORTED
     assert lib.aqlm_bf16_gemm(A16, B16, C16, 16, 128, 64, NULL, NULL) == ac.AQLM_ERR_INVALID_ARG
     assert lib.aqlm_gemm_check(NULL, 0, NULL) == ac.AQLM_ERR_WORKSPACE
