@@ -323,6 +323,31 @@ def test_gemm_overlapped_decode_equals_two_kernels(M, B, tokens, d_out, d_in):
     _gemm_check(bf16_to_np_bits(Y), L, spec, L["x"], tokens_idx=toks)
 
 
+@pytest.mark.parametrize("M,B", FORMATS)
+def test_gemm_overlap_and_pair_repeatable(M, B):
+    """Cross-CTA protocols under repetition: 12 calls of aqlm_gemm_overlap
+    (units claimed from global counters, handed to the publisher warp,
+    panels counted, TMA loads gated on the counts) and of the CTA-pair GEMM
+    leave the same Y bit for bit every time; a load that ran ahead of its
+    panel's stores, or a pair whose halves lost step, would not."""
+    spec = LayerSpec(4864, 1088, M, B)   # 4864 = 20.3 bands of 240; 17 k blocks
+    L = make_layer(spec, seed=77, tokens=1530, x_dtype="bf16")
+    d = to_dev(L)
+    ws = torch.empty(ac.gemm_workspace_bytes(ac.shape_of(d["codes"]), 1530), dtype=torch.uint8, device=DEV)
+    Y0, _ = ac.aqlm_gemm_overlap(d["codes"], d["codebooks"], d["scales"], d["x"], workspace=ws)
+    assert ac.aqlm_gemm_check(ws) == ac.AQLM_OK
+    W = ac.aqlm_dequant(d["codes"], d["codebooks"], d["scales"])
+    P0, st = ac.aqlm_bf16_gemm_config(d["x"], W, 1, 0)
+    for _ in range(12):
+        Y, _ = ac.aqlm_gemm_overlap(d["codes"], d["codebooks"], d["scales"], d["x"], workspace=ws)
+        P, st2 = ac.aqlm_bf16_gemm_config(d["x"], W, 1, 0)
+        torch.cuda.synchronize()
+        assert ac.aqlm_gemm_check(ws) == ac.AQLM_OK and int(st2.item()) == 0
+        assert torch.equal(Y.view(torch.int16), Y0.view(torch.int16))
+        assert torch.equal(P.view(torch.int16), P0.view(torch.int16))
+    assert torch.equal(Y0.view(torch.int16), P0.view(torch.int16))
+
+
 @pytest.mark.parametrize("tokens,n,k", [(200, 520, 576), (128, 256, 65536), (130, 264, 64)])
 def test_bf16_gemm_ragged_and_deep(tokens, n, k):
     """Ragged tiles in every dimension (200 x 520 x 576), one tile with a long
