@@ -236,9 +236,14 @@ aqlm_status aqlm_gemm(const void *codes, const uint16_t *codebooks, const uint16
     int32_t *status = static_cast<int32_t *>(workspace);
     uint8_t *counters = static_cast<uint8_t *>(workspace) + kStatusBytes;
     uint16_t *W = reinterpret_cast<uint16_t *>(counters + aqlm::overlap_counter_bytes(shape.d_out, shape.d_in));
-    (void)counters;   // used by aqlm_gemm_overlap only
     cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), cs);
     if (e != cudaSuccess) return AQLM_ERR_CUDA;
+    if (shape.num_codebooks == 2 && shape.codebook_bits == 16 && aqlm::gemm_uses_pair(tokens)) {
+        // two 16-bit codebooks: the decoding (two L2 gathers per group) is long
+        // enough that overlapping it with the MMAs wins (measured on B200)
+        return from_cuda(aqlm::launch_overlap_gemm(codes, codebooks, scales, X, W, Y, tokens,
+                                                   aqlm::make_dims(shape), status, counters, cs));
+    }
     e = aqlm::launch_dequant(codes, codebooks, scales, W, aqlm::make_dims(shape), cs);
     if (e != cudaSuccess) return AQLM_ERR_CUDA;
     return from_cuda(aqlm::launch_bf16_gemm_after_dequant(X, W, Y, tokens, shape.d_out, shape.d_in, status, cs));

@@ -239,7 +239,10 @@ AQLM_API aqlm_status aqlm_dequant(const void *codes, const uint16_t *codebooks, 
  * the workspace (W^, bf16), then the tcgen05 tensor-core GEMM of
  * aqlm_bf16_gemm (bf16 operands, fp32 accumulation in tensor memory, bf16
  * output rounded to nearest even; CTA pairs past 128 tokens, see
- * aqlm_bf16_gemm_plan).  Y equals aqlm_bf16_gemm on aqlm_dequant's W^.
+ * aqlm_bf16_gemm_plan), launched early so that its set-up overlaps the
+ * dequantisation's end.  For two 16-bit codebooks past 128 tokens, the one
+ * kernel of aqlm_gemm_overlap instead (faster there: its decoding is the
+ * longest).  Either way Y equals aqlm_bf16_gemm on aqlm_dequant's W^.
  *   X: [tokens][d_in] bf16.  Y: [tokens][d_out] bf16 (written).  tokens >= 1.
  *   workspace: at least aqlm_gemm_workspace_bytes(shape, tokens) bytes,
  *   16-byte aligned: a 256-byte status word, the counters aqlm_gemm_overlap
