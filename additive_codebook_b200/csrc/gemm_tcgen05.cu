@@ -1452,6 +1452,9 @@ cudaError_t launch_gemm_pair_bn(const uint16_t *X, const uint16_t *W, uint16_t *
     if (!make_map(&mx, X, tokens, k, BM)) return cudaErrorInvalidValue;
     if (!make_map(&mw, W, n, k, C::B_HALF)) return cudaErrorInvalidValue;
     auto fn = gemm_bf16_tcgen05_pair<BN, FM, FB>;
+    // (pair_slots set it once per device; again here, in case the context was reset since)
+    const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+    if (e != cudaSuccess) return e;
     const long long tiles = pair_tiles(tokens, n, BN);
     const int pairs = tiles < slots ? (int)tiles : slots;
     const int m_tiles = (tokens + kPairRows - 1) / kPairRows;
