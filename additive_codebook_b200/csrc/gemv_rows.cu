@@ -408,11 +408,15 @@ static_assert(RowFmt<2, 8>::kWarps >= kRowWarps && RowFmt<1, 16>::kWarps >= kRow
 // wait) while this launch computes; measured on B200 (graph of back-to-back
 // launches, 4096x4096): with every slot taken by one launch the next
 // launch's CTAs started only as this launch's CTAs ended, and each CTA spent
-// 2-3 us on loads before its first multiply.  1x16 / 2x16: every slot, as
-// the random codeword gathers need all the warps the SM holds (one 8-warp CTA
-// per SM and launch measured slower: 4096x4096 10.6 against 9.8 us).
-int ctas_per_sm_per_launch(const Dims &d, int resident) {
-    if (d.B == 8) return resident > 1 ? resident / 2 : 1;
+// 2-3 us on loads before its first multiply.  A 2x8 launch of several layers
+// (aqlm_gemv_multi) takes every slot instead: it has three times the rows per
+// CTA, so its own warps matter more than the next launch's early start
+// (measured: Llama-2-7B q/k/v in one launch 18.3 -> 13.4 us, gate/up 21.4 ->
+// 20.8 us).  1x16 / 2x16: every slot, as the random codeword gathers need all
+// the warps the SM holds (one 8-warp CTA per SM and launch measured slower:
+// 4096x4096 10.6 against 9.8 us).
+int ctas_per_sm_per_launch(const Dims &d, int resident, int n_layers) {
+    if (d.B == 8 && n_layers == 1) return resident > 1 ? resident / 2 : 1;
     return resident;
 }
 
@@ -516,7 +520,7 @@ cudaError_t launch_rows(const RowLayerIn *layers, int n, const uint16_t *x, int 
     const int occ = resident_ctas(reinterpret_cast<const void *>(fn), threads, p.smem);
     int d_outs[kRowMaxLayers], ctas[kRowMaxLayers];
     for (int l = 0; l < n; ++l) d_outs[l] = layers[l].d_out;
-    rows_grid(d_outs, n, d, p, ctas_per_sm_per_launch(d, occ), sms, ctas);
+    rows_grid(d_outs, n, d, p, ctas_per_sm_per_launch(d, occ, n), sms, ctas);
     RowArgs<NL> a = {};
     int cta0 = 0, row0 = 0;
     for (int l = 0; l < n; ++l) {
