@@ -11,6 +11,7 @@ cudaError_t launch_bf16_gemm_ex(const uint16_t *X, const uint16_t *W, uint16_t *
 cudaError_t launch_bf16_gemm_cfg(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n, int k,
                                  int32_t *status, cudaStream_t st, unsigned long long limit_ns, int stall_test,
                                  int cta_pair, int tile_n, bool pdl);
+bool overlap_preferred(const Dims &d, int tokens);
 cudaError_t launch_bf16_gemm_after_dequant(const uint16_t *X, const uint16_t *W, uint16_t *Y, int tokens, int n,
                                           int k, int32_t *status, cudaStream_t st);
 cudaError_t launch_fused_gemm(const void *codes, const uint16_t *codebooks, const uint16_t *scales,
@@ -238,9 +239,8 @@ aqlm_status aqlm_gemm(const void *codes, const uint16_t *codebooks, const uint16
     uint16_t *W = reinterpret_cast<uint16_t *>(counters + aqlm::overlap_counter_bytes(shape.d_out, shape.d_in));
     cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), cs);
     if (e != cudaSuccess) return AQLM_ERR_CUDA;
-    if (shape.num_codebooks == 2 && shape.codebook_bits == 16 && aqlm::gemm_uses_pair(tokens)) {
-        // two 16-bit codebooks: the decoding (two L2 gathers per group) is long
-        // enough that overlapping it with the MMAs wins (measured on B200)
+    if (aqlm::overlap_preferred(aqlm::make_dims(shape), tokens)) {
+        // the one-kernel prefill of aqlm_gemm_overlap, where it was measured faster
         return from_cuda(aqlm::launch_overlap_gemm(codes, codebooks, scales, X, W, Y, tokens,
                                                    aqlm::make_dims(shape), status, counters, cs));
     }

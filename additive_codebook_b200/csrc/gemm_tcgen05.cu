@@ -696,7 +696,8 @@ struct OverlapArgs {
     uint32_t *panel_done;       // [n_bands][kb_pad] finished units, zero at launch
     int d_out, G, row_bytes;
     int n_bands, num_kb, kb_pad, GB;
-    uint32_t total_units;       // n_bands * (BN / 16) * num_kb (< 2^31)
+    int band0;                  // bands [0, band0) are decoded before the launch (complete)
+    uint32_t total_units;       // (n_bands - band0) * (BN / 16) * num_kb (< 2^31)
     FastDiv per_group;          // units of a group of GB bands
     FastDiv per_kb, per_kb_last;   // units of one k block of a full group, of the last group
 };
@@ -740,7 +741,7 @@ __device__ __forceinline__ bool unit_coords(uint32_t u, const OverlapArgs &oa, i
     if (u >= oa.total_units) return false;
     const uint32_t g = oa.per_group.div(u);
     const uint32_t rem = u - g * oa.per_group.d;
-    const int b_lo = (int)g * oa.GB;
+    const int b_lo = oa.band0 + (int)g * oa.GB;
     const FastDiv &fk = oa.n_bands - b_lo < oa.GB ? oa.per_kb_last : oa.per_kb;
     kb = (int)fk.div(rem);
     const uint32_t rem2 = rem - (uint32_t)kb * fk.d;
@@ -1123,7 +1124,11 @@ gemm_bf16_tcgen05_pair(const __grid_constant__ CUtensorMap tmap_x, const __grid_
                     }
                     if constexpr (kDecode) {
                         constexpr int CHUNKS = BN / 16;
-                        if (nb != poll_nb || kb > done_kb) {
+                        if (nb < oa.band0) {
+                            // decoded before the launch: visible after the grid dependency
+                            poll_nb = nb;
+                            done_kb = num_kb - 1;
+                        } else if (nb != poll_nb || kb > done_kb) {
                             int d = -1;
                             if (ahead.nb == nb && ahead.w == kb / kWindow) d = ahead.template scan<CHUNKS>(oa, kb);
                             if (d < 0) d = wait_window<CHUNKS>(oa, ahead, nb, kb, bars, peer_abort, status, limit_ns);
@@ -1144,7 +1149,7 @@ gemm_bf16_tcgen05_pair(const __grid_constant__ CUtensorMap tmap_x, const __grid_
                                 ahead.issue(oa, nb, (done_kb + 1) / kWindow);
                             } else if (tile + pairs < num_tiles) {
                                 const int nb_next = (tile + pairs) / m_tiles;
-                                if (nb_next != nb) ahead.issue(oa, nb_next, 0);
+                                if (nb_next != nb && nb_next >= oa.band0) ahead.issue(oa, nb_next, 0);
                             }
                         }
                     }
@@ -1459,9 +1464,10 @@ cudaError_t launch_gemm_pair_bn(const uint16_t *X, const uint16_t *W, uint16_t *
     const int pairs = tiles < slots ? (int)tiles : slots;
     const int m_tiles = (tokens + kPairRows - 1) / kPairRows;
     oa.GB = (pairs + m_tiles - 1) / m_tiles;   // bands whose first tiles share a wave
-    if (oa.n_bands > 0) {
+    const int rest = oa.n_bands - oa.band0;     // bands the decoder warps decode
+    if (rest > 0) {
         constexpr uint32_t CHUNKS = BN / 16;
-        const int last = oa.n_bands - (oa.n_bands - 1) / oa.GB * oa.GB;   // bands of the last group
+        const int last = rest - (rest - 1) / oa.GB * oa.GB;   // bands of the last group
         oa.per_group = make_fast_div((uint32_t)oa.GB * CHUNKS * (uint32_t)oa.num_kb);
         oa.per_kb = make_fast_div((uint32_t)oa.GB * CHUNKS);
         oa.per_kb_last = make_fast_div((uint32_t)last * CHUNKS);
@@ -1599,12 +1605,29 @@ cudaError_t launch_overlap_bn(const void *codes, const uint16_t *codebooks, cons
     oa.n_bands = (d.d_out + BN - 1) / BN;
     oa.num_kb = (d.d_in + BK - 1) / BK;
     oa.kb_pad = (oa.num_kb + kWindow - 1) / kWindow * kWindow;
-    oa.total_units = (uint32_t)oa.n_bands * (BN / 16) * (uint32_t)oa.num_kb;   // < 2^31 for any layer of 2^20 x 2^20
+    // The bands the first wave of tiles needs are decoded first, by the
+    // dequantisation kernel on the whole GPU (a fraction of its full-layer
+    // time); the GEMM, launched early behind it, then starts its MMAs at once
+    // instead of waiting for the decoder warps' first panels, which decode
+    // the remaining bands in the order the later waves need them.
+    const int slots = pair_slots<BN, FM, FB>(dev);
+    const long long tiles = pair_tiles(tokens, d.d_out, BN);
+    const int pairs = slots < 1 ? 1 : (tiles < slots ? (int)tiles : slots);
+    const int m_tiles = (tokens + kPairRows - 1) / kPairRows;
+    const int gb = (pairs + m_tiles - 1) / m_tiles;
+    oa.band0 = gb < oa.n_bands ? gb : oa.n_bands;
+    oa.total_units = (uint32_t)(oa.n_bands - oa.band0) * (BN / 16) * (uint32_t)oa.num_kb;   // < 2^31
     const size_t bytes = kClaimBytes + (size_t)oa.n_bands * oa.kb_pad * 4;
-    const cudaError_t e = cudaMemsetAsync(counters, 0, bytes, st);
+    cudaError_t e = cudaMemsetAsync(counters, 0, bytes, st);
     if (e != cudaSuccess) return e;
+    if (oa.band0 > 0) {
+        Dims first = d;
+        first.d_out = oa.band0 * BN < d.d_out ? oa.band0 * BN : d.d_out;
+        e = launch_dequant(codes, codebooks, scales, W, first, st);
+        if (e != cudaSuccess) return e;
+    }
     return launch_gemm_pair_bn<BN, FM, FB>(X, W, Y, tokens, d.d_out, d.d_in, status, st, kGemmWaitLimitNs, 0, dev,
-                                           oa);
+                                           oa, oa.band0 > 0);
 }
 
 template <int FM, int FB>
@@ -1626,6 +1649,27 @@ cudaError_t launch_overlap_fmt(const void *codes, const uint16_t *codebooks, con
     }
 }
 }  // namespace
+
+// Whether the one-kernel prefill beats dequantisation + GEMM for a layer
+// (measured on B200, 2048 tokens): always for two 16-bit codebooks (their
+// dequantisation is the longest: 4096x11008 180.2 vs 190.5 us), otherwise when
+// the bands the first wave of tiles needs -- decoded before the kernel -- are
+// at most a third of the layer (1x16 11008x4096 161.9 vs 165.9 us; with 10 of
+// 18 bands first, 4096x11008 lost: 167.9 vs 163.8 us).
+bool overlap_preferred(const Dims &d, int tokens) {
+    if (!gemm_uses_pair(tokens)) return false;
+    if (d.M == 2 && d.B == 16) return true;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int slots = d.M == 1 ? pair_slots<240, 1, 16>(dev) : pair_slots<240, 2, 8>(dev);
+    const int bn = gemm_pair_tile_n(tokens, d.d_out, slots > 0 ? slots : 1);
+    const long long tiles = pair_tiles(tokens, d.d_out, bn);
+    const int pairs = slots < 1 ? 1 : (tiles < slots ? (int)tiles : slots);
+    const int m_tiles = (tokens + kPairRows - 1) / kPairRows;
+    const long long band0 = (pairs + m_tiles - 1) / m_tiles;
+    const long long n_bands = (d.d_out + bn - 1) / bn;
+    return 3 * band0 <= n_bands;
+}
 
 // Y = X . W^T with W^ decoded into W (d_out x d_in bf16) by the GEMM's own
 // decoder warps; counters: overlap_counter_bytes(d_out, d_in) bytes.

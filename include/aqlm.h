@@ -240,9 +240,10 @@ AQLM_API aqlm_status aqlm_dequant(const void *codes, const uint16_t *codebooks, 
  * aqlm_bf16_gemm (bf16 operands, fp32 accumulation in tensor memory, bf16
  * output rounded to nearest even; CTA pairs past 128 tokens, see
  * aqlm_bf16_gemm_plan), launched early so that its set-up overlaps the
- * dequantisation's end.  For two 16-bit codebooks past 128 tokens, the one
- * kernel of aqlm_gemm_overlap instead (faster there: its decoding is the
- * longest).  Either way Y equals aqlm_bf16_gemm on aqlm_dequant's W^.
+ * dequantisation's end.  Past 128 tokens, aqlm_gemm_overlap's path instead
+ * where it was measured faster on B200: two 16-bit codebooks always, the
+ * other formats when the bands its first wave of tiles needs are at most a
+ * third of the layer.  Either way Y equals aqlm_bf16_gemm on aqlm_dequant's W^.
  *   X: [tokens][d_in] bf16.  Y: [tokens][d_out] bf16 (written).  tokens >= 1.
  *   workspace: at least aqlm_gemm_workspace_bytes(shape, tokens) bytes,
  *   16-byte aligned: a 256-byte status word, the counters aqlm_gemm_overlap
@@ -259,8 +260,10 @@ AQLM_API aqlm_status aqlm_gemm(const void *codes, const uint16_t *codebooks, con
 AQLM_API size_t aqlm_gemm_workspace_bytes(aqlm_shape shape, int32_t tokens);
 
 /*
- * aqlm_gemm_overlap -- the product of aqlm_gemm in ONE kernel that decodes
- * each W^ block once and overlaps the decoding with the MMAs: the CTA-pair
+ * aqlm_gemm_overlap -- the product of aqlm_gemm with the decoding overlapped
+ * with the MMAs, each W^ block decoded once: aqlm_dequant's kernel first
+ * decodes the bands of W^ that the GEMM's first wave of tiles needs, then ONE
+ * kernel does the rest: the CTA-pair
  * GEMM (aqlm_bf16_gemm_plan's width for more than 128 tokens; the same
  * kernel with half-empty pair tiles below) with eight decoder warps and a
  * publisher warp in every CTA.  The decoders write W^ into the workspace in
