@@ -651,19 +651,22 @@ __device__ bool wait_bounded_pair(uint32_t bar, uint32_t parity, Bars *bars, uin
 // CTA turn codes into W^ rows in global memory (the workspace), with the
 // binary32 steps of aqlm_dequant, while the tensor cores run; each CTA's TMA
 // producer loads a W tile only once the units that write it are complete.
+// The bands [0, band0) that the first wave of tiles needs are decoded before
+// the launch (by the dequantisation kernel); the decoder warps take the rest.
 // The work is cut into units of 16 rows x 64 inputs (one k block of a 16-row
 // slice of a band of BN rows).  Units are numbered in the order the tiles
 // need them -- bands in groups of about one wave's worth (GB bands, whose
 // first tiles fall in the same wave), k blocks in order within a group -- and
 // decoder warps claim the next ones from global counters, so the whole GPU
-// decodes what the first wave needs first, and no CTA ever waits for a CTA
+// decodes what the next waves need first, and no CTA ever waits for a CTA
 // that is not running (whoever claims a unit is running and finishes it).
 // Claims (U consecutive units) are dealt over kClaimStreams counters: decoder
 // warp w of a CTA takes claims w, w + 8, w + 16, ... from counter w, which
-// keeps the need order while spreading the atomics over eight L2 lines.  A finished unit adds 1 to its panel's counter
-// (release, GPU scope, after a proxy fence that orders the generic stores
-// before asynchronous-proxy reads); the producer reads the counters of 8 k
-// blocks at a time and loads when a panel holds all BN/16 of its units.
+// keeps the need order while spreading the atomics over eight L2 lines.  A
+// finished unit goes to the CTA's publisher warp, which adds it to its
+// panel's counter (see Mailbox); the producer reads the counters of 32 k
+// blocks at a time, ahead of need, and loads when a panel holds all BN/16 of
+// its units.
 // Division of x < 2^31 by an invariant d as a multiply and a shift (the
 // scheme of Granlund and Montgomery, "Division by invariant integers using
 // multiplication", 1994): s = ceil(log2 d), m = floor(2^(31+s) / d) + 1 < 2^32,
